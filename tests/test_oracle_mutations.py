@@ -1,0 +1,117 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and require a pin to catch each.
+
+This shows the pins are strong enough: a dropped term, a wrong sign or index, a
+transposed operand or a wrong tie rule in any step fails at least one check.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle_pins import ALL_CHECKS
+
+O = oracle.hhr_oracle
+_orig = {name: getattr(O, name) for name in dir(O) if not name.startswith("__")}
+
+
+def _rotate_transposed(R, X):
+    return X @ np.asarray(R, dtype=np.float64)
+
+
+def _bounds_min(Qrot, kmin, kmax):
+    return np.minimum(Qrot[:, None, :] * kmin[None], Qrot[:, None, :] * kmax[None]).sum(axis=(0, 2))
+
+
+def _bounds_one_head(Qrot, kmin, kmax):
+    return _orig["page_bounds"](Qrot[:1], kmin, kmax)
+
+
+def _hamming_one_head(qcodes, codes):
+    return _orig["hamming"](qcodes[:1], codes)
+
+
+def _topk_ties_high(dist, tok, k):
+    order = np.lexsort((-np.asarray(tok), dist))
+    return np.sort(np.asarray(tok)[order[:k]])
+
+
+def _topm_ties_high(scores, m):
+    order = np.lexsort((-np.arange(len(scores)), -np.asarray(scores)))
+    return np.sort(order[:m])
+
+
+def _pack_msb_first(proj):
+    n, bits = proj.shape
+    words = np.zeros((n, bits // 32), dtype=np.uint32)
+    for j in range(bits):
+        words[:, j // 32] |= (proj[:, j] > 0).astype(np.uint32) << np.uint32(31 - j % 32)
+    return words
+
+
+def _attn_no_scale(Qg, Ksel, Vsel, scale):
+    return _orig["sparse_attention"](Qg, Ksel, Vsel, 1.0)
+
+
+def _attn_wrong_sign(Qg, Ksel, Vsel, scale):
+    return _orig["sparse_attention"](Qg, Ksel, Vsel, -scale)
+
+
+def _summaries_unrotated_order(Krot, P):
+    # Off-by-one page boundary: pages start one key late.
+    n, d = Krot.shape
+    return _orig["page_summaries"](np.concatenate([Krot[:1], Krot])[:n], P)
+
+
+def _block_sum(K, P):
+    return _orig["block_means"](K, P) * P
+
+
+def _indexer_eligible_late(q, pos, K, mu, n, P, m_blocks, k):
+    return _orig["indexer_select_one"](q, pos + P, K, mu, n, P, m_blocks, k)
+
+
+def _kept_floor(n_units, m_units, keep_div):
+    if m_units > 0:
+        return min(m_units, n_units)
+    return max(1, n_units // keep_div)
+
+
+def _cands_include_tail(kept, n, P):
+    t = (np.asarray(kept, dtype=np.int64)[:, None] * P + np.arange(P)[None, :]).ravel()
+    return t[t <= n]
+
+
+def _topk_largest_ascending(score, tok, k):
+    order = np.lexsort((tok, np.asarray(score)))
+    return np.sort(np.asarray(tok)[order[:k]])
+
+
+MUTATIONS = {
+    "rotate_transposed": ("rotate", _rotate_transposed),
+    "bound_min_not_max": ("page_bounds", _bounds_min),
+    "bound_drops_heads": ("page_bounds", _bounds_one_head),
+    "hamming_drops_heads": ("hamming", _hamming_one_head),
+    "topk_ties_to_higher": ("top_k_smallest", _topk_ties_high),
+    "topm_ties_to_higher": ("top_m", _topm_ties_high),
+    "pack_msb_first": ("pack_sign_bits", _pack_msb_first),
+    "attention_no_scale": ("sparse_attention", _attn_no_scale),
+    "attention_wrong_sign": ("sparse_attention", _attn_wrong_sign),
+    "summaries_page_shift": ("page_summaries", _summaries_unrotated_order),
+    "block_sum_not_mean": ("block_means", _block_sum),
+    "indexer_causal_off": ("indexer_select_one", _indexer_eligible_late),
+    "kept_floor": ("kept_count", _kept_floor),
+    "candidates_past_end": ("candidates_of", _cands_include_tail),
+    "indexer_smallest_scores": ("top_k_largest", _topk_largest_ascending),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check(O)
+        except (AssertionError, IndexError, ValueError):
+            caught.append(check.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
