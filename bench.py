@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the coarse-to-fine retrieval path on B200.
+
+A step is one HHR decode step for a whole batch: append-encode the newest key of
+every sequence (step a0), select (a1-a4: query prep, page bounds, top-m pages,
+Hamming top-k) and GQA sparse attention (a5), all through the C ABI. Default
+workload: Llama-3.1-8B shapes at 128K context, batch 8 (32 query / 8 KV heads,
+d=128, pages of 32, keep 1/16 of the pages, top-2048, 128-bit codes).
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0). Multi-GPU runs are independent replicas (weak
+scaling, no collective on the data path); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode queries/s (all heads) at 128K ctx; select+attn HBM GB/s vs ~8 TB/s peak"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b_128k_b8")
+    ap.add_argument("--layers", type=int, default=0, help="layer caches rotated (0 = auto)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def required_bytes(wl, lens, m_of):
+    """Algorithmic bytes of one step: summaries + kept-page codes + selected K/V rows."""
+    G, P, d = wl.n_kv_heads, wl.page_size, wl.head_dim
+    summ = codes = kv = 0
+    for n in lens:
+        npg = -(-n // P)
+        m = m_of(npg)
+        cand = min(n, m * P)
+        summ += G * npg * 2 * d * 4
+        codes += G * cand * (wl.code_bits // 8)
+        kv += G * min(wl.top_k, cand) * 2 * d * 2
+    return summ, codes, kv
+
+
+def bound_kernel_bytes(wl, lens):
+    """Algorithmic bytes of one page-bound launch: per (page, group) the 1 KB summary
+    read and the 4-byte bound write; per page its 4-byte page-table entry; per
+    (sequence, group) the 1 KB folded query."""
+    G = wl.n_kv_heads
+    tot = 0
+    for n in lens:
+        npg = -(-n // wl.page_size)
+        tot += npg * G * (2 * wl.head_dim * 4 + 4) + npg * 4 + G * 2 * wl.head_dim * 4
+    return tot
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def _once(self):
+        try:
+            r = subprocess.run(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                "--format=csv,noheader,nounits", "-i", self.uuid],
+                               capture_output=True, text=True, timeout=10)
+            return r.stdout.strip().splitlines()
+        except Exception:
+            return []
+
+    def start(self):
+        self.lines += self._once()
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.uuid], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+                self.lines += out.strip().splitlines()
+            except Exception:
+                self.proc.kill()
+        self.lines += self._once()
+
+    def summary(self):
+        mhz, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def traffic_from_profile(kernel_src_hash):
+    """DRAM bytes per launch of the page-bound kernel from the committed ncu summary,
+    or None if the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "page_bound_kernel_llama8b_128k_b8.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for ln in f:
+            if "=" in ln and not ln.startswith("#"):
+                k, v = ln.split("=", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256") != kernel_src_hash:
+        return None
+    try:
+        return float(vals["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("select.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "hash_hierarchical_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_group_step(O, np_in, wl, b, g, enc, lens_b):
+    """The oracle's decode step for one (sequence, group): append-encode the newest key
+    (its code and its page's summary), select (a1-a4) and attend (a5)."""
+    import numpy as np
+    P, d = wl.page_size, wl.head_dim
+    gs = wl.n_q_heads // wl.n_kv_heads
+    n = lens_b
+    R, W = np_in["R"][g], np_in["W"][g]
+    pt = np_in["page_table"][b]
+    lp = (n - 1) // P
+    page_keys = O.bf16_to_f64(np_in["k_cache"][pt[lp], g, : n - lp * P])
+    kmin, kmax = enc["kmin"].copy(), enc["kmax"].copy()
+    pmin, pmax = O.page_summaries(O.rotate(R, page_keys), P)
+    kmin[lp], kmax[lp] = pmin[0], pmax[0]
+    codes = enc["codes"]
+    codes[n - 1] = O.sign_codes(R, W, page_keys[-1:])[0]
+    m = O.kept_count(-(-n // P), wl.m_pages, wl.keep_div)
+    Qg = O.bf16_to_f64(np_in["q"][b, g * gs:(g + 1) * gs])
+    r = O.select_group(Qg, R, W, kmin, kmax, codes, n, P, m, wl.top_k)
+    idx = r["idx"]
+    rows_k = O.bf16_to_f64(enc["K_rows"](idx))
+    rows_v = O.bf16_to_f64(enc["V_rows"](idx))
+    return O.sparse_attention(Qg, rows_k, rows_v, 1.0 / math.sqrt(d))
+
+
+def oracle_setup(wl, inp, groups):
+    """Host copies of one sequence's cache and the oracle's encoding of `groups` (untimed)."""
+    import numpy as np
+    import hhr_synth as S
+    import oracle
+    O = oracle.hhr_oracle
+    np_in = S.to_numpy_inputs({k: inp[k] for k in ("q", "R", "W", "page_table", "seq_len")})
+    b = 0
+    n = int(np_in["seq_len"][b])
+    P = wl.page_size
+    npg = -(-n // P)
+    pt = np_in["page_table"][b]
+    phys = inp["page_table"][b, :npg].long()
+    kc = inp["k_cache"][phys].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    vc = inp["v_cache"][phys].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    local_pt = np.arange(npg, dtype=np.int32)
+    np_in["k_cache"], np_in["v_cache"] = kc, vc
+    np_in["page_table"] = local_pt[None, :]
+    encs = {}
+    for g in groups:
+        e = O.encode_group(kc, local_pt, g, n, P, np_in["R"][g], np_in["W"][g])
+
+        def rows(cache, g=g):
+            return lambda idx: cache[idx // P, g, idx % P]
+        e["K_rows"], e["V_rows"] = rows(kc), rows(vc)
+        encs[g] = e
+    return O, np_in, encs, n
+
+
+def cpu_threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([1] + [int(i.get("num_threads", 1)) for i in info])
+    except Exception:
+        return 1
+
+
+def run_oracle_timed(wl, inp, seconds=None, steps=None, warmup=0):
+    """Time the oracle's per-group decode step; returns (seconds per group, groups run)."""
+    from threadpoolctl import threadpool_limits
+    groups = list(range(min(2, wl.n_kv_heads)))
+    O, np_in, encs, n = oracle_setup(wl, inp, groups)
+    with threadpool_limits(limits=1):
+        for i in range(warmup):
+            g = groups[i % len(groups)]
+            oracle_group_step(O, np_in, wl, 0, g, encs[g], n)
+        t0 = time.perf_counter()
+        done = 0
+        while True:
+            g = groups[done % len(groups)]
+            oracle_group_step(O, np_in, wl, 0, g, encs[g], n)
+            done += 1
+            el = time.perf_counter() - t0
+            if steps is not None and done >= steps:
+                break
+            if seconds is not None and el >= seconds:
+                break
+        return el / done, done
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    import hhr_synth as S
+    wl = S.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        # The oracle arm: rank 0 alone runs it on the host cores.
+        if rank != 0:
+            return
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        inp = S.make_inputs(wl, device=dev, layer=0)
+        per_group, done = run_oracle_timed(wl, inp, steps=args.steps, warmup=args.warmup)
+        per_query = per_group * wl.n_kv_heads
+        val = 1.0 / per_query
+        cores = 1
+        line = {
+            "metric": METRIC, "value": val, "unit": "queries/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_group * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "batch": wl.batch, "context": wl.seq_lens[0],
+                       "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads,
+                       "page_size": wl.page_size,
+                       "keep": f"1/{wl.keep_div}" if wl.keep_div else f"{wl.m_pages} pages",
+                       "top_k": wl.top_k, "code_bits": wl.code_bits},
+            "cpu_baseline": {"value": val, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step = the fp64 oracle's decode step for one "
+                                       f"(sequence, KV group) of {wl.name} (append-encode the "
+                                       f"newest key, bounds, top-m, Hamming top-k, attention); "
+                                       f"a query = {wl.n_kv_heads} groups"},
+            "e2e": {"value": val, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    from hash_hierarchical_top_b200 import build, hhr
+    from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    lens = S.seq_lens_of(wl)
+    P = wl.page_size
+    m_of = lambda npg: min(npg, -(-npg // wl.keep_div)) if wl.m_pages == 0 else min(wl.m_pages, npg)
+    summ_b, codes_b, kv_b = required_bytes(wl, lens, m_of)
+    req = summ_b + codes_b + kv_b
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    L = args.layers or max(2, math.ceil(4 * l2 / req))
+
+    # Layer caches: inputs drawn on the device (seeded), cache encoded once (untimed).
+    layers = []
+    for l in range(L):
+        inp = S.make_inputs(wl, device=dev, layer=l)
+        d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, P, inp["max_pages"],
+                          inp["n_phys"])
+        cache = LayerCache(d, dev)
+        zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+        hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
+                            int(inp["seq_len"].max()), inp["R"], inp["W"], cache.page_minmax,
+                            cache.codes, None)
+        start = (inp["seq_len"] - 1).to(torch.int32)
+        one = torch.ones(wl.batch, dtype=torch.int32, device=dev)
+        layers.append((inp, d, cache, start, one))
+    d0 = layers[0][1]
+    step = DecodeStep(d0, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def run(i):
+        inp, d, cache, start, one = layers[i % L]
+        step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
+                  inp["R"], inp["W"], cache, start, one)
+
+    kernels_per_step = 7  # encode 1 + select 4 (qprep, bound, top-m, hamming) + attention 2
+    for i in range(max(args.warmup, 3)):
+        run(i)
+    torch.cuda.synchronize()
+    st, bits = hhr.hhr_read_device_status()
+    if st != hhr.HHR_OK:
+        raise RuntimeError(f"device status {bits}")
+
+    # Timed region: K steps, events on the launching stream; per-step events around
+    # the page-bound kernel (the dominant HBM stream) through the library's hook.
+    K = args.steps
+    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = Clocks(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        hhr.hhr_profile_next("bound", ev_b[i][0], ev_b[i][1])
+        run(args.warmup + i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    bound_ms = [a.elapsed_time(b) for a, b in ev_b]
+    ms_t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_total = float(ms_t.item())
+    ms_step = ms_total / K
+    value = world * wl.batch * K / (ms_total / 1e3)
+
+    # Per-kernel averages (separate untimed pass, same launches).
+    kern = {}
+    for name in ("encode", "qprep", "bound", "topm", "hamming", "attn", "combine"):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(50)]
+        for i in range(50):
+            hhr.hhr_profile_next(name, evs[i][0], evs[i][1])
+            run(i)
+        torch.cuda.synchronize()
+        kern[name] = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+
+    # End to end through the public API with host buffers: every step copies the query
+    # and the newest K/V rows from pinned host memory, runs the step, reads the output.
+    e2e = None
+    if not args.no_e2e:
+        from cuda.bindings import runtime as rt
+        inp, d, cache, start, one = layers[0]
+        Bq = wl.batch
+        q_host = inp["q"].cpu().pin_memory()
+        G = wl.n_kv_heads
+        lens_h = inp["seq_len"].cpu().tolist()
+        pt_h = inp["page_table"].cpu()
+        new_k = torch.empty(Bq, G, wl.head_dim, dtype=torch.bfloat16).pin_memory()
+        new_v = torch.empty_like(new_k).pin_memory()
+        for b in range(Bq):
+            t = lens_h[b] - 1
+            phys = int(pt_h[b, t // P])
+            new_k[b] = inp["k_cache"][phys, :, t % P].cpu()
+            new_v[b] = inp["v_cache"][phys, :, t % P].cpu()
+        out_host = torch.empty(Bq, wl.n_q_heads, wl.head_dim, dtype=torch.float32).pin_memory()
+        row_bytes = wl.head_dim * 2
+        sraw = stream.cuda_stream
+        esz = inp["k_cache"].element_size()
+        dsts = []
+        for b in range(Bq):
+            t = lens_h[b] - 1
+            phys = int(pt_h[b, t // P])
+            off = ((phys * G) * P + t % P) * wl.head_dim * esz
+            dsts.append(off)
+
+        def e2e_step():
+            inp["q"].copy_(q_host, non_blocking=True)
+            for b in range(Bq):
+                for cache_t, src in ((inp["k_cache"], new_k), (inp["v_cache"], new_v)):
+                    err, = rt.cudaMemcpy2DAsync(
+                        cache_t.data_ptr() + dsts[b], P * row_bytes,
+                        src.data_ptr() + b * G * row_bytes, row_bytes, row_bytes, G,
+                        rt.cudaMemcpyKind.cudaMemcpyHostToDevice, sraw)
+                    if err != rt.cudaError_t.cudaSuccess:
+                        raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
+            step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
+                      inp["seq_len"], inp["R"], inp["W"], cache, start, one)
+            out_host.copy_(step.out, non_blocking=True)
+
+        for _ in range(5):
+            e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(50, min(K, 2000))
+        a, bev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        bev.record(stream)
+        torch.cuda.synchronize()
+        ms_e = torch.tensor([a.elapsed_time(bev)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(ms_e, op=dist.ReduceOp.MAX)
+        h2d = q_host.numel() * 2 + 2 * new_k.numel() * 2
+        e2e = {"value": world * Bq * Ke / (float(ms_e.item()) / 1e3), "unit": "queries/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * 4,
+               "steps": Ke}
+
+    peak, peak_kind = measured_peaks()
+    bound_bytes = bound_kernel_bytes(wl, lens)
+    bound_avg_ms = statistics.mean(bound_ms)
+    achieved = bound_bytes / (bound_avg_ms / 1e3) / 1e9
+    traffic = traffic_from_profile(kernel_source_hash())
+    step_gbs = req / (ms_step / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_group, done = run_oracle_timed(wl, layers[0][0], seconds=args.cpu_seconds)
+        cpu = {"value": 1.0 / (per_group * wl.n_kv_heads), "unit": "queries/s",
+               "cores": 1, "kind": "oracle",
+               "sample": f"{done} oracle decode steps of single (sequence, KV group) pairs of "
+                         f"{wl.name} (append-encode, bounds, top-m, Hamming top-k, attention) "
+                         f"in {args.cpu_seconds:.0f} s on 1 thread; a query = "
+                         f"{wl.n_kv_heads} groups"}
+
+    if rank == 0:
+        ck = clocks.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "context": lens[0],
+                       "q_heads": wl.n_q_heads, "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
+                       "page_size": P,
+                       "keep": f"1/{wl.keep_div}" if wl.keep_div else f"{wl.m_pages} pages",
+                       "top_k": wl.top_k,
+                       "code_bits": wl.code_bits, "layer_caches_rotated": L,
+                       "l2": f"inputs larger than L2: steps rotate over {L} layer caches, "
+                             f"{L * req / 1e6:.0f} MB of required bytes per cycle vs "
+                             f"{l2 / 1e6:.0f} MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "page_bound_kernel",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "traffic": traffic, "algorithmic_bytes": bound_bytes,
+                         "avg_launch_us": bound_avg_ms * 1e3},
+            "step_hbm": {"required_bytes": req, "summaries": summ_b, "codes": codes_b,
+                         "kv_rows": kv_b, "achieved_gbs": step_gbs,
+                         "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
+                         "frac_of_measured": step_gbs / peak},
+            "kernels_us": kern,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": ck,
+            "gpu_launches": kernels_per_step * K,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

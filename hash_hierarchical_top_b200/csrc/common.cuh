@@ -1,0 +1,113 @@
+// Shared device helpers of the retrieval kernels: bf16 widening, warp/block
+// reductions and scans, order-preserving float keys and the device status word.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hhr {
+
+constexpr int kD = 128;         // head_dim supported by every kernel
+constexpr int kWords = 4;       // 128-bit codes as 4 x uint32
+constexpr int kMaxGroup = 8;    // query heads per KV group
+constexpr unsigned kFull = 0xffffffffu;
+
+// Device-side status bits (never a trap): bad page id, bad token index, clipped append.
+constexpr int kStatusBadPage = 1;
+constexpr int kStatusBadToken = 2;
+constexpr int kStatusClipped = 4;
+
+__device__ int g_status;
+
+__device__ __forceinline__ void flag_status(int bit) {
+  if ((*(volatile int*)&g_status & bit) == 0) atomicOr(&g_status, bit);
+}
+
+// bf16 bit pattern -> float (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(two & 0xffff0000u); }
+__device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Unpack 4 bf16 (two 32-bit words) to 4 floats.
+__device__ __forceinline__ float4 bf16x4_to_f4(uint2 w) {
+  return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+// Transposed warp reduction: on entry every lane holds v[0..31]; on exit lane l
+// holds in v[0] the sum over all lanes of v[l]. 31 shuffles instead of 32 x 5.
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      float send = upper ? v[i] : v[i + s];
+      float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, s);
+    }
+  }
+  return v[0];
+}
+
+// Inclusive warp scan of an int.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Exclusive block scan of one int per thread; blockDim.x a multiple of 32, <= 1024.
+// `scratch` holds >= 33 ints of shared memory. Returns the exclusive prefix and
+// writes the block total to *total. Contains __syncthreads(): call uniformly.
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int incl = warp_incl_scan(v, lane);
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nwarps ? scratch[lane] : 0;
+    int wi = warp_incl_scan(w, lane);
+    if (lane < nwarps) scratch[lane] = wi - w;
+    if (lane == 31) scratch[32] = wi;
+  }
+  __syncthreads();
+  int res = scratch[warp] + incl - v;
+  *total = scratch[32];
+  __syncthreads();
+  return res;
+}
+
+// Order-preserving map of a float to uint32 (larger float -> larger key; -0 < +0).
+__device__ __forceinline__ uint32_t f2key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Kept pages (or blocks) for a row of n units: m_pages > 0 -> min(m_pages, n),
+// else ceil(n / keep_div), never more than n.
+__device__ __host__ __forceinline__ int kept_for(int n, int m_pages, int keep_div) {
+  if (n <= 0) return 0;
+  if (m_pages > 0) return m_pages < n ? m_pages : n;
+  int m = (n + keep_div - 1) / keep_div;
+  return m < n ? m : n;
+}
+
+}  // namespace hhr

@@ -1,0 +1,380 @@
+// C ABI of the retrieval path: argument validation, workspace layout and launches.
+// Every kernel lives in the headers included below (one translation unit, so the
+// device status word is a single symbol).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+
+#include "../../include/hhr.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "encode.cuh"
+#include "select.cuh"
+
+using namespace hhr;
+
+namespace {
+
+constexpr int kMaxPagesPerSeq = 32768;  // top-m keys staged in 128 KB of shared memory
+constexpr int kMaxTokCand = 32768;      // indexer token candidates per query
+constexpr int kMaxDevices = 64;
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int check_dims(const hhr_dims* d) {
+  if (d == nullptr) return HHR_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->page_size < 1 ||
+      d->max_pages_per_seq < 1 || d->n_phys_pages < 1)
+    return HHR_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads != 0) return HHR_ERR_INVALID_ARG;
+  if (d->head_dim != kD || d->code_bits != 32 * kWords) return HHR_ERR_UNSUPPORTED;
+  if (d->page_size > 256 || d->batch > 65535 || d->n_kv_heads > 65535)
+    return HHR_ERR_UNSUPPORTED;
+  if (d->max_pages_per_seq > kMaxPagesPerSeq) return HHR_ERR_UNSUPPORTED;
+  return HHR_OK;
+}
+
+int check_group(const hhr_dims* d) {
+  return (d->n_q_heads / d->n_kv_heads > kMaxGroup) ? HHR_ERR_UNSUPPORTED : HHR_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done_per_dev[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess) done_per_dev[dev] = true;
+  (void)bytes;
+  return e;
+}
+
+bool g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
+    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices];
+
+struct SelectLayout {
+  size_t qpn, q_rot, q_code, bounds, kept, kept_count, tok, total;
+};
+
+int kept_max(const hhr_dims* d, int m_pages, int keep_div) {
+  return kept_for(d->max_pages_per_seq, m_pages, keep_div);
+}
+
+SelectLayout select_layout(const hhr_dims* d, int mode, int m_max) {
+  SelectLayout L{};
+  const size_t B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, maxp = d->max_pages_per_seq;
+  size_t off = 0;
+  if (mode == HHR_MODE_HASH) {
+    L.qpn = off;    off += align256(B * G * 2 * kD * 4);
+    L.q_rot = off;  off += align256(B * Hq * kD * 4);
+    L.q_code = off; off += align256(B * Hq * kWords * 4);
+    L.bounds = off; off += align256(B * G * maxp * 4);
+    L.kept = off;   off += align256(B * G * (size_t)m_max * 4);
+    L.kept_count = off; off += align256(B * G * 4);
+  } else {
+    const size_t T = Hq;
+    L.bounds = off; off += align256(B * T * maxp * 4);
+    L.kept = off;   off += align256(B * T * (size_t)m_max * 4);
+    L.kept_count = off; off += align256(B * T * 4);
+    L.tok = off;    off += align256(B * T * (size_t)m_max * d->page_size * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, int top_k) {
+  int st = check_dims(d);
+  if (st != HHR_OK) return st;
+  if (top_k < 1 || m_pages < 0 || keep_div < 0) return HHR_ERR_INVALID_ARG;
+  if (mode == HHR_MODE_HASH) {
+    if ((m_pages > 0) == (keep_div > 0)) return HHR_ERR_INVALID_ARG;
+    if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
+    if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
+      return HHR_ERR_UNSUPPORTED;
+  } else if (mode == HHR_MODE_INDEXER) {
+    if (m_pages < 1 || keep_div != 0) return HHR_ERR_INVALID_ARG;
+    if (d->n_kv_heads != 1) return HHR_ERR_INVALID_ARG;
+    if ((long long)kept_max(d, m_pages, 0) * d->page_size > kMaxTokCand)
+      return HHR_ERR_UNSUPPORTED;
+    if ((long long)d->batch * d->n_q_heads > 0x7fffffffLL) return HHR_ERR_UNSUPPORTED;
+  } else {
+    return HHR_ERR_INVALID_ARG;
+  }
+  return HHR_OK;
+}
+
+// One-shot event pairs of hhr_profile_next, per host thread.
+struct ProfPair {
+  cudaEvent_t start, stop;
+};
+thread_local ProfPair g_prof[HHR_KERNEL_COUNT];
+
+void prof_begin(int k, cudaStream_t s) {
+  if (g_prof[k].start != nullptr) cudaEventRecord(g_prof[k].start, s);
+}
+void prof_end(int k, cudaStream_t s) {
+  if (g_prof[k].stop != nullptr) cudaEventRecord(g_prof[k].stop, s);
+  g_prof[k].start = nullptr;
+  g_prof[k].stop = nullptr;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? HHR_OK : HHR_ERR_CUDA;
+}
+
+int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
+  if (dst == nullptr || bytes == 0) return HHR_OK;
+  return cudaMemcpyAsync(dst, ws + off, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess
+             ? HHR_OK
+             : HHR_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hhr_status_string(int s) {
+  switch (s) {
+    case HHR_OK: return "HHR_OK";
+    case HHR_ERR_INVALID_ARG: return "HHR_ERR_INVALID_ARG";
+    case HHR_ERR_UNSUPPORTED: return "HHR_ERR_UNSUPPORTED";
+    case HHR_ERR_CUDA: return "HHR_ERR_CUDA";
+    case HHR_ERR_WORKSPACE: return "HHR_ERR_WORKSPACE";
+    case HHR_ERR_DEVICE_STATUS: return "HHR_ERR_DEVICE_STATUS";
+    default: return "HHR_UNKNOWN_STATUS";
+  }
+}
+
+int hhr_profile_next(int kernel, void* start_event, void* stop_event) {
+  if (kernel < 0 || kernel >= HHR_KERNEL_COUNT) return HHR_ERR_INVALID_ARG;
+  g_prof[kernel].start = (cudaEvent_t)start_event;
+  g_prof[kernel].stop = (cudaEvent_t)stop_event;
+  return HHR_OK;
+}
+
+int hhr_kept_max(const hhr_dims* d, int m_pages, int keep_div) {
+  if (check_dims(d) != HHR_OK || m_pages < 0 || keep_div < 0 || (m_pages == 0 && keep_div == 0))
+    return -1;
+  return kept_max(d, m_pages, keep_div);
+}
+
+int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* page_table,
+                    const int32_t* start, const int32_t* n_new, int max_new, const float* R,
+                    const float* W, float* page_minmax, uint32_t* codes, float* block_mean,
+                    void* stream) {
+  int st = check_dims(d);
+  if (st != HHR_OK) return st;
+  if (k_cache == nullptr || page_table == nullptr || start == nullptr || n_new == nullptr)
+    return HHR_ERR_INVALID_ARG;
+  const bool hashing = page_minmax != nullptr || codes != nullptr;
+  if (hashing && (page_minmax == nullptr || codes == nullptr || R == nullptr || W == nullptr))
+    return HHR_ERR_INVALID_ARG;
+  if (!hashing && block_mean == nullptr) return HHR_ERR_INVALID_ARG;
+  if (max_new < 0) return HHR_ERR_INVALID_ARG;
+  if (max_new == 0) return HHR_OK;
+  const long long pages = (long long)(max_new + d->page_size - 1) / d->page_size + 1;
+  if (pages > 0x7fffffffLL) return HHR_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  EncodeArgs a{k_cache, page_table, start, n_new, hashing ? R : nullptr, hashing ? W : nullptr,
+               page_minmax, codes, block_mean, d->n_kv_heads, d->page_size,
+               d->max_pages_per_seq, d->n_phys_pages, max_new};
+  size_t smem = hashing ? encode_page_smem() : 0;
+  if (hashing && allow_smem(encode_page_kernel, smem, g_smem_encode) != cudaSuccess)
+    return HHR_ERR_CUDA;
+  dim3 grid((unsigned)pages, d->n_kv_heads, d->batch);
+  prof_begin(HHR_KERNEL_ENCODE, s);
+  encode_page_kernel<<<grid, 128, smem, s>>>(a);
+  prof_end(HHR_KERNEL_ENCODE, s);
+  return launch_status();
+}
+
+size_t hhr_select_workspace_bytes(const hhr_dims* d, int mode, int m_pages, int keep_div,
+                                  int top_k) {
+  if (check_select_params(d, mode, m_pages, keep_div, top_k) != HHR_OK) return 0;
+  return select_layout(d, mode, kept_max(d, m_pages, keep_div)).total;
+}
+
+int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* seq_len,
+               const int32_t* q_pos, const int32_t* page_table, const float* R, const float* W,
+               const float* page_minmax, const uint32_t* codes, const float* block_mean,
+               const uint16_t* k_cache, int m_pages, int keep_div, int top_k, int32_t* out_idx,
+               int32_t* out_count, void* workspace, size_t ws_bytes, hhr_trace* trace,
+               void* stream) {
+  int st = check_select_params(d, mode, m_pages, keep_div, top_k);
+  if (st != HHR_OK) return st;
+  if (q == nullptr || seq_len == nullptr || page_table == nullptr || out_idx == nullptr ||
+      out_count == nullptr || workspace == nullptr)
+    return HHR_ERR_INVALID_ARG;
+  if (mode == HHR_MODE_HASH &&
+      (R == nullptr || W == nullptr || page_minmax == nullptr || codes == nullptr))
+    return HHR_ERR_INVALID_ARG;
+  if (mode == HHR_MODE_INDEXER && (q_pos == nullptr || block_mean == nullptr || k_cache == nullptr))
+    return HHR_ERR_INVALID_ARG;
+  const int m_max = kept_max(d, m_pages, keep_div);
+  const SelectLayout L = select_layout(d, mode, m_max);
+  if (ws_bytes < L.total) return HHR_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = static_cast<char*>(workspace);
+  const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, P = d->page_size;
+  const int maxp = d->max_pages_per_seq;
+  float* bounds = reinterpret_cast<float*>(ws + L.bounds);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
+  int32_t* kept_count = reinterpret_cast<int32_t*>(ws + L.kept_count);
+  if (allow_smem(select_largest_kernel, 0, g_smem_sel) != cudaSuccess) return HHR_ERR_CUDA;
+
+  if (mode == HHR_MODE_HASH) {
+    float* qpn = reinterpret_cast<float*>(ws + L.qpn);
+    float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
+    uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
+    if (allow_smem(qprep_kernel, 0, g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
+    if (allow_smem(hamming_topk_kernel, 0, g_smem_ham) != cudaSuccess) return HHR_ERR_CUDA;
+    prof_begin(HHR_KERNEL_QPREP, s);
+    qprep_kernel<<<dim3(G, B), 128, qprep_smem(), s>>>(
+        QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
+    prof_end(HHR_KERNEL_QPREP, s);
+    if ((st = launch_status()) != HHR_OK) return st;
+    prof_begin(HHR_KERNEL_BOUND, s);
+    page_bound_kernel<<<dim3((maxp + kPagesPerCta - 1) / kPagesPerCta, G, B), kBoundWarps * 32,
+                        0, s>>>(
+        BoundArgs{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp, d->n_phys_pages});
+    prof_end(HHR_KERNEL_BOUND, s);
+    if ((st = launch_status()) != HHR_OK) return st;
+    SelectArgs sa{};
+    sa.scores = bounds; sa.stride = maxp; sa.rows_per_b = G; sa.seq_len = seq_len;
+    sa.q_pos = nullptr; sa.P = P; sa.mode = 0; sa.m_max = m_max; sa.unit = 0;
+    sa.m_pages = m_pages; sa.keep_div = keep_div; sa.top_k = 0;
+    sa.out = kept; sa.out_stride = m_max; sa.out_count = kept_count; sa.pad_out = 0;
+    prof_begin(HHR_KERNEL_TOPM, s);
+    select_largest_kernel<<<B * G, kSelThreads, (size_t)maxp * 4, s>>>(sa);
+    prof_end(HHR_KERNEL_TOPM, s);
+    if ((st = launch_status()) != HHR_OK) return st;
+    HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
+    prof_begin(HHR_KERNEL_HAMMING, s);
+    hamming_topk_kernel<<<B * G, kHamThreads, hamming_smem(Hq / G, m_max * P), s>>>(ha);
+    prof_end(HHR_KERNEL_HAMMING, s);
+    if ((st = launch_status()) != HHR_OK) return st;
+    if (trace != nullptr) {
+      if ((st = copy_trace(trace->q_rot, ws, L.q_rot, (size_t)B * Hq * kD * 4, s))) return st;
+      if ((st = copy_trace(trace->q_code, ws, L.q_code, (size_t)B * Hq * kWords * 4, s))) return st;
+      if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * G * maxp * 4, s))) return st;
+      if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * G * m_max * 4, s))) return st;
+      if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * G * 4, s))) return st;
+    }
+    return HHR_OK;
+  }
+
+  // Indexer variant (HISA).
+  const int T = Hq;
+  float* tok = reinterpret_cast<float*>(ws + L.tok);
+  if (allow_smem(block_score_kernel, 0, g_smem_blk) != cudaSuccess) return HHR_ERR_CUDA;
+  prof_begin(HHR_KERNEL_BLOCK, s);
+  block_score_kernel<<<dim3((maxp + kBlkTile - 1) / kBlkTile, (T + kQTile - 1) / kQTile, B),
+                       kBlkTile, block_score_smem(), s>>>(
+      BlockScoreArgs{q, block_mean, page_table, seq_len, q_pos, bounds, T, P, maxp,
+                     d->n_phys_pages});
+  prof_end(HHR_KERNEL_BLOCK, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  SelectArgs sb{};
+  sb.scores = bounds; sb.stride = maxp; sb.rows_per_b = T; sb.seq_len = seq_len;
+  sb.q_pos = q_pos; sb.P = P; sb.mode = 0; sb.m_max = m_max; sb.unit = 0;
+  sb.m_pages = m_pages; sb.keep_div = 0; sb.top_k = 0;
+  sb.out = kept; sb.out_stride = m_max; sb.out_count = kept_count; sb.pad_out = 0;
+  prof_begin(HHR_KERNEL_TOPM, s);
+  select_largest_kernel<<<B * T, kSelThreads, (size_t)maxp * 4, s>>>(sb);
+  prof_end(HHR_KERNEL_TOPM, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  const int C = m_max * P;
+  prof_begin(HHR_KERNEL_TOKEN, s);
+  token_score_kernel<<<dim3((C + kTokWarps * 32 - 1) / (kTokWarps * 32), B * T), kTokWarps * 32,
+                       0, s>>>(TokenScoreArgs{q, k_cache, page_table, seq_len, q_pos, kept,
+                                              kept_count, tok, T, P, maxp, d->n_phys_pages,
+                                              m_max});
+  prof_end(HHR_KERNEL_TOKEN, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  SelectArgs sc{};
+  sc.scores = tok; sc.stride = C; sc.rows_per_b = T; sc.seq_len = seq_len; sc.q_pos = q_pos;
+  sc.P = P; sc.mode = 1; sc.kept_count = kept_count; sc.kept_units = kept; sc.m_max = m_max;
+  sc.unit = P; sc.m_pages = 0; sc.keep_div = 0; sc.top_k = top_k;
+  sc.out = out_idx; sc.out_stride = top_k; sc.out_count = out_count; sc.pad_out = 1;
+  prof_begin(HHR_KERNEL_TOKEN_TOPK, s);
+  select_largest_kernel<<<B * T, kSelThreads, (size_t)C * 4, s>>>(sc);
+  prof_end(HHR_KERNEL_TOKEN_TOPK, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  if (trace != nullptr) {
+    if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * T * maxp * 4, s))) return st;
+    if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * T * m_max * 4, s))) return st;
+    if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * T * 4, s))) return st;
+  }
+  return HHR_OK;
+}
+
+size_t hhr_attn_workspace_bytes(const hhr_dims* d, int top_k) {
+  if (check_dims(d) != HHR_OK || check_group(d) != HHR_OK || top_k < 1) return 0;
+  const size_t ns = (top_k + kChunk - 1) / kChunk;
+  const size_t rows = (size_t)d->batch * d->n_kv_heads;
+  const size_t gs = d->n_q_heads / d->n_kv_heads;
+  return align256(rows * ns * gs * kD * 4) + align256(rows * ns * gs * 2 * 4);
+}
+
+int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cache,
+                    const uint16_t* v_cache, const int32_t* page_table, const int32_t* seq_len,
+                    const int32_t* idx, const int32_t* count, int top_k, float scale, float* out,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_dims(d);
+  if (st != HHR_OK) return st;
+  if ((st = check_group(d)) != HHR_OK) return st;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || page_table == nullptr ||
+      seq_len == nullptr || idx == nullptr || count == nullptr || out == nullptr ||
+      workspace == nullptr)
+    return HHR_ERR_INVALID_ARG;
+  if (top_k < 1 || !(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
+  const size_t need = hhr_attn_workspace_bytes(d, top_k);
+  if (ws_bytes < need) return HHR_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads;
+  const int ns = (top_k + kChunk - 1) / kChunk;
+  const int gs = Hq / G;
+  char* ws = static_cast<char*>(workspace);
+  float* part_o = reinterpret_cast<float*>(ws);
+  float* part_ml = reinterpret_cast<float*>(ws + align256((size_t)B * G * ns * gs * kD * 4));
+  if (allow_smem(sparse_attn_kernel, 0, g_smem_attn) != cudaSuccess) return HHR_ERR_CUDA;
+  AttnArgs a{q, k_cache, v_cache, page_table, seq_len, idx, count, part_o, part_ml,
+             scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
+             d->n_phys_pages, top_k, ns};
+  prof_begin(HHR_KERNEL_ATTN, s);
+  sparse_attn_kernel<<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  prof_end(HHR_KERNEL_ATTN, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  prof_begin(HHR_KERNEL_COMBINE, s);
+  attn_combine_kernel<<<dim3(Hq, B), kD, 0, s>>>(
+      CombineArgs{part_o, part_ml, count, out, Hq, G, top_k, ns});
+  prof_end(HHR_KERNEL_COMBINE, s);
+  return launch_status();
+}
+
+int hhr_read_device_status(void* stream, int* bits) {
+  cudaStream_t s = (cudaStream_t)stream;
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return HHR_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HHR_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return HHR_ERR_CUDA;
+  }
+  if (bits != nullptr) *bits = v;
+  return v == 0 ? HHR_OK : HHR_ERR_DEVICE_STATUS;
+}
+
+}  // extern "C"

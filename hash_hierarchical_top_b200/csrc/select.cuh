@@ -1,0 +1,543 @@
+// Steps a1-a4: query preparation, page-level bounds, top-m, Hamming scan and top-k
+// (HHR), and the block filter + token refinement of the indexer variant (HISA).
+#pragma once
+#include "common.cuh"
+#include "encode.cuh"
+
+namespace hhr {
+
+// ---------------------------------------------------------------------------- a1
+// HHR page, Abstract (queries are rotated by the same R_h and encoded like keys).
+// One CTA of 128 threads per (KV group, sequence). For each query head of the
+// group: q' = R_g q (thread i owns channel i), code bits = [W_g q' > 0] (thread j
+// owns bit j). Also folds the group into the two bound vectors
+//   qneg_c = sum_h min(q'_hc, 0),  qpos_c = sum_h max(q'_hc, 0),
+// so that sum_h max(q'_hc*kmin_c, q'_hc*kmax_c) = qneg_c*kmin_c + qpos_c*kmax_c
+// (kmin <= kmax: a positive q' picks kmax, a negative one kmin). The page bound
+// then becomes one 256-long dot product per page.
+struct QPrepArgs {
+  const uint16_t* q;
+  const float* R;
+  const float* W;
+  float* q_rot;      // [B][Hq][d]
+  uint32_t* q_code;  // [B][Hq][4]
+  float* qpn;        // [B][G][2][d]: [0] = qneg, [1] = qpos
+  int Hq, G;
+};
+
+__global__ void __launch_bounds__(128) qprep_kernel(QPrepArgs a) {
+  extern __shared__ float4 smem_f4[];
+  float* RT = reinterpret_cast<float*>(smem_f4);
+  float* WT = RT + kD * kTS;
+  float* qx = WT + kD * kTS;
+  float* qr = qx + kD;
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int gs = a.Hq / a.G;
+  stage_transposed(a.R + (size_t)g * kD * kD, RT);
+  stage_transposed(a.W + (size_t)g * kD * kD, WT);
+  float qneg = 0.f, qpos = 0.f;
+  for (int hh = 0; hh < gs; ++hh) {
+    const int h = g * gs + hh;
+    __syncthreads();
+    qx[tid] = bf16_to_f(a.q[((size_t)b * a.Hq + h) * kD + tid]);
+    __syncthreads();
+    float acc = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < kD; ++c) acc = fmaf(RT[c * kTS + tid], qx[c], acc);
+    qr[tid] = acc;
+    a.q_rot[((size_t)b * a.Hq + h) * kD + tid] = acc;
+    qneg += fminf(acc, 0.f);
+    qpos += fmaxf(acc, 0.f);
+    __syncthreads();
+    float p = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < kD; ++c) p = fmaf(WT[c * kTS + tid], qr[c], p);
+    unsigned word = __ballot_sync(kFull, p > 0.f);
+    if (lane == 0) a.q_code[((size_t)b * a.Hq + h) * kWords + warp] = word;
+  }
+  float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
+  o[tid] = qneg;
+  o[kD + tid] = qpos;
+}
+
+inline size_t qprep_smem() { return (size_t)(2 * kD * kTS + 2 * kD) * sizeof(float); }
+
+// ---------------------------------------------------------------------------- a2
+// HHR page, Abstract: page-level logit bounds of the rotated keys prune pages.
+// bound_p = qneg . kmin_p + qpos . kmax_p over the page summary (1 KB per page and
+// group). The summaries are the dominant HBM stream of the whole path, so this
+// kernel is a pure streaming GEMV: one warp per page, every lane loads one float4
+// of kmin and one of kmax (a warp reads the page's 1 KB in two coalesced 512-byte
+// transactions), 8 FMAs, one warp sum. Each warp handles kPagesPerWarp pages with
+// all loads issued before any arithmetic so that 2*kPagesPerWarp 16-byte loads per
+// lane are in flight.
+constexpr int kBoundWarps = 8;
+constexpr int kPagesPerWarp = 8;
+constexpr int kPagesPerCta = kBoundWarps * kPagesPerWarp;
+
+struct BoundArgs {
+  const float* qpn;
+  const float* page_minmax;
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  float* bounds;  // [B][G][maxp]
+  int G, P, maxp, n_phys;
+};
+
+__global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int npg = ceil_div(a.seq_len[b], a.P);
+  const int base = blockIdx.x * kPagesPerCta + warp * kPagesPerWarp;
+  if (base >= min(npg, a.maxp)) return;
+  const float4 qn = reinterpret_cast<const float4*>(a.qpn + ((size_t)b * a.G + g) * 2 * kD)[lane];
+  const float4 qp =
+      reinterpret_cast<const float4*>(a.qpn + ((size_t)b * a.G + g) * 2 * kD + kD)[lane];
+  // Page ids of this warp's pages: lane i < kPagesPerWarp reads one, then broadcast.
+  int my_phys = -1;
+  if (lane < kPagesPerWarp && base + lane < min(npg, a.maxp))
+    my_phys = a.page_table[(size_t)b * a.maxp + base + lane];
+  float4 mn[kPagesPerWarp], mx[kPagesPerWarp];
+#pragma unroll
+  for (int i = 0; i < kPagesPerWarp; ++i) {
+    int phys = __shfl_sync(kFull, my_phys, i);
+    if (phys >= 0 && phys < a.n_phys) {
+      const float4* s = reinterpret_cast<const float4*>(a.page_minmax +
+                                                        ((size_t)phys * a.G + g) * 2 * kD);
+      mn[i] = __ldcs(s + lane);
+      mx[i] = __ldcs(s + 32 + lane);
+    } else {
+      mn[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      mx[i] = mn[i];
+    }
+  }
+  float* out = a.bounds + ((size_t)b * a.G + g) * a.maxp;
+#pragma unroll
+  for (int i = 0; i < kPagesPerWarp; ++i) {
+    float v = qn.x * mn[i].x + qn.y * mn[i].y + qn.z * mn[i].z + qn.w * mn[i].w +
+              qp.x * mx[i].x + qp.y * mx[i].y + qp.z * mx[i].z + qp.w * mx[i].w;
+    v = warp_sum(v);
+    int phys = __shfl_sync(kFull, my_phys, i);
+    int lp = base + i;
+    if (lane == 0 && lp < min(npg, a.maxp)) {
+      if (phys < 0 || phys >= a.n_phys) {
+        flag_status(kStatusBadPage);
+        v = -INFINITY;
+      }
+      out[lp] = v;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- top-k
+// Deterministic selection of the k largest finite scores of a row (ties to the
+// lower index), written in ascending index order. Used for the top-m pages (HHR
+// pruning), the top-m blocks and the token top-k of the indexer variant.
+// Scores of -inf are ineligible. One CTA of 1024 threads per row:
+//   1. 4-pass MSB-first radix select (8-bit digits) on order-preserving keys finds
+//      the key T of the k-th largest element;
+//   2. an ordered compaction keeps every key > T and the first (k - #greater)
+//      elements equal to T in index order.
+// `unit` > 0 maps an index i to kept_units[i / unit] * unit + i % unit (a token of
+// a kept block); unit == 0 writes i itself.
+constexpr int kSelThreads = 1024;
+
+struct SelectArgs {
+  const float* scores;    // [rows][stride]
+  int stride;
+  int rows_per_b;         // rows per sequence (G or T)
+  const int32_t* seq_len;
+  const int32_t* q_pos;   // indexer: eligibility uses min(seq_len, q_pos + 1); may be null
+  int P;                  // keys per page/block (for n computation)
+  int mode;               // 0: n = pages of the row; 1: n = kept_count[row] * unit
+  const int32_t* kept_count;  // mode 1
+  const int32_t* kept_units;  // mode 1: [rows][m_max]
+  int m_max;
+  int unit;
+  int m_pages, keep_div;  // mode 0: k = kept_for(n_eligible, m_pages, keep_div)
+  int top_k;              // mode 1: k = min(top_k, #finite)
+  int32_t* out;           // [rows][out_stride]
+  int out_stride;
+  int32_t* out_count;     // [rows]
+  int pad_out;            // write -1 into out[k..out_stride)
+};
+
+__global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
+  __shared__ int hist[256];
+  __shared__ int scratch[33];
+  __shared__ int sh_digit, sh_rem;
+  extern __shared__ uint32_t keys[];  // [n]
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int b = row / a.rows_per_b;
+  int n;
+  if (a.mode == 0) {
+    int len = a.seq_len[b];
+    if (a.q_pos != nullptr) len = min(len, a.q_pos[row] + 1);
+    n = min(ceil_div(max(len, 0), a.P), a.stride);
+  } else {
+    n = min(a.kept_count[row] * a.unit, a.stride);
+  }
+  const float* sc = a.scores + (size_t)row * a.stride;
+  int nfin = 0;
+  for (int i = tid; i < n; i += kSelThreads) {
+    float f = sc[i];
+    bool fin = f > -INFINITY;
+    keys[i] = fin ? f2key(f) : 0u;
+    nfin += fin;
+  }
+  int total;
+  block_excl_scan(nfin, scratch, &total);
+  nfin = total;
+  int k = (a.mode == 0) ? kept_for(nfin, a.m_pages, a.keep_div) : min(a.top_k, nfin);
+
+  // Radix select of the k-th largest key among the finite ones (key 0 = ineligible).
+  uint32_t prefix = 0, mask = 0;
+  int rem = k;
+  if (k > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      if (tid < 256) hist[tid] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kSelThreads) {
+        uint32_t kk = keys[i];
+        if (kk != 0u && (kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // Lane l covers digits 255-8l .. 248-8l (descending); find the digit where the
+        // running count from the top reaches rem.
+        int c[8], s = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * tid - q]; s += c[q]; }
+        int incl = warp_incl_scan(s, tid);
+        int excl = incl - s;
+        bool here = excl < rem && rem <= incl;
+        unsigned who = __ballot_sync(kFull, here);
+        if (here) {
+          int run = excl;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (run < rem && rem <= run + c[q]) {
+              sh_digit = 255 - 8 * tid - q;
+              sh_rem = rem - run;
+            }
+            run += c[q];
+          }
+        }
+        (void)who;
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sh_digit << shift;
+      mask |= 255u << shift;
+      rem = sh_rem;
+      __syncthreads();
+    }
+  }
+  // Now: keys > prefix are all selected; the first `rem` keys == prefix in index order.
+  const int per = ceil_div(n, kSelThreads);
+  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+  int eq = 0;
+  if (k > 0)
+    for (int i = i0; i < i1; ++i) eq += (keys[i] == prefix);
+  int eq_before = block_excl_scan(eq, scratch, &total);
+  int cnt = 0;
+  if (k > 0) {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      uint32_t kk = keys[i];
+      if (kk != 0u && kk > prefix) ++cnt;
+      else if (kk == prefix) { if (e < rem) ++cnt; ++e; }
+    }
+  }
+  int pos = block_excl_scan(cnt, scratch, &total);
+  int32_t* out = a.out + (size_t)row * a.out_stride;
+  if (k > 0) {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      uint32_t kk = keys[i];
+      bool take = false;
+      if (kk != 0u && kk > prefix) take = true;
+      else if (kk == prefix) { take = e < rem; ++e; }
+      if (take && pos < a.out_stride) {
+        int v = i;
+        if (a.unit > 0) v = a.kept_units[(size_t)row * a.m_max + i / a.unit] * a.unit + i % a.unit;
+        out[pos++] = v;
+      }
+    }
+  }
+  if (a.pad_out)
+    for (int i = k + tid; i < a.out_stride; i += kSelThreads) out[i] = -1;
+  if (tid == 0) a.out_count[row] = k;
+}
+
+// ---------------------------------------------------------------------------- a3 + a4
+// HHR page, Abstract (LHP: Hamming distance between binary codes ranks the keys of
+// the pages that survive pruning). One CTA of 1024 threads per (sequence, group).
+// Candidates are the valid keys of the kept pages, in ascending token order.
+//   delta_t = sum over the group's heads of popcount(qcode_h ^ code_t)  (0..gs*128)
+// Selection of the k smallest (delta, t): a shared-memory histogram of delta gives
+// the threshold bucket; an ordered compaction keeps every key below it and the
+// first ones inside it in token order. Output ascending; -1 past k_eff.
+constexpr int kHamThreads = 1024;
+constexpr int kMaxCand = 65536;
+
+struct HammingArgs {
+  const uint32_t* q_code;    // [B][Hq][4]
+  const uint32_t* codes;     // [n_phys][G][P][4]
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  const int32_t* kept;       // [B][G][m_max]
+  const int32_t* kept_count; // [B][G]
+  int32_t* out_idx;          // [B][G][top_k]
+  int32_t* out_count;        // [B][G]
+  int Hq, G, P, maxp, n_phys, m_max, top_k;
+};
+
+__global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a) {
+  extern __shared__ uint32_t hsm[];
+  const int row = blockIdx.x, b = row / a.G, g = row % a.G;
+  const int tid = threadIdx.x;
+  const int gs = a.Hq / a.G;
+  const int nbins = gs * 128 + 1;
+  int* hist = reinterpret_cast<int*>(hsm);                    // [nbins]
+  int* scratch = hist + ((nbins + 31) & ~31);                 // [33]
+  int* sh = scratch + 33;                                     // [2]
+  uint16_t* dist = reinterpret_cast<uint16_t*>(sh + 3);       // [C]
+  const int n = a.seq_len[b];
+  const int m = a.kept_count[row];
+  const int C = min(m * a.P, kMaxCand);
+  for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
+  uint32_t qc[kMaxGroup][kWords];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+    for (int w = 0; w < kWords; ++w)
+      qc[h][w] = h < gs ? a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] : 0u;
+  __syncthreads();
+  const int32_t* kp = a.kept + (size_t)row * a.m_max;
+  for (int c = tid; c < C; c += kHamThreads) {
+    const int lp = kp[c / a.P], slot = c % a.P;
+    const int t = lp * a.P + slot;
+    uint16_t dv = 0xffff;
+    if (t < n && lp < a.maxp) {
+      const int phys = a.page_table[(size_t)b * a.maxp + lp];
+      if (phys >= 0 && phys < a.n_phys) {
+        const uint4 code = __ldcs(reinterpret_cast<const uint4*>(
+            a.codes + (((size_t)phys * a.G + g) * a.P + slot) * kWords));
+        int d = 0;
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+          if (h < gs)
+            d += __popc(qc[h][0] ^ code.x) + __popc(qc[h][1] ^ code.y) +
+                 __popc(qc[h][2] ^ code.z) + __popc(qc[h][3] ^ code.w);
+        dv = (uint16_t)d;
+        atomicAdd(&hist[d], 1);
+      } else {
+        flag_status(kStatusBadPage);
+      }
+    }
+    dist[c] = dv;
+  }
+  __syncthreads();
+  // Threshold bucket: smallest T with #(delta <= T) >= k_eff. Warp 0 scans the bins.
+  if (tid < 32) {
+    const int per = ceil_div(nbins, 32);
+    const int b0 = min(nbins, tid * per), b1 = min(nbins, b0 + per);
+    int s = 0;
+    for (int i = b0; i < b1; ++i) s += hist[i];
+    int incl = warp_incl_scan(s, tid);
+    int nvalid = __shfl_sync(kFull, incl, 31);
+    int keff = min(a.top_k, nvalid);
+    int excl = incl - s;
+    if (tid == 0) { sh[0] = -1; sh[1] = 0; sh[2] = keff; }
+    __syncwarp();
+    if (keff > 0 && excl < keff && keff <= incl) {
+      int run = excl;
+      for (int i = b0; i < b1; ++i) {
+        if (run < keff && keff <= run + hist[i]) { sh[0] = i; sh[1] = keff - run; }
+        run += hist[i];
+      }
+    }
+  }
+  __syncthreads();
+  const int T = sh[0], need_eq = sh[1], keff = sh[2];
+  const int per = ceil_div(C, kHamThreads);
+  const int i0 = min(C, tid * per), i1 = min(C, i0 + per);
+  int eq = 0;
+  for (int i = i0; i < i1; ++i) eq += (dist[i] == T);
+  int total;
+  int eq_before = block_excl_scan(eq, scratch, &total);
+  int cnt = 0;
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      int dv = dist[i];
+      if (dv < T) ++cnt;
+      else if (dv == T) { if (e < need_eq) ++cnt; ++e; }
+    }
+  }
+  int pos = block_excl_scan(cnt, scratch, &total);
+  int32_t* out = a.out_idx + (size_t)row * a.top_k;
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      int dv = dist[i];
+      bool take = false;
+      if (dv < T) take = true;
+      else if (dv == T) { take = e < need_eq; ++e; }
+      if (take && pos < a.top_k) out[pos++] = kp[i / a.P] * a.P + i % a.P;
+    }
+  }
+  for (int i = keff + tid; i < a.top_k; i += kHamThreads) out[i] = -1;
+  if (tid == 0) a.out_count[row] = keff;
+}
+
+inline size_t hamming_smem(int gs, int C) {
+  int nbins = gs * 128 + 1;
+  return (size_t)(((nbins + 31) & ~31) + 33 + 3) * 4 + (size_t)C * 2 + 16;
+}
+
+// ---------------------------------------------------------------------------- HISA a1'
+// HISA page, Abstract: the block-level coarse filter scores pooled block
+// representatives (block_mean) against each query. Blocks whose start lies after
+// the query position are ineligible (-inf). One CTA of 128 threads handles 128
+// blocks for up to 16 chunk queries; the block tile is staged in shared memory as
+// float4 columns so thread j reads block j's channels without bank conflicts.
+constexpr int kBlkTile = 128;
+constexpr int kQTile = 16;
+
+struct BlockScoreArgs {
+  const uint16_t* q;        // [B][T][d]
+  const float* block_mean;  // [n_phys][1][d]
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  const int32_t* q_pos;     // [B][T]
+  float* scores;            // [B][T][maxp]
+  int T, P, maxp, n_phys;
+};
+
+constexpr int kBlkStride = kBlkTile + 1;  // float4 row stride of the staged tile (padded)
+
+__global__ void __launch_bounds__(kBlkTile) block_score_kernel(BlockScoreArgs a) {
+  extern __shared__ float4 bs_smem[];
+  float4* Ms = bs_smem;                         // [kD/4][kBlkStride]
+  float4* Qs = bs_smem + (kD / 4) * kBlkStride; // [kQTile][kD/4]
+  const int b = blockIdx.z, q0 = blockIdx.y * kQTile, blk0 = blockIdx.x * kBlkTile;
+  const int tid = threadIdx.x;
+  const int nblk = min(ceil_div(a.seq_len[b], a.P), a.maxp);
+  if (blk0 >= nblk) return;
+  const int nq = min(kQTile, a.T - q0);
+  for (int idx = tid; idx < kQTile * (kD / 4); idx += kBlkTile) {
+    int qi = idx / (kD / 4), c4 = idx % (kD / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (qi < nq) {
+      uint2 w = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * a.T + q0 + qi) * kD + 4 * c4);
+      v = bf16x4_to_f4(w);
+    }
+    Qs[qi * (kD / 4) + c4] = v;
+  }
+  // Stage the block means: warp-cooperative coalesced reads of each 512-byte row.
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int r = warp; r < kBlkTile; r += kBlkTile / 32) {
+    int blk = blk0 + r;
+    int phys = -1;
+    if (blk < nblk) phys = a.page_table[(size_t)b * a.maxp + blk];
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (phys >= 0 && phys < a.n_phys)
+      v = reinterpret_cast<const float4*>(a.block_mean + (size_t)phys * kD)[lane];
+    else if (blk < nblk && lane == 0)
+      flag_status(kStatusBadPage);
+    Ms[lane * kBlkStride + r] = v;
+  }
+  __syncthreads();
+  float acc[kQTile];
+#pragma unroll
+  for (int i = 0; i < kQTile; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int c4 = 0; c4 < kD / 4; ++c4) {
+    float4 mv = Ms[c4 * kBlkStride + tid];
+#pragma unroll
+    for (int i = 0; i < kQTile; ++i) {
+      float4 qv = Qs[i * (kD / 4) + c4];
+      acc[i] = fmaf(qv.x, mv.x, fmaf(qv.y, mv.y, fmaf(qv.z, mv.z, fmaf(qv.w, mv.w, acc[i]))));
+    }
+  }
+  const int blk = blk0 + tid;
+  if (blk < nblk) {
+#pragma unroll
+    for (int i = 0; i < kQTile; ++i) {
+      if (i >= nq) break;
+      int pos = a.q_pos[(size_t)b * a.T + q0 + i];
+      bool elig = (long long)blk * a.P <= (long long)pos;
+      a.scores[((size_t)b * a.T + q0 + i) * a.maxp + blk] = elig ? acc[i] : -INFINITY;
+    }
+  }
+}
+
+inline size_t block_score_smem() {
+  return (size_t)((kD / 4) * kBlkStride + kQTile * (kD / 4)) * sizeof(float4);
+}
+
+// ---------------------------------------------------------------------------- HISA a3
+// HISA page, Abstract: the original token indexer runs only inside the kept blocks.
+// sigma_t = q . k_t in fp32 (bf16 products are exact in fp32). One warp scores 32
+// candidates: lane l loads channels 4l..4l+3 of each candidate row (a coalesced
+// 256-byte row read per candidate), then a transposed warp reduction leaves the
+// score of candidate j on lane j. Ineligible candidates (t > pos or t >= n) get -inf.
+constexpr int kTokWarps = 8;
+
+struct TokenScoreArgs {
+  const uint16_t* q;        // [B][T][d]
+  const uint16_t* k_cache;  // [n_phys][1][P][d]
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  const int32_t* q_pos;
+  const int32_t* kept;      // [B][T][m_max]
+  const int32_t* kept_count;
+  float* tok_scores;        // [B][T][m_max * P]
+  int T, P, maxp, n_phys, m_max;
+};
+
+__global__ void __launch_bounds__(kTokWarps * 32) token_score_kernel(TokenScoreArgs a) {
+  const int row = blockIdx.y, b = row / a.T;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int C = a.kept_count[row] * a.P;
+  const int c0 = (blockIdx.x * kTokWarps + warp) * 32;
+  if (c0 >= C) return;
+  const int n = a.seq_len[b], pos = a.q_pos[row];
+  const float4 qv = bf16x4_to_f4(*reinterpret_cast<const uint2*>(a.q + (size_t)row * kD + 4 * lane));
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int c = c0 + j;
+    float s = 0.f;
+    if (c < C) {
+      const int lp = a.kept[(size_t)row * a.m_max + c / a.P];
+      const int t = lp * a.P + c % a.P;
+      if (t < n && t <= pos) {
+        const int phys = a.page_table[(size_t)b * a.maxp + lp];
+        if (phys >= 0 && phys < a.n_phys) {
+          uint2 w = *reinterpret_cast<const uint2*>(
+              a.k_cache + ((size_t)phys * a.P + c % a.P) * kD + 4 * lane);
+          float4 kv = bf16x4_to_f4(w);
+          s = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+        }
+      }
+    }
+    v[j] = s;
+  }
+  float sc = warp_transpose_sum32(v, lane);
+  const int c = c0 + lane;
+  if (c < C) {
+    const int lp = a.kept[(size_t)row * a.m_max + c / a.P];
+    const int t = lp * a.P + c % a.P;
+    bool ok = t < n && t <= pos;
+    if (ok) {
+      const int phys = a.page_table[(size_t)b * a.maxp + lp];
+      if (phys < 0 || phys >= a.n_phys) { ok = false; flag_status(kStatusBadPage); }
+    }
+    a.tok_scores[(size_t)row * a.m_max * a.P + c] = ok ? sc : -INFINITY;
+  }
+}
+
+}  // namespace hhr

@@ -1,0 +1,129 @@
+"""The C ABI on the host (no GPU): the library loads, exports every declared symbol, and
+host-side validation rejects bad arguments before any launch or CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hash_hierarchical_top_b200 import build, hhr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return hhr.lib()
+
+
+def declared_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(hhr_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(hhr.EXPORTED) == names
+
+
+def test_status_strings(L):
+    assert hhr.status_string(0) == "HHR_OK"
+    assert hhr.status_string(-4) == "HHR_ERR_WORKSPACE"
+    assert hhr.status_string(12345) == "HHR_UNKNOWN_STATUS"
+
+
+def _d(**kw):
+    base = dict(batch=1, n_q_heads=32, n_kv_heads=8, page_size=32, max_pages_per_seq=4096,
+                n_phys_pages=4096)
+    base.update(kw)
+    return hhr.make_dims(**base)
+
+
+def test_workspace_and_kept_sizes(L):
+    d = _d()
+    assert hhr.hhr_kept_max(d, 0, 16) == 256
+    assert hhr.hhr_kept_max(d, 64, 0) == 64
+    assert hhr.hhr_kept_max(_d(max_pages_per_seq=10), 64, 0) == 10
+    ws = hhr.hhr_select_workspace_bytes(d, hhr.HHR_MODE_HASH, 0, 16, 2048)
+    assert ws > 0 and ws % 256 == 0
+    # bounds alone need B*G*max_pages floats
+    assert ws >= 8 * 4096 * 4
+    assert hhr.hhr_attn_workspace_bytes(d, 2048) % 256 == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=64), dict(code_bits=64), dict(n_q_heads=30), dict(n_q_heads=72),
+    dict(page_size=0), dict(page_size=512), dict(batch=0), dict(max_pages_per_seq=40000),
+])
+def test_bad_dims_rejected(L, bad):
+    d = _d(**bad)
+    assert hhr.hhr_select_workspace_bytes(d, hhr.HHR_MODE_HASH, 0, 16, 2048) == 0
+    st = L.hhr_select(ctypes.byref(d), 0, *([None] * 10), 0, 16, 2048, None, None, None, 0,
+                      None, None)
+    assert st in (hhr.HHR_ERR_INVALID_ARG, hhr.HHR_ERR_UNSUPPORTED)
+
+
+def test_select_validation_order(L):
+    d = _d()
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    args = [p] * 10
+    # both m_pages and keep_div given
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 16, 16, 2048, p, p, p, 1 << 30, None,
+                        None) == hhr.HHR_ERR_INVALID_ARG
+    # top_k < 1
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 0, p, p, p, 1 << 30, None,
+                        None) == hhr.HHR_ERR_INVALID_ARG
+    # null query
+    assert L.hhr_select(ctypes.byref(d), 0, None, *args[1:], 0, 16, 2048, p, p, p, 1 << 30, None,
+                        None) == hhr.HHR_ERR_INVALID_ARG
+    # workspace too small
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 2048, p, p, p, 16, None,
+                        None) == hhr.HHR_ERR_WORKSPACE
+    # too many candidates per row (m * P > 65536)
+    assert L.hhr_select(ctypes.byref(_d(page_size=256)), 0, *args, 512, 0, 2048, p, p, p,
+                        1 << 30, None, None) == hhr.HHR_ERR_UNSUPPORTED
+    # indexer mode needs a single KV head and m_pages
+    assert L.hhr_select(ctypes.byref(d), 1, *args, 64, 0, 2048, p, p, p, 1 << 30, None,
+                        None) == hhr.HHR_ERR_INVALID_ARG
+    # unknown mode
+    assert L.hhr_select(ctypes.byref(d), 7, *args, 0, 16, 2048, p, p, p, 1 << 30, None,
+                        None) == hhr.HHR_ERR_INVALID_ARG
+
+
+def test_encode_and_attn_validation(L):
+    d = _d()
+    p = ctypes.c_void_p(256)
+    # codes without page_minmax
+    assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, 1, p, p, None, p, None,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    # neither hashing nor block means requested
+    assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, 1, None, None, None, None, None,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, -1, p, p, p, p, None,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, 0, p, p, p, p, None, None) == hhr.HHR_OK
+    a = [p] * 7
+    assert L.hhr_sparse_attn(ctypes.byref(d), *a, 2048, ctypes.c_float(0.1), p, p, 16,
+                             None) == hhr.HHR_ERR_WORKSPACE
+    assert L.hhr_sparse_attn(ctypes.byref(d), *a, 0, ctypes.c_float(0.1), p, p, 1 << 30,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_sparse_attn(ctypes.byref(d), *a, 2048, ctypes.c_float(float("nan")), p, p,
+                             1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_sparse_attn(ctypes.byref(_d(n_q_heads=72)), *a, 2048, ctypes.c_float(0.1), p,
+                             p, 1 << 30, None) == hhr.HHR_ERR_UNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(hhr, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(hhr, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        hhr.lib()

@@ -1,0 +1,153 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import hhr_synth as S
+from parity_helpers import check_hash_group, check_indexer_query, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(wl, with_values=True):
+    inp = S.make_inputs(wl, device="cuda", with_values=with_values)
+    return inp, S.to_numpy_inputs(inp)
+
+
+def _check_all_groups(wl, inp_np, g_out, groups=None):
+    report = {}
+    B = wl.batch
+    for b in range(B):
+        for g in range(wl.n_kv_heads):
+            if groups is None or (b, g) in groups:
+                check_hash_group(wl, inp_np, g_out, b, g, report)
+    return report
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from hash_hierarchical_top_b200 import build
+    build.build()
+
+
+def test_tiny_single_head():
+    wl = S.WORKLOADS["tiny_1h_4k"]
+    inp, inp_np = _inputs(wl)
+    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    print(rep)
+
+
+def test_llama_32k_full():
+    wl = S.WORKLOADS["llama8b_32k"]
+    inp, inp_np = _inputs(wl)
+    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    print(rep)
+
+
+def test_llama_32k_appended_in_pieces():
+    """The append path (pieces of 37 keys, pages filled across calls) equals a bulk encode."""
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(5000,), top_k=400)
+    inp, inp_np = _inputs(wl)
+    a = run_gpu(wl, inp)
+    c = run_gpu(wl, inp, encode_chunks=37)
+    assert np.array_equal(a["codes"], c["codes"])
+    assert np.array_equal(a["page_minmax"][:157], c["page_minmax"][:157])
+    assert np.array_equal(a["idx"], c["idx"])
+    _check_all_groups(wl, inp_np, c)
+
+
+def test_llama_128k_sampled_groups():
+    """Full 128K context, batch 1: every group's selection and attention, oracle on 3 groups."""
+    wl = S.WORKLOADS["llama8b_128k_b1"]
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp)
+    assert np.all(out["count"] == wl.top_k)
+    _check_all_groups(wl, inp_np, out, groups={(0, 0), (0, 3), (0, 7)})
+
+
+def test_ragged_small():
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=6, ragged=(1, 5000))
+    inp, inp_np = _inputs(wl)
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+
+
+def test_ragged_full_sampled():
+    wl = S.WORKLOADS["ragged_b32"]
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp)
+    lens = inp_np["seq_len"]
+    short = int(np.argmin(lens))
+    longest = int(np.argmax(lens))
+    _check_all_groups(wl, inp_np, out, groups={(short, 0), (short, 5), (longest, 2), (7, 6)})
+
+
+@pytest.mark.parametrize("case", [
+    dict(seq_lens=(17,), page_size=32, m_pages=0, keep_div=16, top_k=1024),   # one partial page
+    dict(seq_lens=(300,), page_size=32, m_pages=64, keep_div=0, top_k=5),     # keep all pages
+    dict(seq_lens=(1000,), page_size=1, m_pages=40, keep_div=0, top_k=40),    # P = 1
+    dict(seq_lens=(3000,), page_size=256, m_pages=3, keep_div=0, top_k=700),  # P max, k_eff < k
+    dict(seq_lens=(2048,), page_size=32, m_pages=0, keep_div=4, top_k=1),     # k = 1
+])
+def test_edge_cases(case):
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], **case)
+    inp, inp_np = _inputs(wl)
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+
+
+@pytest.mark.parametrize("heads", [(8, 1), (8, 8), (6, 2)])
+def test_group_shapes(heads):
+    hq, g = heads
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], n_q_heads=hq, n_kv_heads=g, seq_lens=(3000, 1234),
+                  batch=2, top_k=300)
+    inp, inp_np = _inputs(wl)
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+
+
+def test_deterministic():
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(9000,), top_k=900)
+    inp, _ = _inputs(wl)
+    a, b = run_gpu(wl, inp), run_gpu(wl, inp)
+    for key in ("idx", "count", "codes", "page_minmax", "bounds", "kept"):
+        assert np.array_equal(a[key], b[key]), key
+    assert np.array_equal(a["out"].view(np.uint32), b["out"].view(np.uint32))
+
+
+def test_indexer_decode_small():
+    wl = S.scaled(S.WORKLOADS["hisa_128k_t1"], seq_lens=(20000,), m_pages=16, top_k=700)
+    inp, inp_np = _inputs(wl, with_values=False)
+    out = run_gpu(wl, inp)
+    rep = {}
+    check_indexer_query(wl, inp_np, out, 0, 0, rep)
+
+
+def test_indexer_chunk_small():
+    wl = S.scaled(S.WORKLOADS["hisa_128k_t64"], seq_lens=(9000,), m_pages=8, top_k=300,
+                  n_queries=20)
+    inp, inp_np = _inputs(wl, with_values=False)
+    out = run_gpu(wl, inp)
+    rep = {}
+    for i in range(20):
+        check_indexer_query(wl, inp_np, out, 0, i, rep)
+
+
+def test_indexer_128k_full():
+    for name in ("hisa_128k_t1", "hisa_128k_t64"):
+        wl = S.WORKLOADS[name]
+        inp, inp_np = _inputs(wl, with_values=False)
+        out = run_gpu(wl, inp)
+        rep = {}
+        for i in sorted({0, wl.n_queries // 2, wl.n_queries - 1}):
+            check_indexer_query(wl, inp_np, out, 0, i, rep)
+        if wl.n_queries == 1:
+            # Sanity (not parity): the planted needles are all selected.
+            n = int(inp_np["seq_len"][0])
+            K = S_logical_norms(inp_np, wl, n)
+            needles = np.nonzero(K > 2.5 * np.sqrt(128))[0]
+            assert set(needles.tolist()) <= set(out["idx"][0, 0].tolist())
+
+
+def S_logical_norms(inp_np, wl, n):
+    import oracle
+    K = oracle.hhr_oracle.logical_rows(inp_np["k_cache"], inp_np["page_table"][0], 0, n,
+                                       wl.page_size)
+    return np.linalg.norm(K, axis=1)
