@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--select-only", action="store_true",
+                    help="profiling case: no V cache and no attention (step = encode + select)")
     return ap.parse_args()
 
 
@@ -256,6 +258,19 @@ def run_oracle_timed(wl, inp, seconds=None, steps=None, warmup=0):
         return el / done, done
 
 
+def timing_events(n, stream):
+    """n pairs of timing events, each recorded once so that the CUDA event exists
+    (torch creates it lazily) before its handle is given to the library's hook."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    stream.synchronize()
+    return evs
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -322,7 +337,7 @@ def main():
     # Layer caches: inputs drawn on the device (seeded), cache encoded once (untimed).
     layers = []
     for l in range(L):
-        inp = S.make_inputs(wl, device=dev, layer=l)
+        inp = S.make_inputs(wl, device=dev, layer=l, with_values=not args.select_only)
         d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, P, inp["max_pages"],
                           inp["n_phys"])
         cache = LayerCache(d, dev)
@@ -334,15 +349,23 @@ def main():
         one = torch.ones(wl.batch, dtype=torch.int32, device=dev)
         layers.append((inp, d, cache, start, one))
     d0 = layers[0][1]
-    step = DecodeStep(d0, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev)
+    step = DecodeStep(d0, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev,
+                      attention=not args.select_only)
     stream = torch.cuda.current_stream(dev)
 
     def run(i):
         inp, d, cache, start, one = layers[i % L]
+        if args.select_only:
+            step.encode(inp["k_cache"], inp["page_table"], start, one, 1, inp["R"], inp["W"],
+                        cache)
+            step.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"],
+                        W=inp["W"])
+            return
         step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
                   inp["R"], inp["W"], cache, start, one)
 
-    kernels_per_step = 7  # encode 1 + select 4 (qprep, bound, top-m, hamming) + attention 2
+    # encode 1 + select 4 (qprep, bound, top-m, hamming) + attention 2 (chunks, combine)
+    kernels_per_step = 5 if args.select_only else 7
     for i in range(max(args.warmup, 3)):
         run(i)
     torch.cuda.synchronize()
@@ -353,8 +376,7 @@ def main():
     # Timed region: K steps, events on the launching stream; per-step events around
     # the page-bound kernel (the dominant HBM stream) through the library's hook.
     K = args.steps
-    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(K)]
+    ev_b = timing_events(K, stream)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = Clocks(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
@@ -382,9 +404,10 @@ def main():
 
     # Per-kernel averages (separate untimed pass, same launches).
     kern = {}
-    for name in ("encode", "qprep", "bound", "topm", "hamming", "attn", "combine"):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(50)]
+    names = ("encode", "qprep", "bound", "topm", "hamming") + (
+        () if args.select_only else ("attn", "combine"))
+    for name in names:
+        evs = timing_events(50, stream)
         for i in range(50):
             hhr.hhr_profile_next(name, evs[i][0], evs[i][1])
             run(i)
@@ -394,7 +417,7 @@ def main():
     # End to end through the public API with host buffers: every step copies the query
     # and the newest K/V rows from pinned host memory, runs the step, reads the output.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.select_only:
         from cuda.bindings import runtime as rt
         inp, d, cache, start, one = layers[0]
         Bq = wl.batch
@@ -463,7 +486,7 @@ def main():
     step_gbs = req / (ms_step / 1e3) / 1e9
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.select_only:
         per_group, done = run_oracle_timed(wl, layers[0][0], seconds=args.cpu_seconds)
         cpu = {"value": 1.0 / (per_group * wl.n_kv_heads), "unit": "queries/s",
                "cores": 1, "kind": "oracle",

@@ -38,17 +38,28 @@ int check_group(const hhr_dims* d) {
   return (d->n_q_heads / d->n_kv_heads > kMaxGroup) ? HHR_ERR_UNSUPPORTED : HHR_OK;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device.
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+// Raise a kernel's dynamic shared-memory limit (opt-in maximum minus the kernel's
+// static shared memory) once per device, and check that `bytes` fits under it.
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (e != cudaSuccess) return g_last_cuda = e;
+  if (dev < 0 || dev >= kMaxDevices) return g_last_cuda = cudaErrorInvalidDevice;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return g_last_cuda = e;
+  int optin = 0;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+      cudaSuccess)
+    return g_last_cuda = e;
+  const size_t limit = (size_t)optin - fa.sharedSizeBytes;
+  if (bytes > limit) return g_last_cuda = cudaErrorInvalidValue;
   if (done_per_dev[dev]) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)limit);
   if (e == cudaSuccess) done_per_dev[dev] = true;
-  (void)bytes;
+  else g_last_cuda = e;
   return e;
 }
 
@@ -123,14 +134,15 @@ void prof_end(int k, cudaStream_t s) {
 
 int launch_status() {
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) g_last_cuda = e;
   return e == cudaSuccess ? HHR_OK : HHR_ERR_CUDA;
 }
 
 int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
   if (dst == nullptr || bytes == 0) return HHR_OK;
-  return cudaMemcpyAsync(dst, ws + off, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess
-             ? HHR_OK
-             : HHR_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(dst, ws + off, bytes, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) g_last_cuda = e;
+  return e == cudaSuccess ? HHR_OK : HHR_ERR_CUDA;
 }
 
 }  // namespace
@@ -147,6 +159,10 @@ const char* hhr_status_string(int s) {
     case HHR_ERR_DEVICE_STATUS: return "HHR_ERR_DEVICE_STATUS";
     default: return "HHR_UNKNOWN_STATUS";
   }
+}
+
+const char* hhr_last_cuda_error(void) {
+  return g_last_cuda == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda);
 }
 
 int hhr_profile_next(int kernel, void* start_event, void* stop_event) {
@@ -225,14 +241,18 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
   float* bounds = reinterpret_cast<float*>(ws + L.bounds);
   int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
   int32_t* kept_count = reinterpret_cast<int32_t*>(ws + L.kept_count);
-  if (allow_smem(select_largest_kernel, 0, g_smem_sel) != cudaSuccess) return HHR_ERR_CUDA;
+  if (allow_smem(select_largest_kernel,
+                 (size_t)4 * (mode == HHR_MODE_HASH ? maxp : max(maxp, m_max * P)),
+                 g_smem_sel) != cudaSuccess)
+    return HHR_ERR_CUDA;
 
   if (mode == HHR_MODE_HASH) {
     float* qpn = reinterpret_cast<float*>(ws + L.qpn);
     float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
     uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
-    if (allow_smem(qprep_kernel, 0, g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(hamming_topk_kernel, 0, g_smem_ham) != cudaSuccess) return HHR_ERR_CUDA;
+    if (allow_smem(qprep_kernel, qprep_smem(), g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
+    if (allow_smem(hamming_topk_kernel, hamming_smem(Hq / G, m_max * P), g_smem_ham) != cudaSuccess)
+      return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qprep_kernel<<<dim3(G, B), 128, qprep_smem(), s>>>(
         QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
@@ -272,7 +292,8 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
   // Indexer variant (HISA).
   const int T = Hq;
   float* tok = reinterpret_cast<float*>(ws + L.tok);
-  if (allow_smem(block_score_kernel, 0, g_smem_blk) != cudaSuccess) return HHR_ERR_CUDA;
+  if (allow_smem(block_score_kernel, block_score_smem(), g_smem_blk) != cudaSuccess)
+    return HHR_ERR_CUDA;
   prof_begin(HHR_KERNEL_BLOCK, s);
   block_score_kernel<<<dim3((maxp + kBlkTile - 1) / kBlkTile, (T + kQTile - 1) / kQTile, B),
                        kBlkTile, block_score_smem(), s>>>(
@@ -344,7 +365,7 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
   char* ws = static_cast<char*>(workspace);
   float* part_o = reinterpret_cast<float*>(ws);
   float* part_ml = reinterpret_cast<float*>(ws + align256((size_t)B * G * ns * gs * kD * 4));
-  if (allow_smem(sparse_attn_kernel, 0, g_smem_attn) != cudaSuccess) return HHR_ERR_CUDA;
+  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess) return HHR_ERR_CUDA;
   AttnArgs a{q, k_cache, v_cache, page_table, seq_len, idx, count, part_o, part_ml,
              scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
              d->n_phys_pages, top_k, ns};

@@ -28,7 +28,7 @@ HHR_MODE_INDEXER = 1
 EXPORTED = [
     "hhr_encode_keys", "hhr_kept_max", "hhr_select_workspace_bytes", "hhr_select",
     "hhr_attn_workspace_bytes", "hhr_sparse_attn", "hhr_read_device_status",
-    "hhr_status_string", "hhr_profile_next",
+    "hhr_status_string", "hhr_profile_next", "hhr_last_cuda_error",
 ]
 
 KERNELS = ["encode", "qprep", "bound", "topm", "hamming", "block", "token", "token_topk", "attn",
@@ -39,7 +39,10 @@ KERNEL_ID = {name: i for i, name in enumerate(KERNELS)}
 class HHRError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        msg = f"{fn} failed: {status_string(status)} ({status})"
+        if status == HHR_ERR_CUDA:
+            msg += ": " + lib().hhr_last_cuda_error().decode()
+        super().__init__(msg)
 
 
 class Dims(ctypes.Structure):
@@ -83,6 +86,8 @@ def lib():
         L.hhr_read_device_status.restype = i32
         L.hhr_profile_next.argtypes = [i32, vp, vp]
         L.hhr_profile_next.restype = i32
+        L.hhr_last_cuda_error.argtypes = []
+        L.hhr_last_cuda_error.restype = ctypes.c_char_p
         L.hhr_status_string.argtypes = [i32]
         L.hhr_status_string.restype = ctypes.c_char_p
         _lib = L

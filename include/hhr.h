@@ -198,6 +198,10 @@ int hhr_profile_next(int kernel, void* start_event, void* stop_event);
  * index, 4 = n_new clipped to max_new). */
 int hhr_read_device_status(void* stream, int* bits);
 
+/* The text of the last CUDA error any hhr_* call met on the calling host thread
+ * (the cause behind an HHR_ERR_CUDA), or "no error". Static storage. */
+const char* hhr_last_cuda_error(void);
+
 /* A static, human-readable name of a status code. */
 const char* hhr_status_string(int status);
 
