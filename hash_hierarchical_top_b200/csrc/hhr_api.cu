@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "../../include/hhr.h"
 #include "attn.cuh"
 #include "common.cuh"
@@ -396,6 +398,64 @@ int hhr_read_device_status(void* stream, int* bits) {
   }
   if (bits != nullptr) *bits = v;
   return v == 0 ? HHR_OK : HHR_ERR_DEVICE_STATUS;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free attention: the split-K partials live in a fixed device array.
+//
+// For callers that cannot allocate device memory at call time (for example an
+// allocator-less runtime, code that runs while a memory pool is frozen, or a
+// host that is not allowed to call cudaMalloc on its own), this variant takes
+// no workspace. Its scratch is the file-scope array below, which every GPU that
+// loads the library holds until the process exits. Host code cannot pass the
+// array's name to a kernel (in host code it names a host-side shadow, not device
+// memory), so the first call on each device looks up the array's device address
+// with cudaGetSymbolAddress while that device is current, and caches it.
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+}  // namespace
+
+extern "C" {
+
+int hhr_sparse_attn_noalloc(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cache,
+                            const uint16_t* v_cache, const int32_t* page_table,
+                            const int32_t* seq_len, const int32_t* idx, const int32_t* count,
+                            int top_k, float scale, float* out, void* stream) {
+  // Size check first: the partials must fit in the fixed array.
+  const size_t need = hhr_attn_workspace_bytes(d, top_k);
+  if (need == 0) {
+    int st = check_dims(d);
+    if (st != HHR_OK) return st;
+    if ((st = check_group(d)) != HHR_OK) return st;
+    return HHR_ERR_INVALID_ARG;
+  }
+  if (need > kNoAllocScratchBytes) return HHR_ERR_WORKSPACE;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    g_last_cuda = e;
+    return HHR_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return HHR_ERR_UNSUPPORTED;
+  void* scratch = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {
+    e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+    if (e != cudaSuccess || scratch == nullptr) {
+      g_last_cuda = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+      return HHR_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev].store(scratch, std::memory_order_release);
+  }
+  // The partials are written by the chunk kernel before the merge kernel reads
+  // them (same stream), so nothing in the array has to start at zero.
+  return hhr_sparse_attn(d, q, k_cache, v_cache, page_table, seq_len, idx, count, top_k, scale,
+                         out, scratch, kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

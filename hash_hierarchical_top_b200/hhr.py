@@ -28,7 +28,7 @@ HHR_MODE_INDEXER = 1
 EXPORTED = [
     "hhr_encode_keys", "hhr_kept_max", "hhr_select_workspace_bytes", "hhr_select",
     "hhr_attn_workspace_bytes", "hhr_sparse_attn", "hhr_read_device_status",
-    "hhr_status_string", "hhr_profile_next", "hhr_last_cuda_error",
+    "hhr_status_string", "hhr_profile_next", "hhr_last_cuda_error", "hhr_sparse_attn_noalloc",
 ]
 
 KERNELS = ["encode", "qprep", "bound", "topm", "hamming", "block", "token", "token_topk", "attn",
@@ -86,6 +86,9 @@ def lib():
         L.hhr_read_device_status.restype = i32
         L.hhr_profile_next.argtypes = [i32, vp, vp]
         L.hhr_profile_next.restype = i32
+        L.hhr_sparse_attn_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, i32,
+                                              ctypes.c_float, vp, vp]
+        L.hhr_sparse_attn_noalloc.restype = i32
         L.hhr_last_cuda_error.argtypes = []
         L.hhr_last_cuda_error.restype = ctypes.c_char_p
         L.hhr_status_string.argtypes = [i32]
@@ -207,3 +210,14 @@ def hhr_profile_next(kernel, start_event, stop_event):
     k = KERNEL_ID[kernel] if isinstance(kernel, str) else int(kernel)
     ev = lambda e: ctypes.c_void_p(e.cuda_event) if e is not None else None
     _check("hhr_profile_next", lib().hhr_profile_next(k, ev(start_event), ev(stop_event)))
+
+
+def hhr_sparse_attn_noalloc(d, q, k_cache, v_cache, page_table, seq_len, idx, count, top_k,
+                            scale, out, stream=None):
+    """hhr_sparse_attn with the library's fixed 8 MiB device scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/hhr.h)."""
+    _check("hhr_sparse_attn_noalloc", lib().hhr_sparse_attn_noalloc(
+        ctypes.byref(d), _p(q, _BF16, "q"), _p(k_cache, _BF16, "k_cache"),
+        _p(v_cache, _BF16, "v_cache"), _p(page_table, I32, "page_table"),
+        _p(seq_len, I32, "seq_len"), _p(idx, I32, "idx"), _p(count, I32, "count"), int(top_k),
+        float(scale), _p(out, F32, "out"), _s(stream)))

@@ -170,6 +170,33 @@ int hhr_sparse_attn(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_c
                     const int32_t* idx, const int32_t* count, int top_k, float scale, float* out,
                     void* workspace, size_t ws_bytes, void* stream);
 
+/* hhr_sparse_attn without a workspace argument, for callers that cannot allocate
+ * device memory themselves: runtimes without a device allocator, code running
+ * while a memory pool is frozen or being captured, or plugins whose host forbids
+ * cudaMalloc. The pages have no counterpart of this call (it is a deployment
+ * convenience): it computes the same attention as hhr_sparse_attn, with the
+ * split-K partials kept in a fixed 8 MiB device array inside the library instead
+ * of a caller workspace.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *     The 8 MiB array is part of the library image, so every GPU that loads the
+ *     library holds it until the process exits.
+ *   - Limit: hhr_attn_workspace_bytes(dims, top_k) must be at most 8 MiB (8388608
+ *     bytes), e.g. batch 8 x 8 KV heads x 4-head groups at top_k 2048 needs about
+ *     2.1 MB; a larger problem returns HHR_ERR_WORKSPACE before any launch.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call outside any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each partial is written before it is
+ *     read, in stream order), but calls that can overlap on the GPU (different
+ *     streams, or different host threads, on one device) race on it: serialise
+ *     them.
+ * Arguments, outputs and other errors are those of hhr_sparse_attn. */
+int hhr_sparse_attn_noalloc(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_cache,
+                            const uint16_t* v_cache, const int32_t* page_table,
+                            const int32_t* seq_len, const int32_t* idx, const int32_t* count,
+                            int top_k, float scale, float* out, void* stream);
+
 /* Kernels that hhr_profile_next can bracket with events. */
 typedef enum {
   HHR_KERNEL_ENCODE = 0,     /* hhr_encode_keys */
