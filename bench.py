@@ -163,11 +163,13 @@ def traffic_from_profile(kernel_src_hash):
 
 
 def kernel_source_hash():
-    h = hashlib.sha256()
-    for f in ("select.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "hash_hierarchical_top_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()
+    """sha256 of the page-bound kernel's section of select.cuh (its step-a2 block)."""
+    with open(os.path.join(ROOT, "hash_hierarchical_top_b200", "csrc", "select.cuh")) as fh:
+        s = fh.read()
+    mark = "// " + "-" * 76
+    a = s.index(mark + " a2")
+    b = s.index(mark, a + len(mark))
+    return hashlib.sha256(s[a:b].encode()).hexdigest()
 
 
 # ----------------------------------------------------------------------------- oracle arm
