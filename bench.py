@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama8b_128k_b8")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling: override the workload's batch (same context per sequence)")
     ap.add_argument("--layers", type=int, default=0, help="layer caches rotated (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -286,6 +288,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     import hhr_synth as S
     wl = S.WORKLOADS[args.workload]
+    if args.batch > 0 and wl.ragged is None:
+        wl = S.scaled(wl, batch=args.batch, seq_lens=(wl.seq_lens[0],) * args.batch)
 
     if args.impl == "reference":
         # The oracle arm: rank 0 alone runs it on the host cores.

@@ -93,6 +93,18 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
   return res;
 }
 
+// Histogram increment aggregated over the warp's lanes that hit the same bin: one
+// shared-memory atomic per distinct bin instead of one per lane (similar scores
+// crowd into few bins). `active` = lanes that want to add (the call itself must be
+// made by every lane of the warp).
+__device__ __forceinline__ void hist_add_aggregated(int* hist, int bin, bool active) {
+  const unsigned want = __ballot_sync(kFull, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(want, bin);
+  const int leader = __ffs(peers) - 1;
+  if ((threadIdx.x & 31) == leader) atomicAdd(&hist[bin], __popc(peers));
+}
+
 // Order-preserving map of a float to uint32 (larger float -> larger key; -0 < +0).
 __device__ __forceinline__ uint32_t f2key(float f) {
   uint32_t u = __float_as_uint(f);

@@ -7,9 +7,6 @@
 // [(W_g R_g k)_j > 0]. HISA page, Abstract: the pooled block representative, read
 // here as the mean of the block's keys.
 //
-// One CTA of 128 threads per (touched page, KV group, sequence). Thread i owns
-// channel i of the rotated key and bit i of the code. R_g^T and W_g^T are staged
-// in shared memory (transposed, so thread i reads column i without bank conflicts).
 // Summaries are updated incrementally: if the page already held keys before this
 // append, the new min/max are merged into the stored ones (min/max are exact, so
 // this equals recomputing the whole page).
@@ -19,15 +16,35 @@
 namespace hhr {
 
 // Row stride of a transposed 128x128 matrix in shared memory (padded: conflict-free
-// for both the transposing stores and the column reads).
+// for both the transposing stores and the column reads). Used by the bulk SIMT path.
 constexpr int kTS = kD + 1;
 
-// T[c][r] = M[r][c] for a 128x128 row-major fp32 matrix M; coalesced global reads.
-__device__ __forceinline__ void stage_transposed(const float* __restrict__ M, float* T) {
-  for (int idx = threadIdx.x; idx < kD * kD; idx += blockDim.x) {
-    int r = idx >> 7, c = idx & 127;
-    T[c * kTS + r] = M[idx];
+// y_v = M x_v for up to kVecChunk vectors at once, M a 128x128 row-major fp32 matrix
+// in global memory (L1/L2-resident: it is shared by every CTA of a group).
+// Warp w computes rows 32w..32w+31: lane l reads float4 l of each row (a coalesced
+// 512-byte row read per instruction), multiplies it with channels 4l..4l+3 of every
+// vector, and a transposed warp reduction leaves y_v[32w + l] on lane l. Each row of
+// M is read once per call for all vectors. Requires blockDim.x == 128.
+constexpr int kVecChunk = 4;
+
+template <int NV>
+__device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const float* xs,
+                                            int xs_stride, float (&y)[NV]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float4 xv[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) xv[v] = reinterpret_cast<const float4*>(xs + v * xs_stride)[lane];
+  float acc[NV][32];
+  const float4* Mr = reinterpret_cast<const float4*>(M + (size_t)(warp * 32) * kD) + lane;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float4 m = __ldg(Mr + j * (kD / 4));
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+      acc[v][j] = m.x * xv[v].x + m.y * xv[v].y + m.z * xv[v].z + m.w * xv[v].w;
   }
+#pragma unroll
+  for (int v = 0; v < NV; ++v) y[v] = warp_transpose_sum32(acc[v], lane);
 }
 
 struct EncodeArgs {
@@ -43,12 +60,13 @@ struct EncodeArgs {
   int G, P, maxp, n_phys, max_new;
 };
 
+// One CTA of 128 threads per (touched page, KV group, sequence). The new keys of
+// the page are processed kVecChunk at a time: k' = R_g k (thread 32w+l ends up
+// owning channel 32w+l), min/max folded per channel, then p = W_g k' and the code
+// word of warp w is the ballot of its 32 sign bits.
 __global__ void __launch_bounds__(128) encode_page_kernel(EncodeArgs a) {
-  extern __shared__ float4 smem_f4[];
-  float* RT = reinterpret_cast<float*>(smem_f4);        // [128][kTS], RT[j][i] = R[i][j]
-  float* WT = RT + kD * kTS;                             // [128][kTS], WT[i][j] = W[j][i]
-  float* kx = WT + kD * kTS;                              // raw key (fp32)
-  float* kr = kx + kD;                                    // rotated key
+  __shared__ __align__(16) float kx[kVecChunk][kD];  // raw keys (fp32)
+  __shared__ __align__(16) float kr[kVecChunk][kD];  // rotated keys
 
   const int b = blockIdx.z, g = blockIdx.y, j = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -75,36 +93,39 @@ __global__ void __launch_bounds__(128) encode_page_kernel(EncodeArgs a) {
   }
   const int pstart = lp * P;
   const int t0 = max(s, pstart), t1 = min(e, pstart + P);
-  const bool hashing = (a.R != nullptr);
   const uint16_t* kpage = a.k_cache + ((size_t)phys * G + g) * P * kD;
 
-  if (hashing) {
+  if (a.R != nullptr) {
     const float* Rg = a.R + (size_t)g * kD * kD;
     const float* Wg = a.W + (size_t)g * kD * kD;
-    stage_transposed(Rg, RT);
-    stage_transposed(Wg, WT);
-  }
-  __syncthreads();
-
-  float mn = INFINITY, mx = -INFINITY;
-  if (hashing) {
-    for (int t = t0; t < t1; ++t) {
-      kx[tid] = bf16_to_f(kpage[(size_t)(t - pstart) * kD + tid]);
+    float mn = INFINITY, mx = -INFINITY;
+    for (int t = t0; t < t1; t += kVecChunk) {
+      const int nv = min(kVecChunk, t1 - t);
       __syncthreads();
-      float acc = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < kD; ++c) acc = fmaf(RT[c * kTS + tid], kx[c], acc);
-      kr[tid] = acc;
-      mn = fminf(mn, acc);
-      mx = fmaxf(mx, acc);
+      for (int v = 0; v < kVecChunk; ++v)
+        kx[v][tid] = v < nv ? bf16_to_f(kpage[(size_t)(t + v - pstart) * kD + tid]) : 0.f;
       __syncthreads();
-      float p = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < kD; ++c) p = fmaf(WT[c * kTS + tid], kr[c], p);
-      unsigned word = __ballot_sync(kFull, p > 0.f);
-      if (lane == 0)
-        a.codes[(((size_t)phys * G + g) * P + (t - pstart)) * kWords + warp] = word;
+      float y[kVecChunk];
+      matvec_rows<kVecChunk>(Rg, &kx[0][0], kD, y);
+#pragma unroll
+      for (int v = 0; v < kVecChunk; ++v) {
+        if (v < nv) {
+          kr[v][tid] = y[v];
+          mn = fminf(mn, y[v]);
+          mx = fmaxf(mx, y[v]);
+        } else {
+          kr[v][tid] = 0.f;
+        }
+      }
       __syncthreads();
+      float p[kVecChunk];
+      matvec_rows<kVecChunk>(Wg, &kr[0][0], kD, p);
+#pragma unroll
+      for (int v = 0; v < kVecChunk; ++v) {
+        const unsigned word = __ballot_sync(kFull, p[v] > 0.f);
+        if (v < nv && lane == 0)
+          a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + warp] = word;
+      }
     }
     float* mm = a.page_minmax + ((size_t)phys * G + g) * 2 * kD;
     if (t0 > pstart) {  // the page already held keys: merge with its stored summary
@@ -122,6 +143,6 @@ __global__ void __launch_bounds__(128) encode_page_kernel(EncodeArgs a) {
   }
 }
 
-inline size_t encode_page_smem() { return (size_t)(2 * kD * kTS + 2 * kD) * sizeof(float); }
+inline size_t encode_page_smem() { return 0; }
 
 }  // namespace hhr

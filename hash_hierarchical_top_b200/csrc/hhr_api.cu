@@ -20,6 +20,7 @@ namespace {
 constexpr int kMaxPagesPerSeq = 32768;  // top-m keys staged in 128 KB of shared memory
 constexpr int kMaxTokCand = 32768;      // indexer token candidates per query
 constexpr int kMaxDevices = 64;
+constexpr size_t kMaxKernelSmem = 200 * 1024;  // below the 227 KB opt-in of sm_100
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -66,7 +67,8 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
 }
 
 bool g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
-    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices];
+    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
+    g_smem_attn8[kMaxDevices];
 
 struct SelectLayout {
   size_t qpn, q_rot, q_code, bounds, kept, kept_count, tok, total;
@@ -106,6 +108,9 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
     if ((m_pages > 0) == (keep_div > 0)) return HHR_ERR_INVALID_ARG;
     if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
     if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
+      return HHR_ERR_UNSUPPORTED;
+    if (hamming_smem(d->n_q_heads / d->n_kv_heads, kept_max(d, m_pages, keep_div),
+                     d->page_size) > kMaxKernelSmem)
       return HHR_ERR_UNSUPPORTED;
   } else if (mode == HHR_MODE_INDEXER) {
     if (m_pages < 1 || keep_div != 0) return HHR_ERR_INVALID_ARG;
@@ -253,7 +258,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
     uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
     if (allow_smem(qprep_kernel, qprep_smem(), g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(hamming_topk_kernel, hamming_smem(Hq / G, m_max * P), g_smem_ham) != cudaSuccess)
+    if (allow_smem(hamming_topk_kernel, hamming_smem(Hq / G, m_max, P), g_smem_ham) != cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qprep_kernel<<<dim3(G, B), 128, qprep_smem(), s>>>(
@@ -278,7 +283,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
     prof_begin(HHR_KERNEL_HAMMING, s);
-    hamming_topk_kernel<<<B * G, kHamThreads, hamming_smem(Hq / G, m_max * P), s>>>(ha);
+    hamming_topk_kernel<<<B * G, kHamThreads, hamming_smem(Hq / G, m_max, P), s>>>(ha);
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
     if (trace != nullptr) {
@@ -339,7 +344,8 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
 
 size_t hhr_attn_workspace_bytes(const hhr_dims* d, int top_k) {
   if (check_dims(d) != HHR_OK || check_group(d) != HHR_OK || top_k < 1) return 0;
-  const size_t ns = (top_k + kChunk - 1) / kChunk;
+  const AttnPlan plan = attn_plan(d->batch, d->n_kv_heads, top_k);
+  const size_t ns = plan.n_splits;
   const size_t rows = (size_t)d->batch * d->n_kv_heads;
   const size_t gs = d->n_q_heads / d->n_kv_heads;
   return align256(rows * ns * gs * kD * 4) + align256(rows * ns * gs * 2 * 4);
@@ -362,23 +368,33 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
   if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads;
-  const int ns = (top_k + kChunk - 1) / kChunk;
+  const AttnPlan plan = attn_plan(B, G, top_k);
+  const int ns = plan.n_splits;
   const int gs = Hq / G;
   char* ws = static_cast<char*>(workspace);
   float* part_o = reinterpret_cast<float*>(ws);
   float* part_ml = reinterpret_cast<float*>(ws + align256((size_t)B * G * ns * gs * kD * 4));
-  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess) return HHR_ERR_CUDA;
-  AttnArgs a{q, k_cache, v_cache, page_table, seq_len, idx, count, part_o, part_ml,
+  AttnArgs a{q, k_cache, v_cache, page_table, seq_len, idx, count, part_o, part_ml, out,
              scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
-             d->n_phys_pages, top_k, ns};
+             d->n_phys_pages, top_k, ns, plan.split_rows};
   prof_begin(HHR_KERNEL_ATTN, s);
-  sparse_attn_kernel<<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  if (gs <= 4) {
+    if (allow_smem(sparse_attn_kernel<4>, attn_smem(), g_smem_attn) != cudaSuccess)
+      return HHR_ERR_CUDA;
+    sparse_attn_kernel<4><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  } else {
+    if (allow_smem(sparse_attn_kernel<8>, attn_smem(), g_smem_attn8) != cudaSuccess)
+      return HHR_ERR_CUDA;
+    sparse_attn_kernel<8><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  }
   prof_end(HHR_KERNEL_ATTN, s);
   if ((st = launch_status()) != HHR_OK) return st;
-  prof_begin(HHR_KERNEL_COMBINE, s);
-  attn_combine_kernel<<<dim3(Hq, B), kD, 0, s>>>(
-      CombineArgs{part_o, part_ml, count, out, Hq, G, top_k, ns});
-  prof_end(HHR_KERNEL_COMBINE, s);
+  if (ns > 1) {
+    prof_begin(HHR_KERNEL_COMBINE, s);
+    attn_combine_kernel<<<dim3(Hq, B), kD, 0, s>>>(
+        CombineArgs{part_o, part_ml, count, out, Hq, G, top_k, ns, plan.split_rows});
+    prof_end(HHR_KERNEL_COMBINE, s);
+  }
   return launch_status();
 }
 

@@ -26,42 +26,49 @@ struct QPrepArgs {
 };
 
 __global__ void __launch_bounds__(128) qprep_kernel(QPrepArgs a) {
-  extern __shared__ float4 smem_f4[];
-  float* RT = reinterpret_cast<float*>(smem_f4);
-  float* WT = RT + kD * kTS;
-  float* qx = WT + kD * kTS;
-  float* qr = qx + kD;
+  __shared__ __align__(16) float qx[kMaxGroup][kD];
+  __shared__ __align__(16) float qr[kMaxGroup][kD];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int gs = a.Hq / a.G;
-  stage_transposed(a.R + (size_t)g * kD * kD, RT);
-  stage_transposed(a.W + (size_t)g * kD * kD, WT);
+  const float* Rg = a.R + (size_t)g * kD * kD;
+  const float* Wg = a.W + (size_t)g * kD * kD;
+  for (int h = 0; h < kMaxGroup; ++h) {
+    qx[h][tid] = h < gs ? bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + h) * kD + tid]) : 0.f;
+    qr[h][tid] = 0.f;
+  }
+  __syncthreads();
   float qneg = 0.f, qpos = 0.f;
-  for (int hh = 0; hh < gs; ++hh) {
-    const int h = g * gs + hh;
-    __syncthreads();
-    qx[tid] = bf16_to_f(a.q[((size_t)b * a.Hq + h) * kD + tid]);
-    __syncthreads();
-    float acc = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < kD; ++c) acc = fmaf(RT[c * kTS + tid], qx[c], acc);
-    qr[tid] = acc;
-    a.q_rot[((size_t)b * a.Hq + h) * kD + tid] = acc;
-    qneg += fminf(acc, 0.f);
-    qpos += fmaxf(acc, 0.f);
-    __syncthreads();
-    float p = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < kD; ++c) p = fmaf(WT[c * kTS + tid], qr[c], p);
-    unsigned word = __ballot_sync(kFull, p > 0.f);
-    if (lane == 0) a.q_code[((size_t)b * a.Hq + h) * kWords + warp] = word;
+  for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
+    float y[kVecChunk];
+    matvec_rows<kVecChunk>(Rg, &qx[h0][0], kD, y);
+#pragma unroll
+    for (int v = 0; v < kVecChunk; ++v) {
+      if (h0 + v < gs) {
+        qr[h0 + v][tid] = y[v];
+        a.q_rot[((size_t)b * a.Hq + g * gs + h0 + v) * kD + tid] = y[v];
+        qneg += fminf(y[v], 0.f);
+        qpos += fmaxf(y[v], 0.f);
+      }
+    }
+  }
+  __syncthreads();
+  for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
+    float p[kVecChunk];
+    matvec_rows<kVecChunk>(Wg, &qr[h0][0], kD, p);
+#pragma unroll
+    for (int v = 0; v < kVecChunk; ++v) {
+      const unsigned word = __ballot_sync(kFull, p[v] > 0.f);
+      if (h0 + v < gs && lane == 0)
+        a.q_code[((size_t)b * a.Hq + g * gs + h0 + v) * kWords + warp] = word;
+    }
   }
   float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
   o[tid] = qneg;
   o[kD + tid] = qpos;
 }
 
-inline size_t qprep_smem() { return (size_t)(2 * kD * kTS + 2 * kD) * sizeof(float); }
+inline size_t qprep_smem() { return 0; }
 
 // ---------------------------------------------------------------------------- a2
 // HHR page, Abstract: page-level logit bounds of the rotated keys prune pages.
@@ -163,11 +170,35 @@ struct SelectArgs {
   int pad_out;            // write -1 into out[k..out_stride)
 };
 
+// Block-wide min and max of one uint32 per thread (contains __syncthreads).
+__device__ __forceinline__ void block_minmax_u32(uint32_t lo, uint32_t hi, uint32_t* sh,
+                                                 uint32_t* out_lo, uint32_t* out_hi) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(kFull, lo, o));
+    hi = max(hi, __shfl_xor_sync(kFull, hi, o));
+  }
+  if (lane == 0) { sh[warp] = lo; sh[32 + warp] = hi; }
+  __syncthreads();
+  lo = lane < nw ? sh[lane] : 0xffffffffu;
+  hi = lane < nw ? sh[32 + lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(kFull, lo, o));
+    hi = max(hi, __shfl_xor_sync(kFull, hi, o));
+  }
+  *out_lo = lo;
+  *out_hi = hi;
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
   __shared__ int hist[256];
   __shared__ int scratch[33];
-  __shared__ int sh_digit, sh_rem;
-  extern __shared__ uint32_t keys[];  // [n]
+  __shared__ uint32_t mm[64];
+  __shared__ int sh_digit, sh_rem, sh_cnt;
+  extern __shared__ uint32_t keys[];  // [n], 16-byte aligned
   const int row = blockIdx.x, tid = threadIdx.x;
   const int b = row / a.rows_per_b;
   int n;
@@ -179,85 +210,113 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
     n = min(a.kept_count[row] * a.unit, a.stride);
   }
   const float* sc = a.scores + (size_t)row * a.stride;
-  int nfin = 0;
-  for (int i = tid; i < n; i += kSelThreads) {
-    float f = sc[i];
-    bool fin = f > -INFINITY;
-    keys[i] = fin ? f2key(f) : 0u;
-    nfin += fin;
-  }
-  int total;
-  block_excl_scan(nfin, scratch, &total);
-  nfin = total;
-  int k = (a.mode == 0) ? kept_for(nfin, a.m_pages, a.keep_div) : min(a.top_k, nfin);
-
-  // Radix select of the k-th largest key among the finite ones (key 0 = ineligible).
-  uint32_t prefix = 0, mask = 0;
-  int rem = k;
-  if (k > 0) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      if (tid < 256) hist[tid] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += kSelThreads) {
-        uint32_t kk = keys[i];
-        if (kk != 0u && (kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // Lane l covers digits 255-8l .. 248-8l (descending); find the digit where the
-        // running count from the top reaches rem.
-        int c[8], s = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * tid - q]; s += c[q]; }
-        int incl = warp_incl_scan(s, tid);
-        int excl = incl - s;
-        bool here = excl < rem && rem <= incl;
-        unsigned who = __ballot_sync(kFull, here);
-        if (here) {
-          int run = excl;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (run < rem && rem <= run + c[q]) {
-              sh_digit = 255 - 8 * tid - q;
-              sh_rem = rem - run;
-            }
-            run += c[q];
-          }
-        }
-        (void)who;
-      }
-      __syncthreads();
-      prefix |= (uint32_t)sh_digit << shift;
-      mask |= 255u << shift;
-      rem = sh_rem;
-      __syncthreads();
-    }
-  }
-  // Now: keys > prefix are all selected; the first `rem` keys == prefix in index order.
+  // Contiguous chunk of each thread (index order is needed by the compaction).
   const int per = ceil_div(n, kSelThreads);
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
-  int eq = 0;
-  if (k > 0)
-    for (int i = i0; i < i1; ++i) eq += (keys[i] == prefix);
-  int eq_before = block_excl_scan(eq, scratch, &total);
-  int cnt = 0;
+  int nfin = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i = tid; i < n; i += kSelThreads) {
+    const float f = sc[i];
+    const bool fin = f > -INFINITY;
+    const uint32_t kk = fin ? f2key(f) : 0u;
+    keys[i] = kk;
+    nfin += fin;
+    if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
+  }
+  int total;
+  block_excl_scan(nfin, scratch, &total);  // also orders the key stores before any read
+  nfin = total;
+  block_minmax_u32(kmin, kmax, mm, &kmin, &kmax);
+  const int k = (a.mode == 0) ? kept_for(nfin, a.m_pages, a.keep_div) : min(a.top_k, nfin);
+
+  // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
+  // keys at sel_shift == 0 are taken in index order until `rem` of them are taken; at
+  // sel_shift > 0 the whole bin is taken (>=).
+  uint32_t prefix = 0;
+  int rem = k, sel_shift = 0;
+  bool whole_bin = false;
   if (k > 0) {
-    int e = eq_before;
-    for (int i = i0; i < i1; ++i) {
-      uint32_t kk = keys[i];
-      if (kk != 0u && kk > prefix) ++cnt;
-      else if (kk == prefix) { if (e < rem) ++cnt; ++e; }
+    if (k == nfin) {
+      whole_bin = true;            // everything finite is selected
+      prefix = kmin;
+      sel_shift = 0;
+    } else if (kmin == kmax) {
+      prefix = kmin;               // all equal: the first k in index order
+    } else {
+      const int hb = 31 - __clz(kmin ^ kmax);          // highest differing bit
+      int shift = max(hb - 7, 0);
+      uint32_t mask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);   // common high bits
+      prefix = kmin & mask;
+      while (true) {
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += kSelThreads) {
+          const uint32_t kk = keys[i];
+          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+          // Lane l covers digits 255-8l .. 248-8l (descending).
+          int c[8], s = 0;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * tid - q]; s += c[q]; }
+          const int incl = warp_incl_scan(s, tid);
+          const int excl = incl - s;
+          if (excl < rem && rem <= incl) {
+            int run = excl;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (run < rem && rem <= run + c[q]) {
+                sh_digit = 255 - 8 * tid - q;
+                sh_rem = rem - run;
+                sh_cnt = c[q];
+              }
+              run += c[q];
+            }
+          }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sh_digit << shift;
+        mask |= 255u << shift;
+        rem = sh_rem;
+        const int cnt_bin = sh_cnt;
+        __syncthreads();
+        if (rem == cnt_bin) {  // the whole bin is needed: no tie-break required
+          whole_bin = true;
+          sel_shift = shift;
+          break;
+        }
+        if (shift == 0) break;
+        // Next 8 bits; when fewer than 8 remain, the last pass covers bits [0, 8) and
+        // its already-fixed upper bits are constant across the candidates.
+        shift = max(shift - 8, 0);
+      }
     }
   }
+  // Compaction in index order.
+  auto take_gt = [&](uint32_t kk) -> bool {
+    if (kk == 0u) return false;
+    if (whole_bin) return (kk >> sel_shift) >= (prefix >> sel_shift);
+    return kk > prefix;
+  };
+  int eq = 0, cnt = 0;
+  if (k > 0) {
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t kk = keys[i];
+      if (take_gt(kk)) ++cnt;
+      else if (!whole_bin && kk == prefix) ++eq;
+    }
+  }
+  const int eq_before = block_excl_scan(eq, scratch, &total);
+  if (k > 0 && !whole_bin) cnt += max(0, min(eq, rem - eq_before));
   int pos = block_excl_scan(cnt, scratch, &total);
   int32_t* out = a.out + (size_t)row * a.out_stride;
   if (k > 0) {
     int e = eq_before;
     for (int i = i0; i < i1; ++i) {
-      uint32_t kk = keys[i];
-      bool take = false;
-      if (kk != 0u && kk > prefix) take = true;
-      else if (kk == prefix) { take = e < rem; ++e; }
+      const uint32_t kk = keys[i];
+      bool take = take_gt(kk);
+      if (!take && !whole_bin && kk == prefix) { take = e < rem; ++e; }
       if (take && pos < a.out_stride) {
         int v = i;
         if (a.unit > 0) v = a.kept_units[(size_t)row * a.m_max + i / a.unit] * a.unit + i % a.unit;
@@ -293,20 +352,36 @@ struct HammingArgs {
   int Hq, G, P, maxp, n_phys, m_max, top_k;
 };
 
+constexpr int kHamUnroll = 8;
+
 __global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a) {
   extern __shared__ uint32_t hsm[];
   const int row = blockIdx.x, b = row / a.G, g = row % a.G;
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.G;
   const int nbins = gs * 128 + 1;
+  const int m = min(a.kept_count[row], a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                    // [nbins]
   int* scratch = hist + ((nbins + 31) & ~31);                 // [33]
-  int* sh = scratch + 33;                                     // [2]
-  uint16_t* dist = reinterpret_cast<uint16_t*>(sh + 3);       // [C]
+  int* sh = scratch + 33;                                     // [3]
+  int* kphys = sh + 3;                                        // [m_max] physical page
+  int* klp = kphys + a.m_max;                                 // [m_max] logical page
+  uint16_t* dist = reinterpret_cast<uint16_t*>(kphys + ((2 * a.m_max + 3) & ~3));  // [C], 16B-aligned
   const int n = a.seq_len[b];
-  const int m = a.kept_count[row];
   const int C = min(m * a.P, kMaxCand);
   for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
+  // Resolve the kept pages once: logical id and physical page (-1 if invalid).
+  for (int i = tid; i < m; i += kHamThreads) {
+    const int lp = a.kept[(size_t)row * a.m_max + i];
+    int phys = -1;
+    if (lp >= 0 && lp < a.maxp) phys = a.page_table[(size_t)b * a.maxp + lp];
+    if (phys < 0 || phys >= a.n_phys) {
+      flag_status(kStatusBadPage);
+      phys = -1;
+    }
+    kphys[i] = phys;
+    klp[i] = lp;
+  }
   uint32_t qc[kMaxGroup][kWords];
 #pragma unroll
   for (int h = 0; h < kMaxGroup; ++h)
@@ -314,29 +389,41 @@ __global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a
     for (int w = 0; w < kWords; ++w)
       qc[h][w] = h < gs ? a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] : 0u;
   __syncthreads();
-  const int32_t* kp = a.kept + (size_t)row * a.m_max;
-  for (int c = tid; c < C; c += kHamThreads) {
-    const int lp = kp[c / a.P], slot = c % a.P;
-    const int t = lp * a.P + slot;
-    uint16_t dv = 0xffff;
-    if (t < n && lp < a.maxp) {
-      const int phys = a.page_table[(size_t)b * a.maxp + lp];
-      if (phys >= 0 && phys < a.n_phys) {
-        const uint4 code = __ldcs(reinterpret_cast<const uint4*>(
-            a.codes + (((size_t)phys * a.G + g) * a.P + slot) * kWords));
-        int d = 0;
+  // Candidates c = tid + j*1024: consecutive threads read consecutive 16-byte codes of a
+  // page (coalesced); all kHamUnroll code loads of a thread are issued before any math.
+  // c / P by multiply-high: exact for c < 2^24 with magic = floor(2^32 / P) + 1.
+  const uint32_t magic = (uint32_t)(0xffffffffu / (uint32_t)a.P) + 1u;
+  for (int c0 = 0; c0 < C; c0 += kHamThreads * kHamUnroll) {
+    uint4 code[kHamUnroll];
+    bool ok[kHamUnroll];
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-          if (h < gs)
-            d += __popc(qc[h][0] ^ code.x) + __popc(qc[h][1] ^ code.y) +
-                 __popc(qc[h][2] ^ code.z) + __popc(qc[h][3] ^ code.w);
-        dv = (uint16_t)d;
-        atomicAdd(&hist[d], 1);
-      } else {
-        flag_status(kStatusBadPage);
+    for (int j = 0; j < kHamUnroll; ++j) {
+      const int c = c0 + j * kHamThreads + tid;
+      ok[j] = false;
+      code[j] = make_uint4(0, 0, 0, 0);
+      if (c < C) {
+        const int i = (a.P == 1) ? c : (int)__umulhi((uint32_t)c, magic);
+        const int slot = c - i * a.P;
+        const int phys = kphys[i];
+        if (phys >= 0 && klp[i] * a.P + slot < n) {
+          ok[j] = true;
+          code[j] = __ldcs(reinterpret_cast<const uint4*>(
+              a.codes + (((size_t)phys * a.G + g) * a.P + slot) * kWords));
+        }
       }
     }
-    dist[c] = dv;
+#pragma unroll
+    for (int j = 0; j < kHamUnroll; ++j) {
+      const int c = c0 + j * kHamThreads + tid;
+      int d = 0;
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h)
+        if (h < gs)
+          d += __popc(qc[h][0] ^ code[j].x) + __popc(qc[h][1] ^ code[j].y) +
+               __popc(qc[h][2] ^ code[j].z) + __popc(qc[h][3] ^ code[j].w);
+      if (ok[j]) atomicAdd(&hist[d], 1);
+      if (c < C) dist[c] = ok[j] ? (uint16_t)d : (uint16_t)0xffff;
+    }
   }
   __syncthreads();
   // Threshold bucket: smallest T with #(delta <= T) >= k_eff. Warp 0 scans the bins.
@@ -361,40 +448,63 @@ __global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a
   }
   __syncthreads();
   const int T = sh[0], need_eq = sh[1], keff = sh[2];
-  const int per = ceil_div(C, kHamThreads);
-  const int i0 = min(C, tid * per), i1 = min(C, i0 + per);
-  int eq = 0;
-  for (int i = i0; i < i1; ++i) eq += (dist[i] == T);
-  int total;
-  int eq_before = block_excl_scan(eq, scratch, &total);
-  int cnt = 0;
-  {
-    int e = eq_before;
-    for (int i = i0; i < i1; ++i) {
-      int dv = dist[i];
-      if (dv < T) ++cnt;
-      else if (dv == T) { if (e < need_eq) ++cnt; ++e; }
+  // Ordered compaction: thread t owns the contiguous candidates [t*cpt, (t+1)*cpt), cpt a
+  // multiple of 8, read as 16-byte groups of 8 distances.
+  const int cpt = ((ceil_div(C, kHamThreads) + 7) / 8) * 8;
+  const int ngrp = cpt / 8;
+  auto load8 = [&](int i0, uint16_t (&dv)[8]) {
+    uint4 raw = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+    if (i0 < C) raw = *reinterpret_cast<const uint4*>(dist + i0);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      dv[2 * q] = (i0 + 2 * q < C) ? (uint16_t)(w[q] & 0xffff) : (uint16_t)0xffff;
+      dv[2 * q + 1] = (i0 + 2 * q + 1 < C) ? (uint16_t)(w[q] >> 16) : (uint16_t)0xffff;
+    }
+  };
+  int eq = 0, lt = 0;
+  for (int gi = 0; gi < ngrp; ++gi) {
+    uint16_t dv[8];
+    load8(tid * cpt + gi * 8, dv);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      eq += (dv[q] == T);
+      lt += (dv[q] < T);
     }
   }
+  int total;
+  const int eq_before = block_excl_scan(eq, scratch, &total);
+  const int cnt = lt + max(0, min(eq, need_eq - eq_before));
   int pos = block_excl_scan(cnt, scratch, &total);
   int32_t* out = a.out_idx + (size_t)row * a.top_k;
   {
     int e = eq_before;
-    for (int i = i0; i < i1; ++i) {
-      int dv = dist[i];
-      bool take = false;
-      if (dv < T) take = true;
-      else if (dv == T) { take = e < need_eq; ++e; }
-      if (take && pos < a.top_k) out[pos++] = kp[i / a.P] * a.P + i % a.P;
+    for (int gi = 0; gi < ngrp; ++gi) {
+      uint16_t dv[8];
+      const int i0 = tid * cpt + gi * 8;
+      load8(i0, dv);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        bool take = dv[q] < T;
+        if (dv[q] == T) { take = e < need_eq; ++e; }
+        if (take && pos < a.top_k) {
+          const int i = i0 + q;
+          const int pi = (a.P == 1) ? i : (int)__umulhi((uint32_t)i, magic);
+          out[pos++] = klp[pi] * a.P + (i - pi * a.P);
+        }
+      }
     }
   }
   for (int i = keff + tid; i < a.top_k; i += kHamThreads) out[i] = -1;
   if (tid == 0) a.out_count[row] = keff;
 }
 
-inline size_t hamming_smem(int gs, int C) {
-  int nbins = gs * 128 + 1;
-  return (size_t)(((nbins + 31) & ~31) + 33 + 3) * 4 + (size_t)C * 2 + 16;
+inline size_t hamming_smem(int gs, int m_max, int P) {
+  const int nbins = gs * 128 + 1;
+  const size_t ints = (size_t)((nbins + 31) & ~31) + 36 + (size_t)((2 * m_max + 3) & ~3);
+  // Distances padded so the 16-byte group reads of the last thread stay inside.
+  const size_t cand = ((size_t)m_max * P + 8 + 7) & ~(size_t)7;
+  return ints * 4 + cand * 2 + 16;
 }
 
 // ---------------------------------------------------------------------------- HISA a1'

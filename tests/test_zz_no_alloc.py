@@ -67,9 +67,15 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_rejects_sizes_beyond_the_array():
     build.build()
     L = hhr.lib()
-    # 32 sequences x 8 KV heads x 8-head groups at top_k 8192 needs ~ 69 MB of partials.
-    d = hhr.make_dims(32, 64, 8, 32, 4096, 4096 * 32)
-    assert hhr.hhr_attn_workspace_bytes(d, 8192) > 8 * 1024 * 1024
+    # Grow the batch (8 KV heads, 8-head groups, top_k 8192) until the split-K partials
+    # no longer fit in the 8 MiB array.
+    batch = 32
+    while True:
+        d = hhr.make_dims(batch, 64, 8, 32, 4096, 4096 * 32)
+        if hhr.hhr_attn_workspace_bytes(d, 8192) > 8 * 1024 * 1024:
+            break
+        batch *= 2
+        assert batch <= 65535
     p = ctypes.c_void_p(256)  # never dereferenced: the size check comes first
     st = L.hhr_sparse_attn_noalloc(ctypes.byref(d), p, p, p, p, p, p, p, 8192,
                                    ctypes.c_float(0.1), p, None)
