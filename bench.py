@@ -44,6 +44,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--summary", default="f16", choices=["f16", "f32"],
+                    help="page-summary storage (f16 rounded outward, or f32)")
+    ap.add_argument("--path", default="fused", choices=["fused", "calls"],
+                    help="fused: hhr_decode_step; calls: encode + select + attention calls")
     ap.add_argument("--select-only", action="store_true",
                     help="profiling case: no V cache and no attention (step = encode + select)")
     return ap.parse_args()
@@ -58,7 +62,7 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def required_bytes(wl, lens, m_of):
+def required_bytes(wl, lens, m_of, sbytes=4):
     """Algorithmic bytes of one step: summaries + kept-page codes + selected K/V rows."""
     G, P, d = wl.n_kv_heads, wl.page_size, wl.head_dim
     summ = codes = kv = 0
@@ -66,21 +70,21 @@ def required_bytes(wl, lens, m_of):
         npg = -(-n // P)
         m = m_of(npg)
         cand = min(n, m * P)
-        summ += G * npg * 2 * d * 4
+        summ += G * npg * 2 * d * sbytes
         codes += G * cand * (wl.code_bits // 8)
         kv += G * min(wl.top_k, cand) * 2 * d * 2
     return summ, codes, kv
 
 
-def bound_kernel_bytes(wl, lens):
-    """Algorithmic bytes of one page-bound launch: per (page, group) the 1 KB summary
-    read and the 4-byte bound write; per page its 4-byte page-table entry; per
-    (sequence, group) the 1 KB folded query."""
+def bound_kernel_bytes(wl, lens, sbytes=4):
+    """Algorithmic bytes of one page-bound launch: per (page, group) the summary read
+    (2 x 128 x sbytes) and the 4-byte bound write; per page its 4-byte page-table entry;
+    per (sequence, group) the 1 KB folded query."""
     G = wl.n_kv_heads
     tot = 0
     for n in lens:
         npg = -(-n // wl.page_size)
-        tot += npg * G * (2 * wl.head_dim * 4 + 4) + npg * 4 + G * 2 * wl.head_dim * 4
+        tot += npg * G * (2 * wl.head_dim * sbytes + 4) + npg * 4 + G * 2 * wl.head_dim * 4
     return tot
 
 
@@ -144,10 +148,10 @@ class Clocks:
                 "samples": len(mhz)}
 
 
-def traffic_from_profile(kernel_src_hash):
+def traffic_from_profile(kernel_src_hash, fmt):
     """DRAM bytes per launch of the page-bound kernel from the committed ncu summary,
     or None if the kernel source changed since the counters were taken."""
-    p = os.path.join(ROOT, "profiles", "page_bound_kernel_llama8b_128k_b8.txt")
+    p = os.path.join(ROOT, "profiles", f"page_bound_{fmt}_kernel_llama8b_128k_b8.txt")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -335,7 +339,9 @@ def main():
     lens = S.seq_lens_of(wl)
     P = wl.page_size
     m_of = lambda npg: min(npg, -(-npg // wl.keep_div)) if wl.m_pages == 0 else min(wl.m_pages, npg)
-    summ_b, codes_b, kv_b = required_bytes(wl, lens, m_of)
+    f16 = 1 if args.summary == "f16" else 0
+    sbytes = 2 if f16 else 4
+    summ_b, codes_b, kv_b = required_bytes(wl, lens, m_of, sbytes)
     req = summ_b + codes_b + kv_b
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     L = args.layers or max(2, math.ceil(4 * l2 / req))
@@ -345,7 +351,7 @@ def main():
     for l in range(L):
         inp = S.make_inputs(wl, device=dev, layer=l, with_values=not args.select_only)
         d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, P, inp["max_pages"],
-                          inp["n_phys"])
+                          inp["n_phys"], summary_fp16=f16)
         cache = LayerCache(d, dev)
         zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
         hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
@@ -357,7 +363,11 @@ def main():
     d0 = layers[0][1]
     step = DecodeStep(d0, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev,
                       attention=not args.select_only)
-    stream = torch.cuda.current_stream(dev)
+    # All work runs on one non-default stream (graph capture needs one); the library
+    # launches on torch's current stream.
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
 
     def run(i):
         inp, d, cache, start, one = layers[i % L]
@@ -367,22 +377,61 @@ def main():
             step.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"],
                         W=inp["W"])
             return
+        if args.path == "fused":
+            # The newest row of every sequence is already in the cache: re-append it.
+            step.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
+                            inp["seq_len"], inp["R"], inp["W"], cache)
+            return
         step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
                   inp["R"], inp["W"], cache, start, one)
 
-    # encode 1 + select 4 (qprep, bound, top-m, hamming) + attention 2 (chunks, combine)
-    kernels_per_step = 5 if args.select_only else 7
-    for i in range(max(args.warmup, 3)):
+    if args.select_only:
+        names = ("encode", "qprep", "bound", "hamming")
+    elif args.path == "fused":
+        names = ("encode", "bound", "hamming", "attn", "combine")
+    else:
+        names = ("encode", "qprep", "bound", "hamming", "attn", "combine")
+    for i in range(3):  # eager warm-up: sets kernel attributes outside any capture
         run(i)
     torch.cuda.synchronize()
     st, bits = hhr.hhr_read_device_status()
     if st != hhr.HHR_OK:
         raise RuntimeError(f"device status {bits}")
 
-    # Timed region: K steps, events on the launching stream; per-step events around
-    # the page-bound kernel (the dominant HBM stream) through the library's hook.
+    # Each decode step is one CUDA graph replay (one launch from the host). NG graphs cycle
+    # over the L layer caches; graph j carries its own event pair around the page-bound
+    # kernel, so the last NG replays of the timed region give the kernel's duration.
+    NG = L * max(1, 48 // L)
+    ev_b = timing_events(NG, stream)
+    graphs = []
+    for j in range(NG):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            hhr.hhr_profile_next("bound", ev_b[j][0], ev_b[j][1])
+            run(j)
+        graphs.append(gr)
+    # Per-kernel breakdown graphs (events around every kernel), one per layer.
+    ev_k = {name: timing_events(L, stream) for name in names}
+    kgraphs = []
+    for l in range(L):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for name in names:
+                hhr.hhr_profile_next(name, ev_k[name][l][0], ev_k[name][l][1])
+            run(l)
+            for name in names:  # drop pairs of kernels this configuration did not launch
+                hhr.hhr_profile_next(name, None, None)
+        kgraphs.append(gr)
+    torch.cuda.synchronize()
+
+    for i in range(max(args.warmup, 3)):
+        graphs[i % NG].replay()
+    torch.cuda.synchronize()
+    st, bits = hhr.hhr_read_device_status()
+    if st != hhr.HHR_OK:
+        raise RuntimeError(f"device status {bits}")
+
     K = args.steps
-    ev_b = timing_events(K, stream)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = Clocks(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
@@ -392,15 +441,16 @@ def main():
     clocks.start()
     t0.record(stream)
     for i in range(K):
-        hhr.hhr_profile_next("bound", ev_b[i][0], ev_b[i][1])
-        run(args.warmup + i)
+        graphs[i % NG].replay()
     t1.record(stream)
     torch.cuda.synchronize()
     clocks.stop()
     if world > 1:
         dist.barrier()
     ms_total = t0.elapsed_time(t1)
-    bound_ms = [a.elapsed_time(b) for a, b in ev_b]
+    # The last NG replays of the timed region hold the page-bound kernel's events.
+    bound_ms = [a.elapsed_time(b) for a, b in ev_b] if K >= NG else [
+        ev_b[i % NG][0].elapsed_time(ev_b[i % NG][1]) for i in range(K)]
     ms_t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
@@ -408,87 +458,85 @@ def main():
     ms_step = ms_total / K
     value = world * wl.batch * K / (ms_total / 1e3)
 
-    # Per-kernel averages (separate untimed pass, same launches).
-    kern = {}
-    names = ("encode", "qprep", "bound", "topm", "hamming") + (
-        () if args.select_only else ("attn", "combine"))
-    for name in names:
-        evs = timing_events(50, stream)
-        for i in range(50):
-            hhr.hhr_profile_next(name, evs[i][0], evs[i][1])
-            run(i)
+    # Per-kernel averages: replays of the breakdown graphs, read after each replay.
+    kern = {name: [] for name in names}
+    for r in range(30):
+        kgraphs[r % L].replay()
         torch.cuda.synchronize()
-        kern[name] = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+        for name in names:
+            a_, b_ = ev_k[name][r % L]
+            kern[name].append(a_.elapsed_time(b_) * 1e3)
+    kern = {k: statistics.mean(v) for k, v in kern.items()}
+    # Launches per step: every kernel of the breakdown that ran (an unlaunched kernel's
+    # events are the two pre-recorded ones, 0 us apart).
+    kernels_per_step = sum(1 for v in kern.values() if v > 0.5)
 
     # End to end through the public API with host buffers: every step copies the query
-    # and the newest K/V rows from pinned host memory, runs the step, reads the output.
+    # and the newest K/V rows from pinned host memory, runs the step, reads the output;
+    # the whole sequence is captured once as a CUDA graph and replayed.
     e2e = None
     if not args.no_e2e and not args.select_only:
-        from cuda.bindings import runtime as rt
         inp, d, cache, start, one = layers[0]
-        Bq = wl.batch
-        q_host = inp["q"].cpu().pin_memory()
-        G = wl.n_kv_heads
+        Bq, G = wl.batch, wl.n_kv_heads
         lens_h = inp["seq_len"].cpu().tolist()
         pt_h = inp["page_table"].cpu()
-        new_k = torch.empty(Bq, G, wl.head_dim, dtype=torch.bfloat16).pin_memory()
-        new_v = torch.empty_like(new_k).pin_memory()
+        nq = Bq * wl.n_q_heads * wl.head_dim
+        nkv = Bq * G * wl.head_dim
+        # One pinned host buffer per step: [query | newest K rows | newest V rows] (bf16).
+        host_in = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16).pin_memory()
+        host_in[:nq] = inp["q"].reshape(-1).cpu()
         for b in range(Bq):
             t = lens_h[b] - 1
             phys = int(pt_h[b, t // P])
-            new_k[b] = inp["k_cache"][phys, :, t % P].cpu()
-            new_v[b] = inp["v_cache"][phys, :, t % P].cpu()
+            host_in[nq + b * G * wl.head_dim: nq + (b + 1) * G * wl.head_dim] = \
+                inp["k_cache"][phys, :, t % P].reshape(-1).cpu()
+            host_in[nq + nkv + b * G * wl.head_dim: nq + nkv + (b + 1) * G * wl.head_dim] = \
+                inp["v_cache"][phys, :, t % P].reshape(-1).cpu()
+        dev_in = torch.empty_like(host_in, device=dev)
+        q_d = dev_in[:nq].view(Bq, wl.n_q_heads, wl.head_dim)
+        k_d = dev_in[nq:nq + nkv].view(Bq, G, wl.head_dim)
+        v_d = dev_in[nq + nkv:].view(Bq, G, wl.head_dim)
         out_host = torch.empty(Bq, wl.n_q_heads, wl.head_dim, dtype=torch.float32).pin_memory()
-        row_bytes = wl.head_dim * 2
-        sraw = stream.cuda_stream
-        esz = inp["k_cache"].element_size()
-        dsts = []
-        for b in range(Bq):
-            t = lens_h[b] - 1
-            phys = int(pt_h[b, t // P])
-            off = ((phys * G) * P + t % P) * wl.head_dim * esz
-            dsts.append(off)
 
         def e2e_step():
-            inp["q"].copy_(q_host, non_blocking=True)
-            for b in range(Bq):
-                for cache_t, src in ((inp["k_cache"], new_k), (inp["v_cache"], new_v)):
-                    err, = rt.cudaMemcpy2DAsync(
-                        cache_t.data_ptr() + dsts[b], P * row_bytes,
-                        src.data_ptr() + b * G * row_bytes, row_bytes, row_bytes, G,
-                        rt.cudaMemcpyKind.cudaMemcpyHostToDevice, sraw)
-                    if err != rt.cudaError_t.cudaSuccess:
-                        raise RuntimeError(f"cudaMemcpy2DAsync: {err}")
-            step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
-                      inp["seq_len"], inp["R"], inp["W"], cache, start, one)
+            dev_in.copy_(host_in, non_blocking=True)
+            step.fused_step(q_d, inp["k_cache"], inp["v_cache"], inp["page_table"],
+                            inp["seq_len"], inp["R"], inp["W"], cache, k_new=k_d, v_new=v_d)
             out_host.copy_(step.out, non_blocking=True)
 
-        for _ in range(5):
-            e2e_step()
+        e2e_step()
         torch.cuda.synchronize()
-        Ke = max(50, min(K, 2000))
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=stream):
+            e2e_step()
+        for _ in range(5):
+            ge.replay()
+        torch.cuda.synchronize()
+        Ke = max(50, min(K, 5000))
         a, bev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         a.record(stream)
         for _ in range(Ke):
-            e2e_step()
+            ge.replay()
         bev.record(stream)
         torch.cuda.synchronize()
         ms_e = torch.tensor([a.elapsed_time(bev)], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(ms_e, op=dist.ReduceOp.MAX)
-        h2d = q_host.numel() * 2 + 2 * new_k.numel() * 2
         e2e = {"value": world * Bq * Ke / (float(ms_e.item()) / 1e3), "unit": "queries/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * 4,
-               "steps": Ke}
+               "h2d_bytes_per_step": host_in.numel() * 2,
+               "d2h_bytes_per_step": out_host.numel() * 4, "steps": Ke,
+               "how": "graph replay of: one H2D copy of the pinned [query | newest K | newest V] "
+                      "buffer, hhr_decode_step (which appends the rows), one D2H copy of the "
+                      "output"}
 
     peak, peak_kind = measured_peaks()
-    bound_bytes = bound_kernel_bytes(wl, lens)
+    bound_bytes = bound_kernel_bytes(wl, lens, sbytes)
     bound_avg_ms = statistics.mean(bound_ms)
     achieved = bound_bytes / (bound_avg_ms / 1e3) / 1e9
-    traffic = traffic_from_profile(kernel_source_hash())
+    traffic = traffic_from_profile(kernel_source_hash(), args.summary)
     step_gbs = req / (ms_step / 1e3) / 1e9
 
     cpu = None
@@ -513,11 +561,15 @@ def main():
                        "keep": f"1/{wl.keep_div}" if wl.keep_div else f"{wl.m_pages} pages",
                        "top_k": wl.top_k,
                        "code_bits": wl.code_bits, "layer_caches_rotated": L,
+                       "summaries": args.summary,
                        "l2": f"inputs larger than L2: steps rotate over {L} layer caches, "
                              f"{L * req / 1e6:.0f} MB of required bytes per cycle vs "
                              f"{l2 / 1e6:.0f} MB L2",
-                       "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": "page_bound_kernel",
+                       "parallelism": f"replicas x{world}",
+                       "api": "hhr_decode_step" if args.path == "fused" else
+                              "hhr_encode_keys + hhr_select + hhr_sparse_attn",
+                       "timing": "CUDA-graph replay per step, CUDA events on the stream"},
+            "roofline": {"bound": "hbm", "kernel": f"page_bound_{args.summary}_kernel",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
                          "traffic": traffic, "algorithmic_bytes": bound_bytes,

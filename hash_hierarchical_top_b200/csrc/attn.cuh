@@ -19,6 +19,8 @@
 //      sum, output) per head, or the final output when the group is not split; a
 //      combine kernel merges the splits (standard split softmax rescaling).
 #pragma once
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace hhr {
@@ -26,10 +28,10 @@ namespace hhr {
 constexpr int kAttnWarps = 8;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kTile = 64;                        // selected rows per pipeline stage
-constexpr int kRowsPerWarp = kTile / kAttnWarps; // 8
 constexpr int kStages = 3;
 constexpr int kMaxSplitRows = 2048;              // rows of one split (offsets in smem)
 constexpr int kTargetCtas = 2 * 148;             // two resident CTAs on each of 148 SMs
+constexpr uint32_t kNoRow = 0xffffffffu;          // offset table: row to skip
 
 struct AttnArgs {
   const uint16_t* q;        // [B][Hq][d]
@@ -54,23 +56,69 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Shared memory: kStages x (K tile + V tile) of 64 rows x 256 B, the split's row
-// offsets, and per-warp softmax weights. The merge area reuses the stage buffers.
-inline size_t attn_smem() {
-  return (size_t)kStages * 2 * kTile * kD * 2 + (size_t)kMaxSplitRows * 8 +
-         (size_t)kAttnWarps * kRowsPerWarp * kMaxGroup * 4 + 64;
+// ---- tensor-core fragments (bf16 mma.sync, fp32 accumulate) ----------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D = A(16x16, row) * B(16x8, col) + D
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// D = A(16x8, row) * B(8x8, col) + D
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+  const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+  const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y));
+  return lo | (hi << 16);
+}
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
 }
 
-// GS: compile-time capacity of query heads per group (4 or 8); gs <= GS is masked.
-template <int GS>
-__global__ void __launch_bounds__(kAttnThreads, GS <= 4 ? 2 : 1) sparse_attn_kernel(AttnArgs a) {
+// Shared memory: kStages x (K tile + V tile) of 64 rows x 256 B (16-byte chunks of a row
+// XOR-swizzled by row % 8, so ldmatrix reads of 8 rows hit 8 distinct bank groups), the
+// split's row offsets, and the merge area (reusing the stage buffers).
+inline size_t attn_smem() {
+  return (size_t)kStages * 2 * kTile * kD * 2 + (size_t)kMaxSplitRows * 4 + 64;
+}
+
+__device__ __forceinline__ int swz(int r, int chunk) { return r * kD + ((chunk ^ (r & 7)) << 3); }
+
+// Per warp and tile: the warp's 8 keys. Logits S = Q K^T with Q rows = heads (padded to
+// 16, rows >= gs are zero) on mma.m16n8k16 over 8 channel steps; the accumulator lane
+// (g = lane/4, t = lane%4) holds S[head g][keys 2t, 2t+1], which is exactly the B
+// fragment of O^T = V^T P^T on mma.m16n8k8 (channels on M, heads on N). P is split into
+// bf16 hi + lo parts (two MMAs) so its rounding stays near 2^-16 relative.
+__global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a) {
   extern __shared__ float4 at_smem[];
+  pdl_wait();
+  pdl_trigger();
   uint16_t* stage_base = reinterpret_cast<uint16_t*>(at_smem);             // [kStages][2][kTile][d]
-  long long* offs = reinterpret_cast<long long*>(stage_base + (size_t)kStages * 2 * kTile * kD);
-  float* pbuf = reinterpret_cast<float*>(offs + kMaxSplitRows);             // [warps][8 rows][8 heads]
+  uint32_t* offs = reinterpret_cast<uint32_t*>(stage_base + (size_t)kStages * 2 * kTile * kD);
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;   // fragment coordinates
   const int gs = a.Hq / a.G;
   const int row = b * a.G + g;
   const int cnt = min(a.count[row], a.top_k);
@@ -80,16 +128,16 @@ __global__ void __launch_bounds__(kAttnThreads, GS <= 4 ? 2 : 1) sparse_attn_ker
   const int ntiles = (nrows + kTile - 1) / kTile;
   const int n = a.seq_len[b];
 
-  // Element offsets of the split's rows (-1: skip the row).
+  // Cache row index (phys*G + g)*P + slot of each of the split's rows (kNoRow: skip).
   for (int r = tid; r < ntiles * kTile; r += kAttnThreads) {
-    long long o = -1;
+    uint32_t o = kNoRow;
     if (r < nrows) {
       const int t = a.idx[(size_t)row * a.top_k + base + r];
       const int lp = t / a.P;
       if (t >= 0 && t < n && lp < a.maxp) {
         const int phys = a.page_table[(size_t)b * a.maxp + lp];
         if (phys >= 0 && phys < a.n_phys)
-          o = (((long long)phys * a.G + g) * a.P + (t % a.P)) * kD;
+          o = ((uint32_t)phys * (uint32_t)a.G + (uint32_t)g) * (uint32_t)a.P + (uint32_t)(t % a.P);
         else
           flag_status(kStatusBadPage);
       } else {
@@ -100,8 +148,6 @@ __global__ void __launch_bounds__(kAttnThreads, GS <= 4 ? 2 : 1) sparse_attn_ker
   }
   __syncthreads();
 
-  // Issue the K and V rows of tile t into stage slot t % kStages: 64 rows x 32 pieces of
-  // 16 B; consecutive threads copy consecutive pieces of a row (coalesced 256-byte rows).
   auto issue = [&](int t) {
     uint16_t* Ks = stage_base + (size_t)(t % kStages) * 2 * kTile * kD;
     uint16_t* Vs = Ks + kTile * kD;
@@ -109,12 +155,12 @@ __global__ void __launch_bounds__(kAttnThreads, GS <= 4 ? 2 : 1) sparse_attn_ker
     for (int i = 0; i < (kTile * 16) / kAttnThreads; ++i) {
       const int c = tid + i * kAttnThreads;
       const int r = c >> 4, piece = c & 15;
-      const long long o = offs[t * kTile + r];
-      uint16_t* kd = Ks + r * kD + piece * 8;
-      uint16_t* vd = Vs + r * kD + piece * 8;
-      if (o >= 0) {
-        cp_async16(kd, a.k_cache + o + piece * 8);
-        cp_async16(vd, a.v_cache + o + piece * 8);
+      const uint32_t o = offs[t * kTile + r];
+      uint16_t* kd = Ks + swz(r, piece);
+      uint16_t* vd = Vs + swz(r, piece);
+      if (o != kNoRow) {
+        cp_async16(kd, a.k_cache + (size_t)o * kD + piece * 8);
+        cp_async16(vd, a.v_cache + (size_t)o * kD + piece * 8);
       } else {
         *reinterpret_cast<uint4*>(kd) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
@@ -127,120 +173,106 @@ __global__ void __launch_bounds__(kAttnThreads, GS <= 4 ? 2 : 1) sparse_attn_ker
     cp_async_commit();
   }
 
-  // Query channels 4*lane..4*lane+3 of the group's heads, pre-scaled by scale*log2(e).
-  float4 qv[GS];
+  // A fragments of Q (row gq = head; rows >= gs and the upper 8 rows are zero).
+  uint32_t qa0[8], qa2[8];
+  {
+    const bool hv = gq < gs;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + ((size_t)b * a.Hq + g * gs + (hv ? gq : 0)) * kD);
 #pragma unroll
-  for (int h = 0; h < GS; ++h) {
-    qv[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (h < gs) {
-      const float4 f = bf16x4_to_f4(*reinterpret_cast<const uint2*>(
-          a.q + ((size_t)b * a.Hq + g * gs + h) * kD + 4 * lane));
-      qv[h] = make_float4(f.x * a.scale_log2, f.y * a.scale_log2, f.z * a.scale_log2,
-                          f.w * a.scale_log2);
+    for (int s8 = 0; s8 < 8; ++s8) {
+      qa0[s8] = hv ? qrow[(16 * s8 + 2 * tq) >> 1] : 0u;
+      qa2[s8] = hv ? qrow[(16 * s8 + 2 * tq + 8) >> 1] : 0u;
     }
   }
-  // Per-warp running softmax state of every head (lane-replicated m and l).
-  float m_run[GS], l_run[GS];
-  float4 o_acc[GS];
+  const bool head_ok = gq < gs;
+  float m_run = -INFINITY, l_run = 0.f;      // of head gq (replicated over tq)
+  float oacc[8][4];                          // O^T[channel 16i + gq (+8)][head 2tq (+1)]
 #pragma unroll
-  for (int h = 0; h < GS; ++h) {
-    m_run[h] = -INFINITY;
-    l_run[h] = 0.f;
-    o_acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  float* pw = pbuf + warp * kRowsPerWarp * kMaxGroup;  // [8 rows][8 heads]
+  for (int i = 0; i < 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  const uint32_t smem0 = (uint32_t)__cvta_generic_to_shared(stage_base);
+  const int kr = warp * 8 + (lane & 7);       // ldmatrix row (key) supplied by this lane
+  const int mj = lane >> 3;                   // which of the 4 matrices it addresses
 
   for (int t = 0; t < ntiles; ++t) {
     cp_async_wait<kStages - 2>();
     __syncthreads();
     if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
     cp_async_commit();
-    const uint16_t* Ks = stage_base + (size_t)(t % kStages) * 2 * kTile * kD;
-    const uint16_t* Vs = Ks + kTile * kD;
-    const int r0 = warp * kRowsPerWarp;          // this warp's 8 rows of the tile
-    const int rbase = t * kTile + r0;            // their index within the split
-    float4 kf[kRowsPerWarp];
+    const uint32_t ks = smem0 + (uint32_t)((t % kStages) * 2 * kTile * kD) * 2;
+    const uint32_t vs = ks + (uint32_t)(kTile * kD) * 2;
+    // S = Q K^T for the warp's 8 keys: 8 k-steps, ldmatrix.x4 covers two of them.
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r)
-      kf[r] = bf16x4_to_f4(*reinterpret_cast<const uint2*>(Ks + (r0 + r) * kD + 4 * lane));
-    // Heads in passes of 4: value index r*4 + hh -> after the transposed reduction lane l
-    // holds the logit of row l/4 and head (pass*4 + l%4).
-#pragma unroll
-    for (int h0 = 0; h0 < GS; h0 += 4) {
-      if (h0 >= gs) break;
-      float acc[32];
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r)
-#pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
-          const float4 qq = qv[h0 + hh];
-          acc[r * 4 + hh] = qq.x * kf[r].x + qq.y * kf[r].y + qq.z * kf[r].z + qq.w * kf[r].w;
-        }
-      float lg = warp_transpose_sum32(acc, lane);
-      const int my_r = lane >> 2, my_h = h0 + (lane & 3);
-      const bool valid = (my_h < gs) && (rbase + my_r < nrows) && offs[rbase + my_r] >= 0;
-      lg = valid ? lg : -INFINITY;
-      // Max over the 8 rows of each head: lanes with equal lane%4 (xor 4, 8, 16).
-      float mx = lg;
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-      // Lane l now knows the tile max of head h0 + l%4; fetch each head's onto every lane.
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) {
-        const int h = h0 + hh;
-        const float tmax = __shfl_sync(kFull, mx, hh);
-        const float m_new = fmaxf(m_run[h], tmax);
-        const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run[h] - m_new);
-        m_run[h] = m_new;
-        l_run[h] *= corr;
-        o_acc[h].x *= corr; o_acc[h].y *= corr; o_acc[h].z *= corr; o_acc[h].w *= corr;
-      }
-      float m_h = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh)
-        if ((lane & 3) == hh) m_h = m_run[h0 + hh];
-      const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - m_h);
-      float ps = p;
-      ps += __shfl_xor_sync(kFull, ps, 4);
-      ps += __shfl_xor_sync(kFull, ps, 8);
-      ps += __shfl_xor_sync(kFull, ps, 16);
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) l_run[h0 + hh] += __shfl_sync(kFull, ps, hh);
-      pw[my_r * kMaxGroup + (lane & 3) + h0] = p;
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(ks + (uint32_t)swz(kr, 4 * q4 + mj) * 2, b0, b1, b2, b3);
+      mma_16816(sacc, qa0[2 * q4], 0u, qa2[2 * q4], 0u, b0, b1);
+      mma_16816(sacc, qa0[2 * q4 + 1], 0u, qa2[2 * q4 + 1], 0u, b2, b3);
     }
-    __syncwarp();
-    // P.V over the warp's 8 rows; lane l owns channels 4l..4l+3.
+    // Keys 2tq, 2tq+1 of the warp's 8 for head gq; mask padding and skipped rows.
+    const int kbase = t * kTile + warp * 8 + 2 * tq;
+    const bool v0 = head_ok && kbase < nrows && offs[kbase] != kNoRow;
+    const bool v1 = head_ok && kbase + 1 < nrows && offs[kbase + 1] != kNoRow;
+    const float s0 = v0 ? sacc[0] * a.scale_log2 : -INFINITY;
+    const float s1 = v1 ? sacc[1] * a.scale_log2 : -INFINITY;
+    float mx = fmaxf(s0, s1);
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    const float p0 = v0 ? exp2f(s0 - m_new) : 0.f;
+    const float p1 = v1 ? exp2f(s1 - m_new) : 0.f;
+    float ps = p0 + p1;
+    ps += __shfl_xor_sync(kFull, ps, 1);
+    ps += __shfl_xor_sync(kFull, ps, 2);
+    l_run = l_run * corr + ps;
+    m_run = m_new;
+    // Rescale O^T columns (heads 2tq, 2tq+1): their factors live on lanes 8tq and 8tq+4.
+    const float ca = __shfl_sync(kFull, corr, 8 * tq);
+    const float cb = __shfl_sync(kFull, corr, 8 * tq + 4);
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const float4 vf = bf16x4_to_f4(*reinterpret_cast<const uint2*>(Vs + (r0 + r) * kD + 4 * lane));
-#pragma unroll
-      for (int h = 0; h < GS; ++h) {
-        if (h < gs) {
-          const float p = pw[r * kMaxGroup + h];
-          o_acc[h].x = fmaf(p, vf.x, o_acc[h].x);
-          o_acc[h].y = fmaf(p, vf.y, o_acc[h].y);
-          o_acc[h].z = fmaf(p, vf.z, o_acc[h].z);
-          o_acc[h].w = fmaf(p, vf.w, o_acc[h].w);
-        }
-      }
+    for (int i = 0; i < 8; ++i) {
+      oacc[i][0] *= ca; oacc[i][2] *= ca;
+      oacc[i][1] *= cb; oacc[i][3] *= cb;
     }
-    __syncwarp();
+    const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+    const uint32_t phi = pack_bf16(h0, h1);
+    const uint32_t plo = pack_bf16(p0 - h0, p1 - h1);
+    // O^T += V^T P^T: 8 channel tiles of 16; ldmatrix.x4.trans covers two of them.
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(vs + (uint32_t)swz(kr, 4 * q4 + mj) * 2, a0, a1, a2, a3);
+      mma_1688(oacc[2 * q4], a0, a1, phi);
+      mma_1688(oacc[2 * q4], a0, a1, plo);
+      mma_1688(oacc[2 * q4 + 1], a2, a3, phi);
+      mma_1688(oacc[2 * q4 + 1], a2, a3, plo);
+    }
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Merge the 8 warps' states: o = sum_w 2^(m_w - M) o_w, l = sum_w 2^(m_w - M) l_w.
+  // Merge the 8 warps: o = sum_w 2^(m_w - M) o_w, l = sum_w 2^(m_w - M) l_w.
   float* mo = reinterpret_cast<float*>(stage_base);             // [warps][8 heads][d]
   float* mml = mo + (size_t)kAttnWarps * kMaxGroup * kD;         // [warps][8 heads][2]
+  {
+    float* mw = mo + (size_t)warp * kMaxGroup * kD;
 #pragma unroll
-  for (int h = 0; h < GS; ++h) {
-    if (h < gs) {
-      reinterpret_cast<float4*>(mo + ((size_t)warp * kMaxGroup + h) * kD)[lane] = o_acc[h];
-      if (lane == 0) {
-        mml[(warp * kMaxGroup + h) * 2] = m_run[h];
-        mml[(warp * kMaxGroup + h) * 2 + 1] = l_run[h];
+    for (int i = 0; i < 8; ++i) {
+      const int c0 = 16 * i + gq;
+      if (2 * tq < gs) {
+        mw[(2 * tq) * kD + c0] = oacc[i][0];
+        mw[(2 * tq) * kD + c0 + 8] = oacc[i][2];
       }
+      if (2 * tq + 1 < gs) {
+        mw[(2 * tq + 1) * kD + c0] = oacc[i][1];
+        mw[(2 * tq + 1) * kD + c0 + 8] = oacc[i][3];
+      }
+    }
+    if (tq == 0 && head_ok) {
+      mml[(warp * kMaxGroup + gq) * 2] = m_run;
+      mml[(warp * kMaxGroup + gq) * 2 + 1] = l_run;
     }
   }
   __syncthreads();
@@ -303,6 +335,8 @@ struct CombineArgs {
 };
 
 __global__ void __launch_bounds__(kD) attn_combine_kernel(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int gs = a.Hq / a.G, g = h / gs, hh = h % gs;
   const int row = b * a.G + g;

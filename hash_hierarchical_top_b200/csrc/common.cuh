@@ -2,6 +2,7 @@
 // reductions and scans, order-preserving float keys and the device status word.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -91,6 +92,14 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
   *total = scratch[32];
   __syncthreads();
   return res;
+}
+
+// Programmatic dependent launch: wait until the preceding kernel in the stream has
+// completed and its writes are visible (a no-op when the launch did not ask for
+// programmatic serialisation), and let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
 // Histogram increment aggregated over the warp's lanes that hit the same bin: one

@@ -19,32 +19,52 @@ namespace hhr {
 // for both the transposing stores and the column reads). Used by the bulk SIMT path.
 constexpr int kTS = kD + 1;
 
-// y_v = M x_v for up to kVecChunk vectors at once, M a 128x128 row-major fp32 matrix
-// in global memory (L1/L2-resident: it is shared by every CTA of a group).
-// Warp w computes rows 32w..32w+31: lane l reads float4 l of each row (a coalesced
-// 512-byte row read per instruction), multiplies it with channels 4l..4l+3 of every
-// vector, and a transposed warp reduction leaves y_v[32w + l] on lane l. Each row of
-// M is read once per call for all vectors. Requires blockDim.x == 128.
+// y_v = M x_v for up to kVecChunk vectors at once, M a 128x128 row-major fp32 matrix,
+// with kMvThreads = 512 threads: 4 threads per row. Thread (row r = 8*warp + lane/4,
+// quarter q = lane%4) holds float4s q, q+4, ..., q+28 of row r in registers (the four
+// threads of a row read 64 contiguous bytes per load), dots them with the same float4s
+// of each vector (shared-memory broadcasts), and two shuffles sum the four quarters.
+// Every thread of a row ends up with y_v[r].
 constexpr int kVecChunk = 4;
+constexpr int kMvThreads = 512;
+
+__device__ __forceinline__ int mv_row() { return (threadIdx.x >> 5) * 8 + ((threadIdx.x & 31) >> 2); }
+
+// This thread's quarter of its row of M (8 float4).
+__device__ __forceinline__ void load_rows8(const float* __restrict__ M, float4 (&m)[8]) {
+  const int q = threadIdx.x & 3;
+  const float4* Mr = reinterpret_cast<const float4*>(M + (size_t)mv_row() * kD);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m[j] = __ldg(Mr + 4 * j + q);
+}
 
 template <int NV>
-__device__ __forceinline__ void matvec_rows(const float* __restrict__ M, const float* xs,
-                                            int xs_stride, float (&y)[NV]) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float4 xv[NV];
+__device__ __forceinline__ void matvec8(const float4 (&m)[8], const float* xs, int xs_stride,
+                                        float (&y)[NV]) {
+  const int q = threadIdx.x & 3;
 #pragma unroll
-  for (int v = 0; v < NV; ++v) xv[v] = reinterpret_cast<const float4*>(xs + v * xs_stride)[lane];
-  float acc[NV][32];
-  const float4* Mr = reinterpret_cast<const float4*>(M + (size_t)(warp * 32) * kD) + lane;
+  for (int v = 0; v < NV; ++v) {
+    const float4* xv = reinterpret_cast<const float4*>(xs + v * xs_stride);
+    float acc = 0.f;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float4 m = __ldg(Mr + j * (kD / 4));
-#pragma unroll
-    for (int v = 0; v < NV; ++v)
-      acc[v][j] = m.x * xv[v].x + m.y * xv[v].y + m.z * xv[v].z + m.w * xv[v].w;
+    for (int j = 0; j < 8; ++j) {
+      const float4 x = xv[4 * j + q];
+      acc = fmaf(m[j].x, x.x, fmaf(m[j].y, x.y, fmaf(m[j].z, x.z, fmaf(m[j].w, x.w, acc))));
+    }
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    y[v] = acc;
   }
+}
+
+// The 8 sign bits of this warp's rows (8*warp .. 8*warp+7) from a ballot in which the
+// lanes 4i carry row 8*warp + i.
+__device__ __forceinline__ uint32_t row_bits8(bool positive) {
+  const unsigned b = __ballot_sync(kFull, positive);
+  uint32_t byte = 0;
 #pragma unroll
-  for (int v = 0; v < NV; ++v) y[v] = warp_transpose_sum32(acc[v], lane);
+  for (int i = 0; i < 8; ++i) byte |= ((b >> (4 * i)) & 1u) << i;
+  return byte;
 }
 
 struct EncodeArgs {
@@ -54,19 +74,21 @@ struct EncodeArgs {
   const int32_t* n_new;
   const float* R;
   const float* W;
-  float* page_minmax;
+  void* page_minmax;   // f32 or f16 [n_phys][G][2][d]
   uint32_t* codes;
   float* block_mean;
   int G, P, maxp, n_phys, max_new;
+  int summary_fp16;    // 1: store min rounded down and max rounded up to f16
 };
 
-// One CTA of 128 threads per (touched page, KV group, sequence). The new keys of
-// the page are processed kVecChunk at a time: k' = R_g k (thread 32w+l ends up
-// owning channel 32w+l), min/max folded per channel, then p = W_g k' and the code
-// word of warp w is the ballot of its 32 sign bits.
-__global__ void __launch_bounds__(128) encode_page_kernel(EncodeArgs a) {
+// One CTA of kMvThreads threads per (touched page, KV group, sequence). The new keys of
+// the page are processed kVecChunk at a time: k' = R_g k (the 4 threads of row r own
+// channel r), min/max folded per channel, then p = W_g k'; each warp contributes the 8
+// sign bits of its rows as one byte of the code.
+__global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   __shared__ __align__(16) float kx[kVecChunk][kD];  // raw keys (fp32)
   __shared__ __align__(16) float kr[kVecChunk][kD];  // rotated keys
+  __shared__ __align__(16) uint8_t cbytes[kVecChunk][16];
 
   const int b = blockIdx.z, g = blockIdx.y, j = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -94,48 +116,78 @@ __global__ void __launch_bounds__(128) encode_page_kernel(EncodeArgs a) {
   const int pstart = lp * P;
   const int t0 = max(s, pstart), t1 = min(e, pstart + P);
   const uint16_t* kpage = a.k_cache + ((size_t)phys * G + g) * P * kD;
+  const int row = mv_row();  // channel / code bit owned after a matvec
+  const bool row_lead = (lane & 3) == 0;
 
   if (a.R != nullptr) {
-    const float* Rg = a.R + (size_t)g * kD * kD;
-    const float* Wg = a.W + (size_t)g * kD * kD;
+    // R_g and W_g rows of this thread, and the page's stored summary when the page already
+    // held keys, are fetched up front (one memory latency for all of them).
+    float4 rrow[8], wrow[8];
+    load_rows8(a.R + (size_t)g * kD * kD, rrow);
+    load_rows8(a.W + (size_t)g * kD * kD, wrow);
+    const size_t sbase = ((size_t)phys * G + g) * 2 * kD;
     float mn = INFINITY, mx = -INFINITY;
+    if (t0 > pstart && row_lead) {
+      if (a.summary_fp16) {
+        const __half* mm = reinterpret_cast<const __half*>(a.page_minmax) + sbase;
+        mn = __half2float(mm[row]);
+        mx = __half2float(mm[kD + row]);
+      } else {
+        const float* mm = reinterpret_cast<const float*>(a.page_minmax) + sbase;
+        mn = mm[row];
+        mx = mm[kD + row];
+      }
+    }
     for (int t = t0; t < t1; t += kVecChunk) {
       const int nv = min(kVecChunk, t1 - t);
       __syncthreads();
-      for (int v = 0; v < kVecChunk; ++v)
-        kx[v][tid] = v < nv ? bf16_to_f(kpage[(size_t)(t + v - pstart) * kD + tid]) : 0.f;
+      for (int i = tid; i < kVecChunk * kD; i += kMvThreads) {
+        const int v = i / kD, c = i % kD;
+        kx[v][c] = v < nv ? bf16_to_f(kpage[(size_t)(t + v - pstart) * kD + c]) : 0.f;
+      }
       __syncthreads();
       float y[kVecChunk];
-      matvec_rows<kVecChunk>(Rg, &kx[0][0], kD, y);
+      matvec8<kVecChunk>(rrow, &kx[0][0], kD, y);
 #pragma unroll
       for (int v = 0; v < kVecChunk; ++v) {
         if (v < nv) {
-          kr[v][tid] = y[v];
           mn = fminf(mn, y[v]);
           mx = fmaxf(mx, y[v]);
-        } else {
-          kr[v][tid] = 0.f;
         }
+        if (row_lead) kr[v][row] = v < nv ? y[v] : 0.f;
       }
       __syncthreads();
       float p[kVecChunk];
-      matvec_rows<kVecChunk>(Wg, &kr[0][0], kD, p);
+      matvec8<kVecChunk>(wrow, &kr[0][0], kD, p);
 #pragma unroll
       for (int v = 0; v < kVecChunk; ++v) {
-        const unsigned word = __ballot_sync(kFull, p[v] > 0.f);
-        if (v < nv && lane == 0)
-          a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + warp] = word;
+        const uint32_t bits = row_bits8(p[v] > 0.f);  // rows 8w..8w+7
+        if (lane == 0) cbytes[v][warp] = (uint8_t)bits;
+      }
+      __syncthreads();
+      if (tid < kVecChunk * kWords) {
+        const int v = tid / kWords, w = tid % kWords;
+        if (v < nv)
+          a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + w] =
+              reinterpret_cast<const uint32_t*>(cbytes[v])[w];
       }
     }
-    float* mm = a.page_minmax + ((size_t)phys * G + g) * 2 * kD;
-    if (t0 > pstart) {  // the page already held keys: merge with its stored summary
-      mn = fminf(mn, mm[tid]);
-      mx = fmaxf(mx, mm[kD + tid]);
+    if (row_lead) {
+      // mn/mx started from the stored summary when the page already held keys (min and
+      // max are exact, so merging equals recomputing the whole page).
+      if (a.summary_fp16) {
+        __half* mm = reinterpret_cast<__half*>(a.page_minmax) + sbase;
+        // Outward rounding keeps the stored interval around every rotated key.
+        mm[row] = __float2half_rd(mn);
+        mm[kD + row] = __float2half_ru(mx);
+      } else {
+        float* mm = reinterpret_cast<float*>(a.page_minmax) + sbase;
+        mm[row] = mn;
+        mm[kD + row] = mx;
+      }
     }
-    mm[tid] = mn;
-    mm[kD + tid] = mx;
   }
-  if (a.block_mean != nullptr) {
+  if (a.block_mean != nullptr && tid < kD) {
     // Mean of every valid raw key of the page, summed in ascending position order.
     float sum = 0.f;
     for (int t = pstart; t < t1; ++t) sum += bf16_to_f(kpage[(size_t)(t - pstart) * kD + tid]);

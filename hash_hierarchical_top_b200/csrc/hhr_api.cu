@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "encode.cuh"
 #include "select.cuh"
+#include "step.cuh"
 
 using namespace hhr;
 
@@ -34,6 +35,7 @@ int check_dims(const hhr_dims* d) {
   if (d->page_size > 256 || d->batch > 65535 || d->n_kv_heads > 65535)
     return HHR_ERR_UNSUPPORTED;
   if (d->max_pages_per_seq > kMaxPagesPerSeq) return HHR_ERR_UNSUPPORTED;
+  if (d->summary_fp16 != 0 && d->summary_fp16 != 1) return HHR_ERR_INVALID_ARG;
   return HHR_OK;
 }
 
@@ -66,9 +68,8 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   return e;
 }
 
-bool g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
-    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
-    g_smem_attn8[kMaxDevices];
+bool g_smem_step[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
+    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices];
 
 struct SelectLayout {
   size_t qpn, q_rot, q_code, bounds, kept, kept_count, tok, total;
@@ -109,8 +110,8 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
     if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
     if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
       return HHR_ERR_UNSUPPORTED;
-    if (hamming_smem(d->n_q_heads / d->n_kv_heads, kept_max(d, m_pages, keep_div),
-                     d->page_size) > kMaxKernelSmem)
+    if (topm_hamming_smem(d->n_q_heads / d->n_kv_heads, kept_max(d, m_pages, keep_div),
+                          d->page_size, d->max_pages_per_seq) > kMaxKernelSmem)
       return HHR_ERR_UNSUPPORTED;
   } else if (mode == HHR_MODE_INDEXER) {
     if (m_pages < 1 || keep_div != 0) return HHR_ERR_INVALID_ARG;
@@ -130,11 +131,15 @@ struct ProfPair {
 };
 thread_local ProfPair g_prof[HHR_KERNEL_COUNT];
 
+// External records, so that inside a stream capture they become event-record nodes of
+// the graph (timestamps taken at every replay) rather than internal dependencies.
 void prof_begin(int k, cudaStream_t s) {
-  if (g_prof[k].start != nullptr) cudaEventRecord(g_prof[k].start, s);
+  if (g_prof[k].start != nullptr)
+    cudaEventRecordWithFlags(g_prof[k].start, s, cudaEventRecordExternal);
 }
 void prof_end(int k, cudaStream_t s) {
-  if (g_prof[k].stop != nullptr) cudaEventRecord(g_prof[k].stop, s);
+  if (g_prof[k].stop != nullptr)
+    cudaEventRecordWithFlags(g_prof[k].stop, s, cudaEventRecordExternal);
   g_prof[k].start = nullptr;
   g_prof[k].stop = nullptr;
 }
@@ -143,6 +148,24 @@ int launch_status() {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) g_last_cuda = e;
   return e == cudaSuccess ? HHR_OK : HHR_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel of the stream finishes; it calls griddepcontrol.wait before touching memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
@@ -187,7 +210,7 @@ int hhr_kept_max(const hhr_dims* d, int m_pages, int keep_div) {
 
 int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* page_table,
                     const int32_t* start, const int32_t* n_new, int max_new, const float* R,
-                    const float* W, float* page_minmax, uint32_t* codes, float* block_mean,
+                    const float* W, void* page_minmax, uint32_t* codes, float* block_mean,
                     void* stream) {
   int st = check_dims(d);
   if (st != HHR_OK) return st;
@@ -204,13 +227,13 @@ int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* p
   cudaStream_t s = (cudaStream_t)stream;
   EncodeArgs a{k_cache, page_table, start, n_new, hashing ? R : nullptr, hashing ? W : nullptr,
                page_minmax, codes, block_mean, d->n_kv_heads, d->page_size,
-               d->max_pages_per_seq, d->n_phys_pages, max_new};
+               d->max_pages_per_seq, d->n_phys_pages, max_new, d->summary_fp16};
   size_t smem = hashing ? encode_page_smem() : 0;
   if (hashing && allow_smem(encode_page_kernel, smem, g_smem_encode) != cudaSuccess)
     return HHR_ERR_CUDA;
   dim3 grid((unsigned)pages, d->n_kv_heads, d->batch);
   prof_begin(HHR_KERNEL_ENCODE, s);
-  encode_page_kernel<<<grid, 128, smem, s>>>(a);
+  encode_page_kernel<<<grid, kMvThreads, smem, s>>>(a);
   prof_end(HHR_KERNEL_ENCODE, s);
   return launch_status();
 }
@@ -223,7 +246,7 @@ size_t hhr_select_workspace_bytes(const hhr_dims* d, int mode, int m_pages, int 
 
 int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* seq_len,
                const int32_t* q_pos, const int32_t* page_table, const float* R, const float* W,
-               const float* page_minmax, const uint32_t* codes, const float* block_mean,
+               const void* page_minmax, const uint32_t* codes, const float* block_mean,
                const uint16_t* k_cache, int m_pages, int keep_div, int top_k, int32_t* out_idx,
                int32_t* out_count, void* workspace, size_t ws_bytes, hhr_trace* trace,
                void* stream) {
@@ -258,32 +281,32 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
     uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
     if (allow_smem(qprep_kernel, qprep_smem(), g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(hamming_topk_kernel, hamming_smem(Hq / G, m_max, P), g_smem_ham) != cudaSuccess)
+    if (allow_smem(topm_hamming_kernel, topm_hamming_smem(Hq / G, m_max, P, maxp), g_smem_ham) !=
+        cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
-    qprep_kernel<<<dim3(G, B), 128, qprep_smem(), s>>>(
+    qprep_kernel<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
         QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
     prof_end(HHR_KERNEL_QPREP, s);
     if ((st = launch_status()) != HHR_OK) return st;
     prof_begin(HHR_KERNEL_BOUND, s);
-    page_bound_kernel<<<dim3((maxp + kPagesPerCta - 1) / kPagesPerCta, G, B), kBoundWarps * 32,
-                        0, s>>>(
-        BoundArgs{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp, d->n_phys_pages});
+    {
+      const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
+                         d->n_phys_pages};
+      const dim3 grid = bound_grid(G, (maxp + kPagesPerCtaB - 1) / kPagesPerCtaB, B);
+      if (d->summary_fp16)
+        page_bound_kernel<true><<<grid, kBoundWarps * 32, 0, s>>>(ba);
+      else
+        page_bound_kernel<false><<<grid, kBoundWarps * 32, 0, s>>>(ba);
+    }
     prof_end(HHR_KERNEL_BOUND, s);
-    if ((st = launch_status()) != HHR_OK) return st;
-    SelectArgs sa{};
-    sa.scores = bounds; sa.stride = maxp; sa.rows_per_b = G; sa.seq_len = seq_len;
-    sa.q_pos = nullptr; sa.P = P; sa.mode = 0; sa.m_max = m_max; sa.unit = 0;
-    sa.m_pages = m_pages; sa.keep_div = keep_div; sa.top_k = 0;
-    sa.out = kept; sa.out_stride = m_max; sa.out_count = kept_count; sa.pad_out = 0;
-    prof_begin(HHR_KERNEL_TOPM, s);
-    select_largest_kernel<<<B * G, kSelThreads, (size_t)maxp * 4, s>>>(sa);
-    prof_end(HHR_KERNEL_TOPM, s);
     if ((st = launch_status()) != HHR_OK) return st;
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
+    const size_t fsm = topm_hamming_smem(Hq / G, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
-    hamming_topk_kernel<<<B * G, kHamThreads, hamming_smem(Hq / G, m_max, P), s>>>(ha);
+    topm_hamming_kernel<<<B * G, kHamThreads, fsm, s>>>(
+        TopmHammingArgs{ha, bounds, m_pages, keep_div});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
     if (trace != nullptr) {
@@ -363,6 +386,9 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
       workspace == nullptr)
     return HHR_ERR_INVALID_ARG;
   if (top_k < 1 || !(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
+  // Cache rows are addressed with 32-bit row indices.
+  if ((unsigned long long)d->n_phys_pages * d->n_kv_heads * d->page_size >= 0xffffffffull)
+    return HHR_ERR_UNSUPPORTED;
   const size_t need = hhr_attn_workspace_bytes(d, top_k);
   if (ws_bytes < need) return HHR_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
@@ -378,15 +404,9 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
              scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
              d->n_phys_pages, top_k, ns, plan.split_rows};
   prof_begin(HHR_KERNEL_ATTN, s);
-  if (gs <= 4) {
-    if (allow_smem(sparse_attn_kernel<4>, attn_smem(), g_smem_attn) != cudaSuccess)
-      return HHR_ERR_CUDA;
-    sparse_attn_kernel<4><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
-  } else {
-    if (allow_smem(sparse_attn_kernel<8>, attn_smem(), g_smem_attn8) != cudaSuccess)
-      return HHR_ERR_CUDA;
-    sparse_attn_kernel<8><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
-  }
+  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess)
+    return HHR_ERR_CUDA;
+  sparse_attn_kernel<<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
   prof_end(HHR_KERNEL_ATTN, s);
   if ((st = launch_status()) != HHR_OK) return st;
   if (ns > 1) {
@@ -396,6 +416,108 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
     prof_end(HHR_KERNEL_COMBINE, s);
   }
   return launch_status();
+}
+
+size_t hhr_decode_step_workspace_bytes(const hhr_dims* d, int m_pages, int keep_div,
+                                       int top_k) {
+  const size_t sel = hhr_select_workspace_bytes(d, HHR_MODE_HASH, m_pages, keep_div, top_k);
+  const size_t att = hhr_attn_workspace_bytes(d, top_k);
+  if (sel == 0 || att == 0) return 0;
+  return sel + att;
+}
+
+int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
+                    const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
+                    const int32_t* page_table, const int32_t* seq_len, const float* R,
+                    const float* W, void* page_minmax, uint32_t* codes, int m_pages,
+                    int keep_div, int top_k, float scale, int32_t* out_idx, int32_t* out_count,
+                    float* out, void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_select_params(d, HHR_MODE_HASH, m_pages, keep_div, top_k);
+  if (st != HHR_OK) return st;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || page_table == nullptr ||
+      seq_len == nullptr || R == nullptr || W == nullptr || page_minmax == nullptr ||
+      codes == nullptr || out_idx == nullptr || out_count == nullptr || out == nullptr ||
+      workspace == nullptr)
+    return HHR_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return HHR_ERR_INVALID_ARG;
+  if (!(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
+  if ((unsigned long long)d->n_phys_pages * d->n_kv_heads * d->page_size >= 0xffffffffull)
+    return HHR_ERR_UNSUPPORTED;
+  const size_t need = hhr_decode_step_workspace_bytes(d, m_pages, keep_div, top_k);
+  if (need == 0) return HHR_ERR_INVALID_ARG;
+  if (ws_bytes < need) return HHR_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, P = d->page_size;
+  const int maxp = d->max_pages_per_seq, gs = Hq / G;
+  const int m_max = kept_max(d, m_pages, keep_div);
+  const SelectLayout L = select_layout(d, HHR_MODE_HASH, m_max);
+  char* ws = static_cast<char*>(workspace);
+  float* qpn = reinterpret_cast<float*>(ws + L.qpn);
+  float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
+  uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
+  float* bounds = reinterpret_cast<float*>(ws + L.bounds);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
+  int32_t* kept_count = reinterpret_cast<int32_t*>(ws + L.kept_count);
+  char* aws = ws + L.total;
+  const AttnPlan plan = attn_plan(B, G, top_k);
+  const int ns = plan.n_splits;
+  float* part_o = reinterpret_cast<float*>(aws);
+  float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
+  const size_t fsm = topm_hamming_smem(gs, m_max, P, maxp);
+  if (allow_smem(topm_hamming_kernel, fsm, g_smem_ham) != cudaSuccess) return HHR_ERR_CUDA;
+  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess)
+    return HHR_ERR_CUDA;
+  cudaError_t e;
+
+  // a0 + a1: append and encode the newest key rows, rotate and encode the queries.
+  prof_begin(HHR_KERNEL_ENCODE, s);
+  step_prologue_kernel<<<dim3(G, B), kMvThreads, 0, s>>>(
+      PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
+                   codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
+                   d->summary_fp16});
+  prof_end(HHR_KERNEL_ENCODE, s);
+  if ((st = launch_status()) != HHR_OK) return st;
+  // a2: page bounds.
+  {
+    const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
+                       d->n_phys_pages};
+    const dim3 grid = bound_grid(G, (maxp + kPagesPerCtaB - 1) / kPagesPerCtaB, B);
+    prof_begin(HHR_KERNEL_BOUND, s);
+    e = d->summary_fp16 ? launch_pdl(page_bound_kernel<true>, grid, dim3(kBoundWarps * 32), 0, s, ba)
+                        : launch_pdl(page_bound_kernel<false>, grid, dim3(kBoundWarps * 32), 0, s, ba);
+    prof_end(HHR_KERNEL_BOUND, s);
+    if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+  }
+  // a2 top-m + a3 + a4: kept pages, Hamming distances, deterministic top-k.
+  {
+    HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
+    prof_begin(HHR_KERNEL_HAMMING, s);
+    e = launch_pdl(topm_hamming_kernel, dim3(B * G), dim3(kHamThreads), fsm, s,
+                   TopmHammingArgs{ha, bounds, m_pages, keep_div});
+    prof_end(HHR_KERNEL_HAMMING, s);
+    if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+  }
+  // a5: sparse attention over the selected rows.
+  {
+    AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, part_o, part_ml,
+                out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k, ns,
+                plan.split_rows};
+    prof_begin(HHR_KERNEL_ATTN, s);
+    e = launch_pdl(sparse_attn_kernel, dim3(ns, G, B), dim3(kAttnThreads), attn_smem(), s, aa);
+    prof_end(HHR_KERNEL_ATTN, s);
+    if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+    if (ns > 1) {
+      prof_begin(HHR_KERNEL_COMBINE, s);
+      e = launch_pdl(attn_combine_kernel, dim3(Hq, B), dim3(kD), 0, s,
+                     CombineArgs{part_o, part_ml, out_count, out, Hq, G, top_k, ns,
+                                 plan.split_rows});
+      prof_end(HHR_KERNEL_COMBINE, s);
+      if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+    }
+  }
+  return HHR_OK;
 }
 
 int hhr_read_device_status(void* stream, int* bits) {

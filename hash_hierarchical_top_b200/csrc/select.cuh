@@ -8,9 +8,9 @@ namespace hhr {
 
 // ---------------------------------------------------------------------------- a1
 // HHR page, Abstract (queries are rotated by the same R_h and encoded like keys).
-// One CTA of 128 threads per (KV group, sequence). For each query head of the
-// group: q' = R_g q (thread i owns channel i), code bits = [W_g q' > 0] (thread j
-// owns bit j). Also folds the group into the two bound vectors
+// One CTA of kMvThreads threads per (KV group, sequence). For each query head of the
+// group: q' = R_g q, code bits = [W_g q' > 0] (the 4 threads of row r own channel
+// and bit r). Also folds the group into the two bound vectors
 //   qneg_c = sum_h min(q'_hc, 0),  qpos_c = sum_h max(q'_hc, 0),
 // so that sum_h max(q'_hc*kmin_c, q'_hc*kmax_c) = qneg_c*kmin_c + qpos_c*kmax_c
 // (kmin <= kmax: a positive q' picks kmax, a negative one kmin). The page bound
@@ -25,47 +25,62 @@ struct QPrepArgs {
   int Hq, G;
 };
 
-__global__ void __launch_bounds__(128) qprep_kernel(QPrepArgs a) {
+__global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
   __shared__ __align__(16) float qx[kMaxGroup][kD];
   __shared__ __align__(16) float qr[kMaxGroup][kD];
+  __shared__ __align__(16) uint8_t cbytes[kMaxGroup][16];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
+  const int row = mv_row();
+  const bool row_lead = (lane & 3) == 0;
   const int gs = a.Hq / a.G;
-  const float* Rg = a.R + (size_t)g * kD * kD;
-  const float* Wg = a.W + (size_t)g * kD * kD;
-  for (int h = 0; h < kMaxGroup; ++h) {
-    qx[h][tid] = h < gs ? bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + h) * kD + tid]) : 0.f;
-    qr[h][tid] = 0.f;
+  // R_g and W_g rows of this warp are fetched up front (one memory latency for both).
+  float4 rrow[8], wrow[8];
+  load_rows8(a.R + (size_t)g * kD * kD, rrow);
+  load_rows8(a.W + (size_t)g * kD * kD, wrow);
+  for (int i = tid; i < kMaxGroup * kD; i += kMvThreads) {
+    const int h = i / kD, c = i % kD;
+    qx[h][c] = h < gs ? bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + h) * kD + c]) : 0.f;
+    qr[h][c] = 0.f;
   }
   __syncthreads();
   float qneg = 0.f, qpos = 0.f;
   for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
     float y[kVecChunk];
-    matvec_rows<kVecChunk>(Rg, &qx[h0][0], kD, y);
+    matvec8<kVecChunk>(rrow, &qx[h0][0], kD, y);
 #pragma unroll
     for (int v = 0; v < kVecChunk; ++v) {
       if (h0 + v < gs) {
-        qr[h0 + v][tid] = y[v];
-        a.q_rot[((size_t)b * a.Hq + g * gs + h0 + v) * kD + tid] = y[v];
         qneg += fminf(y[v], 0.f);
         qpos += fmaxf(y[v], 0.f);
+        if (row_lead) {
+          qr[h0 + v][row] = y[v];
+          a.q_rot[((size_t)b * a.Hq + g * gs + h0 + v) * kD + row] = y[v];
+        }
       }
     }
   }
   __syncthreads();
   for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
     float p[kVecChunk];
-    matvec_rows<kVecChunk>(Wg, &qr[h0][0], kD, p);
+    matvec8<kVecChunk>(wrow, &qr[h0][0], kD, p);
 #pragma unroll
     for (int v = 0; v < kVecChunk; ++v) {
-      const unsigned word = __ballot_sync(kFull, p[v] > 0.f);
-      if (h0 + v < gs && lane == 0)
-        a.q_code[((size_t)b * a.Hq + g * gs + h0 + v) * kWords + warp] = word;
+      const uint32_t bits = row_bits8(p[v] > 0.f);
+      if (lane == 0 && h0 + v < kMaxGroup) cbytes[h0 + v][warp] = (uint8_t)bits;
     }
   }
-  float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
-  o[tid] = qneg;
-  o[kD + tid] = qpos;
+  __syncthreads();
+  if (tid < gs * kWords) {
+    const int h = tid / kWords, w = tid % kWords;
+    a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] =
+        reinterpret_cast<const uint32_t*>(cbytes[h])[w];
+  }
+  if (row_lead) {
+    float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
+    o[row] = qneg;
+    o[kD + row] = qpos;
+  }
 }
 
 inline size_t qprep_smem() { return 0; }
@@ -73,66 +88,137 @@ inline size_t qprep_smem() { return 0; }
 // ---------------------------------------------------------------------------- a2
 // HHR page, Abstract: page-level logit bounds of the rotated keys prune pages.
 // bound_p = qneg . kmin_p + qpos . kmax_p over the page summary (1 KB per page and
-// group). The summaries are the dominant HBM stream of the whole path, so this
-// kernel is a pure streaming GEMV: one warp per page, every lane loads one float4
-// of kmin and one of kmax (a warp reads the page's 1 KB in two coalesced 512-byte
-// transactions), 8 FMAs, one warp sum. Each warp handles kPagesPerWarp pages with
-// all loads issued before any arithmetic so that 2*kPagesPerWarp 16-byte loads per
-// lane are in flight.
-constexpr int kBoundWarps = 8;
-constexpr int kPagesPerWarp = 8;
-constexpr int kPagesPerCta = kBoundWarps * kPagesPerWarp;
+// group in f32, 512 B in f16). The summaries are the dominant HBM stream of the whole
+// path, so this kernel is a pure streaming GEMV.
+// Tuned on B200 at 128K context, batch 8 (4096 pages x 8 groups x 8 sequences).
+#ifndef HHR_BOUND_WARPS
+#define HHR_BOUND_WARPS 4
+#endif
+#ifndef HHR_BOUND_ROUNDS
+#define HHR_BOUND_ROUNDS 1
+#endif
+constexpr int kBoundWarps = HHR_BOUND_WARPS;
+
+// Grid of the bound kernels: (page chunk, group, sequence), or (group, page chunk,
+// sequence) when HHR_BOUND_GROUP_FAST is set.
+#ifdef HHR_BOUND_GROUP_FAST
+__device__ __forceinline__ int bound_group() { return blockIdx.x; }
+__device__ __forceinline__ int bound_chunk() { return blockIdx.y; }
+inline dim3 bound_grid(int G, int chunks, int B) { return dim3(G, chunks, B); }
+#else
+__device__ __forceinline__ int bound_group() { return blockIdx.y; }
+__device__ __forceinline__ int bound_chunk() { return blockIdx.x; }
+inline dim3 bound_grid(int G, int chunks, int B) { return dim3(chunks, G, B); }
+#endif
 
 struct BoundArgs {
   const float* qpn;
-  const float* page_minmax;
+  const void* page_minmax;  // f32 or f16 [n_phys][G][2][d]
   const int32_t* page_table;
   const int32_t* seq_len;
   float* bounds;  // [B][G][maxp]
   int G, P, maxp, n_phys;
 };
 
-__global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
-  const int g = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int npg = ceil_div(a.seq_len[b], a.P);
-  const int base = blockIdx.x * kPagesPerCta + warp * kPagesPerWarp;
-  if (base >= min(npg, a.maxp)) return;
-  const float4 qn = reinterpret_cast<const float4*>(a.qpn + ((size_t)b * a.G + g) * 2 * kD)[lane];
-  const float4 qp =
-      reinterpret_cast<const float4*>(a.qpn + ((size_t)b * a.G + g) * 2 * kD + kD)[lane];
-  // Page ids of this warp's pages: lane i < kPagesPerWarp reads one, then broadcast.
-  int my_phys = -1;
-  if (lane < kPagesPerWarp && base + lane < min(npg, a.maxp))
-    my_phys = a.page_table[(size_t)b * a.maxp + base + lane];
-  float4 mn[kPagesPerWarp], mx[kPagesPerWarp];
+// Sum over the warp of 8 per-lane partials (one per page): a butterfly over lane bits 4
+// and 3, then a transposition over bits 2..0; lane l ends with the total of page l & 7.
+__device__ __forceinline__ float warp_sum8_transposed(float (&v)[8], int lane) {
 #pragma unroll
-  for (int i = 0; i < kPagesPerWarp; ++i) {
-    int phys = __shfl_sync(kFull, my_phys, i);
-    if (phys >= 0 && phys < a.n_phys) {
-      const float4* s = reinterpret_cast<const float4*>(a.page_minmax +
-                                                        ((size_t)phys * a.G + g) * 2 * kD);
-      mn[i] = __ldcs(s + lane);
-      mx[i] = __ldcs(s + 32 + lane);
-    } else {
-      mn[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      mx[i] = mn[i];
+  for (int i = 0; i < 8; ++i) {
+    v[i] += __shfl_xor_sync(kFull, v[i], 16);
+    v[i] += __shfl_xor_sync(kFull, v[i], 8);
+  }
+#pragma unroll
+  for (int s = 4; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, s);
     }
   }
+  return v[0];
+}
+
+// One warp per page and load instruction (coalesced: lane l reads 16-byte piece l of the
+// page's summary), 8 pages per round, kBoundRounds rounds per warp; the 8 page sums of a
+// round are folded by one transposed reduction. f32 pages are 1 KB (two pieces per lane:
+// channels 4l..4l+3 of the min and of the max row); f16 pages are 512 B (one piece: lanes
+// 0-15 hold 8 channels of the min row, lanes 16-31 of the max row). Each piece is paired
+// with the matching channels of the folded query (qneg with min, qpos with max).
+constexpr int kBoundRounds = HHR_BOUND_ROUNDS;
+constexpr int kPagesPerCtaB = kBoundWarps * 8 * kBoundRounds;
+
+__device__ __forceinline__ float dot8_h(const uint4 h, const float4 q0, const float4 q1) {
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+  const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&h.z));
+  const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&h.w));
+  return q0.x * a.x + q0.y * a.y + q0.z * b.x + q0.w * b.y + q1.x * c.x + q1.y * c.y +
+         q1.z * d.x + q1.w * d.y;
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int g = bound_group(), b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
+  const int cta_base = bound_chunk() * kPagesPerCtaB;
+  if (cta_base >= npg) return;
+  const float* qb = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
+  float4 q0, q1;
+  if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
+    const float4* qv = reinterpret_cast<const float4*>(qb + (lane >> 4) * kD + 8 * (lane & 15));
+    q0 = qv[0];
+    q1 = qv[1];
+  } else {              // channels 4l..4l+3 of qneg and of qpos
+    q0 = reinterpret_cast<const float4*>(qb)[lane];
+    q1 = reinterpret_cast<const float4*>(qb + kD)[lane];
+  }
+  // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
+  constexpr int kPieces = F16 ? 32 : 64;
+  const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
   float* out = a.bounds + ((size_t)b * a.G + g) * a.maxp;
 #pragma unroll
-  for (int i = 0; i < kPagesPerWarp; ++i) {
-    float v = qn.x * mn[i].x + qn.y * mn[i].y + qn.z * mn[i].z + qn.w * mn[i].w +
-              qp.x * mx[i].x + qp.y * mx[i].y + qp.z * mx[i].z + qp.w * mx[i].w;
-    v = warp_sum(v);
-    int phys = __shfl_sync(kFull, my_phys, i);
-    int lp = base + i;
-    if (lane == 0 && lp < min(npg, a.maxp)) {
-      if (phys < 0 || phys >= a.n_phys) {
-        flag_status(kStatusBadPage);
-        v = -INFINITY;
+  for (int r = 0; r < kBoundRounds; ++r) {
+    const int p0 = cta_base + (r * kBoundWarps + warp) * 8;
+    if (p0 >= npg) break;
+    int my_phys = -1;  // lane i < 8 resolves page p0 + i
+    if (lane < 8 && p0 + lane < npg) my_phys = a.page_table[(size_t)b * a.maxp + p0 + lane];
+    uint4 x[8], y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int phys = __shfl_sync(kFull, my_phys, i);
+      x[i] = make_uint4(0, 0, 0, 0);
+      y[i] = x[i];
+      if (phys >= 0 && phys < a.n_phys) {
+        const uint4* src = base4 + ((size_t)phys * a.G + g) * kPieces + lane;
+        x[i] = __ldcs(src);
+        if constexpr (!F16) y[i] = __ldcs(src + 32);
       }
-      out[lp] = v;
+    }
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if constexpr (F16) {
+        v[i] = dot8_h(x[i], q0, q1);
+      } else {
+        const float4 mn = *reinterpret_cast<const float4*>(&x[i]);
+        const float4 mx = *reinterpret_cast<const float4*>(&y[i]);
+        v[i] = q0.x * mn.x + q0.y * mn.y + q0.z * mn.z + q0.w * mn.w + q1.x * mx.x +
+               q1.y * mx.y + q1.z * mx.z + q1.w * mx.w;
+      }
+    }
+    const float tot = warp_sum8_transposed(v, lane);
+    // Lane l (< 8) now holds the bound of page p0 + l.
+    const int lp = p0 + lane;
+    if (lane < 8 && lp < npg) {
+      const bool ok = my_phys >= 0 && my_phys < a.n_phys;
+      if (!ok) flag_status(kStatusBadPage);
+      out[lp] = ok ? tot : -INFINITY;
     }
   }
 }
@@ -193,24 +279,23 @@ __device__ __forceinline__ void block_minmax_u32(uint32_t lo, uint32_t hi, uint3
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
-  __shared__ int hist[256];
-  __shared__ int scratch[33];
-  __shared__ uint32_t mm[64];
-  __shared__ int sh_digit, sh_rem, sh_cnt;
-  extern __shared__ uint32_t keys[];  // [n], 16-byte aligned
-  const int row = blockIdx.x, tid = threadIdx.x;
-  const int b = row / a.rows_per_b;
-  int n;
-  if (a.mode == 0) {
-    int len = a.seq_len[b];
-    if (a.q_pos != nullptr) len = min(len, a.q_pos[row] + 1);
-    n = min(ceil_div(max(len, 0), a.P), a.stride);
-  } else {
-    n = min(a.kept_count[row] * a.unit, a.stride);
-  }
-  const float* sc = a.scores + (size_t)row * a.stride;
-  // Contiguous chunk of each thread (index order is needed by the compaction).
+struct SelShared {
+  int hist[256];
+  int scratch[33];
+  uint32_t mm[64];
+  int digit, rem, cnt;
+};
+
+// Block-wide selection (kSelThreads threads, call uniformly): the k largest finite scores
+// of sc[0..n), ties to the lower index, written in ascending index order to out[0..k)
+// (global or shared memory). k = kept_for(#finite, m_pages, keep_div) when by_kept, else
+// min(top_k, #finite). unit > 0 maps index i to kept_units[i / unit] * unit + i % unit.
+// keys: shared scratch of n words (16-byte aligned). Returns k.
+__device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
+                                    bool by_kept, int m_pages, int keep_div, int top_k,
+                                    int32_t* out, int out_stride, const int32_t* kept_units,
+                                    int unit) {
+  const int tid = threadIdx.x;
   const int per = ceil_div(n, kSelThreads);
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
   int nfin = 0;
@@ -224,10 +309,10 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
     if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
   }
   int total;
-  block_excl_scan(nfin, scratch, &total);  // also orders the key stores before any read
+  block_excl_scan(nfin, sh.scratch, &total);  // also orders the key stores before any read
   nfin = total;
-  block_minmax_u32(kmin, kmax, mm, &kmin, &kmax);
-  const int k = (a.mode == 0) ? kept_for(nfin, a.m_pages, a.keep_div) : min(a.top_k, nfin);
+  block_minmax_u32(kmin, kmax, sh.mm, &kmin, &kmax);
+  const int k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
 
   // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
   // keys at sel_shift == 0 are taken in index order until `rem` of them are taken; at
@@ -248,18 +333,18 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
       uint32_t mask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);   // common high bits
       prefix = kmin & mask;
       while (true) {
-        if (tid < 256) hist[tid] = 0;
+        if (tid < 256) sh.hist[tid] = 0;
         __syncthreads();
         for (int i = tid; i < n; i += kSelThreads) {
           const uint32_t kk = keys[i];
-          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&sh.hist[(kk >> shift) & 255], 1);
         }
         __syncthreads();
         if (tid < 32) {
           // Lane l covers digits 255-8l .. 248-8l (descending).
           int c[8], s = 0;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * tid - q]; s += c[q]; }
+          for (int q = 0; q < 8; ++q) { c[q] = sh.hist[255 - 8 * tid - q]; s += c[q]; }
           const int incl = warp_incl_scan(s, tid);
           const int excl = incl - s;
           if (excl < rem && rem <= incl) {
@@ -267,19 +352,19 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (run < rem && rem <= run + c[q]) {
-                sh_digit = 255 - 8 * tid - q;
-                sh_rem = rem - run;
-                sh_cnt = c[q];
+                sh.digit = 255 - 8 * tid - q;
+                sh.rem = rem - run;
+                sh.cnt = c[q];
               }
               run += c[q];
             }
           }
         }
         __syncthreads();
-        prefix |= (uint32_t)sh_digit << shift;
+        prefix |= (uint32_t)sh.digit << shift;
         mask |= 255u << shift;
-        rem = sh_rem;
-        const int cnt_bin = sh_cnt;
+        rem = sh.rem;
+        const int cnt_bin = sh.cnt;
         __syncthreads();
         if (rem == cnt_bin) {  // the whole bin is needed: no tie-break required
           whole_bin = true;
@@ -307,23 +392,43 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
       else if (!whole_bin && kk == prefix) ++eq;
     }
   }
-  const int eq_before = block_excl_scan(eq, scratch, &total);
+  const int eq_before = block_excl_scan(eq, sh.scratch, &total);
   if (k > 0 && !whole_bin) cnt += max(0, min(eq, rem - eq_before));
-  int pos = block_excl_scan(cnt, scratch, &total);
-  int32_t* out = a.out + (size_t)row * a.out_stride;
+  int pos = block_excl_scan(cnt, sh.scratch, &total);
   if (k > 0) {
     int e = eq_before;
     for (int i = i0; i < i1; ++i) {
       const uint32_t kk = keys[i];
       bool take = take_gt(kk);
       if (!take && !whole_bin && kk == prefix) { take = e < rem; ++e; }
-      if (take && pos < a.out_stride) {
+      if (take && pos < out_stride) {
         int v = i;
-        if (a.unit > 0) v = a.kept_units[(size_t)row * a.m_max + i / a.unit] * a.unit + i % a.unit;
+        if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
         out[pos++] = v;
       }
     }
   }
+  return k;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
+  __shared__ SelShared sh;
+  extern __shared__ uint32_t keys[];  // [n], 16-byte aligned
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int b = row / a.rows_per_b;
+  int n;
+  if (a.mode == 0) {
+    int len = a.seq_len[b];
+    if (a.q_pos != nullptr) len = min(len, a.q_pos[row] + 1);
+    n = min(ceil_div(max(len, 0), a.P), a.stride);
+  } else {
+    n = min(a.kept_count[row] * a.unit, a.stride);
+  }
+  int32_t* out = a.out + (size_t)row * a.out_stride;
+  const int k = block_select_largest(
+      a.scores + (size_t)row * a.stride, n, keys, sh, a.mode == 0, a.m_pages, a.keep_div,
+      a.top_k, out, a.out_stride,
+      a.unit > 0 ? a.kept_units + (size_t)row * a.m_max : nullptr, a.unit);
   if (a.pad_out)
     for (int i = k + tid; i < a.out_stride; i += kSelThreads) out[i] = -1;
   if (tid == 0) a.out_count[row] = k;
@@ -354,13 +459,15 @@ struct HammingArgs {
 
 constexpr int kHamUnroll = 8;
 
-__global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a) {
-  extern __shared__ uint32_t hsm[];
-  const int row = blockIdx.x, b = row / a.G, g = row % a.G;
+// Steps a3-a4 for one (sequence, group) row, given its kept logical pages kept_list[0..m)
+// (ascending; global or shared memory). hsm: hamming_smem() bytes of shared memory.
+__device__ void hamming_topk_block(const HammingArgs& a, int row, const int32_t* kept_list,
+                                   int m, uint32_t* hsm) {
+  const int b = row / a.G, g = row % a.G;
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.G;
   const int nbins = gs * 128 + 1;
-  const int m = min(a.kept_count[row], a.m_max);
+  m = min(m, a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                    // [nbins]
   int* scratch = hist + ((nbins + 31) & ~31);                 // [33]
   int* sh = scratch + 33;                                     // [3]
@@ -372,7 +479,7 @@ __global__ void __launch_bounds__(kHamThreads) hamming_topk_kernel(HammingArgs a
   for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
   // Resolve the kept pages once: logical id and physical page (-1 if invalid).
   for (int i = tid; i < m; i += kHamThreads) {
-    const int lp = a.kept[(size_t)row * a.m_max + i];
+    const int lp = kept_list[i];
     int phys = -1;
     if (lp >= 0 && lp < a.maxp) phys = a.page_table[(size_t)b * a.maxp + lp];
     if (phys < 0 || phys >= a.n_phys) {
@@ -505,6 +612,41 @@ inline size_t hamming_smem(int gs, int m_max, int P) {
   // Distances padded so the 16-byte group reads of the last thread stay inside.
   const size_t cand = ((size_t)m_max * P + 8 + 7) & ~(size_t)7;
   return ints * 4 + cand * 2 + 16;
+}
+
+// Top-m pages and the Hamming top-k fused in one CTA per (sequence, group): the kept page
+// list never leaves shared memory (a copy goes to `kept`/`kept_count` for inspection).
+// Shared memory: [kept list: m_max words][union of: top-m keys (maxp words) | Hamming
+// scratch (hamming_smem bytes)].
+struct TopmHammingArgs {
+  HammingArgs h;
+  const float* bounds;  // [B][G][maxp]
+  int m_pages, keep_div;
+};
+
+__global__ void __launch_bounds__(kHamThreads) topm_hamming_kernel(TopmHammingArgs a) {
+  __shared__ SelShared sh;
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ uint32_t fsm[];
+  const HammingArgs& h = a.h;
+  const int row = blockIdx.x, b = row / h.G;
+  int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
+  uint32_t* work = fsm + ((h.m_max + 3) & ~3);
+  const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
+  const int m = block_select_largest(a.bounds + (size_t)row * h.maxp, n, work, sh, true,
+                                     a.m_pages, a.keep_div, 0, kept_s, h.m_max, nullptr, 0);
+  __syncthreads();
+  int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
+  for (int i = threadIdx.x; i < m; i += kHamThreads) kept_g[i] = kept_s[i];
+  if (threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
+  hamming_topk_block(h, row, kept_s, m, work);
+}
+
+inline size_t topm_hamming_smem(int gs, int m_max, int P, int maxp) {
+  const size_t sel = (size_t)maxp * 4;
+  const size_t ham = hamming_smem(gs, m_max, P);
+  return (size_t)((m_max + 3) & ~3) * 4 + (sel > ham ? sel : ham);
 }
 
 // ---------------------------------------------------------------------------- HISA a1'

@@ -29,6 +29,7 @@ EXPORTED = [
     "hhr_encode_keys", "hhr_kept_max", "hhr_select_workspace_bytes", "hhr_select",
     "hhr_attn_workspace_bytes", "hhr_sparse_attn", "hhr_read_device_status",
     "hhr_status_string", "hhr_profile_next", "hhr_last_cuda_error", "hhr_sparse_attn_noalloc",
+    "hhr_decode_step_workspace_bytes", "hhr_decode_step",
 ]
 
 KERNELS = ["encode", "qprep", "bound", "topm", "hamming", "block", "token", "token_topk", "attn",
@@ -48,7 +49,7 @@ class HHRError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "head_dim", "page_size", "code_bits",
-        "max_pages_per_seq", "n_phys_pages")]
+        "max_pages_per_seq", "n_phys_pages", "summary_fp16")]
 
 
 class Trace(ctypes.Structure):
@@ -86,6 +87,11 @@ def lib():
         L.hhr_read_device_status.restype = i32
         L.hhr_profile_next.argtypes = [i32, vp, vp]
         L.hhr_profile_next.restype = i32
+        L.hhr_decode_step_workspace_bytes.argtypes = [pd, i32, i32, i32]
+        L.hhr_decode_step_workspace_bytes.restype = sz
+        L.hhr_decode_step.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
+                                      i32, ctypes.c_float, vp, vp, vp, vp, sz, vp]
+        L.hhr_decode_step.restype = i32
         L.hhr_sparse_attn_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, i32,
                                               ctypes.c_float, vp, vp]
         L.hhr_sparse_attn_noalloc.restype = i32
@@ -102,9 +108,9 @@ def status_string(status: int) -> str:
 
 
 def make_dims(batch, n_q_heads, n_kv_heads, page_size, max_pages_per_seq, n_phys_pages,
-              head_dim=128, code_bits=128) -> Dims:
+              head_dim=128, code_bits=128, summary_fp16=0) -> Dims:
     return Dims(batch, n_q_heads, n_kv_heads, head_dim, page_size, code_bits,
-                max_pages_per_seq, n_phys_pages)
+                max_pages_per_seq, n_phys_pages, int(summary_fp16))
 
 
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
@@ -140,6 +146,7 @@ def _check(fn, st):
 
 I32 = (torch.int32,)
 F32 = (torch.float32,)
+SUMMARY = (torch.float32, torch.float16)
 U32 = (torch.int32, torch.uint32) if hasattr(torch, "uint32") else (torch.int32,)
 
 
@@ -148,7 +155,7 @@ def hhr_encode_keys(d, k_cache, page_table, start, n_new, max_new, R, W, page_mi
     _check("hhr_encode_keys", lib().hhr_encode_keys(
         ctypes.byref(d), _p(k_cache, _BF16, "k_cache"), _p(page_table, I32, "page_table"),
         _p(start, I32, "start"), _p(n_new, I32, "n_new"), int(max_new), _p(R, F32, "R"),
-        _p(W, F32, "W"), _p(page_minmax, F32, "page_minmax"), _p(codes, U32, "codes"),
+        _p(W, F32, "W"), _p(page_minmax, SUMMARY, "page_minmax"), _p(codes, U32, "codes"),
         _p(block_mean, F32, "block_mean"), _s(stream)))
 
 
@@ -180,7 +187,7 @@ def hhr_select(d, mode, q, seq_len, q_pos, page_table, R, W, page_minmax, codes,
     _check("hhr_select", lib().hhr_select(
         ctypes.byref(d), int(mode), _p(q, _BF16, "q"), _p(seq_len, I32, "seq_len"),
         _p(q_pos, I32, "q_pos"), _p(page_table, I32, "page_table"), _p(R, F32, "R"),
-        _p(W, F32, "W"), _p(page_minmax, F32, "page_minmax"), _p(codes, U32, "codes"),
+        _p(W, F32, "W"), _p(page_minmax, SUMMARY, "page_minmax"), _p(codes, U32, "codes"),
         _p(block_mean, F32, "block_mean"), _p(k_cache, _BF16, "k_cache"), int(m_pages),
         int(keep_div), int(top_k), _p(out_idx, I32, "out_idx"), _p(out_count, I32, "out_count"),
         _p(workspace, (torch.uint8,), "workspace"), workspace.numel(), tr, _s(stream)))
@@ -221,3 +228,21 @@ def hhr_sparse_attn_noalloc(d, q, k_cache, v_cache, page_table, seq_len, idx, co
         _p(v_cache, _BF16, "v_cache"), _p(page_table, I32, "page_table"),
         _p(seq_len, I32, "seq_len"), _p(idx, I32, "idx"), _p(count, I32, "count"), int(top_k),
         float(scale), _p(out, F32, "out"), _s(stream)))
+
+
+def hhr_decode_step_workspace_bytes(d, m_pages, keep_div, top_k) -> int:
+    return int(lib().hhr_decode_step_workspace_bytes(ctypes.byref(d), int(m_pages),
+                                                     int(keep_div), int(top_k)))
+
+
+def hhr_decode_step(d, q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W,
+                    page_minmax, codes, m_pages, keep_div, top_k, scale, out_idx, out_count, out,
+                    workspace, stream=None):
+    _check("hhr_decode_step", lib().hhr_decode_step(
+        ctypes.byref(d), _p(q, _BF16, "q"), _p(k_new, _BF16, "k_new"), _p(v_new, _BF16, "v_new"),
+        _p(k_cache, _BF16, "k_cache"), _p(v_cache, _BF16, "v_cache"),
+        _p(page_table, I32, "page_table"), _p(seq_len, I32, "seq_len"), _p(R, F32, "R"),
+        _p(W, F32, "W"), _p(page_minmax, SUMMARY, "page_minmax"), _p(codes, U32, "codes"),
+        int(m_pages), int(keep_div), int(top_k), float(scale), _p(out_idx, I32, "out_idx"),
+        _p(out_count, I32, "out_count"), _p(out, F32, "out"),
+        _p(workspace, (torch.uint8,), "workspace"), workspace.numel(), _s(stream)))

@@ -20,11 +20,13 @@ class LayerCache:
 
     def __init__(self, d: hhr.Dims, device, hashing=True, block_means=False):
         n, G, P = d.n_phys_pages, d.n_kv_heads, d.page_size
-        self.page_minmax = (torch.empty(n, G, 2, d.head_dim, dtype=torch.float32, device=device)
+        # Zero-filled, so that slots past a sequence's end have deterministic contents.
+        sdt = torch.float16 if d.summary_fp16 else torch.float32
+        self.page_minmax = (torch.zeros(n, G, 2, d.head_dim, dtype=sdt, device=device)
                             if hashing else None)
-        self.codes = (torch.empty(n, G, P, d.code_bits // 32, dtype=torch.int32, device=device)
+        self.codes = (torch.zeros(n, G, P, d.code_bits // 32, dtype=torch.int32, device=device)
                       if hashing else None)
-        self.block_mean = (torch.empty(n, G, d.head_dim, dtype=torch.float32, device=device)
+        self.block_mean = (torch.zeros(n, G, d.head_dim, dtype=torch.float32, device=device)
                            if block_means else None)
 
 
@@ -43,6 +45,7 @@ class DecodeStep:
         self.count = torch.empty(d.batch, rows, dtype=torch.int32, device=device)
         self.m_max = hhr.hhr_kept_max(d, m_pages, keep_div)
         self.attention = attention and mode == hhr.HHR_MODE_HASH
+        self.fused_ws = None
         if self.attention:
             aws = hhr.hhr_attn_workspace_bytes(d, top_k)
             self.attn_ws = torch.empty(aws, dtype=torch.uint8, device=device)
@@ -65,6 +68,21 @@ class DecodeStep:
             scale = 1.0 / math.sqrt(self.d.head_dim)
         hhr.hhr_sparse_attn(self.d, q, k_cache, v_cache, page_table, seq_len, self.idx,
                             self.count, self.top_k, scale, self.out, self.attn_ws, stream)
+
+    def fused_step(self, q, k_cache, v_cache, page_table, seq_len, R, W, cache: LayerCache,
+                   k_new=None, v_new=None, scale=None, stream=None):
+        """One decode step through hhr_decode_step (the fused single-call path)."""
+        if self.fused_ws is None:
+            n = hhr.hhr_decode_step_workspace_bytes(self.d, self.m_pages, self.keep_div,
+                                                    self.top_k)
+            self.fused_ws = torch.empty(n, dtype=torch.uint8, device=self.idx.device)
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.d.head_dim)
+        hhr.hhr_decode_step(self.d, q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W,
+                            cache.page_minmax, cache.codes, self.m_pages, self.keep_div,
+                            self.top_k, scale, self.idx, self.count, self.out, self.fused_ws,
+                            stream)
+        return self.out
 
     def step(self, q, k_cache, v_cache, page_table, seq_len, R, W, cache: LayerCache,
              append_start, append_n, stream=None):

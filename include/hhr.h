@@ -33,8 +33,9 @@
  *   seq_len          : int32 [B], keys currently in each sequence (after appends)
  *   R                : f32 [G][d][d], orthogonal, applied as x' = R x
  *   W                : f32 [G][code_bits][d], applied to the rotated vector x'
- *   page_minmax      : f32 [n_phys_pages][G][2][d]; [..][0][:] = per-channel min
- *                      and [..][1][:] = per-channel max of the rotated valid keys
+ *   page_minmax      : f32 or f16 (dims.summary_fp16) [n_phys_pages][G][2][d];
+ *                      [..][0][:] = per-channel min and [..][1][:] = per-channel max
+ *                      of the rotated valid keys
  *   codes            : uint32 [n_phys_pages][G][P][W]; bit j of a code is
  *                      [(W R x)_j > 0], stored in word j/32 at bit j%32
  *   block_mean       : f32 [n_phys_pages][G][d], mean of the page's valid raw keys
@@ -76,6 +77,9 @@ typedef struct {
   int code_bits;          /* must be 128 */
   int max_pages_per_seq;  /* columns of page_table */
   int n_phys_pages;       /* pages in the pool */
+  int summary_fp16;       /* page_minmax element type: 0 = f32; 1 = f16 rounded outward
+                             (min toward -inf, max toward +inf), so the page bound stays an
+                             upper bound; values beyond the f16 range saturate to -inf/+inf */
 } hhr_dims;
 
 /* Optional copies of the intermediates of hhr_select, for inspection and layered
@@ -108,7 +112,7 @@ typedef struct {
  * small ones on the per-page encoder. Both produce the same layout. */
 int hhr_encode_keys(const hhr_dims* dims, const uint16_t* k_cache, const int32_t* page_table,
                     const int32_t* start, const int32_t* n_new, int max_new, const float* R,
-                    const float* W, float* page_minmax, uint32_t* codes, float* block_mean,
+                    const float* W, void* page_minmax, uint32_t* codes, float* block_mean,
                     void* stream);
 
 /* Kept pages (or blocks) per row for the given sizes: m_pages > 0 keeps
@@ -147,7 +151,7 @@ size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, i
  * trace: may be NULL. workspace: at least hhr_select_workspace_bytes(). */
 int hhr_select(const hhr_dims* dims, int mode, const uint16_t* q, const int32_t* seq_len,
                const int32_t* q_pos, const int32_t* page_table, const float* R, const float* W,
-               const float* page_minmax, const uint32_t* codes, const float* block_mean,
+               const void* page_minmax, const uint32_t* codes, const float* block_mean,
                const uint16_t* k_cache, int m_pages, int keep_div, int top_k, int32_t* out_idx,
                int32_t* out_count, void* workspace, size_t ws_bytes, hhr_trace* trace,
                void* stream);
@@ -169,6 +173,30 @@ int hhr_sparse_attn(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_c
                     const uint16_t* v_cache, const int32_t* page_table, const int32_t* seq_len,
                     const int32_t* idx, const int32_t* count, int top_k, float scale, float* out,
                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace needed by hhr_decode_step (bytes, 256-byte multiple); 0 on invalid input. */
+size_t hhr_decode_step_workspace_bytes(const hhr_dims* dims, int m_pages, int keep_div,
+                                       int top_k);
+
+/* One whole HHR decode step (steps a0-a5) in one call, for a decode loop that appends one
+ * key/value row per sequence and then attends: equal, bit for bit, to
+ *   hhr_encode_keys(start = seq_len - 1, n_new = 1) + hhr_select(HHR_MODE_HASH) +
+ *   hhr_sparse_attn,
+ * but with the append encoder and the query preparation fused into one kernel (one read
+ * of R and W), top-m fused with the Hamming top-k, and the kernels chained with
+ * programmatic dependent launch.
+ *   seq_len : lengths after the append; the newest row of sequence b is position
+ *             seq_len[b] - 1 (its page must be mapped in page_table).
+ *   k_new, v_new : bf16 [B][G][d] newest rows, written into k_cache/v_cache at that
+ *             position before encoding; both NULL when the caller already wrote them.
+ *   out_idx, out_count, out, scale : as in hhr_select / hhr_sparse_attn.
+ * workspace: at least hhr_decode_step_workspace_bytes(). Errors as in the separate calls. */
+int hhr_decode_step(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_new,
+                    const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
+                    const int32_t* page_table, const int32_t* seq_len, const float* R,
+                    const float* W, void* page_minmax, uint32_t* codes, int m_pages,
+                    int keep_div, int top_k, float scale, int32_t* out_idx, int32_t* out_count,
+                    float* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* hhr_sparse_attn without a workspace argument, for callers that cannot allocate
  * device memory themselves: runtimes without a device allocator, code running
@@ -199,11 +227,11 @@ int hhr_sparse_attn_noalloc(const hhr_dims* dims, const uint16_t* q, const uint1
 
 /* Kernels that hhr_profile_next can bracket with events. */
 typedef enum {
-  HHR_KERNEL_ENCODE = 0,     /* hhr_encode_keys */
+  HHR_KERNEL_ENCODE = 0,     /* hhr_encode_keys; hhr_decode_step's fused prologue */
   HHR_KERNEL_QPREP = 1,      /* hhr_select, hash mode, step a1 */
   HHR_KERNEL_BOUND = 2,      /* hhr_select, hash mode, step a2 bounds */
-  HHR_KERNEL_TOPM = 3,       /* hhr_select, top-m pages (or blocks) */
-  HHR_KERNEL_HAMMING = 4,    /* hhr_select, hash mode, steps a3-a4 */
+  HHR_KERNEL_TOPM = 3,       /* hhr_select, indexer mode, top-m blocks */
+  HHR_KERNEL_HAMMING = 4,    /* hhr_select, hash mode, top-m pages + steps a3-a4 (fused) */
   HHR_KERNEL_BLOCK = 5,      /* hhr_select, indexer mode, block scores */
   HHR_KERNEL_TOKEN = 6,      /* hhr_select, indexer mode, token scores */
   HHR_KERNEL_TOKEN_TOPK = 7, /* hhr_select, indexer mode, token top-k */
@@ -214,8 +242,9 @@ typedef enum {
 
 /* Measurement hook (no counterpart on the pages): the next launch of `kernel` by
  * the calling host thread is bracketed by cudaEventRecord(start_event) and
- * cudaEventRecord(stop_event) on that launch's stream. One-shot: the pair is
- * forgotten after use. Events are cudaEvent_t passed as void*; NULL, NULL clears
+ * cudaEventRecord(stop_event) on that launch's stream (recorded as external events,
+ * so inside a stream capture they become event-record nodes of the graph). One-shot:
+ * the pair is forgotten after use. Events are cudaEvent_t passed as void*; NULL, NULL clears
  * a pending pair. Returns HHR_ERR_INVALID_ARG for an unknown kernel id. */
 int hhr_profile_next(int kernel, void* start_event, void* stop_event);
 

@@ -32,16 +32,17 @@ BOUND_TOL = 1e-3
 FP32_TOL = 1e-5
 
 
-def dims_of(wl, inp):
+def dims_of(wl, inp, summary_fp16=0):
     return hhr.make_dims(wl.batch, wl.n_queries if wl.mode == "indexer" else wl.n_q_heads,
                          wl.n_kv_heads, wl.page_size, inp["max_pages"], inp["n_phys"],
-                         head_dim=wl.head_dim, code_bits=wl.code_bits)
+                         head_dim=wl.head_dim, code_bits=wl.code_bits,
+                         summary_fp16=summary_fp16)
 
 
-def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None):
+def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
     """Encode the whole cache, select and (hash mode) attend. Returns numpy results."""
     dev = inp["k_cache"].device
-    d = dims_of(wl, inp)
+    d = dims_of(wl, inp, summary_fp16)
     hashing = wl.mode == "hash"
     mode = hhr.HHR_MODE_HASH if hashing else hhr.HHR_MODE_INDEXER
     cache = LayerCache(d, dev, hashing=hashing, block_means=not hashing)
@@ -81,7 +82,8 @@ def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None):
     out = dict(idx=step.idx.cpu().numpy(), count=step.count.cpu().numpy(), m_max=step.m_max)
     if hashing:
         out["out"] = step.out.cpu().numpy()
-        out["page_minmax"] = cache.page_minmax.cpu().numpy()
+        out["page_minmax"] = cache.page_minmax.float().cpu().numpy()
+        out["summary_fp16"] = bool(summary_fp16)
         out["codes"] = cache.codes.cpu().numpy().view(np.uint32)
     else:
         out["block_mean"] = cache.block_mean.cpu().numpy()
@@ -124,10 +126,15 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
         sum(bin(int(x)).count("1") for x in diff.ravel()))
     phys = np.asarray(pt[:n_pages], dtype=np.int64)
     gmm = g_out["page_minmax"][phys, g].astype(np.float64)     # [n_pages][2][d]
-    for ref, got in ((enc["kmin"], gmm[:, 0]), (enc["kmax"], gmm[:, 1])):
-        err = np.abs(got - ref).max(axis=1)
-        lim = FP32_TOL * (1 + np.abs(ref).max(axis=1))
-        assert np.all(err <= lim), f"summary error {err.max()} (b={b}, g={g})"
+    for side, ref, got in ((0, enc["kmin"], gmm[:, 0]), (1, enc["kmax"], gmm[:, 1])):
+        lim = FP32_TOL * (1 + np.abs(ref).max(axis=1, keepdims=True))
+        if g_out.get("summary_fp16"):
+            # f16 storage rounded outward: within one f16 step, and on the outer side.
+            assert np.all(np.abs(got - ref) <= 2.0 ** -10 * np.abs(ref) + 6e-8 + lim)
+            outward = (got <= ref + lim) if side == 0 else (got >= ref - lim)
+            assert np.all(outward), f"f16 summary not rounded outward (b={b}, g={g})"
+        else:
+            assert np.all(np.abs(got - ref) <= lim), f"summary error (b={b}, g={g})"
 
     # a1: rotated queries and query codes.
     Qg = O.bf16_to_f64(inp_np["q"][b, g * gs:(g + 1) * gs])
@@ -148,6 +155,12 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
     beta_gpu = g_out["bounds"][b, g, :n_pages].astype(np.float64)
     scale = (np.abs(qr)[:, None, :] * np.maximum(np.abs(kmin_g), np.abs(kmax_g))[None]).sum(axis=(0, 2))
     assert np.all(np.abs(beta_gpu - beta_ref) <= BOUND_TOL * scale), "page bound out of tolerance"
+    # Invariant at any size: the GPU's bound dominates every true summed logit of its page.
+    Krot = O.rotate(R, O.logical_rows(inp_np["k_cache"], pt, g, n, P))
+    summed = (Krot @ Qrot.T).sum(axis=1)
+    page_max = np.full(n_pages, -np.inf)
+    np.maximum.at(page_max, np.arange(n) // P, summed)
+    assert np.all(beta_gpu >= page_max - 1e-5 * scale), "bound below a true logit"
     m = O.kept_count(n_pages, wl.m_pages, wl.keep_div)
     kc = int(g_out["kept_count"][b, g])
     assert kc == m

@@ -1,0 +1,104 @@
+"""hhr_decode_step (one fused call) against the separate calls it replaces: encode the newest
+key, select, attend. Same kernels' arithmetic, so every output must be bit-identical."""
+import numpy as np
+import pytest
+import torch
+
+import hhr_synth as S
+from hash_hierarchical_top_b200 import build, hhr
+from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+from parity_helpers import check_hash_group, dims_of
+
+pytestmark = pytest.mark.gpu
+
+
+def _prefill(wl, inp, d, upto):
+    """Encode positions [0, upto[b]) of every sequence; returns the cache."""
+    cache = LayerCache(d, "cuda")
+    step = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    z = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
+    step.encode(inp["k_cache"], inp["page_table"], z, upto, int(upto.max()), inp["R"], inp["W"],
+                cache)
+    return cache
+
+
+@pytest.mark.parametrize("f16", [0, 1])
+@pytest.mark.parametrize("with_new_rows", [False, True])
+def test_fused_step_equals_separate_calls(f16, with_new_rows):
+    build.build()
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=5, ragged=(33, 6000), top_k=300)
+    inp = S.make_inputs(wl, device="cuda")
+    d = dims_of(wl, inp, f16)
+    lens = inp["seq_len"]
+    G, P = wl.n_kv_heads, wl.page_size
+    # The newest row of each sequence: remember it, and (for the k_new path) wipe it from
+    # the caches so that only the fused call can put it back.
+    t = (lens - 1).long()
+    pt = inp["page_table"].long()
+    phys = pt[torch.arange(wl.batch, device="cuda"), t // P]
+    k_new = inp["k_cache"][phys, :, t % P].contiguous()
+    v_new = inp["v_cache"][phys, :, t % P].contiguous()
+
+    # Reference: separate calls.
+    ref_cache = _prefill(wl, inp, d, lens - 1)
+    ref = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    one = torch.ones(wl.batch, dtype=torch.int32, device="cuda")
+    ref.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], lens, inp["R"],
+             inp["W"], ref_cache, (lens - 1).to(torch.int32), one)
+
+    # Fused.
+    cache = _prefill(wl, inp, d, lens - 1)
+    kc, vc = inp["k_cache"].clone(), inp["v_cache"].clone()
+    if with_new_rows:
+        kc[phys, :, t % P] = 0
+        vc[phys, :, t % P] = 0
+    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    fs.fused_step(inp["q"], kc, vc, inp["page_table"], lens, inp["R"], inp["W"], cache,
+                  k_new=k_new if with_new_rows else None, v_new=v_new if with_new_rows else None)
+    torch.cuda.synchronize()
+    assert hhr.hhr_read_device_status() == (hhr.HHR_OK, 0)
+    assert torch.equal(kc, inp["k_cache"]) and torch.equal(vc, inp["v_cache"])
+    assert torch.equal(cache.codes, ref_cache.codes)
+    assert torch.equal(cache.page_minmax, ref_cache.page_minmax)
+    assert torch.equal(fs.count, ref.count)
+    assert torch.equal(fs.idx, ref.idx)
+    assert torch.equal(fs.out.view(torch.int32), ref.out.view(torch.int32))
+
+
+def test_fused_step_against_oracle():
+    """The fused call's outputs through the layered oracle checks (selection + attention)."""
+    build.build()
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(7777,), top_k=700)
+    inp = S.make_inputs(wl, device="cuda")
+    inp_np = S.to_numpy_inputs(inp)
+    d = dims_of(wl, inp, 1)
+    cache = _prefill(wl, inp, d, inp["seq_len"] - 1)
+    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    B, Hq = wl.batch, wl.n_q_heads
+    tr = dict(q_rot=torch.empty(B, Hq, 128, device="cuda"),
+              q_code=torch.empty(B, Hq, 4, dtype=torch.int32, device="cuda"))
+    fs.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
+                  inp["R"], inp["W"], cache)
+    torch.cuda.synchronize()
+    # Intermediates live in the fused workspace; recompute them with the select call to
+    # feed the layered checks (the fused selection must equal it).
+    sel = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    bounds = torch.empty(B, wl.n_kv_heads, d.max_pages_per_seq, device="cuda")
+    kept = torch.empty(B, wl.n_kv_heads, sel.m_max, dtype=torch.int32, device="cuda")
+    kc = torch.empty(B, wl.n_kv_heads, dtype=torch.int32, device="cuda")
+    trace = hhr.make_trace(q_rot=tr["q_rot"], q_code=tr["q_code"], bounds=bounds, kept=kept,
+                           kept_count=kc)
+    sel.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"], W=inp["W"],
+               trace=trace)
+    torch.cuda.synchronize()
+    assert torch.equal(sel.idx, fs.idx) and torch.equal(sel.count, fs.count)
+    g_out = dict(idx=fs.idx.cpu().numpy(), count=fs.count.cpu().numpy(),
+                 out=fs.out.cpu().numpy(), page_minmax=cache.page_minmax.float().cpu().numpy(),
+                 summary_fp16=True, codes=cache.codes.cpu().numpy().view(np.uint32),
+                 q_rot=tr["q_rot"].cpu().numpy(),
+                 q_code=tr["q_code"].cpu().numpy().view(np.uint32),
+                 bounds=bounds.cpu().numpy(), kept=kept.cpu().numpy(),
+                 kept_count=kc.cpu().numpy())
+    rep = {}
+    for g in range(wl.n_kv_heads):
+        check_hash_group(wl, inp_np, g_out, 0, g, rep)

@@ -30,51 +30,59 @@ def _built():
     build.build()
 
 
-def test_tiny_single_head():
+F16 = pytest.mark.parametrize("f16", [0, 1], ids=["f32sum", "f16sum"])
+
+
+@F16
+def test_tiny_single_head(f16):
     wl = S.WORKLOADS["tiny_1h_4k"]
     inp, inp_np = _inputs(wl)
-    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=f16))
     print(rep)
 
 
-def test_llama_32k_full():
+@F16
+def test_llama_32k_full(f16):
     wl = S.WORKLOADS["llama8b_32k"]
     inp, inp_np = _inputs(wl)
-    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    rep = _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=f16))
     print(rep)
 
 
-def test_llama_32k_appended_in_pieces():
+@F16
+def test_llama_32k_appended_in_pieces(f16):
     """The append path (pieces of 37 keys, pages filled across calls) equals a bulk encode."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(5000,), top_k=400)
     inp, inp_np = _inputs(wl)
-    a = run_gpu(wl, inp)
-    c = run_gpu(wl, inp, encode_chunks=37)
+    a = run_gpu(wl, inp, summary_fp16=f16)
+    c = run_gpu(wl, inp, encode_chunks=37, summary_fp16=f16)
     assert np.array_equal(a["codes"], c["codes"])
     assert np.array_equal(a["page_minmax"][:157], c["page_minmax"][:157])
     assert np.array_equal(a["idx"], c["idx"])
     _check_all_groups(wl, inp_np, c)
 
 
-def test_llama_128k_sampled_groups():
+@F16
+def test_llama_128k_sampled_groups(f16):
     """Full 128K context, batch 1: every group's selection and attention, oracle on 3 groups."""
     wl = S.WORKLOADS["llama8b_128k_b1"]
     inp, inp_np = _inputs(wl)
-    out = run_gpu(wl, inp)
+    out = run_gpu(wl, inp, summary_fp16=f16)
     assert np.all(out["count"] == wl.top_k)
     _check_all_groups(wl, inp_np, out, groups={(0, 0), (0, 3), (0, 7)})
 
 
-def test_ragged_small():
+@F16
+def test_ragged_small(f16):
     wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=6, ragged=(1, 5000))
     inp, inp_np = _inputs(wl)
-    _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=f16))
 
 
 def test_ragged_full_sampled():
     wl = S.WORKLOADS["ragged_b32"]
     inp, inp_np = _inputs(wl)
-    out = run_gpu(wl, inp)
+    out = run_gpu(wl, inp, summary_fp16=1)
     lens = inp_np["seq_len"]
     short = int(np.argmin(lens))
     longest = int(np.argmax(lens))
@@ -88,10 +96,11 @@ def test_ragged_full_sampled():
     dict(seq_lens=(3000,), page_size=256, m_pages=3, keep_div=0, top_k=700),  # P max, k_eff < k
     dict(seq_lens=(2048,), page_size=32, m_pages=0, keep_div=4, top_k=1),     # k = 1
 ])
-def test_edge_cases(case):
+@F16
+def test_edge_cases(case, f16):
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], **case)
     inp, inp_np = _inputs(wl)
-    _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=f16))
 
 
 @pytest.mark.parametrize("heads", [(8, 1), (8, 8), (6, 2)])
