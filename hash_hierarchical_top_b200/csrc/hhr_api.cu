@@ -11,6 +11,7 @@
 #include "attn.cuh"
 #include "common.cuh"
 #include "encode.cuh"
+#include "encode_tc.cuh"
 #include "select.cuh"
 #include "step.cuh"
 
@@ -21,6 +22,8 @@ namespace {
 constexpr int kMaxPagesPerSeq = 32768;  // top-m keys staged in 128 KB of shared memory
 constexpr int kMaxTokCand = 32768;      // indexer token candidates per query
 constexpr int kMaxDevices = 64;
+constexpr int kTcMinBulk = 4096;  // appends at least this long use the tensor-core encoder
+constexpr int kTcSlots = 148;     // persistent encoder CTAs (one per SM of a B200)
 constexpr size_t kMaxKernelSmem = 200 * 1024;  // below the 227 KB opt-in of sm_100
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -68,7 +71,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   return e;
 }
 
-bool g_smem_step[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
+bool g_smem_tc[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
     g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices];
 
 struct SelectLayout {
@@ -225,6 +228,20 @@ int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* p
   const long long pages = (long long)(max_new + d->page_size - 1) / d->page_size + 1;
   if (pages > 0x7fffffffLL) return HHR_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
+  if (hashing && block_mean == nullptr && d->page_size == kTcPage && max_new >= kTcMinBulk) {
+    // Bulk append (e.g. a prefill): the tensor-core encoder.
+    if (allow_smem(encode_tc_kernel, kTcSmem, g_smem_tc) != cudaSuccess) return HHR_ERR_CUDA;
+    const int G = d->n_kv_heads;
+    int cpg = kTcSlots / G;
+    if (cpg < 1) cpg = 1;
+    EncodeTcArgs ta{k_cache, page_table, start, n_new, R, W, page_minmax, codes, d->batch, G,
+                    d->max_pages_per_seq, d->n_phys_pages, max_new, d->summary_fp16, cpg,
+                    (d->max_pages_per_seq * kTcPage + kTcTile - 1) / kTcTile};
+    prof_begin(HHR_KERNEL_ENCODE, s);
+    encode_tc_kernel<<<dim3(cpg, G), kTcThreads, kTcSmem, s>>>(ta);
+    prof_end(HHR_KERNEL_ENCODE, s);
+    return launch_status();
+  }
   EncodeArgs a{k_cache, page_table, start, n_new, hashing ? R : nullptr, hashing ? W : nullptr,
                page_minmax, codes, block_mean, d->n_kv_heads, d->page_size,
                d->max_pages_per_seq, d->n_phys_pages, max_new, d->summary_fp16};

@@ -108,8 +108,10 @@ typedef struct {
  *   max_new      : host int, an upper bound on every n_new[b] (sizes the launch;
  *                  a larger n_new[b] is clipped to it and flagged in the device
  *                  status word)
- * Large appends (whole pages, e.g. a prefill) run on the tensor-core encoder;
- * small ones on the per-page encoder. Both produce the same layout. */
+ * Appends of at least 4096 keys (max_new) with page_size 32 and no block means run
+ * on the tensor-core encoder (tcgen05: one GEMM per 128-key tile against [R; W R],
+ * fp32 operands split into three bf16 terms); others on the per-page encoder. Both
+ * produce the same layout; their results agree within the code and bound tolerances. */
 int hhr_encode_keys(const hhr_dims* dims, const uint16_t* k_cache, const int32_t* page_table,
                     const int32_t* start, const int32_t* n_new, int max_new, const float* R,
                     const float* W, void* page_minmax, uint32_t* codes, float* block_mean,
@@ -251,7 +253,8 @@ int hhr_profile_next(int kernel, void* start_event, void* stop_event);
 /* Synchronises `stream`, then returns HHR_OK if no device-side check fired since
  * the last call, else HHR_ERR_DEVICE_STATUS; clears the status word. If `bits` is
  * not NULL (host), receives the raw status bits (1 = bad page id, 2 = bad token
- * index, 4 = n_new clipped to max_new). */
+ * index, 4 = n_new clipped to max_new, 8 = a bounded wait in the tensor-core encoder
+ * gave up). */
 int hhr_read_device_status(void* stream, int* bits);
 
 /* The text of the last CUDA error any hhr_* call met on the calling host thread

@@ -51,15 +51,19 @@ def test_llama_32k_full(f16):
 
 @F16
 def test_llama_32k_appended_in_pieces(f16):
-    """The append path (pieces of 37 keys, pages filled across calls) equals a bulk encode."""
+    """Bulk encoding (tensor cores) and appends in pieces of 37 keys (pages filled across
+    calls, per-page encoder) both match the oracle and each other."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(5000,), top_k=400)
     inp, inp_np = _inputs(wl)
-    a = run_gpu(wl, inp, summary_fp16=f16)
-    c = run_gpu(wl, inp, encode_chunks=37, summary_fp16=f16)
-    assert np.array_equal(a["codes"], c["codes"])
-    assert np.array_equal(a["page_minmax"][:157], c["page_minmax"][:157])
-    assert np.array_equal(a["idx"], c["idx"])
+    a = run_gpu(wl, inp, summary_fp16=f16)          # bulk: the tensor-core encoder
+    c = run_gpu(wl, inp, encode_chunks=37, summary_fp16=f16)  # appends: per-page encoder
+    # Both paths against the oracle (codes exact outside fragile bits, summaries within
+    # tolerance, selection and attention layered checks).
+    _check_all_groups(wl, inp_np, a)
     _check_all_groups(wl, inp_np, c)
+    # And against each other: codes differ in at most a handful of (fragile) bits.
+    diff = np.bitwise_count(a["codes"][:157] ^ c["codes"][:157]).sum()
+    assert diff <= 16, diff
 
 
 @F16
@@ -110,6 +114,14 @@ def test_group_shapes(heads):
                   batch=2, top_k=300)
     inp, inp_np = _inputs(wl)
     _check_all_groups(wl, inp_np, run_gpu(wl, inp))
+
+
+def test_bulk_encoder_partial_start():
+    """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp, encode_chunks=6007, summary_fp16=1)
+    _check_all_groups(wl, inp_np, out)
 
 
 def test_deterministic():
