@@ -19,6 +19,7 @@
 //      sum, output) per head, or the final output when the group is not split; a
 //      combine kernel merges the splits (standard split softmax rescaling).
 #pragma once
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -109,6 +110,10 @@ __device__ __forceinline__ int swz(int r, int chunk) { return r * kD + ((chunk ^
 // (g = lane/4, t = lane%4) holds S[head g][keys 2t, 2t+1], which is exactly the B
 // fragment of O^T = V^T P^T on mma.m16n8k8 (channels on M, heads on N). P is split into
 // bf16 hi + lo parts (two MMAs) so its rounding stays near 2^-16 relative.
+// kCluster: the splits of a group form one thread-block cluster; after each CTA has
+// merged its warps, the cluster's rank 0 merges the splits through distributed shared
+// memory and writes the output (no partials in global memory, no combine kernel).
+template <bool kCluster>
 __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a) {
   extern __shared__ float4 at_smem[];
   pdl_wait();
@@ -123,8 +128,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   const int row = b * a.G + g;
   const int cnt = min(a.count[row], a.top_k);
   const int base = split * a.split_rows;
-  if (base >= cnt) return;
-  const int nrows = min(a.split_rows, cnt - base);
+  // A split past the selection does no work (in a cluster it still joins the merge).
+  const int nrows = max(0, min(a.split_rows, cnt - base));
+  if (!kCluster && nrows == 0) return;
   const int ntiles = (nrows + kTile - 1) / kTile;
   const int n = a.seq_len[b];
 
@@ -291,7 +297,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
         O = fmaf(sc, mo[((size_t)w * kMaxGroup + h) * kD + c], O);
       }
     }
-    if (a.n_splits == 1) {
+    if constexpr (kCluster) {
+      // This CTA's merged state, in the (now free) offset table: [gs][d] outputs, [gs][2].
+      float* res = reinterpret_cast<float*>(offs);
+      res[h * kD + c] = O;
+      if (c == 0) {
+        res[kMaxGroup * kD + 2 * h] = M;
+        res[kMaxGroup * kD + 2 * h + 1] = L;
+      }
+    } else if (a.n_splits == 1) {
       a.out[((size_t)b * a.Hq + g * gs + h) * kD + c] = (L > 0.f) ? O / L : 0.f;
     } else {
       const size_t p = ((size_t)row * a.n_splits + split) * gs + h;
@@ -302,6 +316,33 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
       }
     }
   }
+  if constexpr (kCluster) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();  // every split's state is in its shared memory
+    if (cl.block_rank() == 0) {
+      const int ns = (int)cl.num_blocks();
+      float* res_local = reinterpret_cast<float*>(offs);
+      for (int i = tid; i < gs * kD; i += kAttnThreads) {
+        const int h = i / kD, c = i % kD;
+        float M = -INFINITY;
+        for (int r = 0; r < ns; ++r)
+          M = fmaxf(M, cl.map_shared_rank(res_local, r)[kMaxGroup * kD + 2 * h]);
+        float L = 0.f, O = 0.f;
+        if (M > -INFINITY) {
+          for (int r = 0; r < ns; ++r) {
+            const float* rr = cl.map_shared_rank(res_local, r);
+            const float mr = rr[kMaxGroup * kD + 2 * h];
+            const float sc = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
+            L = fmaf(sc, rr[kMaxGroup * kD + 2 * h + 1], L);
+            O = fmaf(sc, rr[h * kD + c], O);
+          }
+        }
+        a.out[((size_t)b * a.Hq + g * gs + h) * kD + c] = (L > 0.f) ? O / L : 0.f;
+      }
+    }
+    cl.sync();  // keep every CTA's shared memory alive until rank 0 has read it
+  }
 }
 
 // Split plan: about two resident CTAs per SM over the whole batch, at most
@@ -309,11 +350,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
 struct AttnPlan {
   int n_splits, split_rows;
 };
-inline AttnPlan attn_plan(int B, int G, int top_k) {
+// Cluster variant (fused decode step): at most kMaxClusterSplits splits per group.
+constexpr int kMaxClusterSplits = 8;
+inline AttnPlan attn_plan(int B, int G, int top_k, int max_splits = 1 << 30) {
   const long long rows = (long long)B * G;
   int s = (int)(kTargetCtas / (rows > 0 ? rows : 1));
   if (s < 1) s = 1;
-  const int max_s = (top_k + kTile - 1) / kTile;
+  int max_s = (top_k + kTile - 1) / kTile;
+  if (max_s > max_splits) max_s = max_splits;
   if (s > max_s) s = max_s;
   const int min_s = (top_k + kMaxSplitRows - 1) / kMaxSplitRows;
   if (s < min_s) s = min_s;

@@ -72,7 +72,8 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
 }
 
 bool g_smem_tc[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
-    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices];
+    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
+    g_smem_attn_cl[kMaxDevices];
 
 struct SelectLayout {
   size_t qpn, q_rot, q_code, bounds, kept, kept_count, tok, total;
@@ -134,15 +135,22 @@ struct ProfPair {
 };
 thread_local ProfPair g_prof[HHR_KERNEL_COUNT];
 
-// External records, so that inside a stream capture they become event-record nodes of
-// the graph (timestamps taken at every replay) rather than internal dependencies.
+// Inside a stream capture the records are external, so that they become event-record
+// nodes of the graph (timestamps taken at every replay) rather than internal
+// dependencies; outside a capture they are plain records.
+void prof_record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) cs = cudaStreamCaptureStatusNone;
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
 void prof_begin(int k, cudaStream_t s) {
-  if (g_prof[k].start != nullptr)
-    cudaEventRecordWithFlags(g_prof[k].start, s, cudaEventRecordExternal);
+  if (g_prof[k].start != nullptr) prof_record(g_prof[k].start, s);
 }
 void prof_end(int k, cudaStream_t s) {
-  if (g_prof[k].stop != nullptr)
-    cudaEventRecordWithFlags(g_prof[k].stop, s, cudaEventRecordExternal);
+  if (g_prof[k].stop != nullptr) prof_record(g_prof[k].stop, s);
   g_prof[k].start = nullptr;
   g_prof[k].stop = nullptr;
 }
@@ -310,7 +318,8 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     {
       const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                          d->n_phys_pages};
-      const dim3 grid = bound_grid(G, (maxp + kPagesPerCtaB - 1) / kPagesPerCtaB, B);
+      const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
+      const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
       if (d->summary_fp16)
         page_bound_kernel<true><<<grid, kBoundWarps * 32, 0, s>>>(ba);
       else
@@ -421,9 +430,9 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
              scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
              d->n_phys_pages, top_k, ns, plan.split_rows};
   prof_begin(HHR_KERNEL_ATTN, s);
-  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess)
+  if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
-  sparse_attn_kernel<<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  sparse_attn_kernel<false><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
   prof_end(HHR_KERNEL_ATTN, s);
   if ((st = launch_status()) != HHR_OK) return st;
   if (ns > 1) {
@@ -483,7 +492,9 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
   const size_t fsm = topm_hamming_smem(gs, m_max, P, maxp);
   if (allow_smem(topm_hamming_kernel, fsm, g_smem_ham) != cudaSuccess) return HHR_ERR_CUDA;
-  if (allow_smem(sparse_attn_kernel, attn_smem(), g_smem_attn) != cudaSuccess)
+  if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
+    return HHR_ERR_CUDA;
+  if (allow_smem(sparse_attn_kernel<true>, attn_smem(), g_smem_attn_cl) != cudaSuccess)
     return HHR_ERR_CUDA;
   cudaError_t e;
 
@@ -499,7 +510,8 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   {
     const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                        d->n_phys_pages};
-    const dim3 grid = bound_grid(G, (maxp + kPagesPerCtaB - 1) / kPagesPerCtaB, B);
+    const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
+    const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
     prof_begin(HHR_KERNEL_BOUND, s);
     e = d->summary_fp16 ? launch_pdl(page_bound_kernel<true>, grid, dim3(kBoundWarps * 32), 0, s, ba)
                         : launch_pdl(page_bound_kernel<false>, grid, dim3(kBoundWarps * 32), 0, s, ba);
@@ -516,22 +528,49 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   }
-  // a5: sparse attention over the selected rows.
+  // a5: sparse attention over the selected rows. The splits of a group form a cluster
+  // merged through distributed shared memory when they fit one (at most 8 splits).
   {
-    AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, part_o, part_ml,
-                out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k, ns,
-                plan.split_rows};
-    prof_begin(HHR_KERNEL_ATTN, s);
-    e = launch_pdl(sparse_attn_kernel, dim3(ns, G, B), dim3(kAttnThreads), attn_smem(), s, aa);
-    prof_end(HHR_KERNEL_ATTN, s);
-    if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
-    if (ns > 1) {
-      prof_begin(HHR_KERNEL_COMBINE, s);
-      e = launch_pdl(attn_combine_kernel, dim3(Hq, B), dim3(kD), 0, s,
-                     CombineArgs{part_o, part_ml, out_count, out, Hq, G, top_k, ns,
-                                 plan.split_rows});
-      prof_end(HHR_KERNEL_COMBINE, s);
+    const AttnPlan cp = attn_plan(B, G, top_k, kMaxClusterSplits);
+    if (cp.n_splits <= kMaxClusterSplits) {
+      AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, nullptr, nullptr,
+                  out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k,
+                  cp.n_splits, cp.split_rows};
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cp.n_splits, G, B);
+      cfg.blockDim = dim3(kAttnThreads);
+      cfg.dynamicSmemBytes = attn_smem();
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cp.n_splits;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      prof_begin(HHR_KERNEL_ATTN, s);
+      e = cudaLaunchKernelEx(&cfg, sparse_attn_kernel<true>, aa);
+      prof_end(HHR_KERNEL_ATTN, s);
       if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+    } else {
+      AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, part_o, part_ml,
+                  out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k, ns,
+                  plan.split_rows};
+      prof_begin(HHR_KERNEL_ATTN, s);
+      e = launch_pdl(sparse_attn_kernel<false>, dim3(ns, G, B), dim3(kAttnThreads), attn_smem(),
+                     s, aa);
+      prof_end(HHR_KERNEL_ATTN, s);
+      if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+      if (ns > 1) {
+        prof_begin(HHR_KERNEL_COMBINE, s);
+        e = launch_pdl(attn_combine_kernel, dim3(Hq, B), dim3(kD), 0, s,
+                       CombineArgs{part_o, part_ml, out_count, out, Hq, G, top_k, ns,
+                                   plan.split_rows});
+        prof_end(HHR_KERNEL_COMBINE, s);
+        if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+      }
     }
   }
   return HHR_OK;

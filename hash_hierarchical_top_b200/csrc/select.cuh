@@ -90,12 +90,16 @@ inline size_t qprep_smem() { return 0; }
 // bound_p = qneg . kmin_p + qpos . kmax_p over the page summary (1 KB per page and
 // group in f32, 512 B in f16). The summaries are the dominant HBM stream of the whole
 // path, so this kernel is a pure streaming GEMV.
-// Tuned on B200 at 128K context, batch 8 (4096 pages x 8 groups x 8 sequences).
+// Tuned on B200 at 128K context, batch 8 (4096 pages x 8 groups x 8 sequences); the
+// macros below exist for such sweeps.
 #ifndef HHR_BOUND_WARPS
 #define HHR_BOUND_WARPS 4
 #endif
-#ifndef HHR_BOUND_ROUNDS
-#define HHR_BOUND_ROUNDS 1
+#ifndef HHR_BOUND_SETS_F16
+#define HHR_BOUND_SETS_F16 2
+#endif
+#ifndef HHR_BOUND_SETS_F32
+#define HHR_BOUND_SETS_F32 2
 #endif
 constexpr int kBoundWarps = HHR_BOUND_WARPS;
 
@@ -142,14 +146,13 @@ __device__ __forceinline__ float warp_sum8_transposed(float (&v)[8], int lane) {
 }
 
 // One warp per page and load instruction (coalesced: lane l reads 16-byte piece l of the
-// page's summary), 8 pages per round, kBoundRounds rounds per warp; the 8 page sums of a
-// round are folded by one transposed reduction. f32 pages are 1 KB (two pieces per lane:
-// channels 4l..4l+3 of the min and of the max row); f16 pages are 512 B (one piece: lanes
-// 0-15 hold 8 channels of the min row, lanes 16-31 of the max row). Each piece is paired
-// with the matching channels of the folded query (qneg with min, qpos with max).
-constexpr int kBoundRounds = HHR_BOUND_ROUNDS;
-constexpr int kPagesPerCtaB = kBoundWarps * 8 * kBoundRounds;
-
+// page's summary); each warp loads 16 pages (two sets of 8) before any arithmetic and
+// folds each set of 8 page sums with one transposed reduction. f32 pages are 1 KB (two
+// pieces per lane: channels 4l..4l+3 of the min and of the max row); f16 pages are 512 B
+// (one piece: lanes 0-15 hold 8 channels of the min row, lanes 16-31 of the max row).
+// Each piece is paired with the matching channels of the folded query (qneg with min,
+// qpos with max). Measured on B200 (128K context, batch 8): 16 pages per warp and 4 warps
+// per CTA stream fastest (f32 6.25 TB/s, f16 5.07 TB/s); 8 or 24+ pages per warp are slower.
 __device__ __forceinline__ float dot8_h(const uint4 h, const float4 q0, const float4 q1) {
   const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
   const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
@@ -159,15 +162,39 @@ __device__ __forceinline__ float dot8_h(const uint4 h, const float4 q0, const fl
          q1.z * d.x + q1.w * d.y;
 }
 
+// 16-byte summary load; the variant is a build-time choice (streaming by default).
+#ifndef HHR_BOUND_LOAD
+#define HHR_BOUND_LOAD 0
+#endif
+__device__ __forceinline__ uint4 load_summary16(const uint4* p) {
+#if HHR_BOUND_LOAD == 0
+  return __ldcs(p);
+#elif HHR_BOUND_LOAD == 1
+  return __ldg(p);
+#elif HHR_BOUND_LOAD == 2
+  return *p;
+#else
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+#endif
+}
+
 template <bool F16>
 __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
+  // kSets groups of 8 pages per warp are loaded together (all page ids first, then all
+  // summary pieces), so that each warp keeps kSets * 8 page summaries in flight.
+  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
+  constexpr int kPagesPerWarp = 8 * kSets;
   pdl_wait();
   pdl_trigger();
   const int g = bound_group(), b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
-  const int cta_base = bound_chunk() * kPagesPerCtaB;
-  if (cta_base >= npg) return;
+  const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
+  if (p0 >= npg) return;
   const float* qb = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
   float4 q0, q1;
   if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
@@ -181,46 +208,51 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
   // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
   constexpr int kPieces = F16 ? 32 : 64;
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
+  int my_phys = -1;  // lane i < kPagesPerWarp resolves page p0 + i
+  if (lane < kPagesPerWarp && p0 + lane < npg)
+    my_phys = a.page_table[(size_t)b * a.maxp + p0 + lane];
+  uint4 x[kPagesPerWarp], y[F16 ? 1 : kPagesPerWarp];
+#pragma unroll
+  for (int i = 0; i < kPagesPerWarp; ++i) {
+    const int phys = __shfl_sync(kFull, my_phys, i);
+    x[i] = make_uint4(0, 0, 0, 0);
+    if constexpr (!F16) y[i] = x[i];
+    if (phys >= 0 && phys < a.n_phys) {
+      const uint4* src = base4 + ((size_t)phys * a.G + g) * kPieces + lane;
+      x[i] = load_summary16(src);
+      if constexpr (!F16) y[i] = load_summary16(src + 32);
+    }
+  }
   float* out = a.bounds + ((size_t)b * a.G + g) * a.maxp;
 #pragma unroll
-  for (int r = 0; r < kBoundRounds; ++r) {
-    const int p0 = cta_base + (r * kBoundWarps + warp) * 8;
-    if (p0 >= npg) break;
-    int my_phys = -1;  // lane i < 8 resolves page p0 + i
-    if (lane < 8 && p0 + lane < npg) my_phys = a.page_table[(size_t)b * a.maxp + p0 + lane];
-    uint4 x[8], y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int phys = __shfl_sync(kFull, my_phys, i);
-      x[i] = make_uint4(0, 0, 0, 0);
-      y[i] = x[i];
-      if (phys >= 0 && phys < a.n_phys) {
-        const uint4* src = base4 + ((size_t)phys * a.G + g) * kPieces + lane;
-        x[i] = __ldcs(src);
-        if constexpr (!F16) y[i] = __ldcs(src + 32);
-      }
-    }
+  for (int st = 0; st < kSets; ++st) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if constexpr (F16) {
-        v[i] = dot8_h(x[i], q0, q1);
+        v[i] = dot8_h(x[st * 8 + i], q0, q1);
       } else {
-        const float4 mn = *reinterpret_cast<const float4*>(&x[i]);
-        const float4 mx = *reinterpret_cast<const float4*>(&y[i]);
+        const float4 mn = *reinterpret_cast<const float4*>(&x[st * 8 + i]);
+        const float4 mx = *reinterpret_cast<const float4*>(&y[st * 8 + i]);
         v[i] = q0.x * mn.x + q0.y * mn.y + q0.z * mn.z + q0.w * mn.w + q1.x * mx.x +
                q1.y * mx.y + q1.z * mx.z + q1.w * mx.w;
       }
     }
     const float tot = warp_sum8_transposed(v, lane);
-    // Lane l (< 8) now holds the bound of page p0 + l.
-    const int lp = p0 + lane;
+    // Lane l (< 8) holds the bound of page p0 + st*8 + l; its page id is on lane st*8 + l.
+    const int phys_l = __shfl_sync(kFull, my_phys, (st * 8 + lane) & 31);
+    const int lp = p0 + st * 8 + lane;
     if (lane < 8 && lp < npg) {
-      const bool ok = my_phys >= 0 && my_phys < a.n_phys;
+      const bool ok = phys_l >= 0 && phys_l < a.n_phys;
       if (!ok) flag_status(kStatusBadPage);
       out[lp] = ok ? tot : -INFINITY;
     }
   }
+}
+
+// Pages covered by one CTA of page_bound_kernel.
+inline int bound_pages_per_cta(bool f16) {
+  return kBoundWarps * 8 * (f16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32);
 }
 
 // ---------------------------------------------------------------------------- top-k
