@@ -19,52 +19,43 @@ namespace hhr {
 // for both the transposing stores and the column reads). Used by the bulk SIMT path.
 constexpr int kTS = kD + 1;
 
-// y_v = M x_v for up to kVecChunk vectors at once, M a 128x128 row-major fp32 matrix,
-// with kMvThreads = 512 threads: 4 threads per row. Thread (row r = 8*warp + lane/4,
-// quarter q = lane%4) holds float4s q, q+4, ..., q+28 of row r in registers (the four
-// threads of a row read 64 contiguous bytes per load), dots them with the same float4s
-// of each vector (shared-memory broadcasts), and two shuffles sum the four quarters.
-// Every thread of a row ends up with y_v[r].
+// Mat-vecs with 128x128 row-major fp32 matrices (R_g, W_g) use one canonical row dot
+// product everywhere (append encoder, query prep, fused prologues), so that their results
+// are bit-identical: the 16 threads of a row (consecutive lanes) each hold float4s part and
+// part+16 of the row, multiply them with the same channels of the vector in a fixed fmaf
+// order, and sum over the 16 threads with a 4-step butterfly. With kMvThreads = 512, a
+// CTA covers 32 rows at a time: thread t owns rows 32*rb + t/16 for row blocks rb = 0..3.
 constexpr int kVecChunk = 4;
 constexpr int kMvThreads = 512;
+constexpr int kRowBlocks = kD / 32;
 
-__device__ __forceinline__ int mv_row() { return (threadIdx.x >> 5) * 8 + ((threadIdx.x & 31) >> 2); }
+__device__ __forceinline__ int mv_lrow() { return (int)threadIdx.x >> 4; }  // 0..31
 
-// This thread's quarter of its row of M (8 float4).
-__device__ __forceinline__ void load_rows8(const float* __restrict__ M, float4 (&m)[8]) {
-  const int q = threadIdx.x & 3;
-  const float4* Mr = reinterpret_cast<const float4*>(M + (size_t)mv_row() * kD);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) m[j] = __ldg(Mr + 4 * j + q);
+// Row `row` of M, this thread's part (float4s part and part + 16).
+__device__ __forceinline__ void load_row16(const float* __restrict__ M, int row, float4 (&m)[2]) {
+  const int part = threadIdx.x & 15;
+  const float4* r4 = reinterpret_cast<const float4*>(M + (size_t)row * kD);
+  m[0] = __ldg(r4 + part);
+  m[1] = __ldg(r4 + part + 16);
 }
 
-template <int NV>
-__device__ __forceinline__ void matvec8(const float4 (&m)[8], const float* xs, int xs_stride,
-                                        float (&y)[NV]) {
-  const int q = threadIdx.x & 3;
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const float4* xv = reinterpret_cast<const float4*>(xs + v * xs_stride);
-    float acc = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 x = xv[4 * j + q];
-      acc = fmaf(m[j].x, x.x, fmaf(m[j].y, x.y, fmaf(m[j].z, x.z, fmaf(m[j].w, x.w, acc))));
-    }
-    acc += __shfl_xor_sync(kFull, acc, 1);
-    acc += __shfl_xor_sync(kFull, acc, 2);
-    y[v] = acc;
-  }
-}
-
-// The 8 sign bits of this warp's rows (8*warp .. 8*warp+7) from a ballot in which the
-// lanes 4i carry row 8*warp + i.
-__device__ __forceinline__ uint32_t row_bits8(bool positive) {
-  const unsigned b = __ballot_sync(kFull, positive);
-  uint32_t byte = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) byte |= ((b >> (4 * i)) & 1u) << i;
-  return byte;
+__device__ __forceinline__ float row_dot16(const float4 (&m)[2], const float* x) {
+  const int part = threadIdx.x & 15;
+  const float4 x0 = reinterpret_cast<const float4*>(x)[part];
+  const float4 x1 = reinterpret_cast<const float4*>(x)[part + 16];
+  float acc = m[0].x * x0.x;
+  acc = fmaf(m[0].y, x0.y, acc);
+  acc = fmaf(m[0].z, x0.z, acc);
+  acc = fmaf(m[0].w, x0.w, acc);
+  acc = fmaf(m[1].x, x1.x, acc);
+  acc = fmaf(m[1].y, x1.y, acc);
+  acc = fmaf(m[1].z, x1.z, acc);
+  acc = fmaf(m[1].w, x1.w, acc);
+  acc += __shfl_xor_sync(kFull, acc, 1);
+  acc += __shfl_xor_sync(kFull, acc, 2);
+  acc += __shfl_xor_sync(kFull, acc, 4);
+  acc += __shfl_xor_sync(kFull, acc, 8);
+  return acc;
 }
 
 struct EncodeArgs {
@@ -82,16 +73,16 @@ struct EncodeArgs {
 };
 
 // One CTA of kMvThreads threads per (touched page, KV group, sequence). The new keys of
-// the page are processed kVecChunk at a time: k' = R_g k (the 4 threads of row r own
-// channel r), min/max folded per channel, then p = W_g k'; each warp contributes the 8
-// sign bits of its rows as one byte of the code.
+// the page are processed kVecChunk at a time: k' = R_g k (row_dot16; the 16 threads of
+// row r own channel r), min/max folded per channel, then p = W_g k' and the sign bit of
+// row r is OR-ed into the key's code word r / 32.
 __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   __shared__ __align__(16) float kx[kVecChunk][kD];  // raw keys (fp32)
   __shared__ __align__(16) float kr[kVecChunk][kD];  // rotated keys
-  __shared__ __align__(16) uint8_t cbytes[kVecChunk][16];
+  __shared__ uint32_t cword[kVecChunk][kWords];
 
   const int b = blockIdx.z, g = blockIdx.y, j = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int P = a.P, G = a.G;
 
   int nn = a.n_new[b];
@@ -116,26 +107,35 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   const int pstart = lp * P;
   const int t0 = max(s, pstart), t1 = min(e, pstart + P);
   const uint16_t* kpage = a.k_cache + ((size_t)phys * G + g) * P * kD;
-  const int row = mv_row();  // channel / code bit owned after a matvec
-  const bool row_lead = (lane & 3) == 0;
+  const int lrow = mv_lrow();
+  const bool row_lead = (tid & 15) == 0;
 
   if (a.R != nullptr) {
     // R_g and W_g rows of this thread, and the page's stored summary when the page already
     // held keys, are fetched up front (one memory latency for all of them).
-    float4 rrow[8], wrow[8];
-    load_rows8(a.R + (size_t)g * kD * kD, rrow);
-    load_rows8(a.W + (size_t)g * kD * kD, wrow);
+    float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];
+#pragma unroll
+    for (int rb = 0; rb < kRowBlocks; ++rb) {
+      load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
+      load_row16(a.W + (size_t)g * kD * kD, rb * 32 + lrow, wrow[rb]);
+    }
     const size_t sbase = ((size_t)phys * G + g) * 2 * kD;
-    float mn = INFINITY, mx = -INFINITY;
-    if (t0 > pstart && row_lead) {
-      if (a.summary_fp16) {
-        const __half* mm = reinterpret_cast<const __half*>(a.page_minmax) + sbase;
-        mn = __half2float(mm[row]);
-        mx = __half2float(mm[kD + row]);
-      } else {
-        const float* mm = reinterpret_cast<const float*>(a.page_minmax) + sbase;
-        mn = mm[row];
-        mx = mm[kD + row];
+    float mn[kRowBlocks], mx[kRowBlocks];
+#pragma unroll
+    for (int rb = 0; rb < kRowBlocks; ++rb) {
+      mn[rb] = INFINITY;
+      mx[rb] = -INFINITY;
+      if (t0 > pstart && row_lead) {
+        const int row = rb * 32 + lrow;
+        if (a.summary_fp16) {
+          const __half* mm = reinterpret_cast<const __half*>(a.page_minmax) + sbase;
+          mn[rb] = __half2float(mm[row]);
+          mx[rb] = __half2float(mm[kD + row]);
+        } else {
+          const float* mm = reinterpret_cast<const float*>(a.page_minmax) + sbase;
+          mn[rb] = mm[row];
+          mx[rb] = mm[kD + row];
+        }
       }
     }
     for (int t = t0; t < t1; t += kVecChunk) {
@@ -145,45 +145,51 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
         const int v = i / kD, c = i % kD;
         kx[v][c] = v < nv ? bf16_to_f(kpage[(size_t)(t + v - pstart) * kD + c]) : 0.f;
       }
+      if (tid < kVecChunk * kWords) cword[tid / kWords][tid % kWords] = 0u;
       __syncthreads();
-      float y[kVecChunk];
-      matvec8<kVecChunk>(rrow, &kx[0][0], kD, y);
 #pragma unroll
-      for (int v = 0; v < kVecChunk; ++v) {
-        if (v < nv) {
-          mn = fminf(mn, y[v]);
-          mx = fmaxf(mx, y[v]);
+      for (int rb = 0; rb < kRowBlocks; ++rb) {
+#pragma unroll
+        for (int v = 0; v < kVecChunk; ++v) {
+          const float y = row_dot16(rrow[rb], &kx[v][0]);
+          if (v < nv) {
+            mn[rb] = fminf(mn[rb], y);
+            mx[rb] = fmaxf(mx[rb], y);
+          }
+          if (row_lead) kr[v][rb * 32 + lrow] = v < nv ? y : 0.f;
         }
-        if (row_lead) kr[v][row] = v < nv ? y[v] : 0.f;
       }
       __syncthreads();
-      float p[kVecChunk];
-      matvec8<kVecChunk>(wrow, &kr[0][0], kD, p);
 #pragma unroll
-      for (int v = 0; v < kVecChunk; ++v) {
-        const uint32_t bits = row_bits8(p[v] > 0.f);  // rows 8w..8w+7
-        if (lane == 0) cbytes[v][warp] = (uint8_t)bits;
+      for (int rb = 0; rb < kRowBlocks; ++rb) {
+#pragma unroll
+        for (int v = 0; v < kVecChunk; ++v) {
+          const float p = row_dot16(wrow[rb], &kr[v][0]);
+          if (row_lead && p > 0.f) atomicOr(&cword[v][rb], 1u << lrow);
+        }
       }
       __syncthreads();
       if (tid < kVecChunk * kWords) {
         const int v = tid / kWords, w = tid % kWords;
-        if (v < nv)
-          a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + w] =
-              reinterpret_cast<const uint32_t*>(cbytes[v])[w];
+        if (v < nv) a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + w] = cword[v][w];
       }
     }
     if (row_lead) {
       // mn/mx started from the stored summary when the page already held keys (min and
       // max are exact, so merging equals recomputing the whole page).
-      if (a.summary_fp16) {
-        __half* mm = reinterpret_cast<__half*>(a.page_minmax) + sbase;
-        // Outward rounding keeps the stored interval around every rotated key.
-        mm[row] = __float2half_rd(mn);
-        mm[kD + row] = __float2half_ru(mx);
-      } else {
-        float* mm = reinterpret_cast<float*>(a.page_minmax) + sbase;
-        mm[row] = mn;
-        mm[kD + row] = mx;
+#pragma unroll
+      for (int rb = 0; rb < kRowBlocks; ++rb) {
+        const int row = rb * 32 + lrow;
+        if (a.summary_fp16) {
+          __half* mm = reinterpret_cast<__half*>(a.page_minmax) + sbase;
+          // Outward rounding keeps the stored interval around every rotated key.
+          mm[row] = __float2half_rd(mn[rb]);
+          mm[kD + row] = __float2half_ru(mx[rb]);
+        } else {
+          float* mm = reinterpret_cast<float*>(a.page_minmax) + sbase;
+          mm[row] = mn[rb];
+          mm[kD + row] = mx[rb];
+        }
       }
     }
   }

@@ -500,7 +500,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
 
   // a0 + a1: append and encode the newest key rows, rotate and encode the queries.
   prof_begin(HHR_KERNEL_ENCODE, s);
-  step_prologue_kernel<<<dim3(G, B), kMvThreads, 0, s>>>(
+  step_prologue_cluster_kernel<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
                    d->summary_fp16});

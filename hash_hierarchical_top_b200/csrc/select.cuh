@@ -9,8 +9,8 @@ namespace hhr {
 // ---------------------------------------------------------------------------- a1
 // HHR page, Abstract (queries are rotated by the same R_h and encoded like keys).
 // One CTA of kMvThreads threads per (KV group, sequence). For each query head of the
-// group: q' = R_g q, code bits = [W_g q' > 0] (the 4 threads of row r own channel
-// and bit r). Also folds the group into the two bound vectors
+// group: q' = R_g q, code bits = [W_g q' > 0] (row_dot16: the 16 threads of row r own
+// channel and bit r). Also folds the group into the two bound vectors
 //   qneg_c = sum_h min(q'_hc, 0),  qpos_c = sum_h max(q'_hc, 0),
 // so that sum_h max(q'_hc*kmin_c, q'_hc*kmax_c) = qneg_c*kmin_c + qpos_c*kmax_c
 // (kmin <= kmax: a positive q' picks kmax, a negative one kmin). The page bound
@@ -28,58 +28,59 @@ struct QPrepArgs {
 __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
   __shared__ __align__(16) float qx[kMaxGroup][kD];
   __shared__ __align__(16) float qr[kMaxGroup][kD];
-  __shared__ __align__(16) uint8_t cbytes[kMaxGroup][16];
+  __shared__ uint32_t cword[kMaxGroup][kWords];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int row = mv_row();
-  const bool row_lead = (lane & 3) == 0;
+  const int lrow = mv_lrow();
+  const bool row_lead = (tid & 15) == 0;
   const int gs = a.Hq / a.G;
-  // R_g and W_g rows of this warp are fetched up front (one memory latency for both).
-  float4 rrow[8], wrow[8];
-  load_rows8(a.R + (size_t)g * kD * kD, rrow);
-  load_rows8(a.W + (size_t)g * kD * kD, wrow);
+  // R_g and W_g rows of this thread are fetched up front (one memory latency for both).
+  float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];
+#pragma unroll
+  for (int rb = 0; rb < kRowBlocks; ++rb) {
+    load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
+    load_row16(a.W + (size_t)g * kD * kD, rb * 32 + lrow, wrow[rb]);
+  }
   for (int i = tid; i < kMaxGroup * kD; i += kMvThreads) {
     const int h = i / kD, c = i % kD;
     qx[h][c] = h < gs ? bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + h) * kD + c]) : 0.f;
-    qr[h][c] = 0.f;
   }
+  if (tid < kMaxGroup * kWords) cword[tid / kWords][tid % kWords] = 0u;
   __syncthreads();
-  float qneg = 0.f, qpos = 0.f;
-  for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
-    float y[kVecChunk];
-    matvec8<kVecChunk>(rrow, &qx[h0][0], kD, y);
+  float qneg[kRowBlocks], qpos[kRowBlocks];
 #pragma unroll
-    for (int v = 0; v < kVecChunk; ++v) {
-      if (h0 + v < gs) {
-        qneg += fminf(y[v], 0.f);
-        qpos += fmaxf(y[v], 0.f);
-        if (row_lead) {
-          qr[h0 + v][row] = y[v];
-          a.q_rot[((size_t)b * a.Hq + g * gs + h0 + v) * kD + row] = y[v];
-        }
+  for (int rb = 0; rb < kRowBlocks; ++rb) {
+    qneg[rb] = 0.f;
+    qpos[rb] = 0.f;
+    for (int h = 0; h < gs; ++h) {
+      const float y = row_dot16(rrow[rb], &qx[h][0]);
+      qneg[rb] += fminf(y, 0.f);
+      qpos[rb] += fmaxf(y, 0.f);
+      if (row_lead) {
+        qr[h][rb * 32 + lrow] = y;
+        a.q_rot[((size_t)b * a.Hq + g * gs + h) * kD + rb * 32 + lrow] = y;
       }
     }
   }
   __syncthreads();
-  for (int h0 = 0; h0 < gs; h0 += kVecChunk) {
-    float p[kVecChunk];
-    matvec8<kVecChunk>(wrow, &qr[h0][0], kD, p);
 #pragma unroll
-    for (int v = 0; v < kVecChunk; ++v) {
-      const uint32_t bits = row_bits8(p[v] > 0.f);
-      if (lane == 0 && h0 + v < kMaxGroup) cbytes[h0 + v][warp] = (uint8_t)bits;
+  for (int rb = 0; rb < kRowBlocks; ++rb) {
+    for (int h = 0; h < gs; ++h) {
+      const float p = row_dot16(wrow[rb], &qr[h][0]);
+      if (row_lead && p > 0.f) atomicOr(&cword[h][rb], 1u << lrow);
     }
   }
   __syncthreads();
   if (tid < gs * kWords) {
     const int h = tid / kWords, w = tid % kWords;
-    a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] =
-        reinterpret_cast<const uint32_t*>(cbytes[h])[w];
+    a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] = cword[h][w];
   }
   if (row_lead) {
     float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
-    o[row] = qneg;
-    o[kD + row] = qpos;
+#pragma unroll
+    for (int rb = 0; rb < kRowBlocks; ++rb) {
+      o[rb * 32 + lrow] = qneg[rb];
+      o[kD + rb * 32 + lrow] = qpos[rb];
+    }
   }
 }
 
