@@ -94,6 +94,51 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
   return res;
 }
 
+// Exclusive block scan of two ints per thread in one pass of barriers (same contract as
+// block_excl_scan; `scratch` holds >= 66 ints). Returns both prefixes; *total the totals.
+__device__ __forceinline__ int2 block_excl_scan2(int2 v, int* scratch, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int a = v.x, b = v.y;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int na = __shfl_up_sync(kFull, a, o), nb = __shfl_up_sync(kFull, b, o);
+    if (lane >= o) { a += na; b += nb; }
+  }
+  if (lane == 31) { scratch[warp] = a; scratch[33 + warp] = b; }
+  __syncthreads();
+  if (warp == 0) {
+    const int wa = lane < nwarps ? scratch[lane] : 0, wb = lane < nwarps ? scratch[33 + lane] : 0;
+    int ia = wa, ib = wb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int na = __shfl_up_sync(kFull, ia, o), nb = __shfl_up_sync(kFull, ib, o);
+      if (lane >= o) { ia += na; ib += nb; }
+    }
+    if (lane < nwarps) { scratch[lane] = ia - wa; scratch[33 + lane] = ib - wb; }
+    if (lane == 31) { scratch[32] = ia; scratch[65] = ib; }
+  }
+  __syncthreads();
+  const int2 res = make_int2(scratch[warp] + a - v.x, scratch[33 + warp] + b - v.y);
+  *total = make_int2(scratch[32], scratch[65]);
+  __syncthreads();
+  return res;
+}
+
+// Cluster barrier in two halves: every thread of every CTA of the cluster arrives (release:
+// its earlier shared-memory writes become visible cluster-wide) and later waits (acquire).
+// arrive + wait together act as cluster.sync(), which also covers __syncthreads().
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  cluster_arrive();
+  cluster_wait();
+}
+
 // Programmatic dependent launch: wait until the preceding kernel in the stream has
 // completed and its writes are visible (a no-op when the launch did not ask for
 // programmatic serialisation), and let the next kernel start launching.

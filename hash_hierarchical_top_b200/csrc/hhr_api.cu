@@ -72,7 +72,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
 }
 
 bool g_smem_tc[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
-    g_smem_ham[kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
+    g_smem_ham[4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
     g_smem_attn_cl[kMaxDevices];
 
 struct SelectLayout {
@@ -306,8 +306,8 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
     uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
     if (allow_smem(qprep_kernel, qprep_smem(), g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(topm_hamming_kernel, topm_hamming_smem(Hq / G, m_max, P, maxp), g_smem_ham) !=
-        cudaSuccess)
+    if (allow_smem(topm_hamming_for(Hq / G), topm_hamming_smem(Hq / G, m_max, P, maxp),
+                   g_smem_ham[hamming_planes(Hq / G) - 1]) != cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qprep_kernel<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
@@ -331,7 +331,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
     const size_t fsm = topm_hamming_smem(Hq / G, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
-    topm_hamming_kernel<<<B * G, kHamThreads, fsm, s>>>(
+    topm_hamming_for(Hq / G)<<<B * G * kHamRanks, kHamThreads, fsm, s>>>(
         TopmHammingArgs{ha, bounds, m_pages, keep_div});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
@@ -491,7 +491,8 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   float* part_o = reinterpret_cast<float*>(aws);
   float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
   const size_t fsm = topm_hamming_smem(gs, m_max, P, maxp);
-  if (allow_smem(topm_hamming_kernel, fsm, g_smem_ham) != cudaSuccess) return HHR_ERR_CUDA;
+  if (allow_smem(topm_hamming_for(gs), fsm, g_smem_ham[hamming_planes(gs) - 1]) != cudaSuccess)
+    return HHR_ERR_CUDA;
   if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
   if (allow_smem(sparse_attn_kernel<true>, attn_smem(), g_smem_attn_cl) != cudaSuccess)
@@ -523,7 +524,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
     prof_begin(HHR_KERNEL_HAMMING, s);
-    e = launch_pdl(topm_hamming_kernel, dim3(B * G), dim3(kHamThreads), fsm, s,
+    e = launch_pdl(topm_hamming_for(gs), dim3(B * G * kHamRanks), dim3(kHamThreads), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div});
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }

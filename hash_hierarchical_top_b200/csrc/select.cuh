@@ -1,6 +1,8 @@
 // Steps a1-a4: query preparation, page-level bounds, top-m, Hamming scan and top-k
 // (HHR), and the block filter + token refinement of the indexer variant (HISA).
 #pragma once
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "encode.cuh"
 
@@ -289,24 +291,30 @@ struct SelectArgs {
   int pad_out;            // write -1 into out[k..out_stride)
 };
 
-// Block-wide min and max of one uint32 per thread (contains __syncthreads).
-__device__ __forceinline__ void block_minmax_u32(uint32_t lo, uint32_t hi, uint32_t* sh,
-                                                 uint32_t* out_lo, uint32_t* out_hi) {
+// Block-wide sum of one int and min / max of one uint32 per thread, in one pass of
+// barriers (contains __syncthreads). sh: 96 words of shared memory.
+__device__ __forceinline__ void block_count_minmax(int cnt, uint32_t lo, uint32_t hi, uint32_t* sh,
+                                                   int* out_cnt, uint32_t* out_lo,
+                                                   uint32_t* out_hi) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
+    cnt += __shfl_xor_sync(kFull, cnt, o);
     lo = min(lo, __shfl_xor_sync(kFull, lo, o));
     hi = max(hi, __shfl_xor_sync(kFull, hi, o));
   }
-  if (lane == 0) { sh[warp] = lo; sh[32 + warp] = hi; }
+  if (lane == 0) { sh[warp] = (uint32_t)cnt; sh[32 + warp] = lo; sh[64 + warp] = hi; }
   __syncthreads();
-  lo = lane < nw ? sh[lane] : 0xffffffffu;
-  hi = lane < nw ? sh[32 + lane] : 0u;
+  cnt = lane < nw ? (int)sh[lane] : 0;
+  lo = lane < nw ? sh[32 + lane] : 0xffffffffu;
+  hi = lane < nw ? sh[64 + lane] : 0u;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
+    cnt += __shfl_xor_sync(kFull, cnt, o);
     lo = min(lo, __shfl_xor_sync(kFull, lo, o));
     hi = max(hi, __shfl_xor_sync(kFull, hi, o));
   }
+  *out_cnt = cnt;
   *out_lo = lo;
   *out_hi = hi;
   __syncthreads();
@@ -314,10 +322,21 @@ __device__ __forceinline__ void block_minmax_u32(uint32_t lo, uint32_t hi, uint3
 
 struct SelShared {
   int hist[256];
-  int scratch[33];
-  uint32_t mm[64];
+  int scratch[66];
+  uint32_t mm[96];
   int digit, rem, cnt;
 };
+
+// Optional page resolution during the compaction of a page selection: the physical page
+// of every kept logical page i is read from ptab[i] and written beside it (-1, and the
+// bad-page status bit, when it is out of range).
+struct PageResolve {
+  const int32_t* ptab;  // the sequence's page-table row, or null
+  int n_phys;
+  int32_t* out_phys;    // parallel to `out`
+};
+
+constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 
 // Block-wide selection (kSelThreads threads, call uniformly): the k largest finite scores
 // of sc[0..n), ties to the lower index, written in ascending index order to out[0..k)
@@ -327,24 +346,31 @@ struct SelShared {
 __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
                                     bool by_kept, int m_pages, int keep_div, int top_k,
                                     int32_t* out, int out_stride, const int32_t* kept_units,
-                                    int unit) {
+                                    int unit, PageResolve pr = PageResolve{nullptr, 0, nullptr}) {
   const int tid = threadIdx.x;
   const int per = ceil_div(n, kSelThreads);
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = tid; i < n; i += kSelThreads) {
-    const float f = sc[i];
-    const bool fin = f > -INFINITY;
-    const uint32_t kk = fin ? f2key(f) : 0u;
-    keys[i] = kk;
-    nfin += fin;
-    if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
+  for (int base = 0; base < n; base += kSelLoadUnroll * kSelThreads) {
+    float f[kSelLoadUnroll];
+#pragma unroll
+    for (int j = 0; j < kSelLoadUnroll; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      f[j] = i < n ? sc[i] : -INFINITY;
+    }
+#pragma unroll
+    for (int j = 0; j < kSelLoadUnroll; ++j) {
+      const int i = base + j * kSelThreads + tid;
+      const bool fin = f[j] > -INFINITY;
+      const uint32_t kk = fin ? f2key(f[j]) : 0u;
+      if (i < n) keys[i] = kk;
+      nfin += fin;
+      if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
+    }
   }
-  int total;
-  block_excl_scan(nfin, sh.scratch, &total);  // also orders the key stores before any read
-  nfin = total;
-  block_minmax_u32(kmin, kmax, sh.mm, &kmin, &kmax);
+  // Also orders the key stores before any read.
+  block_count_minmax(nfin, kmin, kmax, sh.mm, &nfin, &kmin, &kmax);
   const int k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
 
   // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
@@ -411,25 +437,26 @@ __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelS
       }
     }
   }
-  // Compaction in index order.
+  // Compaction in index order. Before thread t's range are gt_before keys above the
+  // threshold and eq_before equal to it, of which the first min(eq_before, rem) are taken.
   auto take_gt = [&](uint32_t kk) -> bool {
     if (kk == 0u) return false;
     if (whole_bin) return (kk >> sel_shift) >= (prefix >> sel_shift);
     return kk > prefix;
   };
-  int eq = 0, cnt = 0;
+  int eq = 0, gt = 0;
   if (k > 0) {
     for (int i = i0; i < i1; ++i) {
       const uint32_t kk = keys[i];
-      if (take_gt(kk)) ++cnt;
+      if (take_gt(kk)) ++gt;
       else if (!whole_bin && kk == prefix) ++eq;
     }
   }
-  const int eq_before = block_excl_scan(eq, sh.scratch, &total);
-  if (k > 0 && !whole_bin) cnt += max(0, min(eq, rem - eq_before));
-  int pos = block_excl_scan(cnt, sh.scratch, &total);
+  int2 tot;
+  const int2 before = block_excl_scan2(make_int2(gt, eq), sh.scratch, &tot);
   if (k > 0) {
-    int e = eq_before;
+    int e = before.y;
+    int pos = before.x + min(e, rem);
     for (int i = i0; i < i1; ++i) {
       const uint32_t kk = keys[i];
       bool take = take_gt(kk);
@@ -437,7 +464,16 @@ __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelS
       if (take && pos < out_stride) {
         int v = i;
         if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
-        out[pos++] = v;
+        out[pos] = v;
+        if (pr.out_phys != nullptr) {
+          int phys = pr.ptab[v];
+          if (phys < 0 || phys >= pr.n_phys) {
+            flag_status(kStatusBadPage);
+            phys = -1;
+          }
+          pr.out_phys[pos] = phys;
+        }
+        ++pos;
       }
     }
   }
@@ -469,14 +505,25 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 
 // ---------------------------------------------------------------------------- a3 + a4
 // HHR page, Abstract (LHP: Hamming distance between binary codes ranks the keys of
-// the pages that survive pruning). One CTA of 1024 threads per (sequence, group).
-// Candidates are the valid keys of the kept pages, in ascending token order.
+// the pages that survive pruning). Candidates are the valid keys of the kept pages, in
+// ascending token order.
 //   delta_t = sum over the group's heads of popcount(qcode_h ^ code_t)  (0..gs*128)
-// Selection of the k smallest (delta, t): a shared-memory histogram of delta gives
-// the threshold bucket; an ordered compaction keeps every key below it and the
-// first ones inside it in token order. Output ascending; -1 past k_eff.
+// Selection of the k smallest (delta, t): a histogram of delta gives the threshold
+// bucket; an ordered compaction keeps every key below it and the first ones inside it
+// in token order. Output ascending; -1 past k_eff.
+//
+// Distance by bit planes: channel j of a candidate contributes z_j = #heads with query
+// bit 0 when the key bit is 1, else n_j = #heads with query bit 1. n and z are kept per
+// code word as NB bit planes (NB = bit width of gs), so one select per plane and word
+// gives the contributions' bits, and a carry-save step over the 4 words leaves 3
+// popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
 constexpr int kHamThreads = 1024;
+constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
+// Code loads in flight per thread (fewer with 4 planes, whose 32 plane words fill registers).
+template <int NB>
+constexpr int ham_load() { return NB >= 4 ? 2 : 4; }
 constexpr int kMaxCand = 65536;
+static_assert(kMaxGroup * 128 + 1 <= 2 * kHamThreads, "threshold search covers 2 bins a thread");
 
 struct HammingArgs {
   const uint32_t* q_code;    // [B][Hq][4]
@@ -490,58 +537,100 @@ struct HammingArgs {
   int Hq, G, P, maxp, n_phys, m_max, top_k;
 };
 
-constexpr int kHamUnroll = 8;
+inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
 
-// Steps a3-a4 for one (sequence, group) row, given its kept logical pages kept_list[0..m)
-// (ascending; global or shared memory). hsm: hamming_smem() bytes of shared memory.
-__device__ void hamming_topk_block(const HammingArgs& a, int row, const int32_t* kept_list,
-                                   int m, uint32_t* hsm) {
+template <int NB>
+struct QueryPlanes {
+  uint32_t n[kWords][NB];  // bit planes of #heads with a 1 bit
+  uint32_t z[kWords][NB];  // bit planes of #heads with a 0 bit
+};
+
+// Bit-sliced counts over the gs query codes qc[h*4 + w] (ripple-carry adds of one bit
+// vector per head).
+template <int NB>
+__device__ __forceinline__ void build_query_planes(const uint32_t* qc, int gs, QueryPlanes<NB>& p) {
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) { p.n[w][b] = 0u; p.z[w][b] = 0u; }
+    for (int h = 0; h < gs; ++h) {
+      uint32_t cn = qc[h * kWords + w], cz = ~cn;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const uint32_t tn = p.n[w][b] & cn, tz = p.z[w][b] & cz;
+        p.n[w][b] ^= cn;
+        p.z[w][b] ^= cz;
+        cn = tn;
+        cz = tz;
+      }
+    }
+  }
+}
+
+template <int NB>
+__device__ __forceinline__ int hamming_delta(const QueryPlanes<NB>& p, const uint4 c) {
+  const uint32_t cw[kWords] = {c.x, c.y, c.z, c.w};
+  int d = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    uint32_t x[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) x[w] = (cw[w] & p.z[w][b]) | (~cw[w] & p.n[w][b]);
+    const uint32_t sum = x[0] ^ x[1] ^ x[2];
+    const uint32_t carry = (x[0] & x[1]) | (x[2] & (x[0] ^ x[1]));
+    d += (__popc(sum) + __popc(x[3]) + 2 * __popc(carry)) << b;
+  }
+  return d;
+}
+
+struct HamShared {
+  int scratch[66];
+  int T, need_eq;
+  int tot[2];  // this CTA's (#below threshold, #equal) for the other ranks
+};
+
+// Steps a3-a4 for one (sequence, group) row on the cluster's CTA `rank`, given the row's
+// kept logical pages klp[0..m) (ascending) and their physical pages kphys (-1 invalid),
+// in shared memory. CTA r scores candidates [r*half, (r+1)*half); the histograms and the
+// compaction offsets are combined through distributed shared memory.
+// hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
+template <int NB>
+__device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
+                                     const int32_t* kphys, int m, const uint32_t* qc,
+                                     uint32_t* hsm, HamShared& hs) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
   const int b = row / a.G, g = row % a.G;
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.G;
   const int nbins = gs * 128 + 1;
   m = min(m, a.m_max);
-  int* hist = reinterpret_cast<int*>(hsm);                    // [nbins]
-  int* scratch = hist + ((nbins + 31) & ~31);                 // [33]
-  int* sh = scratch + 33;                                     // [3]
-  int* kphys = sh + 3;                                        // [m_max] physical page
-  int* klp = kphys + a.m_max;                                 // [m_max] logical page
-  uint16_t* dist = reinterpret_cast<uint16_t*>(kphys + ((2 * a.m_max + 3) & ~3));  // [C], 16B-aligned
+  int* hist = reinterpret_cast<int*>(hsm);                                // [nbins]
+  uint16_t* dist = reinterpret_cast<uint16_t*>(hist + ((nbins + 31) & ~31));  // [half], 16B-aligned
   const int n = a.seq_len[b];
   const int C = min(m * a.P, kMaxCand);
+  const int half = ((ceil_div(C, kHamRanks) + 7) / 8) * 8;
+  const int lo = min(C, rank * half), hi = min(C, lo + half);
+  const int Cr = hi - lo;
   for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
-  // Resolve the kept pages once: logical id and physical page (-1 if invalid).
-  for (int i = tid; i < m; i += kHamThreads) {
-    const int lp = kept_list[i];
-    int phys = -1;
-    if (lp >= 0 && lp < a.maxp) phys = a.page_table[(size_t)b * a.maxp + lp];
-    if (phys < 0 || phys >= a.n_phys) {
-      flag_status(kStatusBadPage);
-      phys = -1;
-    }
-    kphys[i] = phys;
-    klp[i] = lp;
-  }
-  uint32_t qc[kMaxGroup][kWords];
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-    for (int w = 0; w < kWords; ++w)
-      qc[h][w] = h < gs ? a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] : 0u;
+  if (tid == 0) { hs.T = -1; hs.need_eq = 0; }
+  QueryPlanes<NB> qp;
+  build_query_planes<NB>(qc, gs, qp);
   __syncthreads();
-  // Candidates c = tid + j*1024: consecutive threads read consecutive 16-byte codes of a
-  // page (coalesced); all kHamUnroll code loads of a thread are issued before any math.
+  // Candidates c = lo + tid + j*1024: consecutive threads read consecutive 16-byte codes of
+  // a page (coalesced); all ham_load() code loads of a thread are issued before any math.
   // c / P by multiply-high: exact for c < 2^24 with magic = floor(2^32 / P) + 1.
   const uint32_t magic = (uint32_t)(0xffffffffu / (uint32_t)a.P) + 1u;
-  for (int c0 = 0; c0 < C; c0 += kHamThreads * kHamUnroll) {
-    uint4 code[kHamUnroll];
-    bool ok[kHamUnroll];
+  constexpr int kHamLoad = ham_load<NB>();
+  for (int c0 = lo; c0 < hi; c0 += kHamThreads * kHamLoad) {
+    uint4 code[kHamLoad];
+    bool ok[kHamLoad];
 #pragma unroll
-    for (int j = 0; j < kHamUnroll; ++j) {
+    for (int j = 0; j < kHamLoad; ++j) {
       const int c = c0 + j * kHamThreads + tid;
       ok[j] = false;
       code[j] = make_uint4(0, 0, 0, 0);
-      if (c < C) {
+      if (c < hi) {
         const int i = (a.P == 1) ? c : (int)__umulhi((uint32_t)c, magic);
         const int slot = c - i * a.P;
         const int phys = kphys[i];
@@ -553,53 +642,54 @@ __device__ void hamming_topk_block(const HammingArgs& a, int row, const int32_t*
       }
     }
 #pragma unroll
-    for (int j = 0; j < kHamUnroll; ++j) {
+    for (int j = 0; j < kHamLoad; ++j) {
       const int c = c0 + j * kHamThreads + tid;
-      int d = 0;
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h)
-        if (h < gs)
-          d += __popc(qc[h][0] ^ code[j].x) + __popc(qc[h][1] ^ code[j].y) +
-               __popc(qc[h][2] ^ code[j].z) + __popc(qc[h][3] ^ code[j].w);
+      const int d = hamming_delta<NB>(qp, code[j]);
       if (ok[j]) atomicAdd(&hist[d], 1);
-      if (c < C) dist[c] = ok[j] ? (uint16_t)d : (uint16_t)0xffff;
+      if (c < hi) dist[c - lo] = ok[j] ? (uint16_t)d : (uint16_t)0xffff;
     }
   }
-  __syncthreads();
-  // Threshold bucket: smallest T with #(delta <= T) >= k_eff. Warp 0 scans the bins.
-  if (tid < 32) {
-    const int per = ceil_div(nbins, 32);
-    const int b0 = min(nbins, tid * per), b1 = min(nbins, b0 + per);
-    int s = 0;
-    for (int i = b0; i < b1; ++i) s += hist[i];
-    int incl = warp_incl_scan(s, tid);
-    int nvalid = __shfl_sync(kFull, incl, 31);
-    int keff = min(a.top_k, nvalid);
-    int excl = incl - s;
-    if (tid == 0) { sh[0] = -1; sh[1] = 0; sh[2] = keff; }
-    __syncwarp();
-    if (keff > 0 && excl < keff && keff <= incl) {
-      int run = excl;
-      for (int i = b0; i < b1; ++i) {
-        if (run < keff && keff <= run + hist[i]) { sh[0] = i; sh[1] = keff - run; }
-        run += hist[i];
+  cluster_sync_all();  // every rank's histogram is complete
+  // Threshold bucket: smallest T with #(delta <= T) >= k_eff over the summed histograms.
+  // Thread t holds bins [2t, 2t+2) (fewer past nbins).
+  {
+    int hv[2], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int i = 2 * tid + q;
+      hv[q] = 0;
+      if (i < nbins) {
+#pragma unroll
+        for (int r = 0; r < kHamRanks; ++r) hv[q] += cl.map_shared_rank(hist, r)[i];
       }
+      sum += hv[q];
     }
+    int nvalid;
+    const int excl = block_excl_scan(sum, hs.scratch, &nvalid);
+    const int keff = min(a.top_k, nvalid);
+    if (keff > 0 && excl < keff && keff <= excl + sum) {
+      const int first = keff <= excl + hv[0] ? 0 : 1;
+      hs.T = 2 * tid + first;
+      hs.need_eq = keff - excl - (first ? hv[0] : 0);
+    }
+    if (tid == 0) a.out_count[row] = keff;  // every rank writes the same value
+    __syncthreads();
+    for (int i = keff + rank * kHamThreads + tid; i < a.top_k; i += kHamRanks * kHamThreads)
+      a.out_idx[(size_t)row * a.top_k + i] = -1;
   }
-  __syncthreads();
-  const int T = sh[0], need_eq = sh[1], keff = sh[2];
-  // Ordered compaction: thread t owns the contiguous candidates [t*cpt, (t+1)*cpt), cpt a
+  const int T = hs.T, need_eq = hs.need_eq;
+  // Ordered compaction of this rank's candidates: thread t owns [t*cpt, (t+1)*cpt), cpt a
   // multiple of 8, read as 16-byte groups of 8 distances.
-  const int cpt = ((ceil_div(C, kHamThreads) + 7) / 8) * 8;
+  const int cpt = ((ceil_div(Cr, kHamThreads) + 7) / 8) * 8;
   const int ngrp = cpt / 8;
   auto load8 = [&](int i0, uint16_t (&dv)[8]) {
     uint4 raw = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
-    if (i0 < C) raw = *reinterpret_cast<const uint4*>(dist + i0);
+    if (i0 < Cr) raw = *reinterpret_cast<const uint4*>(dist + i0);
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      dv[2 * q] = (i0 + 2 * q < C) ? (uint16_t)(w[q] & 0xffff) : (uint16_t)0xffff;
-      dv[2 * q + 1] = (i0 + 2 * q + 1 < C) ? (uint16_t)(w[q] >> 16) : (uint16_t)0xffff;
+      dv[2 * q] = (i0 + 2 * q < Cr) ? (uint16_t)(w[q] & 0xffff) : (uint16_t)0xffff;
+      dv[2 * q + 1] = (i0 + 2 * q + 1 < Cr) ? (uint16_t)(w[q] >> 16) : (uint16_t)0xffff;
     }
   };
   int eq = 0, lt = 0;
@@ -612,13 +702,21 @@ __device__ void hamming_topk_block(const HammingArgs& a, int row, const int32_t*
       lt += (dv[q] < T);
     }
   }
-  int total;
-  const int eq_before = block_excl_scan(eq, scratch, &total);
-  const int cnt = lt + max(0, min(eq, need_eq - eq_before));
-  int pos = block_excl_scan(cnt, scratch, &total);
+  int2 tot;
+  const int2 before = block_excl_scan2(make_int2(lt, eq), hs.scratch, &tot);
+  if (tid == 0) { hs.tot[0] = tot.x; hs.tot[1] = tot.y; }
+  cluster_sync_all();  // every rank's totals are published
+  int lt_off = 0, eq_off = 0;
+  for (int r = 0; r < rank; ++r) {
+    const int* rt = cl.map_shared_rank(&hs.tot[0], r);
+    lt_off += rt[0];
+    eq_off += rt[1];
+  }
+  cluster_arrive();  // no remote shared-memory access after this point
   int32_t* out = a.out_idx + (size_t)row * a.top_k;
   {
-    int e = eq_before;
+    int e = eq_off + before.y;
+    int pos = lt_off + before.x + min(e, need_eq);
     for (int gi = 0; gi < ngrp; ++gi) {
       uint16_t dv[8];
       const int i0 = tid * cpt + gi * 8;
@@ -628,58 +726,84 @@ __device__ void hamming_topk_block(const HammingArgs& a, int row, const int32_t*
         bool take = dv[q] < T;
         if (dv[q] == T) { take = e < need_eq; ++e; }
         if (take && pos < a.top_k) {
-          const int i = i0 + q;
+          const int i = lo + i0 + q;
           const int pi = (a.P == 1) ? i : (int)__umulhi((uint32_t)i, magic);
           out[pos++] = klp[pi] * a.P + (i - pi * a.P);
         }
       }
     }
   }
-  for (int i = keff + tid; i < a.top_k; i += kHamThreads) out[i] = -1;
-  if (tid == 0) a.out_count[row] = keff;
+  cluster_wait();  // keep this CTA's shared memory alive until every rank has read it
 }
 
 inline size_t hamming_smem(int gs, int m_max, int P) {
   const int nbins = gs * 128 + 1;
-  const size_t ints = (size_t)((nbins + 31) & ~31) + 36 + (size_t)((2 * m_max + 3) & ~3);
-  // Distances padded so the 16-byte group reads of the last thread stay inside.
-  const size_t cand = ((size_t)m_max * P + 8 + 7) & ~(size_t)7;
-  return ints * 4 + cand * 2 + 16;
+  const size_t ints = (size_t)((nbins + 31) & ~31);
+  // This rank's distances, padded so the 16-byte group reads of the last thread stay inside.
+  const size_t c = (size_t)m_max * P < (size_t)kMaxCand ? (size_t)m_max * P : (size_t)kMaxCand;
+  const size_t half = ((c + kHamRanks - 1) / kHamRanks + 7) & ~(size_t)7;
+  return ints * 4 + (half + 8) * 2 + 16;
 }
 
-// Top-m pages and the Hamming top-k fused in one CTA per (sequence, group): the kept page
-// list never leaves shared memory (a copy goes to `kept`/`kept_count` for inspection).
-// Shared memory: [kept list: m_max words][union of: top-m keys (maxp words) | Hamming
-// scratch (hamming_smem bytes)].
+// Top-m pages and the Hamming top-k fused in one cluster of kHamRanks CTAs per (sequence,
+// group): every rank selects the same kept pages (deterministic), resolving their physical
+// pages during the compaction, so the kept list never leaves shared memory (rank 0 copies
+// it to `kept`/`kept_count` for inspection). Shared memory: [kept list: m_max words][their
+// physical pages: m_max words][union of: top-m keys (maxp words) | Hamming scratch].
 struct TopmHammingArgs {
   HammingArgs h;
   const float* bounds;  // [B][G][maxp]
   int m_pages, keep_div;
 };
 
-__global__ void __launch_bounds__(kHamThreads) topm_hamming_kernel(TopmHammingArgs a) {
+template <int NB>
+__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
+    topm_hamming_kernel(TopmHammingArgs a) {
   __shared__ SelShared sh;
+  __shared__ HamShared hs;
+  __shared__ uint32_t qcs[kMaxGroup * kWords];
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t fsm[];
   const HammingArgs& h = a.h;
-  const int row = blockIdx.x, b = row / h.G;
+  const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
+  const int b = row / h.G, g = row % h.G;
+  const int gs = h.Hq / h.G;
+  if (threadIdx.x < gs * kWords)
+    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + g * gs) * kWords + threadIdx.x];
+  const int mw = (h.m_max + 3) & ~3;
   int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
-  uint32_t* work = fsm + ((h.m_max + 3) & ~3);
+  int32_t* kphys_s = kept_s + mw;
+  uint32_t* work = fsm + 2 * mw;
   const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
-  const int m = block_select_largest(a.bounds + (size_t)row * h.maxp, n, work, sh, true,
-                                     a.m_pages, a.keep_div, 0, kept_s, h.m_max, nullptr, 0);
+  const int m = block_select_largest(
+      a.bounds + (size_t)row * h.maxp, n, work, sh, true, a.m_pages, a.keep_div, 0, kept_s,
+      h.m_max, nullptr, 0, PageResolve{h.page_table + (size_t)b * h.maxp, h.n_phys, kphys_s});
   __syncthreads();
-  int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
-  for (int i = threadIdx.x; i < m; i += kHamThreads) kept_g[i] = kept_s[i];
-  if (threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
-  hamming_topk_block(h, row, kept_s, m, work);
+  if (rank == 0) {
+    int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
+    for (int i = threadIdx.x; i < m; i += kHamThreads) kept_g[i] = kept_s[i];
+    if (threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
+  }
+  hamming_topk_cluster<NB>(h, row, rank, kept_s, kphys_s, m, qcs, work, hs);
 }
 
 inline size_t topm_hamming_smem(int gs, int m_max, int P, int maxp) {
   const size_t sel = (size_t)maxp * 4;
   const size_t ham = hamming_smem(gs, m_max, P);
-  return (size_t)((m_max + 3) & ~3) * 4 + (sel > ham ? sel : ham);
+  return (size_t)((m_max + 3) & ~3) * 8 + (sel > ham ? sel : ham);
+}
+
+using TopmHammingFn = void (*)(TopmHammingArgs);
+
+// The instantiation for group size gs (1..kMaxGroup).
+inline TopmHammingFn topm_hamming_for(int gs) {
+  switch (hamming_planes(gs)) {
+    case 1: return topm_hamming_kernel<1>;
+    case 2: return topm_hamming_kernel<2>;
+    case 3: return topm_hamming_kernel<3>;
+    default: return topm_hamming_kernel<4>;
+  }
 }
 
 // ---------------------------------------------------------------------------- HISA a1'

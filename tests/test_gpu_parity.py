@@ -107,7 +107,7 @@ def test_edge_cases(case, f16):
     _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=f16))
 
 
-@pytest.mark.parametrize("heads", [(8, 1), (8, 8), (6, 2)])
+@pytest.mark.parametrize("heads", [(8, 1), (8, 8), (6, 2), (10, 2)])
 def test_group_shapes(heads):
     hq, g = heads
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], n_q_heads=hq, n_kv_heads=g, seq_lens=(3000, 1234),
