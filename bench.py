@@ -359,6 +359,13 @@ def main():
                             cache.codes, None)
         start = (inp["seq_len"] - 1).to(torch.int32)
         one = torch.ones(wl.batch, dtype=torch.int32, device=dev)
+        if not args.select_only:
+            # The newest K/V row of every sequence, as a decode step receives it from the
+            # model ([B][G][d]); appending it rewrites the same cache slot every step.
+            t = start.long()
+            phys = inp["page_table"][torch.arange(wl.batch, device=dev), t // P].long()
+            inp["k_new"] = inp["k_cache"][phys, :, t % P].contiguous()
+            inp["v_new"] = inp["v_cache"][phys, :, t % P].contiguous()
         layers.append((inp, d, cache, start, one))
     d0 = layers[0][1]
     step = DecodeStep(d0, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev,
@@ -378,9 +385,11 @@ def main():
                         W=inp["W"])
             return
         if args.path == "fused":
-            # The newest row of every sequence is already in the cache: re-append it.
+            # Append the newest K/V rows (they equal the cached ones, so every step sees the
+            # same cache), encode the key, select, attend: one hhr_decode_step call.
             step.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
-                            inp["seq_len"], inp["R"], inp["W"], cache)
+                            inp["seq_len"], inp["R"], inp["W"], cache, k_new=inp["k_new"],
+                            v_new=inp["v_new"])
             return
         step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
                   inp["R"], inp["W"], cache, start, one)

@@ -31,12 +31,22 @@ constexpr int kRowBlocks = kD / 32;
 
 __device__ __forceinline__ int mv_lrow() { return (int)threadIdx.x >> 4; }  // 0..31
 
-// Row `row` of M, this thread's part (float4s part and part + 16).
+// Row `row` of M, this thread's part (float4s part and part + 16). The loads are volatile
+// asm so that they are issued here, at kernel start, and not sunk past later barriers to
+// their first use (which would add a memory latency to the critical path).
+__device__ __forceinline__ float4 ldg_f4_now(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ void load_row16(const float* __restrict__ M, int row, float4 (&m)[2]) {
   const int part = threadIdx.x & 15;
   const float4* r4 = reinterpret_cast<const float4*>(M + (size_t)row * kD);
-  m[0] = __ldg(r4 + part);
-  m[1] = __ldg(r4 + part + 16);
+  m[0] = ldg_f4_now(r4 + part);
+  m[1] = ldg_f4_now(r4 + part + 16);
 }
 
 __device__ __forceinline__ float row_dot16(const float4 (&m)[2], const float* x) {

@@ -6,6 +6,7 @@
 #include <stdio.h>
 
 #include <atomic>
+#include <initializer_list>
 
 #include "../../include/hhr.h"
 #include "attn.cuh"
@@ -25,6 +26,13 @@ constexpr int kMaxDevices = 64;
 constexpr int kTcMinBulk = 4096;  // appends at least this long use the tensor-core encoder
 constexpr int kTcSlots = 148;     // persistent encoder CTAs (one per SM of a B200)
 constexpr size_t kMaxKernelSmem = 200 * 1024;  // below the 227 KB opt-in of sm_100
+
+// Every device buffer is read with 16-byte vector loads somewhere on the path.
+bool misaligned16(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (((uintptr_t)p & 15) != 0) return true;
+  return false;
+}
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -231,6 +239,7 @@ int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* p
   if (hashing && (page_minmax == nullptr || codes == nullptr || R == nullptr || W == nullptr))
     return HHR_ERR_INVALID_ARG;
   if (!hashing && block_mean == nullptr) return HHR_ERR_INVALID_ARG;
+  if (misaligned16({k_cache, R, W, page_minmax, codes, block_mean})) return HHR_ERR_INVALID_ARG;
   if (max_new < 0) return HHR_ERR_INVALID_ARG;
   if (max_new == 0) return HHR_OK;
   const long long pages = (long long)(max_new + d->page_size - 1) / d->page_size + 1;
@@ -285,6 +294,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     return HHR_ERR_INVALID_ARG;
   if (mode == HHR_MODE_INDEXER && (q_pos == nullptr || block_mean == nullptr || k_cache == nullptr))
     return HHR_ERR_INVALID_ARG;
+  if (misaligned16({q, R, W, page_minmax, codes, block_mean, k_cache})) return HHR_ERR_INVALID_ARG;
   const int m_max = kept_max(d, m_pages, keep_div);
   const SelectLayout L = select_layout(d, mode, m_max);
   if (ws_bytes < L.total) return HHR_ERR_WORKSPACE;
@@ -412,6 +422,7 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
       workspace == nullptr)
     return HHR_ERR_INVALID_ARG;
   if (top_k < 1 || !(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
+  if (misaligned16({q, k_cache, v_cache, out})) return HHR_ERR_INVALID_ARG;
   // Cache rows are addressed with 32-bit row indices.
   if ((unsigned long long)d->n_phys_pages * d->n_kv_heads * d->page_size >= 0xffffffffull)
     return HHR_ERR_UNSUPPORTED;
@@ -467,6 +478,8 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     return HHR_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return HHR_ERR_INVALID_ARG;
   if (!(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
+  if (misaligned16({q, k_new, v_new, k_cache, v_cache, R, W, page_minmax, codes, out}))
+    return HHR_ERR_INVALID_ARG;
   if ((unsigned long long)d->n_phys_pages * d->n_kv_heads * d->page_size >= 0xffffffffull)
     return HHR_ERR_UNSUPPORTED;
   const size_t need = hhr_decode_step_workspace_bytes(d, m_pages, keep_div, top_k);
@@ -501,7 +514,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
 
   // a0 + a1: append and encode the newest key rows, rotate and encode the queries.
   prof_begin(HHR_KERNEL_ENCODE, s);
-  step_prologue_cluster_kernel<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
+  step_prologue_for(gs)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
                    d->summary_fp16});

@@ -3,11 +3,11 @@
 // all with one read of R_g and W_g.
 //
 // HHR page, Abstract: GKR rotates keys and queries with the head-wise orthogonal R_h and
-// summarises each page for its logit bound; LHP encodes both into binary codes. One CTA
-// of kMvThreads threads per (KV group, sequence): the newest key (position seq_len-1) and
-// the group's query heads form one batch of up to 9 vectors for the two mat-vecs. The key
-// and query arithmetic is the same per-vector code as in encode_page_kernel and
-// qprep_kernel, so the results are bit-identical to the separate calls.
+// summarises each page for its logit bound; LHP encodes both into binary codes. The newest
+// key (position seq_len-1) and the group's query heads form one batch of 1 + gs vectors
+// for the two mat-vecs. Every rotated channel and projection is row_dot16 on the same
+// inputs as in encode_page_kernel and qprep_kernel, and the folds run in the same order, so
+// the results are bit-identical to the separate calls.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -34,9 +34,8 @@ struct PrologueArgs {
   int Hq, G, P, maxp, n_phys, summary_fp16;
 };
 
-constexpr int kMaxStepVecs = 1 + kMaxGroup;  // newest key + query heads
 
-// Loads the stored summary channels `row` of a page that already held keys.
+// Loads the stored summary channel `row` of a page that already held keys.
 __device__ __forceinline__ void load_summary_row(const void* page_minmax, int fp16, size_t sbase,
                                                  int row, float& mn, float& mx) {
   if (fp16) {
@@ -64,14 +63,15 @@ __device__ __forceinline__ void store_summary_row(void* page_minmax, int fp16, s
   }
 }
 
-// Resolves the newest key's slot; phys < 0 when the sequence is empty or its page is bad.
+// The newest key's slot; phys < 0 when the sequence is empty or its page is out of range.
 struct NewestSlot {
   int phys, slot;
   size_t krow, sbase;
 };
 
-__device__ __forceinline__ NewestSlot newest_slot(const PrologueArgs& a, int b, int g, bool report) {
-  const int t = a.seq_len[b] - 1;
+__device__ __forceinline__ NewestSlot newest_slot(const PrologueArgs& a, int len, int b, int g,
+                                                  bool report) {
+  const int t = len - 1;
   const int lp = t >= 0 ? t / a.P : -1;
   int phys = -1;
   if (t >= 0 && lp < a.maxp) {
@@ -87,190 +87,134 @@ __device__ __forceinline__ NewestSlot newest_slot(const PrologueArgs& a, int b, 
   return s;
 }
 
-// Fills xs[0] with the newest key (written to the cache first when given; only when
-// `writer`) and xs[1..gs] with the group's queries.
-__device__ __forceinline__ void load_step_vectors(const PrologueArgs& a, int b, int g, const NewestSlot& s,
-                                                  bool writer, float (*xs)[kD], int nthreads) {
-  const int gs = a.Hq / a.G;
-  for (int i = threadIdx.x; i < (1 + gs) * kD; i += nthreads) {
-    const int v = i / kD, c = i % kD;
-    float x = 0.f;
-    if (v == 0) {
-      if (s.phys >= 0) {
-        uint16_t kb;
-        if (a.k_new != nullptr) {
-          kb = a.k_new[((size_t)b * a.G + g) * kD + c];
-          if (writer) {
-            a.k_cache[s.krow + c] = kb;
-            if (a.v_new != nullptr) a.v_cache[s.krow + c] = a.v_new[((size_t)b * a.G + g) * kD + c];
-          }
-        } else {
-          kb = a.k_cache[s.krow + c];
-        }
-        x = bf16_to_f(kb);
-      }
-    } else {
-      x = bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + (v - 1)) * kD + c]);
-    }
-    xs[v][c] = x;
-  }
+// Eight bf16 values (one 16-byte piece) to fp32, stored at dst[0..8).
+__device__ __forceinline__ void store_bf16x8(const uint4 raw, float* dst) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+  d4[0] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
+  d4[1] = make_float4(__uint_as_float(raw.z << 16), __uint_as_float(raw.z & 0xffff0000u),
+                      __uint_as_float(raw.w << 16), __uint_as_float(raw.w & 0xffff0000u));
 }
 
-__global__ void __launch_bounds__(kMvThreads) step_prologue_kernel(PrologueArgs a) {
-  __shared__ __align__(16) float xs[kMaxStepVecs][kD];  // raw vectors
-  __shared__ __align__(16) float xr[kMaxStepVecs][kD];  // rotated vectors
-  __shared__ uint32_t cword[kMaxStepVecs][kWords];
-  pdl_wait();
-  pdl_trigger();
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int lrow = mv_lrow();
-  const bool row_lead = (tid & 15) == 0;
-  const int gs = a.Hq / a.G;
-
-  float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];
-#pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
-    load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
-    load_row16(a.W + (size_t)g * kD * kD, rb * 32 + lrow, wrow[rb]);
-  }
-  const NewestSlot s = newest_slot(a, b, g, tid == 0);
-  const bool has_key = s.phys >= 0;
-  float mn[kRowBlocks], mx[kRowBlocks];
-#pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
-    mn[rb] = INFINITY;
-    mx[rb] = -INFINITY;
-    if (has_key && s.slot > 0 && row_lead)
-      load_summary_row(a.page_minmax, a.summary_fp16, s.sbase, rb * 32 + lrow, mn[rb], mx[rb]);
-  }
-  load_step_vectors(a, b, g, s, true, xs, kMvThreads);
-  if (tid < kMaxStepVecs * kWords) cword[tid / kWords][tid % kWords] = 0u;
-  __syncthreads();
-
-  // Vector 0 is the newest key, 1..gs the queries: the per-vector arithmetic is that of
-  // encode_page_kernel and qprep_kernel.
-  float qneg[kRowBlocks], qpos[kRowBlocks];
-#pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
-    const int row = rb * 32 + lrow;
-    const float yk = row_dot16(rrow[rb], &xs[0][0]);
-    if (has_key) {
-      mn[rb] = fminf(mn[rb], yk);
-      mx[rb] = fmaxf(mx[rb], yk);
-    }
-    if (row_lead) xr[0][row] = has_key ? yk : 0.f;
-    qneg[rb] = 0.f;
-    qpos[rb] = 0.f;
-    for (int h = 0; h < gs; ++h) {
-      const float y = row_dot16(rrow[rb], &xs[1 + h][0]);
-      qneg[rb] += fminf(y, 0.f);
-      qpos[rb] += fmaxf(y, 0.f);
-      if (row_lead) {
-        xr[1 + h][row] = y;
-        a.q_rot[((size_t)b * a.Hq + g * gs + h) * kD + row] = y;
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
-    for (int v = 0; v <= gs; ++v) {
-      const float p = row_dot16(wrow[rb], &xr[v][0]);
-      if (row_lead && p > 0.f) atomicOr(&cword[v][rb], 1u << lrow);
-    }
-  }
-  __syncthreads();
-  if (tid < (1 + gs) * kWords) {
-    const int v = tid / kWords, w = tid % kWords;
-    if (v == 0) {
-      if (has_key) a.codes[(((size_t)s.phys * a.G + g) * a.P + s.slot) * kWords + w] = cword[0][w];
-    } else {
-      a.q_code[((size_t)b * a.Hq + g * gs + (v - 1)) * kWords + w] = cword[v][w];
-    }
-  }
-  if (row_lead) {
-    float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
-#pragma unroll
-    for (int rb = 0; rb < kRowBlocks; ++rb) {
-      const int row = rb * 32 + lrow;
-      if (has_key) store_summary_row(a.page_minmax, a.summary_fp16, s.sbase, row, mn[rb], mx[rb]);
-      o[row] = qneg[rb];
-      o[kD + row] = qpos[rb];
-    }
-  }
-}
-
-// Cluster form of the prologue: a cluster of kPrologueRanks CTAs per (group, sequence),
-// CTA r owning rows 32r..32r+31 of R_g and W_g (one row block of row_dot16 each, so every
-// thread does 1/16 of a row's dot product). Each CTA rotates every vector on its 32 rows,
-// the rotated vectors are assembled through distributed shared memory, and each CTA
-// projects them on its 32 rows of W_g: its 32 sign bits are code word r. CTA r also owns
-// summary channels and folded-query channels 32r..32r+31. Same arithmetic per value as
-// step_prologue_kernel.
+// A cluster of kPrologueRanks CTAs per (group, sequence). CTA r owns rows 32r..32r+31 of R_g
+// and W_g (one row block of row_dot16, 16 threads per row). It rotates all 1 + GS vectors on
+// its rows and sends the results, as 16-byte pieces, into every CTA's copy of the rotated
+// vectors (distributed shared memory); after one cluster barrier it projects them on its rows of W_g, whose 32
+// sign bits are code word r. CTA r also owns summary channels and folded-query channels
+// 32r..32r+31. Every input load is issued at the start; only the key's cache slot (and the
+// key itself when k_new is null) waits for the page table.
 constexpr int kPrologueRanks = kRowBlocks;
 constexpr int kPrologueThreads = kMvThreads;  // 32 rows x 16 threads
 
+template <int GS>
 __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kPrologueThreads)
     step_prologue_cluster_kernel(PrologueArgs a) {
   namespace cg = cooperative_groups;
-  __shared__ __align__(16) float xs[kMaxStepVecs][kD];     // raw vectors
-  __shared__ __align__(16) float xpart[kMaxStepVecs][32];  // my rows, rotated
-  __shared__ __align__(16) float xr[kMaxStepVecs][kD];     // all rows, rotated
-  __shared__ uint32_t cword[kMaxStepVecs];
+  constexpr int NV = 1 + GS;  // vector 0: the newest key; 1..GS: the query heads
+  static_assert(16 * (NV + 1) <= kPrologueThreads, "one 16-byte piece per thread");
+  __shared__ __align__(16) float xs[NV][kD];  // raw vectors
+  __shared__ __align__(16) float xpart[NV][32];  // rotated vectors, this CTA's rows
+  __shared__ __align__(16) float xr[NV][kD];     // rotated vectors, every row
+  __shared__ uint32_t cpart[NV][kPrologueThreads / 32];  // sign bits of each warp's rows
   pdl_wait();
   pdl_trigger();
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int lrow = mv_lrow();
+  const int lrow = mv_lrow(), part = tid & 15;
   const int row = rank * 32 + lrow;
-  const bool row_lead = (tid & 15) == 0;
-  const int gs = a.Hq / a.G;
+  const bool row_lead = part == 0;
 
   float4 rr[2], wr[2];
   load_row16(a.R + (size_t)g * kD * kD, row, rr);
   load_row16(a.W + (size_t)g * kD * kD, row, wr);
-  if (tid < kMaxStepVecs) cword[tid] = 0u;
-  const NewestSlot s = newest_slot(a, b, g, tid == 0 && rank == 0);
+  const int len = a.seq_len[b];
+  // Threads [16v, 16v + 16) load vector v (k_new, then the queries) as 16-byte pieces of
+  // 8 channels; threads [16 NV, 16 NV + 16) load v_new.
+  const int pv = tid >> 4, c8 = part * 8;
+  const bool append = a.k_new != nullptr;
+  uint4 raw = make_uint4(0, 0, 0, 0);
+  if (pv == 0) {
+    if (append) raw = *reinterpret_cast<const uint4*>(a.k_new + ((size_t)b * a.G + g) * kD + c8);
+  } else if (pv < NV) {
+    raw = *reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + g * GS + pv - 1) * kD + c8);
+  } else if (pv == NV && append && a.v_new != nullptr) {
+    raw = *reinterpret_cast<const uint4*>(a.v_new + ((size_t)b * a.G + g) * kD + c8);
+  }
+  const NewestSlot s = newest_slot(a, len, b, g, tid == 0 && rank == 0);
   const bool has_key = s.phys >= 0;
+  if (pv == 0) {
+    if (!has_key) {
+      raw = make_uint4(0, 0, 0, 0);
+    } else if (!append) {
+      raw = *reinterpret_cast<const uint4*>(a.k_cache + s.krow + c8);
+    } else if (rank == 0) {  // one writer of the new rows
+      *reinterpret_cast<uint4*>(a.k_cache + s.krow + c8) = raw;
+    }
+  } else if (pv == NV && has_key && append && a.v_new != nullptr && rank == 0) {
+    *reinterpret_cast<uint4*>(a.v_cache + s.krow + c8) = raw;
+  }
+  if (pv < NV) store_bf16x8(raw, &xs[pv][c8]);
   float mn = INFINITY, mx = -INFINITY;
   if (has_key && s.slot > 0 && row_lead) load_summary_row(a.page_minmax, a.summary_fp16, s.sbase, row, mn, mx);
-  load_step_vectors(a, b, g, s, rank == 0, xs, kPrologueThreads);
   __syncthreads();
 
-  const float yk = row_dot16(rr, &xs[0][0]);
+  // Rotation (steps a0 and a1) of every vector on this thread's row.
+  float y[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) y[v] = row_dot16(rr, &xs[v][0]);
   if (has_key) {
-    mn = fminf(mn, yk);
-    mx = fmaxf(mx, yk);
+    mn = fminf(mn, y[0]);
+    mx = fmaxf(mx, y[0]);
   }
-  if (row_lead) xpart[0][lrow] = has_key ? yk : 0.f;
   float qneg = 0.f, qpos = 0.f;
-  for (int h = 0; h < gs; ++h) {
-    const float y = row_dot16(rr, &xs[1 + h][0]);
-    qneg += fminf(y, 0.f);
-    qpos += fmaxf(y, 0.f);
-    if (row_lead) {
-      xpart[1 + h][lrow] = y;
-      a.q_rot[((size_t)b * a.Hq + g * gs + h) * kD + row] = y;
+#pragma unroll
+  for (int h = 0; h < GS; ++h) {
+    qneg += fminf(y[1 + h], 0.f);
+    qpos += fmaxf(y[1 + h], 0.f);
+  }
+  if (row_lead) {
+#pragma unroll
+    for (int v = 0; v < NV; ++v) xpart[v][lrow] = v == 0 && !has_key ? 0.f : y[v];
+  }
+#pragma unroll
+  for (int h = 0; h < GS; ++h)
+    if (h == part) a.q_rot[((size_t)b * a.Hq + g * GS + h) * kD + row] = y[1 + h];
+  __syncthreads();
+  // Every rank's copy of the rotated vectors receives this CTA's rows: thread i sends
+  // 16-byte piece j of vector v to rank r.
+  if (tid < NV * 8 * kPrologueRanks) {
+    const int v = tid / (8 * kPrologueRanks), r = (tid / 8) % kPrologueRanks, j = tid % 8;
+    const float4 val = reinterpret_cast<const float4*>(&xpart[v][0])[j];
+    reinterpret_cast<float4*>(cl.map_shared_rank(&xr[v][0], r))[rank * 8 + j] = val;
+  }
+  cluster_sync_all();  // every rank's rows of every rotated vector have landed
+
+  // LHP codes: the sign of W_g x' on this thread's row is bit lrow of code word `rank`.
+  // Warp w holds rows 2w and 2w + 1: an OR-reduction collects the warp's two bits, and
+  // warp 0 merges the warps' pieces.
+  const int lane = tid & 31, warp = tid >> 5;
+  float pj[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) pj[v] = row_dot16(wr, &xr[v][0]);
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const uint32_t bits = __reduce_or_sync(kFull, row_lead && pj[v] > 0.f ? 1u << lrow : 0u);
+    if (lane == 0) cpart[v][warp] = bits;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const uint32_t word =
+          __reduce_or_sync(kFull, lane < kPrologueThreads / 32 ? cpart[v][lane] : 0u);
+      if (lane == v) mine = word;
     }
-  }
-  cl.sync();  // every CTA's rotated rows are ready
-  for (int i = tid; i < (1 + gs) * kD; i += kPrologueThreads) {
-    const int v = i / kD, c = i % kD;
-    xr[v][c] = cl.map_shared_rank(&xpart[0][0], c >> 5)[v * 32 + (c & 31)];
-  }
-  __syncthreads();
-  for (int v = 0; v <= gs; ++v) {
-    const float p = row_dot16(wr, &xr[v][0]);
-    if (row_lead && p > 0.f) atomicOr(&cword[v], 1u << lrow);
-  }
-  __syncthreads();
-  if (tid <= gs) {
-    const uint32_t word = cword[tid];
-    if (tid == 0) {
-      if (has_key) a.codes[(((size_t)s.phys * a.G + g) * a.P + s.slot) * kWords + rank] = word;
-    } else {
-      a.q_code[((size_t)b * a.Hq + g * gs + (tid - 1)) * kWords + rank] = word;
+    if (lane == 0) {
+      if (has_key) a.codes[(((size_t)s.phys * a.G + g) * a.P + s.slot) * kWords + rank] = mine;
+    } else if (lane < NV) {
+      a.q_code[((size_t)b * a.Hq + g * GS + (lane - 1)) * kWords + rank] = mine;
     }
   }
   if (row_lead) {
@@ -279,7 +223,22 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
     o[row] = qneg;
     o[kD + row] = qpos;
   }
-  cl.sync();  // keep xpart alive until every CTA has read it
+}
+
+using PrologueFn = void (*)(PrologueArgs);
+
+// The instantiation for group size gs (1..kMaxGroup).
+inline PrologueFn step_prologue_for(int gs) {
+  switch (gs) {
+    case 1: return step_prologue_cluster_kernel<1>;
+    case 2: return step_prologue_cluster_kernel<2>;
+    case 3: return step_prologue_cluster_kernel<3>;
+    case 4: return step_prologue_cluster_kernel<4>;
+    case 5: return step_prologue_cluster_kernel<5>;
+    case 6: return step_prologue_cluster_kernel<6>;
+    case 7: return step_prologue_cluster_kernel<7>;
+    default: return step_prologue_cluster_kernel<8>;
+  }
 }
 
 }  // namespace hhr

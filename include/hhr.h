@@ -16,10 +16,14 @@
  *   - Every pointer argument is a DEVICE pointer unless its comment says "host".
  *     The caller owns every buffer. The library never allocates or frees memory
  *     and never synchronises, except hhr_read_device_status.
+ *   - Every device buffer starts on a 16-byte boundary (cudaMalloc gives 256);
+ *     a misaligned pointer returns HHR_ERR_INVALID_ARG. Workspaces start on a
+ *     256-byte boundary.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).
  *   - Host-side validation runs first and returns an error before any launch:
- *     HHR_ERR_INVALID_ARG (null pointer, negative size, H % G != 0, ...),
+ *     HHR_ERR_INVALID_ARG (null or misaligned pointer, negative size,
+ *     H % G != 0, ...),
  *     HHR_ERR_UNSUPPORTED (head_dim != 128, code_bits != 128, group > 8, a size
  *     beyond a documented limit), HHR_ERR_WORKSPACE (workspace too small).
  *     A failed launch returns HHR_ERR_CUDA.

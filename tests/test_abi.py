@@ -127,3 +127,23 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(hhr, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         hhr.lib()
+
+
+def test_misaligned_pointers_rejected(L):
+    """Device buffers must start on a 16-byte boundary (checked before any launch)."""
+    d = _d()
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(256 + 8)
+    a = [p] * 7
+    assert L.hhr_sparse_attn(ctypes.byref(d), bad, *a[1:], 2048, ctypes.c_float(0.1), p, p,
+                             1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_encode_keys(ctypes.byref(d), bad, p, p, p, 1, p, p, p, p, None,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, 1, p, bad, p, p, None,
+                             None) == hhr.HHR_ERR_INVALID_ARG
+    step = [p, bad, bad, p, p, p, p, p, p, p, p]  # q, k_new, v_new, k/v cache, ..., codes
+    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, ctypes.c_float(0.1), p, p, p,
+                             p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    step = [p] * 11
+    step[7] = bad  # R
+    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, ctypes.c_float(0.1), p, p, p,
+                             p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG

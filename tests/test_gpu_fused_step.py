@@ -25,8 +25,21 @@ def _prefill(wl, inp, d, upto):
 @pytest.mark.parametrize("f16", [0, 1])
 @pytest.mark.parametrize("with_new_rows", [False, True])
 def test_fused_step_equals_separate_calls(f16, with_new_rows):
-    build.build()
     wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=5, ragged=(33, 6000), top_k=300)
+    _fused_vs_separate(wl, f16, with_new_rows)
+
+
+@pytest.mark.parametrize("heads", [(8, 1), (8, 8), (10, 2), (6, 2), (14, 2)])
+def test_fused_step_group_shapes(heads):
+    """Every group size has its own prologue instantiation: each must match."""
+    hq, g = heads
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=3, ragged=(33, 4000), top_k=200,
+                  n_q_heads=hq, n_kv_heads=g)
+    _fused_vs_separate(wl, 1, True)
+
+
+def _fused_vs_separate(wl, f16, with_new_rows):
+    build.build()
     inp = S.make_inputs(wl, device="cuda")
     d = dims_of(wl, inp, f16)
     lens = inp["seq_len"]
