@@ -334,7 +334,19 @@ struct PageResolve {
   const int32_t* ptab;  // the sequence's page-table row, or null
   int n_phys;
   int32_t* out_phys;    // parallel to `out`
+  // When code_g is set, the code block of every kept page (code_bytes at code_g +
+  // phys * code_page_words) is prefetched into L2 as soon as the page is kept.
+  const uint32_t* code_g;
+  size_t code_page_words;
+  unsigned code_bytes;
 };
+
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
+constexpr int kSelPtabPrefetch = 4;  // page-table entries of a thread loaded up front (the
+                                     // compaction below reads pt[0..3] by name)
 
 constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 
@@ -346,10 +358,16 @@ constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
                                     bool by_kept, int m_pages, int keep_div, int top_k,
                                     int32_t* out, int out_stride, const int32_t* kept_units,
-                                    int unit, PageResolve pr = PageResolve{nullptr, 0, nullptr}) {
+                                    int unit,
+                                    PageResolve pr = PageResolve{nullptr, 0, nullptr, nullptr, 0, 0}) {
   const int tid = threadIdx.x;
   const int per = ceil_div(n, kSelThreads);
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+  // The first page-table entries of this thread's compaction range, loaded with the scores.
+  int pt[kSelPtabPrefetch];
+#pragma unroll
+  for (int k = 0; k < kSelPtabPrefetch; ++k)
+    pt[k] = (pr.out_phys != nullptr && i0 + k < i1) ? pr.ptab[i0 + k] : -1;
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int base = 0; base < n; base += kSelLoadUnroll * kSelThreads) {
@@ -466,10 +484,14 @@ __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelS
         if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
         out[pos] = v;
         if (pr.out_phys != nullptr) {
-          int phys = pr.ptab[v];
+          const int kq = i - i0;
+          int phys = kq == 0 ? pt[0] : kq == 1 ? pt[1] : kq == 2 ? pt[2] : kq == 3 ? pt[3]
+                                                                            : pr.ptab[v];
           if (phys < 0 || phys >= pr.n_phys) {
             flag_status(kStatusBadPage);
             phys = -1;
+          } else if (pr.code_g != nullptr) {
+            prefetch_l2(pr.code_g + (size_t)phys * pr.code_page_words, pr.code_bytes);
           }
           pr.out_phys[pos] = phys;
         }
@@ -545,26 +567,27 @@ struct QueryPlanes {
   uint32_t z[kWords][NB];  // bit planes of #heads with a 0 bit
 };
 
-// Bit-sliced counts over the gs query codes qc[h*4 + w] (ripple-carry adds of one bit
-// vector per head).
+// One plane set of the bit-sliced counts: thread (kind, w) adds, with ripple carries, the
+// bit vector of word w of every head's query code (q_code_w[h * 4], kind 0) or of its
+// complement (kind 1). Result: out[b] for b < NB.
 template <int NB>
-__device__ __forceinline__ void build_query_planes(const uint32_t* qc, int gs, QueryPlanes<NB>& p) {
+__device__ __forceinline__ void build_plane_word(const uint32_t* q_code_w, int gs, int kind,
+                                                 uint32_t* out) {
+  uint32_t pl[NB];
 #pragma unroll
-  for (int w = 0; w < kWords; ++w) {
+  for (int b = 0; b < NB; ++b) pl[b] = 0u;
+  for (int h = 0; h < gs; ++h) {
+    uint32_t c = q_code_w[h * kWords];
+    if (kind) c = ~c;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) { p.n[w][b] = 0u; p.z[w][b] = 0u; }
-    for (int h = 0; h < gs; ++h) {
-      uint32_t cn = qc[h * kWords + w], cz = ~cn;
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const uint32_t tn = p.n[w][b] & cn, tz = p.z[w][b] & cz;
-        p.n[w][b] ^= cn;
-        p.z[w][b] ^= cz;
-        cn = tn;
-        cz = tz;
-      }
+    for (int b = 0; b < NB; ++b) {
+      const uint32_t t = pl[b] & c;
+      pl[b] ^= c;
+      c = t;
     }
   }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) out[b] = pl[b];
 }
 
 template <int NB>
@@ -596,8 +619,8 @@ struct HamShared {
 // hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
 template <int NB>
 __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
-                                     const int32_t* kphys, int m, const uint32_t* qc,
-                                     uint32_t* hsm, HamShared& hs) {
+                                     const int32_t* kphys, int m, const uint32_t* qcs,
+                                     uint32_t (*planes)[kWords][4], uint32_t* hsm, HamShared& hs) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int b = row / a.G, g = row % a.G;
@@ -614,9 +637,20 @@ __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, co
   const int Cr = hi - lo;
   for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
   if (tid == 0) { hs.T = -1; hs.need_eq = 0; }
+  if (tid < 2 * kWords) {
+    const int kind = tid / kWords, w = tid % kWords;
+    build_plane_word<NB>(qcs + w, gs, kind, &planes[kind][w][0]);
+  }
+  __syncthreads();  // histogram zeroed, planes built
   QueryPlanes<NB> qp;
-  build_query_planes<NB>(qc, gs, qp);
-  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+    for (int pb = 0; pb < NB; ++pb) {
+      qp.n[w][pb] = planes[0][w][pb];
+      qp.z[w][pb] = planes[1][w][pb];
+    }
+  }
   // Candidates c = lo + tid + j*1024: consecutive threads read consecutive 16-byte codes of
   // a page (coalesced); all ham_load() code loads of a thread are issued before any math.
   // c / P by multiply-high: exact for c < 2^24 with magic = floor(2^32 / P) + 1.
@@ -761,7 +795,8 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
     topm_hamming_kernel(TopmHammingArgs a) {
   __shared__ SelShared sh;
   __shared__ HamShared hs;
-  __shared__ uint32_t qcs[kMaxGroup * kWords];
+  __shared__ uint32_t qcs[kMaxGroup * kWords];     // the group's query codes
+  __shared__ uint32_t planes[2][kWords][4];         // their bit planes
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t fsm[];
@@ -769,7 +804,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
   const int b = row / h.G, g = row % h.G;
   const int gs = h.Hq / h.G;
-  if (threadIdx.x < gs * kWords)
+  if (threadIdx.x < gs * kWords)  // visible after the selection's first barrier
     qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + g * gs) * kWords + threadIdx.x];
   const int mw = (h.m_max + 3) & ~3;
   int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
@@ -778,14 +813,17 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
   const int m = block_select_largest(
       a.bounds + (size_t)row * h.maxp, n, work, sh, true, a.m_pages, a.keep_div, 0, kept_s,
-      h.m_max, nullptr, 0, PageResolve{h.page_table + (size_t)b * h.maxp, h.n_phys, kphys_s});
+      h.m_max, nullptr, 0,
+      PageResolve{h.page_table + (size_t)b * h.maxp, h.n_phys, kphys_s,
+                  h.codes + (size_t)g * h.P * kWords, (size_t)h.G * h.P * kWords,
+                  (unsigned)(h.P * kWords * 4)});
   __syncthreads();
   if (rank == 0) {
     int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
     for (int i = threadIdx.x; i < m; i += kHamThreads) kept_g[i] = kept_s[i];
     if (threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
   }
-  hamming_topk_cluster<NB>(h, row, rank, kept_s, kphys_s, m, qcs, work, hs);
+  hamming_topk_cluster<NB>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
 }
 
 inline size_t topm_hamming_smem(int gs, int m_max, int P, int maxp) {
