@@ -47,6 +47,8 @@ struct AttnArgs {
   float* out;               // [B][Hq][d]                 (n_splits == 1)
   float scale_log2;
   int Hq, G, P, maxp, n_phys, top_k, n_splits, split_rows;
+  const uint32_t* rows;     // [B][G][top_k] cache rows of the selected keys, already
+                            // resolved and checked (fused step); null: resolve from idx
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -137,7 +139,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   // Cache row index (phys*G + g)*P + slot of each of the split's rows (kNoRow: skip).
   for (int r = tid; r < ntiles * kTile; r += kAttnThreads) {
     uint32_t o = kNoRow;
-    if (r < nrows) {
+    if (r < nrows && a.rows != nullptr) {
+      o = a.rows[(size_t)row * a.top_k + base + r];
+    } else if (r < nrows) {
       const int t = a.idx[(size_t)row * a.top_k + base + r];
       const int lp = t / a.P;
       if (t >= 0 && t < n && lp < a.maxp) {

@@ -460,7 +460,8 @@ size_t hhr_decode_step_workspace_bytes(const hhr_dims* d, int m_pages, int keep_
   const size_t sel = hhr_select_workspace_bytes(d, HHR_MODE_HASH, m_pages, keep_div, top_k);
   const size_t att = hhr_attn_workspace_bytes(d, top_k);
   if (sel == 0 || att == 0) return 0;
-  return sel + att;
+  // + the cache row of every selected key, handed from the selection to the attention.
+  return sel + att + align256((size_t)d->batch * d->n_kv_heads * top_k * 4);
 }
 
 int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
@@ -503,6 +504,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   const int ns = plan.n_splits;
   float* part_o = reinterpret_cast<float*>(aws);
   float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
+  uint32_t* sel_rows = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
   const size_t fsm = topm_hamming_smem(gs, m_max, P, maxp);
   if (allow_smem(topm_hamming_for(gs), fsm, g_smem_ham[hamming_planes(gs) - 1]) != cudaSuccess)
     return HHR_ERR_CUDA;
@@ -535,7 +537,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   // a2 top-m + a3 + a4: kept pages, Hamming distances, deterministic top-k.
   {
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows};
     prof_begin(HHR_KERNEL_HAMMING, s);
     e = launch_pdl(topm_hamming_for(gs), dim3(B * G * kHamRanks), dim3(kHamThreads), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div});
@@ -549,7 +551,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     if (cp.n_splits <= kMaxClusterSplits) {
       AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, nullptr, nullptr,
                   out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k,
-                  cp.n_splits, cp.split_rows};
+                  cp.n_splits, cp.split_rows, sel_rows};
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cp.n_splits, G, B);
       cfg.blockDim = dim3(kAttnThreads);
@@ -571,7 +573,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     } else {
       AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, part_o, part_ml,
                   out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k, ns,
-                  plan.split_rows};
+                  plan.split_rows, sel_rows};
       prof_begin(HHR_KERNEL_ATTN, s);
       e = launch_pdl(sparse_attn_kernel<false>, dim3(ns, G, B), dim3(kAttnThreads), attn_smem(),
                      s, aa);

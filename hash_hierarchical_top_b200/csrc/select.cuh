@@ -557,6 +557,8 @@ struct HammingArgs {
   int32_t* out_idx;          // [B][G][top_k]
   int32_t* out_count;        // [B][G]
   int Hq, G, P, maxp, n_phys, m_max, top_k;
+  uint32_t* out_rows;        // [B][G][top_k] cache row (phys*G + g)*P + slot of each selected
+                             // key, for the attention of the fused step; or null
 };
 
 inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
@@ -762,7 +764,12 @@ __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, co
         if (take && pos < a.top_k) {
           const int i = lo + i0 + q;
           const int pi = (a.P == 1) ? i : (int)__umulhi((uint32_t)i, magic);
-          out[pos++] = klp[pi] * a.P + (i - pi * a.P);
+          const int slot = i - pi * a.P;
+          out[pos] = klp[pi] * a.P + slot;
+          if (a.out_rows != nullptr)
+            a.out_rows[(size_t)row * a.top_k + pos] =
+                ((uint32_t)kphys[pi] * (uint32_t)a.G + (uint32_t)g) * (uint32_t)a.P + (uint32_t)slot;
+          ++pos;
         }
       }
     }
