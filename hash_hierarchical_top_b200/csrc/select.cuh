@@ -345,41 +345,44 @@ __device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
 }
 
-constexpr int kSelPtabPrefetch = 4;  // page-table entries of a thread loaded up front (the
-                                     // compaction below reads pt[0..3] by name)
+
 
 constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 
-// Block-wide selection (kSelThreads threads, call uniformly): the k largest finite scores
+// Block-wide selection (NT threads, call uniformly): the k largest finite scores
 // of sc[0..n), ties to the lower index, written in ascending index order to out[0..k)
 // (global or shared memory). k = kept_for(#finite, m_pages, keep_div) when by_kept, else
 // min(top_k, #finite). unit > 0 maps index i to kept_units[i / unit] * unit + i % unit.
 // keys: shared scratch of n words (16-byte aligned). Returns k.
-__device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
+template <int NT = kSelThreads>
+__device__ __forceinline__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
                                     bool by_kept, int m_pages, int keep_div, int top_k,
                                     int32_t* out, int out_stride, const int32_t* kept_units,
                                     int unit,
                                     PageResolve pr = PageResolve{nullptr, 0, nullptr, nullptr, 0, 0}) {
   const int tid = threadIdx.x;
-  const int per = ceil_div(n, kSelThreads);
+  // Page-table entries of a thread's compaction range loaded with the scores (all of them
+  // up to 4096 pages).
+  constexpr int kPre = 4096 / NT;
+  const int per = ceil_div(n, NT);
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
   // The first page-table entries of this thread's compaction range, loaded with the scores.
-  int pt[kSelPtabPrefetch];
+  int pt[kPre];
 #pragma unroll
-  for (int k = 0; k < kSelPtabPrefetch; ++k)
+  for (int k = 0; k < kPre; ++k)
     pt[k] = (pr.out_phys != nullptr && i0 + k < i1) ? pr.ptab[i0 + k] : -1;
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int base = 0; base < n; base += kSelLoadUnroll * kSelThreads) {
+  for (int base = 0; base < n; base += kSelLoadUnroll * NT) {
     float f[kSelLoadUnroll];
 #pragma unroll
     for (int j = 0; j < kSelLoadUnroll; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NT + tid;
       f[j] = i < n ? sc[i] : -INFINITY;
     }
 #pragma unroll
     for (int j = 0; j < kSelLoadUnroll; ++j) {
-      const int i = base + j * kSelThreads + tid;
+      const int i = base + j * NT + tid;
       const bool fin = f[j] > -INFINITY;
       const uint32_t kk = fin ? f2key(f[j]) : 0u;
       if (i < n) keys[i] = kk;
@@ -412,7 +415,7 @@ __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelS
       while (true) {
         if (tid < 256) sh.hist[tid] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kSelThreads) {
+        for (int i = tid; i < n; i += NT) {
           const uint32_t kk = keys[i];
           if (kk != 0u && (kk & mask) == prefix) atomicAdd(&sh.hist[(kk >> shift) & 255], 1);
         }
@@ -473,27 +476,45 @@ __device__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelS
   int2 tot;
   const int2 before = block_excl_scan2(make_int2(gt, eq), sh.scratch, &tot);
   if (k > 0) {
+    // Keys are visited in chunks of 32: a take mask (keys above the threshold, then the
+    // first equal ones while fewer than rem equal keys precede them) is built from shared
+    // memory, and only its set bits do the writes, in ascending order.
     int e = before.y;
     int pos = before.x + min(e, rem);
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t kk = keys[i];
-      bool take = take_gt(kk);
-      if (!take && !whole_bin && kk == prefix) { take = e < rem; ++e; }
-      if (take && pos < out_stride) {
-        int v = i;
-        if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
-        out[pos] = v;
-        if (pr.out_phys != nullptr) {
-          const int kq = i - i0;
-          int phys = kq == 0 ? pt[0] : kq == 1 ? pt[1] : kq == 2 ? pt[2] : kq == 3 ? pt[3]
-                                                                            : pr.ptab[v];
-          if (phys < 0 || phys >= pr.n_phys) {
-            flag_status(kStatusBadPage);
-            phys = -1;
-          } else if (pr.code_g != nullptr) {
-            prefetch_l2(pr.code_g + (size_t)phys * pr.code_page_words, pr.code_bytes);
+    for (int c0 = i0; c0 < i1; c0 += 32) {
+      const int c1 = min(i1, c0 + 32);
+      uint32_t takem = 0u, eqm = 0u;
+      for (int i = c0; i < c1; ++i) {
+        const uint32_t kk = keys[i];
+        const uint32_t bit = 1u << (i - c0);
+        if (take_gt(kk)) takem |= bit;
+        else if (!whole_bin && kk == prefix) eqm |= bit;
+      }
+      for (int want = rem - e; eqm != 0u; eqm &= eqm - 1u, ++e, --want)
+        if (want > 0) takem |= eqm & (0u - eqm);
+      while (takem != 0u) {
+        const int i = c0 + __ffs(takem) - 1;
+        takem &= takem - 1u;
+        if (pos < out_stride) {
+          int v = i;
+          if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
+          out[pos] = v;
+          if (pr.out_phys != nullptr) {
+            const int kq = i - i0;
+            int phys = 0;
+            bool pre = false;
+#pragma unroll
+            for (int kp = 0; kp < kPre; ++kp)
+              if (kq == kp) { phys = pt[kp]; pre = true; }
+            if (!pre) phys = pr.ptab[v];
+            if (phys < 0 || phys >= pr.n_phys) {
+              flag_status(kStatusBadPage);
+              phys = -1;
+            } else if (pr.code_g != nullptr) {
+              prefetch_l2(pr.code_g + (size_t)phys * pr.code_page_words, pr.code_bytes);
+            }
+            pr.out_phys[pos] = phys;
           }
-          pr.out_phys[pos] = phys;
         }
         ++pos;
       }
@@ -539,13 +560,13 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 // code word as NB bit planes (NB = bit width of gs), so one select per plane and word
 // gives the contributions' bits, and a carry-save step over the 4 words leaves 3
 // popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
-constexpr int kHamThreads = 1024;
+constexpr int kHamThreads = 512;
 constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
 // Code loads in flight per thread (fewer with 4 planes, whose 32 plane words fill registers).
 template <int NB>
-constexpr int ham_load() { return NB >= 4 ? 2 : 4; }
+constexpr int ham_load() { return NB >= 4 ? 4 : 8; }
 constexpr int kMaxCand = 65536;
-static_assert(kMaxGroup * 128 + 1 <= 2 * kHamThreads, "threshold search covers 2 bins a thread");
+constexpr int kHamBins = (kMaxGroup * 128 + 1 + kHamThreads - 1) / kHamThreads;  // per thread
 
 struct HammingArgs {
   const uint32_t* q_code;    // [B][Hq][4]
@@ -620,7 +641,7 @@ struct HamShared {
 // compaction offsets are combined through distributed shared memory.
 // hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
 template <int NB>
-__device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
+__device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
                                      const int32_t* kphys, int m, const uint32_t* qcs,
                                      uint32_t (*planes)[kWords][4], uint32_t* hsm, HamShared& hs) {
   namespace cg = cooperative_groups;
@@ -687,12 +708,12 @@ __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, co
   }
   cluster_sync_all();  // every rank's histogram is complete
   // Threshold bucket: smallest T with #(delta <= T) >= k_eff over the summed histograms.
-  // Thread t holds bins [2t, 2t+2) (fewer past nbins).
+  // Thread t holds bins [kHamBins t, kHamBins (t + 1)) (fewer past nbins).
   {
-    int hv[2], sum = 0;
+    int hv[kHamBins], sum = 0;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int i = 2 * tid + q;
+    for (int q = 0; q < kHamBins; ++q) {
+      const int i = kHamBins * tid + q;
       hv[q] = 0;
       if (i < nbins) {
 #pragma unroll
@@ -704,9 +725,17 @@ __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, co
     const int excl = block_excl_scan(sum, hs.scratch, &nvalid);
     const int keff = min(a.top_k, nvalid);
     if (keff > 0 && excl < keff && keff <= excl + sum) {
-      const int first = keff <= excl + hv[0] ? 0 : 1;
-      hs.T = 2 * tid + first;
-      hs.need_eq = keff - excl - (first ? hv[0] : 0);
+      int run = excl;
+      bool found = false;
+#pragma unroll
+      for (int q = 0; q < kHamBins; ++q) {
+        if (!found && keff <= run + hv[q]) {
+          hs.T = kHamBins * tid + q;
+          hs.need_eq = keff - run;
+          found = true;
+        }
+        run += hv[q];
+      }
     }
     if (tid == 0) a.out_count[row] = keff;  // every rank writes the same value
     __syncthreads();
@@ -757,11 +786,17 @@ __device__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, co
       uint16_t dv[8];
       const int i0 = tid * cpt + gi * 8;
       load8(i0, dv);
+      uint32_t takem = 0u;  // the group's selected candidates, then visited bit by bit
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         bool take = dv[q] < T;
         if (dv[q] == T) { take = e < need_eq; ++e; }
-        if (take && pos < a.top_k) {
+        if (take) takem |= 1u << q;
+      }
+      while (takem != 0u) {
+        const int q = __ffs(takem) - 1;
+        takem &= takem - 1u;
+        if (pos < a.top_k) {
           const int i = lo + i0 + q;
           const int pi = (a.P == 1) ? i : (int)__umulhi((uint32_t)i, magic);
           const int slot = i - pi * a.P;
@@ -818,7 +853,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   int32_t* kphys_s = kept_s + mw;
   uint32_t* work = fsm + 2 * mw;
   const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
-  const int m = block_select_largest(
+  const int m = block_select_largest<kHamThreads>(
       a.bounds + (size_t)row * h.maxp, n, work, sh, true, a.m_pages, a.keep_div, 0, kept_s,
       h.m_max, nullptr, 0,
       PageResolve{h.page_table + (size_t)b * h.maxp, h.n_phys, kphys_s,
