@@ -149,8 +149,8 @@ class Clocks:
 
 
 def traffic_from_profile(kernel_src_hash, fmt):
-    """DRAM bytes per launch of the page-bound kernel from the committed ncu summary,
-    or None if the kernel source changed since the counters were taken."""
+    """(DRAM bytes, algorithmic bytes) of the profiled page-bound launch from the committed
+    ncu summary, or None if the kernel source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", f"page_bound_{fmt}_kernel_llama8b_128k_b8.txt")
     if not os.path.exists(p):
         return None
@@ -163,7 +163,7 @@ def traffic_from_profile(kernel_src_hash, fmt):
     if vals.get("kernel_source_sha256") != kernel_src_hash:
         return None
     try:
-        return float(vals["dram_bytes_per_full_launch"])
+        return float(vals["dram_bytes_per_full_launch"]), float(vals["algorithmic_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
 
@@ -577,7 +577,10 @@ def main():
     bound_bytes = bound_kernel_bytes(wl, lens, sbytes)
     bound_avg_ms = statistics.mean(bound_ms)
     achieved = bound_bytes / (bound_avg_ms / 1e3) / 1e9
-    traffic = traffic_from_profile(kernel_source_hash(), args.summary)
+    # DRAM bytes of the profiled launch, scaled to this launch's algorithmic bytes (the
+    # kernel's traffic grows in proportion to the pages it reads).
+    prof = traffic_from_profile(kernel_source_hash(), args.summary)
+    traffic = prof[0] * bound_bytes / prof[1] if prof is not None else None
     step_gbs = req / (ms_step / 1e3) / 1e9
 
     cpu = None

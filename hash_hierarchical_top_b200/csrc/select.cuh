@@ -327,50 +327,38 @@ struct SelShared {
   int digit, rem, cnt;
 };
 
-// Optional page resolution during the compaction of a page selection: the physical page
-// of every kept logical page i is read from ptab[i] and written beside it (-1, and the
-// bad-page status bit, when it is out of range).
-struct PageResolve {
-  const int32_t* ptab;  // the sequence's page-table row, or null
-  int n_phys;
-  int32_t* out_phys;    // parallel to `out`
-  // When code_g is set, the code block of every kept page (code_bytes at code_g +
-  // phys * code_page_words) is prefetched into L2 as soon as the page is kept.
-  const uint32_t* code_g;
-  size_t code_page_words;
-  unsigned code_bytes;
-};
-
 __device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
 }
 
-
-
 constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 
-// Block-wide selection (NT threads, call uniformly): the k largest finite scores
-// of sc[0..n), ties to the lower index, written in ascending index order to out[0..k)
-// (global or shared memory). k = kept_for(#finite, m_pages, keep_div) when by_kept, else
-// min(top_k, #finite). unit > 0 maps index i to kept_units[i / unit] * unit + i % unit.
-// keys: shared scratch of n words (16-byte aligned). Returns k.
-template <int NT = kSelThreads>
-__device__ __forceinline__ int block_select_largest(const float* sc, int n, uint32_t* keys, SelShared& sh,
-                                    bool by_kept, int m_pages, int keep_div, int top_k,
-                                    int32_t* out, int out_stride, const int32_t* kept_units,
-                                    int unit,
-                                    PageResolve pr = PageResolve{nullptr, 0, nullptr, nullptr, 0, 0}) {
+// Where a block selection cuts (after block_select_cut): a key kk (0 = not finite) is taken
+// when above(kk); with !whole_bin, keys equal to prefix (tie(kk)) are taken in index order
+// until rem of them are taken. k = the number taken.
+struct SelCut {
+  int k, rem, sel_shift;
+  uint32_t prefix;
+  bool whole_bin;
+  __device__ __forceinline__ bool above(uint32_t kk) const {
+    if (kk == 0u || k == 0) return false;
+    if (whole_bin) return (kk >> sel_shift) >= (prefix >> sel_shift);
+    return kk > prefix;
+  }
+  __device__ __forceinline__ bool tie(uint32_t kk) const {
+    return k > 0 && !whole_bin && kk != 0u && kk == prefix;
+  }
+};
+
+// Threshold search of a block-wide selection (NT threads, call uniformly) of the k largest
+// finite scores of sc[0..n), ties to the lower index. k = kept_for(#finite, m_pages,
+// keep_div) when by_kept, else min(top_k, #finite). Leaves the order-preserving keys of
+// the scores in keys[0..n) (shared memory, 16-byte aligned).
+template <int NT>
+__device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint32_t* keys,
+                                                   SelShared& sh, bool by_kept, int m_pages,
+                                                   int keep_div, int top_k) {
   const int tid = threadIdx.x;
-  // Page-table entries of a thread's compaction range loaded with the scores (all of them
-  // up to 4096 pages).
-  constexpr int kPre = 4096 / NT;
-  const int per = ceil_div(n, NT);
-  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
-  // The first page-table entries of this thread's compaction range, loaded with the scores.
-  int pt[kPre];
-#pragma unroll
-  for (int k = 0; k < kPre; ++k)
-    pt[k] = (pr.out_phys != nullptr && i0 + k < i1) ? pr.ptab[i0 + k] : -1;
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int base = 0; base < n; base += kSelLoadUnroll * NT) {
@@ -392,26 +380,27 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
   }
   // Also orders the key stores before any read.
   block_count_minmax(nfin, kmin, kmax, sh.mm, &nfin, &kmin, &kmax);
-  const int k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
-
+  SelCut c;
+  c.k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
   // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
   // keys at sel_shift == 0 are taken in index order until `rem` of them are taken; at
   // sel_shift > 0 the whole bin is taken (>=).
-  uint32_t prefix = 0;
-  int rem = k, sel_shift = 0;
-  bool whole_bin = false;
-  if (k > 0) {
-    if (k == nfin) {
-      whole_bin = true;            // everything finite is selected
-      prefix = kmin;
-      sel_shift = 0;
+  c.prefix = 0;
+  c.rem = c.k;
+  c.sel_shift = 0;
+  c.whole_bin = false;
+  if (c.k > 0) {
+    if (c.k == nfin) {
+      c.whole_bin = true;          // everything finite is selected
+      c.prefix = kmin;
     } else if (kmin == kmax) {
-      prefix = kmin;               // all equal: the first k in index order
+      c.prefix = kmin;             // all equal: the first k in index order
     } else {
       const int hb = 31 - __clz(kmin ^ kmax);          // highest differing bit
       int shift = max(hb - 7, 0);
       uint32_t mask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);   // common high bits
-      prefix = kmin & mask;
+      uint32_t prefix = kmin & mask;
+      int rem = c.k;
       while (true) {
         if (tid < 256) sh.hist[tid] = 0;
         __syncthreads();
@@ -422,21 +411,21 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
         __syncthreads();
         if (tid < 32) {
           // Lane l covers digits 255-8l .. 248-8l (descending).
-          int c[8], s = 0;
+          int cq[8], s = 0;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { c[q] = sh.hist[255 - 8 * tid - q]; s += c[q]; }
+          for (int q = 0; q < 8; ++q) { cq[q] = sh.hist[255 - 8 * tid - q]; s += cq[q]; }
           const int incl = warp_incl_scan(s, tid);
           const int excl = incl - s;
           if (excl < rem && rem <= incl) {
             int run = excl;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              if (run < rem && rem <= run + c[q]) {
+              if (run < rem && rem <= run + cq[q]) {
                 sh.digit = 255 - 8 * tid - q;
                 sh.rem = rem - run;
-                sh.cnt = c[q];
+                sh.cnt = cq[q];
               }
-              run += c[q];
+              run += cq[q];
             }
           }
         }
@@ -447,8 +436,8 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
         const int cnt_bin = sh.cnt;
         __syncthreads();
         if (rem == cnt_bin) {  // the whole bin is needed: no tie-break required
-          whole_bin = true;
-          sel_shift = shift;
+          c.whole_bin = true;
+          c.sel_shift = shift;
           break;
         }
         if (shift == 0) break;
@@ -456,71 +445,64 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
         // its already-fixed upper bits are constant across the candidates.
         shift = max(shift - 8, 0);
       }
+      c.prefix = prefix;
+      c.rem = rem;
     }
   }
-  // Compaction in index order. Before thread t's range are gt_before keys above the
-  // threshold and eq_before equal to it, of which the first min(eq_before, rem) are taken.
-  auto take_gt = [&](uint32_t kk) -> bool {
-    if (kk == 0u) return false;
-    if (whole_bin) return (kk >> sel_shift) >= (prefix >> sel_shift);
-    return kk > prefix;
-  };
+  return c;
+}
+
+// Block-wide selection (NT threads, call uniformly): the k largest finite scores of sc[0..n),
+// ties to the lower index, written in ascending index order to out[0..k) (global or shared
+// memory); see block_select_cut for k. unit > 0 maps index i to kept_units[i / unit] * unit
+// + i % unit. keys: shared scratch of n words (16-byte aligned). Returns k.
+template <int NT = kSelThreads>
+__device__ __forceinline__ int block_select_largest(const float* sc, int n, uint32_t* keys,
+                                                    SelShared& sh, bool by_kept, int m_pages,
+                                                    int keep_div, int top_k, int32_t* out,
+                                                    int out_stride, const int32_t* kept_units,
+                                                    int unit) {
+  const int tid = threadIdx.x;
+  const SelCut c = block_select_cut<NT>(sc, n, keys, sh, by_kept, m_pages, keep_div, top_k);
+  // Compaction in index order over contiguous per-thread ranges. Before thread t's range
+  // are gt_before keys above the cut and eq_before equal to it, of which the first
+  // min(eq_before, rem) are taken.
+  const int per = ceil_div(n, NT);
+  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
   int eq = 0, gt = 0;
-  if (k > 0) {
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t kk = keys[i];
-      if (take_gt(kk)) ++gt;
-      else if (!whole_bin && kk == prefix) ++eq;
-    }
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t kk = keys[i];
+    if (c.above(kk)) ++gt;
+    else if (c.tie(kk)) ++eq;
   }
   int2 tot;
   const int2 before = block_excl_scan2(make_int2(gt, eq), sh.scratch, &tot);
-  if (k > 0) {
-    // Keys are visited in chunks of 32: a take mask (keys above the threshold, then the
-    // first equal ones while fewer than rem equal keys precede them) is built from shared
+  if (c.k > 0) {
+    // Keys are visited in chunks of 32: a take mask (keys above the cut, then the first
+    // equal ones while fewer than rem equal keys precede them) is built from shared
     // memory, and only its set bits do the writes, in ascending order.
     int e = before.y;
-    int pos = before.x + min(e, rem);
+    int pos = before.x + min(e, c.rem);
     for (int c0 = i0; c0 < i1; c0 += 32) {
       const int c1 = min(i1, c0 + 32);
       uint32_t takem = 0u, eqm = 0u;
       for (int i = c0; i < c1; ++i) {
         const uint32_t kk = keys[i];
         const uint32_t bit = 1u << (i - c0);
-        if (take_gt(kk)) takem |= bit;
-        else if (!whole_bin && kk == prefix) eqm |= bit;
+        if (c.above(kk)) takem |= bit;
+        else if (c.tie(kk)) eqm |= bit;
       }
-      for (int want = rem - e; eqm != 0u; eqm &= eqm - 1u, ++e, --want)
+      for (int want = c.rem - e; eqm != 0u; eqm &= eqm - 1u, ++e, --want)
         if (want > 0) takem |= eqm & (0u - eqm);
       while (takem != 0u) {
         const int i = c0 + __ffs(takem) - 1;
         takem &= takem - 1u;
-        if (pos < out_stride) {
-          int v = i;
-          if (unit > 0) v = kept_units[i / unit] * unit + i % unit;
-          out[pos] = v;
-          if (pr.out_phys != nullptr) {
-            const int kq = i - i0;
-            int phys = 0;
-            bool pre = false;
-#pragma unroll
-            for (int kp = 0; kp < kPre; ++kp)
-              if (kq == kp) { phys = pt[kp]; pre = true; }
-            if (!pre) phys = pr.ptab[v];
-            if (phys < 0 || phys >= pr.n_phys) {
-              flag_status(kStatusBadPage);
-              phys = -1;
-            } else if (pr.code_g != nullptr) {
-              prefetch_l2(pr.code_g + (size_t)phys * pr.code_page_words, pr.code_bytes);
-            }
-            pr.out_phys[pos] = phys;
-          }
-        }
+        if (pos < out_stride) out[pos] = unit > 0 ? kept_units[i / unit] * unit + i % unit : i;
         ++pos;
       }
     }
   }
-  return k;
+  return c.k;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
@@ -560,11 +542,11 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 // code word as NB bit planes (NB = bit width of gs), so one select per plane and word
 // gives the contributions' bits, and a carry-save step over the 4 words leaves 3
 // popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
-constexpr int kHamThreads = 512;
+constexpr int kHamThreads = 1024;
 constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
 // Code loads in flight per thread (fewer with 4 planes, whose 32 plane words fill registers).
 template <int NB>
-constexpr int ham_load() { return NB >= 4 ? 4 : 8; }
+constexpr int ham_load() { return NB >= 4 ? 2 : 4; }
 constexpr int kMaxCand = 65536;
 constexpr int kHamBins = (kMaxGroup * 128 + 1 + kHamThreads - 1) / kHamThreads;  // per thread
 
@@ -832,6 +814,16 @@ struct TopmHammingArgs {
   int m_pages, keep_div;
 };
 
+// Per-warp ballots of the kept-page pass of topm_hamming_kernel.
+constexpr int kTopmWarps = kHamThreads / 32;
+constexpr int kTopmChunks = 32;   // 32-page chunks per warp: up to 32 * 32 * 32 = 32768 pages
+constexpr int kTopmPtPre = 4;     // chunks whose page-table entries are loaded up front
+struct TopmShared {
+  uint32_t bal[kTopmWarps][kTopmChunks][2];  // (above, tie) ballots per warp and chunk
+  int cnt[kTopmWarps][2];                    // per-warp counts, then their exclusive prefix
+};
+static_assert(kTopmWarps == 32, "the warp-prefix scan covers 32 warps with one warp");
+
 template <int NB>
 __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
     topm_hamming_kernel(TopmHammingArgs a) {
@@ -839,6 +831,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   __shared__ HamShared hs;
   __shared__ uint32_t qcs[kMaxGroup * kWords];     // the group's query codes
   __shared__ uint32_t planes[2][kWords][4];         // their bit planes
+  __shared__ TopmShared ts;
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t fsm[];
@@ -853,18 +846,83 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   int32_t* kphys_s = kept_s + mw;
   uint32_t* work = fsm + 2 * mw;
   const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
-  const int m = block_select_largest<kHamThreads>(
-      a.bounds + (size_t)row * h.maxp, n, work, sh, true, a.m_pages, a.keep_div, 0, kept_s,
-      h.m_max, nullptr, 0,
-      PageResolve{h.page_table + (size_t)b * h.maxp, h.n_phys, kphys_s,
-                  h.codes + (size_t)g * h.P * kWords, (size_t)h.G * h.P * kWords,
-                  (unsigned)(h.P * kWords * 4)});
-  __syncthreads();
-  if (rank == 0) {
-    int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
-    for (int i = threadIdx.x; i < m; i += kHamThreads) kept_g[i] = kept_s[i];
-    if (threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
+  // Kept pages: warp w owns pages [w R, (w + 1) R), R a multiple of 32, visited 32 at a time
+  // (page w R + 32 j + lane), so that kept flags come from ballots and kept positions from
+  // popcounts; every lane with a kept page then does its writes at once.
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int R = ceil_div(ceil_div(n, kTopmWarps), 32) * 32;
+  const int J = R / 32;
+  const int wbase = warp * R;
+  const int32_t* ptab = h.page_table + (size_t)b * h.maxp;
+  int pt[kTopmPtPre];  // page-table entries of the first chunks, loaded with the bounds
+#pragma unroll
+  for (int j = 0; j < kTopmPtPre; ++j) {
+    const int p = wbase + 32 * j + lane;
+    pt[j] = (j < J && p < n) ? ptab[p] : -1;
   }
+  const SelCut cut = block_select_cut<kHamThreads>(a.bounds + (size_t)row * h.maxp, n, work, sh,
+                                                   true, a.m_pages, a.keep_div, 0);
+  int ng = 0, ne = 0;
+  for (int j = 0; j < J; ++j) {
+    const int p = wbase + 32 * j + lane;
+    const uint32_t kk = p < n ? work[p] : 0u;
+    const uint32_t bg = __ballot_sync(kFull, cut.above(kk));
+    const uint32_t be = __ballot_sync(kFull, cut.tie(kk));
+    if (lane == 0) {
+      ts.bal[warp][j][0] = bg;
+      ts.bal[warp][j][1] = be;
+    }
+    ng += __popc(bg);
+    ne += __popc(be);
+  }
+  if (lane == 0) {
+    ts.cnt[warp][0] = ng;
+    ts.cnt[warp][1] = ne;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive prefix over the warps of (above, tie) counts
+    const int xg = ts.cnt[lane][0], xe = ts.cnt[lane][1];
+    const int ig = warp_incl_scan(xg, lane), ie = warp_incl_scan(xe, lane);
+    ts.cnt[lane][0] = ig - xg;
+    ts.cnt[lane][1] = ie - xe;
+  }
+  __syncthreads();
+  const int m = cut.k;
+  int e = ts.cnt[warp][1];                 // ties before this warp's pages
+  int pos = ts.cnt[warp][0] + min(e, cut.rem);
+  int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
+  const uint32_t* code_g = h.codes + (size_t)g * h.P * kWords;
+  const size_t code_page = (size_t)h.G * h.P * kWords;
+  for (int j = 0; j < J; ++j) {
+    uint32_t takem = ts.bal[warp][j][0];
+    uint32_t be = ts.bal[warp][j][1];
+    for (int want = cut.rem - e; be != 0u; be &= be - 1u, ++e, --want)  // ties in index order
+      if (want > 0) takem |= be & (0u - be);
+    if ((takem >> lane) & 1u) {
+      const int kpos = pos + __popc(takem & ((1u << lane) - 1u));
+      const int p = wbase + 32 * j + lane;
+      int phys = 0;
+      bool pre = false;
+#pragma unroll
+      for (int q = 0; q < kTopmPtPre; ++q)
+        if (j == q) { phys = pt[q]; pre = true; }
+      if (!pre) phys = ptab[p];
+      if (phys < 0 || phys >= h.n_phys) {
+        flag_status(kStatusBadPage);
+        phys = -1;
+      } else {
+        prefetch_l2(code_g + (size_t)phys * code_page, (unsigned)(h.P * kWords * 4));
+      }
+      if (kpos < h.m_max) {
+        kept_s[kpos] = p;
+        kphys_s[kpos] = phys;
+        if (rank == 0) kept_g[kpos] = p;
+      }
+    }
+    pos += __popc(takem);
+  }
+  if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
+  __syncthreads();
   hamming_topk_cluster<NB>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
 }
 
