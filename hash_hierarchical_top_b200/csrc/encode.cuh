@@ -21,15 +21,21 @@ constexpr int kTS = kD + 1;
 
 // Mat-vecs with 128x128 row-major fp32 matrices (R_g, W_g) use one canonical row dot
 // product everywhere (append encoder, query prep, fused prologues), so that their results
-// are bit-identical: the 16 threads of a row (consecutive lanes) each hold float4s part and
-// part+16 of the row, multiply them with the same channels of the vector in a fixed fmaf
-// order, and sum over the 16 threads with a 4-step butterfly. With kMvThreads = 512, a
-// CTA covers 32 rows at a time: thread t owns rows 32*rb + t/16 for row blocks rb = 0..3.
+// are bit-identical: the 16 threads of a row each hold float4s part and part+16 of the row,
+// multiply them with the same channels of the vector in a fixed fmaf order, and sum over
+// the 16 parts with a 4-step butterfly (part ^ 1, ^ 2, ^ 4, ^ 8). A warp holds two rows,
+// interleaved (lane = 2 part + row & 1), so that the two rows' reads of the same vector
+// channels fall in the same quarter-warp and are served by one shared-memory broadcast.
+// With kMvThreads = 512, a CTA covers 32 rows at a time: warp w holds rows 2w and 2w + 1
+// of a 32-row block.
 constexpr int kVecChunk = 4;
 constexpr int kMvThreads = 512;
 constexpr int kRowBlocks = kD / 32;
 
-__device__ __forceinline__ int mv_lrow() { return (int)threadIdx.x >> 4; }  // 0..31
+__device__ __forceinline__ int mv_lrow() {  // 0..31
+  return (((int)threadIdx.x >> 5) << 1) | ((int)threadIdx.x & 1);
+}
+__device__ __forceinline__ int mv_part() { return ((int)threadIdx.x & 31) >> 1; }  // 0..15
 
 // Row `row` of M, this thread's part (float4s part and part + 16). The loads are volatile
 // asm so that they are issued here, at kernel start, and not sunk past later barriers to
@@ -43,14 +49,14 @@ __device__ __forceinline__ float4 ldg_f4_now(const float4* p) {
 }
 
 __device__ __forceinline__ void load_row16(const float* __restrict__ M, int row, float4 (&m)[2]) {
-  const int part = threadIdx.x & 15;
+  const int part = mv_part();
   const float4* r4 = reinterpret_cast<const float4*>(M + (size_t)row * kD);
   m[0] = ldg_f4_now(r4 + part);
   m[1] = ldg_f4_now(r4 + part + 16);
 }
 
 __device__ __forceinline__ float row_dot16(const float4 (&m)[2], const float* x) {
-  const int part = threadIdx.x & 15;
+  const int part = mv_part();
   const float4 x0 = reinterpret_cast<const float4*>(x)[part];
   const float4 x1 = reinterpret_cast<const float4*>(x)[part + 16];
   float acc = m[0].x * x0.x;
@@ -61,10 +67,10 @@ __device__ __forceinline__ float row_dot16(const float4 (&m)[2], const float* x)
   acc = fmaf(m[1].y, x1.y, acc);
   acc = fmaf(m[1].z, x1.z, acc);
   acc = fmaf(m[1].w, x1.w, acc);
-  acc += __shfl_xor_sync(kFull, acc, 1);
-  acc += __shfl_xor_sync(kFull, acc, 2);
-  acc += __shfl_xor_sync(kFull, acc, 4);
-  acc += __shfl_xor_sync(kFull, acc, 8);
+  acc += __shfl_xor_sync(kFull, acc, 2);   // part ^ 1
+  acc += __shfl_xor_sync(kFull, acc, 4);   // part ^ 2
+  acc += __shfl_xor_sync(kFull, acc, 8);   // part ^ 4
+  acc += __shfl_xor_sync(kFull, acc, 16);  // part ^ 8
   return acc;
 }
 
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   const int t0 = max(s, pstart), t1 = min(e, pstart + P);
   const uint16_t* kpage = a.k_cache + ((size_t)phys * G + g) * P * kD;
   const int lrow = mv_lrow();
-  const bool row_lead = (tid & 15) == 0;
+  const bool row_lead = mv_part() == 0;
 
   if (a.R != nullptr) {
     // R_g and W_g rows of this thread, and the page's stored summary when the page already

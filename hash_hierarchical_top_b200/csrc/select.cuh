@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
   __shared__ uint32_t cword[kMaxGroup][kWords];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lrow = mv_lrow();
-  const bool row_lead = (tid & 15) == 0;
+  const bool row_lead = mv_part() == 0;
   const int gs = a.Hq / a.G;
   // R_g and W_g rows of this thread are fetched up front (one memory latency for both).
   float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];

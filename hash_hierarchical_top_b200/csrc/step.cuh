@@ -121,7 +121,7 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int lrow = mv_lrow(), part = tid & 15;
+  const int lrow = mv_lrow(), part = mv_part();
   const int row = rank * 32 + lrow;
   const bool row_lead = part == 0;
 
@@ -131,7 +131,7 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   const int len = a.seq_len[b];
   // Threads [16v, 16v + 16) load vector v (k_new, then the queries) as 16-byte pieces of
   // 8 channels; threads [16 NV, 16 NV + 16) load v_new.
-  const int pv = tid >> 4, c8 = part * 8;
+  const int pv = tid >> 4, c8 = (tid & 15) * 8;
   const bool append = a.k_new != nullptr;
   uint4 raw = make_uint4(0, 0, 0, 0);
   if (pv == 0) {
