@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="layer caches rotated (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other SURVEY workloads (other_workloads field)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--summary", default="f16", choices=["f16", "f32"],
                     help="page-summary storage (f16 rounded outward, or f32)")
@@ -176,6 +178,105 @@ def kernel_source_hash():
     a = s.index(mark + " a2")
     b = s.index(mark, a + len(mark))
     return hashlib.sha256(s[a:b].encode()).hexdigest()
+
+
+# ----------------------------------------------------------------------------- other workloads
+
+SECONDARY = ("llama8b_128k_b1", "ragged_b32", "llama8b_32k", "tiny_1h_4k", "hisa_128k_t1",
+             "hisa_128k_t64")
+
+
+def indexer_required_bytes(wl, lens):
+    """Algorithmic bytes of one HISA selection: block means (512 B per block, read once per
+    step) + the kept blocks' keys of every chunk query (256 B per key; the union of the
+    queries' kept blocks would be the minimum, the per-query sum is what the kernel reads)."""
+    d, P = wl.head_dim, wl.page_size
+    tot = 0
+    for n in lens:
+        nblk = -(-n // P)
+        tot += nblk * d * 4 + wl.n_queries * min(wl.m_pages, nblk) * P * d * 2
+    return tot
+
+
+def measure_secondary(name, dev, l2, f16, steps, stream, mem_cap):
+    """Graph-replayed decode steps of another workload; returns its figures."""
+    import torch
+    import hhr_synth as S
+    from hash_hierarchical_top_b200 import hhr
+    from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+    wl = S.WORKLOADS[name]
+    lens = S.seq_lens_of(wl)
+    hashing = wl.mode == "hash"
+    if hashing:
+        m_of = (lambda npg: min(npg, -(-npg // wl.keep_div))) if wl.m_pages == 0 else (
+            lambda npg: min(wl.m_pages, npg))
+        req = sum(required_bytes(wl, lens, m_of, 2 if f16 else 4))
+        queries = wl.batch
+    else:
+        req = indexer_required_bytes(wl, lens)
+        queries = wl.batch * wl.n_queries
+    # Layer caches for an L2-cold rotation (>= 4x L2 of required bytes), within a memory cap.
+    per_layer = sum(lens) * wl.n_kv_heads * wl.head_dim * 2 * (2 if hashing else 1)
+    L = max(2, min(-(-4 * l2 // req), max(2, mem_cap // max(per_layer, 1)), 64))
+    layers, graphs = [], []
+    for l in range(L):
+        inp = S.make_inputs(wl, device=dev, layer=l, with_values=hashing)
+        d = hhr.make_dims(wl.batch, wl.n_q_heads if hashing else wl.n_queries, wl.n_kv_heads,
+                          wl.page_size, inp["max_pages"], inp["n_phys"],
+                          summary_fp16=f16 if hashing else 0)
+        cache = LayerCache(d, dev, hashing=hashing, block_means=not hashing)
+        zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+        hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
+                            int(inp["seq_len"].max()), inp["R"] if hashing else None,
+                            inp["W"] if hashing else None,
+                            cache.page_minmax if hashing else None,
+                            cache.codes if hashing else None,
+                            None if hashing else cache.block_mean)
+        mode = hhr.HHR_MODE_HASH if hashing else hhr.HHR_MODE_INDEXER
+        st = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev, attention=hashing)
+        if hashing:
+            t = (inp["seq_len"] - 1).long()
+            phys = inp["page_table"][torch.arange(wl.batch, device=dev), t // wl.page_size].long()
+            kn = inp["k_cache"][phys, :, t % wl.page_size].contiguous()
+            vn = inp["v_cache"][phys, :, t % wl.page_size].contiguous()
+
+            def run(inp=inp, cache=cache, st=st, kn=kn, vn=vn):
+                st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
+                              inp["seq_len"], inp["R"], inp["W"], cache, k_new=kn, v_new=vn)
+        else:
+            def run(inp=inp, cache=cache, st=st):
+                st.select(inp["q"], inp["seq_len"], inp["page_table"], cache,
+                          k_cache=inp["k_cache"], q_pos=inp["q_pos"])
+        run()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            run()
+        layers.append((inp, cache, st))
+        graphs.append(gr)
+    for i in range(3 * L):
+        graphs[i % L].replay()
+    torch.cuda.synchronize()
+    st_, bits = hhr.hhr_read_device_status()
+    if st_ != hhr.HHR_OK:
+        raise RuntimeError(f"{name}: device status {bits}")
+    K = max(steps, 2 * L)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(K):
+        graphs[i % L].replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / K
+    peak, _ = measured_peaks()
+    gbs = req / (ms / 1e3) / 1e9
+    del graphs, layers
+    torch.cuda.empty_cache()
+    return {"api": "hhr_decode_step" if hashing else "hhr_select (indexer)",
+            "queries_per_s": queries / (ms / 1e3), "us_per_step": ms * 1e3,
+            "queries_per_step": queries, "required_bytes": req, "achieved_gbs": gbs,
+            "frac_of_measured": gbs / peak, "layer_caches_rotated": L,
+            "l2_cold": L * req >= 4 * l2}
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -394,6 +495,7 @@ def main():
         step.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
                   inp["R"], inp["W"], cache, start, one)
 
+    fused = args.path == "fused" and not args.select_only
     if args.select_only:
         names = ("encode", "qprep", "bound", "hamming")
     elif args.path == "fused":
@@ -594,6 +696,13 @@ def main():
     traffic = prof[0] * bound_bytes / prof[1] if prof is not None else None
     step_gbs = req / (ms_step / 1e3) / 1e9
 
+    # The other SURVEY workloads (configs 1, 2, 3 at batch 1, 4 and 5), each graph-timed on
+    # its own layer caches; single-GPU default runs only.
+    other = None
+    if (rank == 0 and world == 1 and not args.no_secondary and fused and args.batch == 0
+            and args.workload == "llama8b_128k_b8"):
+        other = {w: measure_secondary(w, dev, l2, f16, 2000, stream, 24 << 30) for w in SECONDARY}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.select_only:
         per_group, done = run_oracle_timed(wl, layers[0][0], seconds=args.cpu_seconds)
@@ -637,6 +746,7 @@ def main():
                          "frac_of_measured": step_gbs / peak},
             "kernels_us": kern,
             "prefill_encode": prefill,
+            "other_workloads": other,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": ck,
