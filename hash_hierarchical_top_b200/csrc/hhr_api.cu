@@ -372,27 +372,28 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
   sb.q_pos = q_pos; sb.P = P; sb.mode = 0; sb.m_max = m_max; sb.unit = 0;
   sb.m_pages = m_pages; sb.keep_div = 0; sb.top_k = 0;
   sb.out = kept; sb.out_stride = m_max; sb.out_count = kept_count; sb.pad_out = 0;
+  cudaError_t e;
   prof_begin(HHR_KERNEL_TOPM, s);
-  select_largest_kernel<<<B * T, kSelThreads, (size_t)maxp * 4, s>>>(sb);
+  e = launch_pdl(select_largest_kernel, dim3(B * T), dim3(kSelThreads), (size_t)maxp * 4, s, sb);
   prof_end(HHR_KERNEL_TOPM, s);
-  if ((st = launch_status()) != HHR_OK) return st;
+  if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   const int C = m_max * P;
   prof_begin(HHR_KERNEL_TOKEN, s);
-  token_score_kernel<<<dim3((C + kTokWarps * 32 - 1) / (kTokWarps * 32), B * T), kTokWarps * 32,
-                       0, s>>>(TokenScoreArgs{q, k_cache, page_table, seq_len, q_pos, kept,
-                                              kept_count, tok, T, P, maxp, d->n_phys_pages,
-                                              m_max});
+  e = launch_pdl(token_score_kernel, dim3((C + kTokWarps * 32 - 1) / (kTokWarps * 32), B * T),
+                 dim3(kTokWarps * 32), 0, s,
+                 TokenScoreArgs{q, k_cache, page_table, seq_len, q_pos, kept, kept_count, tok, T,
+                                P, maxp, d->n_phys_pages, m_max});
   prof_end(HHR_KERNEL_TOKEN, s);
-  if ((st = launch_status()) != HHR_OK) return st;
+  if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   SelectArgs sc{};
   sc.scores = tok; sc.stride = C; sc.rows_per_b = T; sc.seq_len = seq_len; sc.q_pos = q_pos;
   sc.P = P; sc.mode = 1; sc.kept_count = kept_count; sc.kept_units = kept; sc.m_max = m_max;
   sc.unit = P; sc.m_pages = 0; sc.keep_div = 0; sc.top_k = top_k;
   sc.out = out_idx; sc.out_stride = top_k; sc.out_count = out_count; sc.pad_out = 1;
   prof_begin(HHR_KERNEL_TOKEN_TOPK, s);
-  select_largest_kernel<<<B * T, kSelThreads, (size_t)C * 4, s>>>(sc);
+  e = launch_pdl(select_largest_kernel, dim3(B * T), dim3(kSelThreads), (size_t)C * 4, s, sc);
   prof_end(HHR_KERNEL_TOKEN_TOPK, s);
-  if ((st = launch_status()) != HHR_OK) return st;
+  if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   if (trace != nullptr) {
     if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * T * maxp * 4, s))) return st;
     if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * T * m_max * 4, s))) return st;

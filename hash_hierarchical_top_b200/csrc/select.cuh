@@ -506,6 +506,8 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SelShared sh;
   extern __shared__ uint32_t keys[];  // [n], 16-byte aligned
   const int row = blockIdx.x, tid = threadIdx.x;
@@ -967,6 +969,8 @@ constexpr int kBlkStride = kBlkTile + 1;  // float4 row stride of the staged til
 
 __global__ void __launch_bounds__(kBlkTile) block_score_kernel(BlockScoreArgs a) {
   extern __shared__ float4 bs_smem[];
+  pdl_wait();
+  pdl_trigger();
   float4* Ms = bs_smem;                         // [kD/4][kBlkStride]
   float4* Qs = bs_smem + (kD / 4) * kBlkStride; // [kQTile][kD/4]
   const int b = blockIdx.z, q0 = blockIdx.y * kQTile, blk0 = blockIdx.x * kBlkTile;
@@ -1046,6 +1050,8 @@ struct TokenScoreArgs {
 };
 
 __global__ void __launch_bounds__(kTokWarps * 32) token_score_kernel(TokenScoreArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.y, b = row / a.T;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int C = a.kept_count[row] * a.P;
