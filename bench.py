@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other SURVEY workloads (other_workloads field)")
+    ap.add_argument("--no-quality", action="store_true",
+                    help="skip the selection-quality figures (selection_quality field)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--summary", default="f16", choices=["f16", "f32"],
                     help="page-summary storage (f16 rounded outward, or f32)")
@@ -178,6 +180,163 @@ def kernel_source_hash():
     a = s.index(mark + " a2")
     b = s.index(mark, a + len(mark))
     return hashlib.sha256(s[a:b].encode()).hexdigest()
+
+
+# ----------------------------------------------------------------------------- selection quality
+# Measures how well the GPU path's selections match exact ones on the synthetic workloads
+# (HHR page, Figure 4: recall of the true top-k; Figure 2: Hamming distance against logits;
+# HISA page, Abstract: overlap of the hierarchical with the flat indexer's selection).
+
+
+def recall_at_k(sel, true):
+    """|sel ∩ true| / |true| for two 1-D index tensors (sel may hold -1 padding)."""
+    import torch
+    sel = sel[sel >= 0]
+    if true.numel() == 0:
+        return 1.0
+    return float(torch.isin(true, sel).sum().item()) / true.numel()
+
+
+def iou(a, b):
+    """Intersection over union of two index sets (-1 padding ignored)."""
+    import torch
+    a, b = a[a >= 0], b[b >= 0]
+    inter = int(torch.isin(a, b).sum().item())
+    union = a.numel() + b.numel() - inter
+    return 1.0 if union == 0 else inter / union
+
+
+def mass_recall(logits, sel, scale):
+    """Mean over rows of logits [H][n] of the softmax(scale * logits) mass on sel."""
+    import torch
+    p = torch.softmax(logits.double() * scale, dim=-1)
+    sel = sel[sel >= 0]
+    return float(p[:, sel].sum(dim=-1).mean().item())
+
+
+def spearman(x, y):
+    """Spearman rank correlation of two 1-D tensors (average ranks for ties)."""
+    import torch
+
+    def ranks(v):
+        v = v.double()
+        order = torch.argsort(v)
+        r = torch.empty_like(v)
+        r[order] = torch.arange(v.numel(), dtype=torch.float64, device=v.device)
+        # average the ranks of equal values
+        uniq, inv = torch.unique(v, return_inverse=True)
+        sums = torch.zeros(uniq.numel(), dtype=torch.float64, device=v.device).index_add_(0, inv, r)
+        cnt = torch.zeros(uniq.numel(), dtype=torch.float64, device=v.device).index_add_(
+            0, inv, torch.ones_like(r))
+        return (sums / cnt)[inv]
+
+    rx, ry = ranks(x), ranks(y)
+    rx, ry = rx - rx.mean(), ry - ry.mean()
+    return float((rx * ry).sum().item() / ((rx.square().sum() * ry.square().sum()).sqrt().item()))
+
+
+def popcount32(x):
+    """Per-element popcount of an int32 tensor (bit-parallel sums; int64 result)."""
+    x = x.to(__import__("torch").int64) & 0xFFFFFFFF
+    x = x - ((x >> 1) & 0x55555555)
+    x = (x & 0x33333333) + ((x >> 2) & 0x33333333)
+    x = (x + (x >> 4)) & 0x0F0F0F0F
+    return ((x * 0x01010101) & 0xFFFFFFFF) >> 24
+
+
+def selection_quality(dev):
+    """Recall, attention-mass recall and Hamming/logit correlation of the HHR selection on the
+    128K batch-8 workload, and overlap of the HISA selection with the flat indexer's."""
+    import statistics
+    import torch
+    import hhr_synth as S
+    from hash_hierarchical_top_b200 import hhr
+    from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+    out = {}
+    # HHR: GPU selection (hhr_select on layer 0) against exact group logits.
+    wl = S.WORKLOADS["llama8b_128k_b8"]
+    inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
+    d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.page_size, inp["max_pages"],
+                      inp["n_phys"], summary_fp16=1)
+    cache = LayerCache(d, dev)
+    zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+    hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
+                        int(inp["seq_len"].max()), inp["R"], inp["W"], cache.page_minmax,
+                        cache.codes, None)
+    st = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev, attention=False)
+    B, G, gs, P = wl.batch, wl.n_kv_heads, wl.n_q_heads // wl.n_kv_heads, wl.page_size
+    qcode = torch.empty(B, wl.n_q_heads, 4, dtype=torch.int32, device=dev)
+    kept = torch.empty(B, G, st.m_max, dtype=torch.int32, device=dev)
+    kcnt = torch.empty(B, G, dtype=torch.int32, device=dev)
+    st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"], W=inp["W"],
+              trace=hhr.make_trace(q_code=qcode, kept=kept, kept_count=kcnt))
+    torch.cuda.synchronize()
+    rec, mass, page_rec, ham_rec, rho = [], [], [], [], []
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    gen = torch.Generator(device=dev).manual_seed(0)
+    for b in range(B):
+        n = int(inp["seq_len"][b])
+        npg = -(-n // P)
+        pages = inp["page_table"][b, :npg].long()
+        for g in range(G):
+            K = inp["k_cache"][pages, g].reshape(npg * P, -1)[:n].float()
+            lg = inp["q"][b, g * gs:(g + 1) * gs].float() @ K.T          # [gs][n]
+            grp = lg.sum(0)
+            k = min(wl.top_k, n)
+            true = torch.topk(grp, k).indices
+            sel = st.idx[b, g, :int(st.count[b, g])].long()
+            rec.append(recall_at_k(sel, true))
+            mass.append(mass_recall(lg, sel, scale))
+            kp = kept[b, g, :int(kcnt[b, g])].long()
+            in_kept = torch.isin(true // P, kp)
+            page_rec.append(float(in_kept.float().mean().item()))
+            if bool(in_kept.any()):
+                ham_rec.append(recall_at_k(sel, true[in_kept]))
+            codes = cache.codes[pages, g].reshape(npg * P, 4)[:n]
+            qc = qcode[b, g * gs:(g + 1) * gs]                            # [gs][4]
+            delta = popcount32(qc[:, None, :] ^ codes[None, :, :]).sum(dim=(0, 2))
+            smp = torch.randint(0, n, (16384,), device=dev, generator=gen)
+            rho.append(spearman(-delta[smp].double(), grp[smp].double()))
+    out["hhr_llama8b_128k_b8"] = {
+        "recall_at_k": statistics.mean(rec), "recall_at_k_min": min(rec),
+        "attention_mass_recall": statistics.mean(mass),
+        "true_topk_in_kept_pages": statistics.mean(page_rec),
+        "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
+        "spearman_minus_hamming_vs_logit": statistics.mean(rho),
+        "k": wl.top_k, "keep": f"1/{wl.keep_div}", "rows": B * G,
+        "random_selection_mass": wl.top_k / int(inp["seq_len"].float().mean()),
+        "true_set": "top-k of the group-summed logits sum_h q_h . k_t (one selection per KV group)"}
+    del inp, cache, st
+    # HISA: hierarchical selection against the flat indexer's causal top-k over all keys.
+    for name in ("hisa_128k_t1", "hisa_128k_t64"):
+        wl = S.WORKLOADS[name]
+        inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
+        d = hhr.make_dims(wl.batch, wl.n_queries, 1, wl.page_size, inp["max_pages"], inp["n_phys"])
+        cache = LayerCache(d, dev, hashing=False, block_means=True)
+        zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+        hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
+                            int(inp["seq_len"].max()), None, None, None, None, cache.block_mean)
+        st = DecodeStep(d, hhr.HHR_MODE_INDEXER, wl.m_pages, 0, wl.top_k, dev, attention=False)
+        st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, k_cache=inp["k_cache"],
+                  q_pos=inp["q_pos"])
+        torch.cuda.synchronize()
+        n = int(inp["seq_len"][0])
+        P = wl.page_size
+        npg = -(-n // P)
+        pages = inp["page_table"][0, :npg].long()
+        K = inp["k_cache"][pages, 0].reshape(npg * P, -1)[:n].float()
+        ious = []
+        for t in range(wl.n_queries):
+            pos = int(inp["q_pos"][0, t])
+            sc = inp["q"][0, t].float() @ K[:pos + 1].T
+            flat = torch.topk(sc, min(wl.top_k, pos + 1)).indices
+            ious.append(iou(st.idx[0, t, :int(st.count[0, t])].long(), flat))
+        out[name] = {"iou_with_flat_indexer": statistics.mean(ious),
+                     "iou_min": min(ious), "queries": wl.n_queries, "k": wl.top_k,
+                     "kept_blocks": wl.m_pages}
+        del inp, cache, st
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- other workloads
@@ -702,6 +861,10 @@ def main():
     if (rank == 0 and world == 1 and not args.no_secondary and fused and args.batch == 0
             and args.workload == "llama8b_128k_b8"):
         other = {w: measure_secondary(w, dev, l2, f16, 2000, stream, 24 << 30) for w in SECONDARY}
+    quality = None
+    if (rank == 0 and world == 1 and not args.no_quality and fused and args.batch == 0
+            and args.workload == "llama8b_128k_b8"):
+        quality = selection_quality(dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.select_only:
@@ -747,6 +910,7 @@ def main():
             "kernels_us": kern,
             "prefill_encode": prefill,
             "other_workloads": other,
+            "selection_quality": quality,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": ck,

@@ -362,7 +362,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     return HHR_ERR_CUDA;
   prof_begin(HHR_KERNEL_BLOCK, s);
   block_score_kernel<<<dim3((maxp + kBlkTile - 1) / kBlkTile, (T + kQTile - 1) / kQTile, B),
-                       kBlkTile, block_score_smem(), s>>>(
+                       kBlkThreads, block_score_smem(), s>>>(
       BlockScoreArgs{q, block_mean, page_table, seq_len, q_pos, bounds, T, P, maxp,
                      d->n_phys_pages});
   prof_end(HHR_KERNEL_BLOCK, s);

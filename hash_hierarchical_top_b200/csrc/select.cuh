@@ -949,11 +949,14 @@ inline TopmHammingFn topm_hamming_for(int gs) {
 // ---------------------------------------------------------------------------- HISA a1'
 // HISA page, Abstract: the block-level coarse filter scores pooled block
 // representatives (block_mean) against each query. Blocks whose start lies after
-// the query position are ineligible (-inf). One CTA of 128 threads handles 128
-// blocks for up to 16 chunk queries; the block tile is staged in shared memory as
-// float4 columns so thread j reads block j's channels without bank conflicts.
-constexpr int kBlkTile = 128;
+// the query position are ineligible (-inf). One CTA of 128 threads handles 32 blocks for up
+// to 16 chunk queries: the 32 page ids are read first, then every thread issues its 8
+// block-mean pieces at once (warp w loads whole 512-byte rows, one per instruction), staged
+// transposed in shared memory; thread t then scores block t % 32 for queries 4 (t / 32) ..
+// 4 (t / 32) + 3.
+constexpr int kBlkTile = 32;
 constexpr int kQTile = 16;
+constexpr int kBlkThreads = 128;
 
 struct BlockScoreArgs {
   const uint16_t* q;        // [B][T][d]
@@ -967,67 +970,80 @@ struct BlockScoreArgs {
 
 constexpr int kBlkStride = kBlkTile + 1;  // float4 row stride of the staged tile (padded)
 
-__global__ void __launch_bounds__(kBlkTile) block_score_kernel(BlockScoreArgs a) {
-  extern __shared__ float4 bs_smem[];
+__global__ void __launch_bounds__(kBlkThreads) block_score_kernel(BlockScoreArgs a) {
+  __shared__ float4 Ms[kD / 4][kBlkStride];  // block means, channel-major
+  __shared__ float4 Qs[kQTile][kD / 4];
+  __shared__ int ids[kBlkTile];
   pdl_wait();
   pdl_trigger();
-  float4* Ms = bs_smem;                         // [kD/4][kBlkStride]
-  float4* Qs = bs_smem + (kD / 4) * kBlkStride; // [kQTile][kD/4]
   const int b = blockIdx.z, q0 = blockIdx.y * kQTile, blk0 = blockIdx.x * kBlkTile;
   const int tid = threadIdx.x;
   const int nblk = min(ceil_div(a.seq_len[b], a.P), a.maxp);
   if (blk0 >= nblk) return;
   const int nq = min(kQTile, a.T - q0);
-  for (int idx = tid; idx < kQTile * (kD / 4); idx += kBlkTile) {
-    int qi = idx / (kD / 4), c4 = idx % (kD / 4);
+  if (tid < kBlkTile) {
+    const int blk = blk0 + tid;
+    int phys = -1;
+    if (blk < nblk) {
+      phys = a.page_table[(size_t)b * a.maxp + blk];
+      if (phys < 0 || phys >= a.n_phys) {
+        flag_status(kStatusBadPage);
+        phys = -1;
+      }
+    }
+    ids[tid] = phys;
+  }
+  for (int idx = tid; idx < kQTile * (kD / 4); idx += kBlkThreads) {
+    const int qi = idx / (kD / 4), c4 = idx % (kD / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (qi < nq) {
-      uint2 w = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * a.T + q0 + qi) * kD + 4 * c4);
+      const uint2 w = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * a.T + q0 + qi) * kD + 4 * c4);
       v = bf16x4_to_f4(w);
     }
-    Qs[qi * (kD / 4) + c4] = v;
-  }
-  // Stage the block means: warp-cooperative coalesced reads of each 512-byte row.
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int r = warp; r < kBlkTile; r += kBlkTile / 32) {
-    int blk = blk0 + r;
-    int phys = -1;
-    if (blk < nblk) phys = a.page_table[(size_t)b * a.maxp + blk];
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (phys >= 0 && phys < a.n_phys)
-      v = reinterpret_cast<const float4*>(a.block_mean + (size_t)phys * kD)[lane];
-    else if (blk < nblk && lane == 0)
-      flag_status(kStatusBadPage);
-    Ms[lane * kBlkStride + r] = v;
+    Qs[qi][c4] = v;
   }
   __syncthreads();
-  float acc[kQTile];
+  constexpr int kPer = kBlkTile * (kD / 4) / kBlkThreads;  // 8 pieces per thread
+  float4 mv[kPer];
 #pragma unroll
-  for (int i = 0; i < kQTile; ++i) acc[i] = 0.f;
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = i * kBlkThreads + tid;
+    const int r = idx / (kD / 4), c4 = idx % (kD / 4);
+    const int phys = ids[r];
+    mv[i] = phys >= 0 ? reinterpret_cast<const float4*>(a.block_mean + (size_t)phys * kD)[c4]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = i * kBlkThreads + tid;
+    Ms[idx % (kD / 4)][idx / (kD / 4)] = mv[i];
+  }
+  __syncthreads();
+  const int r = tid % kBlkTile, qg = tid / kBlkTile;  // block r, queries 4 qg .. 4 qg + 3
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
   for (int c4 = 0; c4 < kD / 4; ++c4) {
-    float4 mv = Ms[c4 * kBlkStride + tid];
+    const float4 m = Ms[c4][r];
 #pragma unroll
-    for (int i = 0; i < kQTile; ++i) {
-      float4 qv = Qs[i * (kD / 4) + c4];
-      acc[i] = fmaf(qv.x, mv.x, fmaf(qv.y, mv.y, fmaf(qv.z, mv.z, fmaf(qv.w, mv.w, acc[i]))));
+    for (int i = 0; i < 4; ++i) {
+      const float4 qv = Qs[4 * qg + i][c4];
+      acc[i] = fmaf(qv.x, m.x, fmaf(qv.y, m.y, fmaf(qv.z, m.z, fmaf(qv.w, m.w, acc[i]))));
     }
   }
-  const int blk = blk0 + tid;
+  const int blk = blk0 + r;
   if (blk < nblk) {
 #pragma unroll
-    for (int i = 0; i < kQTile; ++i) {
-      if (i >= nq) break;
-      int pos = a.q_pos[(size_t)b * a.T + q0 + i];
-      bool elig = (long long)blk * a.P <= (long long)pos;
-      a.scores[((size_t)b * a.T + q0 + i) * a.maxp + blk] = elig ? acc[i] : -INFINITY;
+    for (int i = 0; i < 4; ++i) {
+      const int qi = 4 * qg + i;
+      if (qi >= nq) break;
+      const int pos = a.q_pos[(size_t)b * a.T + q0 + qi];
+      const bool elig = (long long)blk * a.P <= (long long)pos;
+      a.scores[((size_t)b * a.T + q0 + qi) * a.maxp + blk] = elig ? acc[i] : -INFINITY;
     }
   }
 }
 
-inline size_t block_score_smem() {
-  return (size_t)((kD / 4) * kBlkStride + kQTile * (kD / 4)) * sizeof(float4);
-}
+inline size_t block_score_smem() { return 0; }
 
 // ---------------------------------------------------------------------------- HISA a3
 // HISA page, Abstract: the original token indexer runs only inside the kept blocks.
@@ -1059,37 +1075,61 @@ __global__ void __launch_bounds__(kTokWarps * 32) token_score_kernel(TokenScoreA
   if (c0 >= C) return;
   const int n = a.seq_len[b], pos = a.q_pos[row];
   const float4 qv = bf16x4_to_f4(*reinterpret_cast<const uint2*>(a.q + (size_t)row * kD + 4 * lane));
+  // Candidate c is slot c % P of kept block kept[c / P]. With P a multiple of 32 the warp's
+  // 32 candidates share one block, resolved once (lane 0) so that the row loads are
+  // independent; otherwise each candidate resolves its own block.
+  const bool one_block = (a.P & 31) == 0;
+  int lp_w = -1, phys_w = -1;
+  if (one_block && lane == 0) {
+    lp_w = a.kept[(size_t)row * a.m_max + c0 / a.P];
+    if (lp_w >= 0 && lp_w < a.maxp) {
+      phys_w = a.page_table[(size_t)b * a.maxp + lp_w];
+      if (phys_w < 0 || phys_w >= a.n_phys) phys_w = -1;
+    }
+  }
+  lp_w = __shfl_sync(kFull, lp_w, 0);
+  phys_w = __shfl_sync(kFull, phys_w, 0);
+  auto resolve = [&](int c, int& t, int& phys) {
+    int lp = lp_w;
+    phys = phys_w;
+    if (!one_block) {
+      lp = a.kept[(size_t)row * a.m_max + c / a.P];
+      phys = -1;
+      if (lp >= 0 && lp < a.maxp) {
+        phys = a.page_table[(size_t)b * a.maxp + lp];
+        if (phys < 0 || phys >= a.n_phys) phys = -1;
+      }
+    }
+    t = lp * a.P + c % a.P;
+  };
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const int c = c0 + j;
-    float s = 0.f;
+    float sc = 0.f;
     if (c < C) {
-      const int lp = a.kept[(size_t)row * a.m_max + c / a.P];
-      const int t = lp * a.P + c % a.P;
-      if (t < n && t <= pos) {
-        const int phys = a.page_table[(size_t)b * a.maxp + lp];
-        if (phys >= 0 && phys < a.n_phys) {
-          uint2 w = *reinterpret_cast<const uint2*>(
-              a.k_cache + ((size_t)phys * a.P + c % a.P) * kD + 4 * lane);
-          float4 kv = bf16x4_to_f4(w);
-          s = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
-        }
+      int t, phys;
+      resolve(c, t, phys);
+      if (t < n && t <= pos && phys >= 0) {
+        const uint2 w = *reinterpret_cast<const uint2*>(
+            a.k_cache + ((size_t)phys * a.P + c % a.P) * kD + 4 * lane);
+        const float4 kv = bf16x4_to_f4(w);
+        sc = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
       }
     }
-    v[j] = s;
+    v[j] = sc;
   }
-  float sc = warp_transpose_sum32(v, lane);
+  const float scv = warp_transpose_sum32(v, lane);
   const int c = c0 + lane;
   if (c < C) {
-    const int lp = a.kept[(size_t)row * a.m_max + c / a.P];
-    const int t = lp * a.P + c % a.P;
+    int t, phys;
+    resolve(c, t, phys);
     bool ok = t < n && t <= pos;
-    if (ok) {
-      const int phys = a.page_table[(size_t)b * a.maxp + lp];
-      if (phys < 0 || phys >= a.n_phys) { ok = false; flag_status(kStatusBadPage); }
+    if (ok && phys < 0) {
+      ok = false;
+      flag_status(kStatusBadPage);
     }
-    a.tok_scores[(size_t)row * a.m_max * a.P + c] = ok ? sc : -INFINITY;
+    a.tok_scores[(size_t)row * a.m_max * a.P + c] = ok ? scv : -INFINITY;
   }
 }
 
