@@ -74,7 +74,9 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 
 // Exclusive block scan of one int per thread; blockDim.x a multiple of 32, <= 1024.
 // `scratch` holds >= 33 ints of shared memory. Returns the exclusive prefix and
-// writes the block total to *total. Contains __syncthreads(): call uniformly.
+// writes the block total to *total. Contains __syncthreads(): call uniformly. Without the
+// tail barrier (kTailSync false) the caller must pass a barrier before scratch is reused.
+template <bool kTailSync = true>
 __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -90,12 +92,13 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
   __syncthreads();
   int res = scratch[warp] + incl - v;
   *total = scratch[32];
-  __syncthreads();
+  if (kTailSync) __syncthreads();  // before scratch is reused
   return res;
 }
 
 // Exclusive block scan of two ints per thread in one pass of barriers (same contract as
 // block_excl_scan; `scratch` holds >= 66 ints). Returns both prefixes; *total the totals.
+template <bool kTailSync = true>
 __device__ __forceinline__ int2 block_excl_scan2(int2 v, int* scratch, int2* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -121,7 +124,7 @@ __device__ __forceinline__ int2 block_excl_scan2(int2 v, int* scratch, int2* tot
   __syncthreads();
   const int2 res = make_int2(scratch[warp] + a - v.x, scratch[33 + warp] + b - v.y);
   *total = make_int2(scratch[32], scratch[65]);
-  __syncthreads();
+  if (kTailSync) __syncthreads();  // before scratch is reused
   return res;
 }
 

@@ -293,6 +293,7 @@ struct SelectArgs {
 
 // Block-wide sum of one int and min / max of one uint32 per thread, in one pass of
 // barriers (contains __syncthreads). sh: 96 words of shared memory.
+template <bool kTailSync = true>
 __device__ __forceinline__ void block_count_minmax(int cnt, uint32_t lo, uint32_t hi, uint32_t* sh,
                                                    int* out_cnt, uint32_t* out_lo,
                                                    uint32_t* out_hi) {
@@ -317,14 +318,14 @@ __device__ __forceinline__ void block_count_minmax(int cnt, uint32_t lo, uint32_
   *out_cnt = cnt;
   *out_lo = lo;
   *out_hi = hi;
-  __syncthreads();
+  if (kTailSync) __syncthreads();  // before sh is reused
 }
 
 struct SelShared {
-  int hist[256];
+  int hist[2][256];  // double-buffered: a pass zeroes the next pass's histogram
   int scratch[66];
   uint32_t mm[96];
-  int digit, rem, cnt;
+  int res[2][3];     // per pass (alternating): digit, rem, cnt
 };
 
 __device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
@@ -378,8 +379,8 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
       if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
     }
   }
-  // Also orders the key stores before any read.
-  block_count_minmax(nfin, kmin, kmax, sh.mm, &nfin, &kmin, &kmax);
+  // Also orders the key stores before any read (sh.mm is not reused: no tail barrier).
+  block_count_minmax<false>(nfin, kmin, kmax, sh.mm, &nfin, &kmin, &kmax);
   SelCut c;
   c.k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
   // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
@@ -401,40 +402,43 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
       uint32_t mask = (hb >= 31) ? 0u : ~((2u << hb) - 1u);   // common high bits
       uint32_t prefix = kmin & mask;
       int rem = c.k;
+      // Two barriers per pass: the histogram and the pass result alternate between two
+      // buffers, and a pass zeroes the other histogram while it fills its own.
+      int cur = 0;
+      if (tid < 256) sh.hist[0][tid] = 0;
+      __syncthreads();
       while (true) {
-        if (tid < 256) sh.hist[tid] = 0;
-        __syncthreads();
         for (int i = tid; i < n; i += NT) {
           const uint32_t kk = keys[i];
-          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&sh.hist[(kk >> shift) & 255], 1);
+          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&sh.hist[cur][(kk >> shift) & 255], 1);
         }
+        if (tid < 256) sh.hist[cur ^ 1][tid] = 0;
         __syncthreads();
         if (tid < 32) {
           // Lane l covers digits 255-8l .. 248-8l (descending).
-          int cq[8], s = 0;
+          int cq[8], sum = 0;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { cq[q] = sh.hist[255 - 8 * tid - q]; s += cq[q]; }
-          const int incl = warp_incl_scan(s, tid);
-          const int excl = incl - s;
+          for (int q = 0; q < 8; ++q) { cq[q] = sh.hist[cur][255 - 8 * tid - q]; sum += cq[q]; }
+          const int incl = warp_incl_scan(sum, tid);
+          const int excl = incl - sum;
           if (excl < rem && rem <= incl) {
             int run = excl;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (run < rem && rem <= run + cq[q]) {
-                sh.digit = 255 - 8 * tid - q;
-                sh.rem = rem - run;
-                sh.cnt = cq[q];
+                sh.res[cur][0] = 255 - 8 * tid - q;
+                sh.res[cur][1] = rem - run;
+                sh.res[cur][2] = cq[q];
               }
               run += cq[q];
             }
           }
         }
         __syncthreads();
-        prefix |= (uint32_t)sh.digit << shift;
+        prefix |= (uint32_t)sh.res[cur][0] << shift;
         mask |= 255u << shift;
-        rem = sh.rem;
-        const int cnt_bin = sh.cnt;
-        __syncthreads();
+        rem = sh.res[cur][1];
+        const int cnt_bin = sh.res[cur][2];
         if (rem == cnt_bin) {  // the whole bin is needed: no tie-break required
           c.whole_bin = true;
           c.sel_shift = shift;
@@ -444,6 +448,7 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
         // Next 8 bits; when fewer than 8 remain, the last pass covers bits [0, 8) and
         // its already-fixed upper bits are constant across the candidates.
         shift = max(shift - 8, 0);
+        cur ^= 1;
       }
       c.prefix = prefix;
       c.rem = rem;
@@ -706,7 +711,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
       sum += hv[q];
     }
     int nvalid;
-    const int excl = block_excl_scan(sum, hs.scratch, &nvalid);
+    const int excl = block_excl_scan<false>(sum, hs.scratch, &nvalid);  // next use: after the barrier below
     const int keff = min(a.top_k, nvalid);
     if (keff > 0 && excl < keff && keff <= excl + sum) {
       int run = excl;
@@ -752,7 +757,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
     }
   }
   int2 tot;
-  const int2 before = block_excl_scan2(make_int2(lt, eq), hs.scratch, &tot);
+  const int2 before = block_excl_scan2<false>(make_int2(lt, eq), hs.scratch, &tot);  // last use
   if (tid == 0) { hs.tot[0] = tot.x; hs.tot[1] = tot.y; }
   cluster_sync_all();  // every rank's totals are published
   int lt_off = 0, eq_off = 0;
