@@ -244,31 +244,26 @@ def popcount32(x):
     return ((x * 0x01010101) & 0xFFFFFFFF) >> 24
 
 
-def selection_quality(dev):
-    """Recall, attention-mass recall and Hamming/logit correlation of the HHR selection on the
-    128K batch-8 workload, and overlap of the HISA selection with the flat indexer's."""
+def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True):
+    """Encode layer inputs `inp` with rotation R, select with the given page budget and score
+    the selection against the exact group logits (see selection_quality)."""
     import statistics
     import torch
-    import hhr_synth as S
     from hash_hierarchical_top_b200 import hhr
     from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
-    out = {}
-    # HHR: GPU selection (hhr_select on layer 0) against exact group logits.
-    wl = S.WORKLOADS["llama8b_128k_b8"]
-    inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
     d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.page_size, inp["max_pages"],
                       inp["n_phys"], summary_fp16=1)
     cache = LayerCache(d, dev)
     zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
     hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
-                        int(inp["seq_len"].max()), inp["R"], inp["W"], cache.page_minmax,
-                        cache.codes, None)
-    st = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, dev, attention=False)
+                        int(inp["seq_len"].max()), R, inp["W"], cache.page_minmax, cache.codes,
+                        None)
+    st = DecodeStep(d, hhr.HHR_MODE_HASH, m_pages, keep_div, wl.top_k, dev, attention=False)
     B, G, gs, P = wl.batch, wl.n_kv_heads, wl.n_q_heads // wl.n_kv_heads, wl.page_size
     qcode = torch.empty(B, wl.n_q_heads, 4, dtype=torch.int32, device=dev)
     kept = torch.empty(B, G, st.m_max, dtype=torch.int32, device=dev)
     kcnt = torch.empty(B, G, dtype=torch.int32, device=dev)
-    st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"], W=inp["W"],
+    st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=R, W=inp["W"],
               trace=hhr.make_trace(q_code=qcode, kept=kept, kept_count=kcnt))
     torch.cuda.synchronize()
     rec, mass, page_rec, ham_rec, rho = [], [], [], [], []
@@ -282,8 +277,7 @@ def selection_quality(dev):
             K = inp["k_cache"][pages, g].reshape(npg * P, -1)[:n].float()
             lg = inp["q"][b, g * gs:(g + 1) * gs].float() @ K.T          # [gs][n]
             grp = lg.sum(0)
-            k = min(wl.top_k, n)
-            true = torch.topk(grp, k).indices
+            true = torch.topk(grp, min(wl.top_k, n)).indices
             sel = st.idx[b, g, :int(st.count[b, g])].long()
             rec.append(recall_at_k(sel, true))
             mass.append(mass_recall(lg, sel, scale))
@@ -292,21 +286,57 @@ def selection_quality(dev):
             page_rec.append(float(in_kept.float().mean().item()))
             if bool(in_kept.any()):
                 ham_rec.append(recall_at_k(sel, true[in_kept]))
-            codes = cache.codes[pages, g].reshape(npg * P, 4)[:n]
-            qc = qcode[b, g * gs:(g + 1) * gs]                            # [gs][4]
-            delta = popcount32(qc[:, None, :] ^ codes[None, :, :]).sum(dim=(0, 2))
-            smp = torch.randint(0, n, (16384,), device=dev, generator=gen)
-            rho.append(spearman(-delta[smp].double(), grp[smp].double()))
-    out["hhr_llama8b_128k_b8"] = {
-        "recall_at_k": statistics.mean(rec), "recall_at_k_min": min(rec),
-        "attention_mass_recall": statistics.mean(mass),
-        "true_topk_in_kept_pages": statistics.mean(page_rec),
-        "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
-        "spearman_minus_hamming_vs_logit": statistics.mean(rho),
-        "k": wl.top_k, "keep": f"1/{wl.keep_div}", "rows": B * G,
-        "random_selection_mass": wl.top_k / int(inp["seq_len"].float().mean()),
-        "true_set": "top-k of the group-summed logits sum_h q_h . k_t (one selection per KV group)"}
-    del inp, cache, st
+            if full:
+                codes = cache.codes[pages, g].reshape(npg * P, 4)[:n]
+                qc = qcode[b, g * gs:(g + 1) * gs]                        # [gs][4]
+                delta = popcount32(qc[:, None, :] ^ codes[None, :, :]).sum(dim=(0, 2))
+                smp = torch.randint(0, n, (16384,), device=dev, generator=gen)
+                rho.append(spearman(-delta[smp].double(), grp[smp].double()))
+    res = {"recall_at_k": statistics.mean(rec), "recall_at_k_min": min(rec),
+           "attention_mass_recall": statistics.mean(mass),
+           "true_topk_in_kept_pages": statistics.mean(page_rec),
+           "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
+           "k": wl.top_k, "kept_pages": st.m_max, "rows": B * G}
+    if full:
+        res["spearman_minus_hamming_vs_logit"] = statistics.mean(rho)
+        res["random_selection_mass"] = wl.top_k / float(inp["seq_len"].float().mean())
+    del cache, st
+    return res
+
+
+def selection_quality(dev):
+    """Recall, attention-mass recall and Hamming/logit correlation of the HHR selection on the
+    128K batch-8 workload, and overlap of the HISA selection with the flat indexer's."""
+    import statistics
+    import torch
+    import hhr_synth as S
+    from hash_hierarchical_top_b200 import hhr
+    from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+    out = {}
+    # HHR: GPU selection (hhr_select on layer 0) against exact group logits.
+    wl = S.WORKLOADS["llama8b_128k_b8"]
+    inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
+    out["hhr_llama8b_128k_b8"] = hhr_quality(wl, inp, dev, inp["R"], wl.m_pages, wl.keep_div)
+    out["hhr_llama8b_128k_b8"]["true_set"] = ("top-k of the group-summed logits sum_h q_h . k_t "
+                                              "(one selection per KV group)")
+    # Stage variants and the page budget (SURVEY §8(f) item 3): bounds without the rotation
+    # (R = I, QUEST-style page min/max of the raw keys), and keep 1/8 and 1/32.
+    eye = torch.eye(wl.head_dim, device=dev).expand(wl.n_kv_heads, -1, -1).contiguous()
+    sweep = {"quest_R_identity_keep_1/16": hhr_quality(wl, inp, dev, eye, 0, 16, full=False)}
+    for kd in (8, 32):
+        sweep[f"gkr_keep_1/{kd}"] = hhr_quality(wl, inp, dev, inp["R"], 0, kd, full=False)
+    out["hhr_variants_llama8b_128k_b8"] = sweep
+    del inp
+    # Flat hash top-k (every page kept, HATA-style) against the hierarchical selection at 32K.
+    wl = S.WORKLOADS["llama8b_32k"]
+    inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
+    npg = -(-int(inp["seq_len"].max()) // wl.page_size)
+    budget = f"{wl.m_pages}_pages" if wl.m_pages else f"keep_1/{wl.keep_div}"
+    out["llama8b_32k_hierarchical_vs_flat"] = {
+        f"hierarchical_{budget}": hhr_quality(wl, inp, dev, inp["R"], wl.m_pages, wl.keep_div,
+                                              full=False),
+        f"flat_all_{npg}_pages": hhr_quality(wl, inp, dev, inp["R"], npg, 0, full=False)}
+    del inp
     # HISA: hierarchical selection against the flat indexer's causal top-k over all keys.
     for name in ("hisa_128k_t1", "hisa_128k_t64"):
         wl = S.WORKLOADS[name]
