@@ -182,6 +182,32 @@ def kernel_source_hash():
     return hashlib.sha256(s[a:b].encode()).hexdigest()
 
 
+# ----------------------------------------------------------------------------- ranks
+# One process per GPU under torchrun; the timing of a multi-GPU run is the slowest rank's.
+
+
+def rank_env():
+    """(world size, rank, local rank) from the torchrun environment; (1, 0, 0) without it."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x, world, device):
+    """x (a duration) maximised over the ranks (every rank must call it, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_step, steps, ms_max):
+    """Whole-job units/s: each of `world` ranks processed `units_per_step` per step for `steps`
+    steps, and the job took the slowest rank's `ms_max` milliseconds."""
+    return world * units_per_step * steps / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- selection quality
 # Measures how well the GPU path's selections match exact ones on the synthetic workloads
 # (HHR page, Figure 4: recall of the true top-k; Figure 2: Hamming distance against logits;
@@ -577,9 +603,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     import hhr_synth as S
     wl = S.WORKLOADS[args.workload]
     if args.batch > 0 and wl.ragged is None:
@@ -762,12 +786,9 @@ def main():
     ms_total = t0.elapsed_time(t1)
     # The last NG replays of the timed region hold the page-bound kernel's events.
     bound_ms = [a.elapsed_time(b) for a, b in ev_b[max(0, NG - K):]]
-    ms_t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_total = float(ms_t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / K
-    value = world * wl.batch * K / (ms_total / 1e3)
+    value = job_throughput(world, wl.batch, K, ms_total)
 
     # Per-kernel averages: replays of the breakdown graphs, read after each replay.
     kern = {name: [] for name in names}
@@ -833,10 +854,8 @@ def main():
             ge.replay()
         bev.record(stream)
         torch.cuda.synchronize()
-        ms_e = torch.tensor([a.elapsed_time(bev)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(ms_e, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * Bq * Ke / (float(ms_e.item()) / 1e3), "unit": "queries/s",
+        ms_e = max_over_ranks(a.elapsed_time(bev), world, dev)
+        e2e = {"value": job_throughput(world, Bq, Ke, ms_e), "unit": "queries/s",
                "h2d_bytes_per_step": host_in.numel() * 2,
                "d2h_bytes_per_step": out_host.numel() * 4, "steps": Ke,
                "how": "graph replay of: one H2D copy of the pinned [query | newest K | newest V] "
