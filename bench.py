@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the other SURVEY workloads (other_workloads field)")
+                    help="skip the other workloads (other_workloads field)")
     ap.add_argument("--no-quality", action="store_true",
                     help="skip the selection-quality figures (selection_quality field)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -270,26 +270,29 @@ def popcount32(x):
     return ((x * 0x01010101) & 0xFFFFFFFF) >> 24
 
 
-def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True):
-    """Encode layer inputs `inp` with rotation R, select with the given page budget and score
-    the selection against the exact group logits (see selection_quality)."""
+def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None):
+    """Encode layer inputs `inp` with rotation R (and projection W, default inp["W"], of
+    wl.code_bits rows), select with the given page budget and score the selection against
+    the exact group logits (see selection_quality)."""
     import statistics
     import torch
     from hash_hierarchical_top_b200 import hhr
     from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
+    W = inp["W"] if W is None else W
+    CW = wl.code_bits // 32
     d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.page_size, inp["max_pages"],
-                      inp["n_phys"], summary_fp16=1)
+                      inp["n_phys"], summary_fp16=1, code_bits=wl.code_bits)
     cache = LayerCache(d, dev)
     zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
     hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
-                        int(inp["seq_len"].max()), R, inp["W"], cache.page_minmax, cache.codes,
+                        int(inp["seq_len"].max()), R, W, cache.page_minmax, cache.codes,
                         None)
     st = DecodeStep(d, hhr.HHR_MODE_HASH, m_pages, keep_div, wl.top_k, dev, attention=False)
     B, G, gs, P = wl.batch, wl.n_kv_heads, wl.n_q_heads // wl.n_kv_heads, wl.page_size
-    qcode = torch.empty(B, wl.n_q_heads, 4, dtype=torch.int32, device=dev)
+    qcode = torch.empty(B, wl.n_q_heads, CW, dtype=torch.int32, device=dev)
     kept = torch.empty(B, G, st.m_max, dtype=torch.int32, device=dev)
     kcnt = torch.empty(B, G, dtype=torch.int32, device=dev)
-    st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=R, W=inp["W"],
+    st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=R, W=W,
               trace=hhr.make_trace(q_code=qcode, kept=kept, kept_count=kcnt))
     torch.cuda.synchronize()
     rec, mass, page_rec, ham_rec, rho = [], [], [], [], []
@@ -313,8 +316,8 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True):
             if bool(in_kept.any()):
                 ham_rec.append(recall_at_k(sel, true[in_kept]))
             if full:
-                codes = cache.codes[pages, g].reshape(npg * P, 4)[:n]
-                qc = qcode[b, g * gs:(g + 1) * gs]                        # [gs][4]
+                codes = cache.codes[pages, g].reshape(npg * P, CW)[:n]
+                qc = qcode[b, g * gs:(g + 1) * gs]                        # [gs][CW]
                 delta = popcount32(qc[:, None, :] ^ codes[None, :, :]).sum(dim=(0, 2))
                 smp = torch.randint(0, n, (16384,), device=dev, generator=gen)
                 rho.append(spearman(-delta[smp].double(), grp[smp].double()))
@@ -345,12 +348,17 @@ def selection_quality(dev):
     out["hhr_llama8b_128k_b8"] = hhr_quality(wl, inp, dev, inp["R"], wl.m_pages, wl.keep_div)
     out["hhr_llama8b_128k_b8"]["true_set"] = ("top-k of the group-summed logits sum_h q_h . k_t "
                                               "(one selection per KV group)")
-    # Stage variants and the page budget: bounds without the rotation
-    # (R = I, QUEST-style page min/max of the raw keys), and keep 1/8 and 1/32.
+    # Stage variants and the page budget: bounds without the rotation (R = I, QUEST-style
+    # page min/max of the raw keys), keep 1/8 and 1/32, and 64- and 256-bit codes.
     eye = torch.eye(wl.head_dim, device=dev).expand(wl.n_kv_heads, -1, -1).contiguous()
     sweep = {"quest_R_identity_keep_1/16": hhr_quality(wl, inp, dev, eye, 0, 16, full=False)}
     for kd in (8, 32):
         sweep[f"gkr_keep_1/{kd}"] = hhr_quality(wl, inp, dev, inp["R"], 0, kd, full=False)
+    for bits in (64, 256):
+        wb = S.scaled(wl, code_bits=bits)
+        Wb = S.lhp_projection(wb, layer=0).to(dev)
+        sweep[f"codes_{bits}_bit_keep_1/16"] = hhr_quality(wb, inp, dev, inp["R"], 0, 16,
+                                                          full=False, W=Wb)
     out["hhr_variants_llama8b_128k_b8"] = sweep
     del inp
     # Flat hash top-k (every page kept, HATA-style) against the hierarchical selection at 32K.
@@ -772,10 +780,15 @@ def main():
     torch.cuda.synchronize()
     clocks.start()
     t0.record(stream)
+    # The last nbr replays (about 1/16 of them, at least one per layer cache, at most NG)
+    # carry the page-bound kernel's events; the rest replay the plain graphs.
+    nbr = min(NG, K, max(L, (K // 16) // L * L))
+    used = []
     for i in range(K):
-        j = i - (K - NG)  # the last NG replays carry the page-bound kernel's events
+        j = i - (K - nbr)
         if j >= 0:  # same layer rotation; each bracketed graph replays once
-            graphs[(j // L) * L + i % L].replay()
+            used.append((j // L) * L + i % L)
+            graphs[used[-1]].replay()
         else:
             plain[i % L].replay()
     t1.record(stream)
@@ -784,8 +797,8 @@ def main():
     if world > 1:
         dist.barrier()
     ms_total = t0.elapsed_time(t1)
-    # The last NG replays of the timed region hold the page-bound kernel's events.
-    bound_ms = [a.elapsed_time(b) for a, b in ev_b[max(0, NG - K):]]
+    # The bracketed replays of the timed region hold the page-bound kernel's events.
+    bound_ms = [ev_b[u][0].elapsed_time(ev_b[u][1]) for u in used]
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / K
     value = job_throughput(world, wl.batch, K, ms_total)
@@ -940,8 +953,8 @@ def main():
     traffic = prof[0] * bound_bytes / prof[1] if prof is not None else None
     step_gbs = req / (ms_step / 1e3) / 1e9
 
-    # The other SURVEY workloads (configs 1, 2, 3 at batch 1, 4 and 5), each graph-timed on
-    # its own layer caches; single-GPU default runs only.
+    # The other workloads (tiny single head, 32K, 128K at batch 1, the HISA indexer and the
+    # ragged batch), each graph-timed on its own layer caches; single-GPU default runs only.
     other = None
     if (rank == 0 and world == 1 and not args.no_secondary and fused and args.batch == 0
             and args.workload == "llama8b_128k_b8"):
@@ -981,7 +994,7 @@ def main():
                        "api": "hhr_decode_step" if args.path == "fused" else
                               "hhr_encode_keys + hhr_select + hhr_sparse_attn",
                        "timing": f"CUDA-graph replay per step, CUDA events on the stream; the "
-                                 f"last {NG} replays carry event nodes around the page-bound "
+                                 f"last {nbr} of {K} replays carry event nodes around the page-bound "
                                  f"kernel (its duration for the roofline)"},
             "roofline": {"bound": "hbm", "kernel": f"page_bound_{args.summary}_kernel",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",

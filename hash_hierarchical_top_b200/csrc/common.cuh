@@ -9,7 +9,7 @@
 namespace hhr {
 
 constexpr int kD = 128;         // head_dim supported by every kernel
-constexpr int kWords = 4;       // 128-bit codes as 4 x uint32
+constexpr int kWords = 4;       // 128-bit codes as 4 x uint32 (the tensor-core encoder)
 constexpr int kMaxGroup = 8;    // query heads per KV group
 constexpr unsigned kFull = 0xffffffffu;
 

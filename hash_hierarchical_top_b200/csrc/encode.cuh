@@ -90,12 +90,13 @@ struct EncodeArgs {
 
 // One CTA of kMvThreads threads per (touched page, KV group, sequence). The new keys of
 // the page are processed kVecChunk at a time: k' = R_g k (row_dot16; the 16 threads of
-// row r own channel r), min/max folded per channel, then p = W_g k' and the sign bit of
-// row r is OR-ed into the key's code word r / 32.
+// row r own channel r), min/max folded per channel, then p = W_g k' (32 CW rows) and the
+// sign bit of row r is OR-ed into the key's code word r / 32. CW: 32-bit code words.
+template <int CW>
 __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   __shared__ __align__(16) float kx[kVecChunk][kD];  // raw keys (fp32)
   __shared__ __align__(16) float kr[kVecChunk][kD];  // rotated keys
-  __shared__ uint32_t cword[kVecChunk][kWords];
+  __shared__ uint32_t cword[kVecChunk][CW];
 
   const int b = blockIdx.z, g = blockIdx.y, j = blockIdx.x;
   const int tid = threadIdx.x;
@@ -129,12 +130,12 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
   if (a.R != nullptr) {
     // R_g and W_g rows of this thread, and the page's stored summary when the page already
     // held keys, are fetched up front (one memory latency for all of them).
-    float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];
+    float4 rrow[kRowBlocks][2], wrow[CW][2];
 #pragma unroll
-    for (int rb = 0; rb < kRowBlocks; ++rb) {
-      load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
-      load_row16(a.W + (size_t)g * kD * kD, rb * 32 + lrow, wrow[rb]);
-    }
+    for (int rb = 0; rb < kRowBlocks; ++rb) load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
+#pragma unroll
+    for (int wb = 0; wb < CW; ++wb)
+      load_row16(a.W + (size_t)g * (32 * CW) * kD, wb * 32 + lrow, wrow[wb]);
     const size_t sbase = ((size_t)phys * G + g) * 2 * kD;
     float mn[kRowBlocks], mx[kRowBlocks];
 #pragma unroll
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
         const int v = i / kD, c = i % kD;
         kx[v][c] = v < nv ? bf16_to_f(kpage[(size_t)(t + v - pstart) * kD + c]) : 0.f;
       }
-      if (tid < kVecChunk * kWords) cword[tid / kWords][tid % kWords] = 0u;
+      if (tid < kVecChunk * CW) cword[tid / CW][tid % CW] = 0u;
       __syncthreads();
 #pragma unroll
       for (int rb = 0; rb < kRowBlocks; ++rb) {
@@ -177,17 +178,17 @@ __global__ void __launch_bounds__(kMvThreads) encode_page_kernel(EncodeArgs a) {
       }
       __syncthreads();
 #pragma unroll
-      for (int rb = 0; rb < kRowBlocks; ++rb) {
+      for (int wb = 0; wb < CW; ++wb) {
 #pragma unroll
         for (int v = 0; v < kVecChunk; ++v) {
-          const float p = row_dot16(wrow[rb], &kr[v][0]);
-          if (row_lead && p > 0.f) atomicOr(&cword[v][rb], 1u << lrow);
+          const float p = row_dot16(wrow[wb], &kr[v][0]);
+          if (row_lead && p > 0.f) atomicOr(&cword[v][wb], 1u << lrow);
         }
       }
       __syncthreads();
-      if (tid < kVecChunk * kWords) {
-        const int v = tid / kWords, w = tid % kWords;
-        if (v < nv) a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * kWords + w] = cword[v][w];
+      if (tid < kVecChunk * CW) {
+        const int v = tid / CW, w = tid % CW;
+        if (v < nv) a.codes[(((size_t)phys * G + g) * P + (t + v - pstart)) * CW + w] = cword[v][w];
       }
     }
     if (row_lead) {

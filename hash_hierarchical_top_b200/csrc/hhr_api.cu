@@ -42,13 +42,18 @@ int check_dims(const hhr_dims* d) {
       d->max_pages_per_seq < 1 || d->n_phys_pages < 1)
     return HHR_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads != 0) return HHR_ERR_INVALID_ARG;
-  if (d->head_dim != kD || d->code_bits != 32 * kWords) return HHR_ERR_UNSUPPORTED;
+  if (d->head_dim != kD) return HHR_ERR_UNSUPPORTED;
+  if (d->code_bits != 64 && d->code_bits != 128 && d->code_bits != 256) return HHR_ERR_UNSUPPORTED;
   if (d->page_size > 256 || d->batch > 65535 || d->n_kv_heads > 65535)
     return HHR_ERR_UNSUPPORTED;
   if (d->max_pages_per_seq > kMaxPagesPerSeq) return HHR_ERR_UNSUPPORTED;
   if (d->summary_fp16 != 0 && d->summary_fp16 != 1) return HHR_ERR_INVALID_ARG;
   return HHR_OK;
 }
+
+// 32-bit code words per key and its index among the supported lengths (2, 4, 8 words).
+inline int code_words(const hhr_dims* d) { return d->code_bits / 32; }
+inline int cw_index(int cw) { return cw == 2 ? 0 : cw == 4 ? 1 : 2; }
 
 int check_group(const hhr_dims* d) {
   return (d->n_q_heads / d->n_kv_heads > kMaxGroup) ? HHR_ERR_UNSUPPORTED : HHR_OK;
@@ -79,8 +84,8 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   return e;
 }
 
-bool g_smem_tc[kMaxDevices], g_smem_encode[kMaxDevices], g_smem_qprep[kMaxDevices], g_smem_sel[kMaxDevices],
-    g_smem_ham[4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
+bool g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
+    g_smem_sel[kMaxDevices], g_smem_ham[3][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
     g_smem_attn_cl[kMaxDevices];
 
 struct SelectLayout {
@@ -98,7 +103,7 @@ SelectLayout select_layout(const hhr_dims* d, int mode, int m_max) {
   if (mode == HHR_MODE_HASH) {
     L.qpn = off;    off += align256(B * G * 2 * kD * 4);
     L.q_rot = off;  off += align256(B * Hq * kD * 4);
-    L.q_code = off; off += align256(B * Hq * kWords * 4);
+    L.q_code = off; off += align256(B * Hq * code_words(d) * 4);
     L.bounds = off; off += align256(B * G * maxp * 4);
     L.kept = off;   off += align256(B * G * (size_t)m_max * 4);
     L.kept_count = off; off += align256(B * G * 4);
@@ -122,8 +127,9 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
     if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
     if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
       return HHR_ERR_UNSUPPORTED;
-    if (topm_hamming_smem(d->n_q_heads / d->n_kv_heads, kept_max(d, m_pages, keep_div),
-                          d->page_size, d->max_pages_per_seq) > kMaxKernelSmem)
+    if (topm_hamming_smem(d->n_q_heads / d->n_kv_heads, code_words(d),
+                          kept_max(d, m_pages, keep_div), d->page_size,
+                          d->max_pages_per_seq) > kMaxKernelSmem)
       return HHR_ERR_UNSUPPORTED;
   } else if (mode == HHR_MODE_INDEXER) {
     if (m_pages < 1 || keep_div != 0) return HHR_ERR_INVALID_ARG;
@@ -245,8 +251,10 @@ int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* p
   const long long pages = (long long)(max_new + d->page_size - 1) / d->page_size + 1;
   if (pages > 0x7fffffffLL) return HHR_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
-  if (hashing && block_mean == nullptr && d->page_size == kTcPage && max_new >= kTcMinBulk) {
-    // Bulk append (e.g. a prefill): the tensor-core encoder.
+  const int cw = code_words(d);
+  if (hashing && block_mean == nullptr && d->page_size == kTcPage && max_new >= kTcMinBulk &&
+      cw == kWords) {
+    // Bulk append (e.g. a prefill) of 128-bit codes: the tensor-core encoder.
     if (allow_smem(encode_tc_kernel, kTcSmem, g_smem_tc) != cudaSuccess) return HHR_ERR_CUDA;
     const int G = d->n_kv_heads;
     int cpg = kTcSlots / G;
@@ -263,11 +271,13 @@ int hhr_encode_keys(const hhr_dims* d, const uint16_t* k_cache, const int32_t* p
                page_minmax, codes, block_mean, d->n_kv_heads, d->page_size,
                d->max_pages_per_seq, d->n_phys_pages, max_new, d->summary_fp16};
   size_t smem = hashing ? encode_page_smem() : 0;
-  if (hashing && allow_smem(encode_page_kernel, smem, g_smem_encode) != cudaSuccess)
+  void (*enc)(EncodeArgs) =
+      cw == 2 ? encode_page_kernel<2> : cw == 8 ? encode_page_kernel<8> : encode_page_kernel<4>;
+  if (hashing && allow_smem(enc, smem, g_smem_encode[cw_index(cw)]) != cudaSuccess)
     return HHR_ERR_CUDA;
   dim3 grid((unsigned)pages, d->n_kv_heads, d->batch);
   prof_begin(HHR_KERNEL_ENCODE, s);
-  encode_page_kernel<<<grid, kMvThreads, smem, s>>>(a);
+  enc<<<grid, kMvThreads, smem, s>>>(a);
   prof_end(HHR_KERNEL_ENCODE, s);
   return launch_status();
 }
@@ -315,12 +325,15 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     float* qpn = reinterpret_cast<float*>(ws + L.qpn);
     float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
     uint32_t* q_code = reinterpret_cast<uint32_t*>(ws + L.q_code);
-    if (allow_smem(qprep_kernel, qprep_smem(), g_smem_qprep) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(topm_hamming_for(Hq / G), topm_hamming_smem(Hq / G, m_max, P, maxp),
-                   g_smem_ham[hamming_planes(Hq / G) - 1]) != cudaSuccess)
+    const int cw = code_words(d);
+    void (*qp)(QPrepArgs) =
+        cw == 2 ? qprep_kernel<2> : cw == 8 ? qprep_kernel<8> : qprep_kernel<4>;
+    if (allow_smem(qp, qprep_smem(), g_smem_qprep[cw_index(cw)]) != cudaSuccess) return HHR_ERR_CUDA;
+    if (allow_smem(topm_hamming_for(Hq / G, cw), topm_hamming_smem(Hq / G, cw, m_max, P, maxp),
+                   g_smem_ham[cw_index(cw)][hamming_planes(Hq / G) - 1]) != cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
-    qprep_kernel<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
+    qp<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
         QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
     prof_end(HHR_KERNEL_QPREP, s);
     if ((st = launch_status()) != HHR_OK) return st;
@@ -339,15 +352,15 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     if ((st = launch_status()) != HHR_OK) return st;
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
-    const size_t fsm = topm_hamming_smem(Hq / G, m_max, P, maxp);
+    const size_t fsm = topm_hamming_smem(Hq / G, cw, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
-    topm_hamming_for(Hq / G)<<<B * G * kHamRanks, kHamThreads, fsm, s>>>(
+    topm_hamming_for(Hq / G, cw)<<<B * G * kHamRanks, topm_hamming_threads(cw), fsm, s>>>(
         TopmHammingArgs{ha, bounds, m_pages, keep_div});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
     if (trace != nullptr) {
       if ((st = copy_trace(trace->q_rot, ws, L.q_rot, (size_t)B * Hq * kD * 4, s))) return st;
-      if ((st = copy_trace(trace->q_code, ws, L.q_code, (size_t)B * Hq * kWords * 4, s))) return st;
+      if ((st = copy_trace(trace->q_code, ws, L.q_code, (size_t)B * Hq * cw * 4, s))) return st;
       if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * G * maxp * 4, s))) return st;
       if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * G * m_max * 4, s))) return st;
       if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * G * 4, s))) return st;
@@ -506,8 +519,10 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   float* part_o = reinterpret_cast<float*>(aws);
   float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
   uint32_t* sel_rows = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
-  const size_t fsm = topm_hamming_smem(gs, m_max, P, maxp);
-  if (allow_smem(topm_hamming_for(gs), fsm, g_smem_ham[hamming_planes(gs) - 1]) != cudaSuccess)
+  const int cw = code_words(d);
+  const size_t fsm = topm_hamming_smem(gs, cw, m_max, P, maxp);
+  if (allow_smem(topm_hamming_for(gs, cw), fsm, g_smem_ham[cw_index(cw)][hamming_planes(gs) - 1]) !=
+      cudaSuccess)
     return HHR_ERR_CUDA;
   if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
@@ -517,7 +532,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
 
   // a0 + a1: append and encode the newest key rows, rotate and encode the queries.
   prof_begin(HHR_KERNEL_ENCODE, s);
-  step_prologue_for(gs)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
+  step_prologue_for(gs, cw)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
                    d->summary_fp16});
@@ -540,7 +555,8 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows};
     prof_begin(HHR_KERNEL_HAMMING, s);
-    e = launch_pdl(topm_hamming_for(gs), dim3(B * G * kHamRanks), dim3(kHamThreads), fsm, s,
+    e = launch_pdl(topm_hamming_for(gs, cw), dim3(B * G * kHamRanks),
+                   dim3(topm_hamming_threads(cw)), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div});
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }

@@ -22,31 +22,32 @@ struct QPrepArgs {
   const float* R;
   const float* W;
   float* q_rot;      // [B][Hq][d]
-  uint32_t* q_code;  // [B][Hq][4]
+  uint32_t* q_code;  // [B][Hq][CW]
   float* qpn;        // [B][G][2][d]: [0] = qneg, [1] = qpos
   int Hq, G;
 };
 
+template <int CW>
 __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
   __shared__ __align__(16) float qx[kMaxGroup][kD];
   __shared__ __align__(16) float qr[kMaxGroup][kD];
-  __shared__ uint32_t cword[kMaxGroup][kWords];
+  __shared__ uint32_t cword[kMaxGroup][CW];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int lrow = mv_lrow();
   const bool row_lead = mv_part() == 0;
   const int gs = a.Hq / a.G;
   // R_g and W_g rows of this thread are fetched up front (one memory latency for both).
-  float4 rrow[kRowBlocks][2], wrow[kRowBlocks][2];
+  float4 rrow[kRowBlocks][2], wrow[CW][2];
 #pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
-    load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
-    load_row16(a.W + (size_t)g * kD * kD, rb * 32 + lrow, wrow[rb]);
-  }
+  for (int rb = 0; rb < kRowBlocks; ++rb) load_row16(a.R + (size_t)g * kD * kD, rb * 32 + lrow, rrow[rb]);
+#pragma unroll
+  for (int wb = 0; wb < CW; ++wb)
+    load_row16(a.W + (size_t)g * (32 * CW) * kD, wb * 32 + lrow, wrow[wb]);
   for (int i = tid; i < kMaxGroup * kD; i += kMvThreads) {
     const int h = i / kD, c = i % kD;
     qx[h][c] = h < gs ? bf16_to_f(a.q[((size_t)b * a.Hq + g * gs + h) * kD + c]) : 0.f;
   }
-  if (tid < kMaxGroup * kWords) cword[tid / kWords][tid % kWords] = 0u;
+  if (tid < kMaxGroup * CW) cword[tid / CW][tid % CW] = 0u;
   __syncthreads();
   float qneg[kRowBlocks], qpos[kRowBlocks];
 #pragma unroll
@@ -65,16 +66,16 @@ __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
   }
   __syncthreads();
 #pragma unroll
-  for (int rb = 0; rb < kRowBlocks; ++rb) {
+  for (int wb = 0; wb < CW; ++wb) {
     for (int h = 0; h < gs; ++h) {
-      const float p = row_dot16(wrow[rb], &qr[h][0]);
-      if (row_lead && p > 0.f) atomicOr(&cword[h][rb], 1u << lrow);
+      const float p = row_dot16(wrow[wb], &qr[h][0]);
+      if (row_lead && p > 0.f) atomicOr(&cword[h][wb], 1u << lrow);
     }
   }
   __syncthreads();
-  if (tid < gs * kWords) {
-    const int h = tid / kWords, w = tid % kWords;
-    a.q_code[((size_t)b * a.Hq + g * gs + h) * kWords + w] = cword[h][w];
+  if (tid < gs * CW) {
+    const int h = tid / CW, w = tid % CW;
+    a.q_code[((size_t)b * a.Hq + g * gs + h) * CW + w] = cword[h][w];
   }
   if (row_lead) {
     float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
@@ -549,17 +550,21 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 // code word as NB bit planes (NB = bit width of gs), so one select per plane and word
 // gives the contributions' bits, and a carry-save step over the 4 words leaves 3
 // popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
-constexpr int kHamThreads = 1024;
 constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
-// Code loads in flight per thread (fewer with 4 planes, whose 32 plane words fill registers).
-template <int NB>
-constexpr int ham_load() { return NB >= 4 ? 2 : 4; }
 constexpr int kMaxCand = 65536;
-constexpr int kHamBins = (kMaxGroup * 128 + 1 + kHamThreads - 1) / kHamThreads;  // per thread
+constexpr int kMaxCodeWords = 8;  // 256-bit codes
+
+// Threads of a top-m + Hamming CTA: 1024, or 512 for 8-word codes (whose query bit planes
+// need the larger register budget).
+template <int CW>
+constexpr int ham_threads() { return CW >= 8 ? 512 : 1024; }
+// Code loads in flight per thread (fewer when the plane words fill the registers).
+template <int NB, int CW>
+constexpr int ham_load() { return NB * CW >= 16 ? 2 : 4; }
 
 struct HammingArgs {
-  const uint32_t* q_code;    // [B][Hq][4]
-  const uint32_t* codes;     // [n_phys][G][P][4]
+  const uint32_t* q_code;    // [B][Hq][CW]
+  const uint32_t* codes;     // [n_phys][G][P][CW]
   const int32_t* page_table;
   const int32_t* seq_len;
   const int32_t* kept;       // [B][G][m_max]
@@ -573,23 +578,23 @@ struct HammingArgs {
 
 inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
 
-template <int NB>
+template <int NB, int CW>
 struct QueryPlanes {
-  uint32_t n[kWords][NB];  // bit planes of #heads with a 1 bit
-  uint32_t z[kWords][NB];  // bit planes of #heads with a 0 bit
+  uint32_t n[CW][NB];  // bit planes of #heads with a 1 bit
+  uint32_t z[CW][NB];  // bit planes of #heads with a 0 bit
 };
 
 // One plane set of the bit-sliced counts: thread (kind, w) adds, with ripple carries, the
-// bit vector of word w of every head's query code (q_code_w[h * 4], kind 0) or of its
+// bit vector of word w of every head's query code (q_code_w[h * stride], kind 0) or of its
 // complement (kind 1). Result: out[b] for b < NB.
 template <int NB>
-__device__ __forceinline__ void build_plane_word(const uint32_t* q_code_w, int gs, int kind,
-                                                 uint32_t* out) {
+__device__ __forceinline__ void build_plane_word(const uint32_t* q_code_w, int stride, int gs,
+                                                 int kind, uint32_t* out) {
   uint32_t pl[NB];
 #pragma unroll
   for (int b = 0; b < NB; ++b) pl[b] = 0u;
   for (int h = 0; h < gs; ++h) {
-    uint32_t c = q_code_w[h * kWords];
+    uint32_t c = q_code_w[h * stride];
     if (kind) c = ~c;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -602,18 +607,48 @@ __device__ __forceinline__ void build_plane_word(const uint32_t* q_code_w, int g
   for (int b = 0; b < NB; ++b) out[b] = pl[b];
 }
 
-template <int NB>
-__device__ __forceinline__ int hamming_delta(const QueryPlanes<NB>& p, const uint4 c) {
-  const uint32_t cw[kWords] = {c.x, c.y, c.z, c.w};
+// CW code words of a candidate (16-byte loads, 8-byte for two words).
+template <int CW>
+__device__ __forceinline__ void load_code(const uint32_t* p, uint32_t (&c)[CW]) {
+  if constexpr (CW == 2) {
+    const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+    c[0] = v.x;
+    c[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < CW / 4; ++i) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+      c[4 * i] = v.x;
+      c[4 * i + 1] = v.y;
+      c[4 * i + 2] = v.z;
+      c[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// Sum over the group's heads of popcount(qcode_h ^ c), from the bit planes: per plane b the
+// selected contribution bits of each word, summed with one carry-save step per 4 words (3
+// popcounts per 4 words), weighted by 2^b.
+template <int NB, int CW>
+__device__ __forceinline__ int hamming_delta(const QueryPlanes<NB, CW>& p, const uint32_t (&cw)[CW]) {
   int d = 0;
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    uint32_t x[kWords];
+    uint32_t x[CW];
 #pragma unroll
-    for (int w = 0; w < kWords; ++w) x[w] = (cw[w] & p.z[w][b]) | (~cw[w] & p.n[w][b]);
-    const uint32_t sum = x[0] ^ x[1] ^ x[2];
-    const uint32_t carry = (x[0] & x[1]) | (x[2] & (x[0] ^ x[1]));
-    d += (__popc(sum) + __popc(x[3]) + 2 * __popc(carry)) << b;
+    for (int w = 0; w < CW; ++w) x[w] = (cw[w] & p.z[w][b]) | (~cw[w] & p.n[w][b]);
+    int cnt = 0;
+    if constexpr (CW == 2) {
+      cnt = __popc(x[0]) + __popc(x[1]);
+    } else {
+#pragma unroll
+      for (int w = 0; w < CW; w += 4) {
+        const uint32_t sum = x[w] ^ x[w + 1] ^ x[w + 2];
+        const uint32_t carry = (x[w] & x[w + 1]) | (x[w + 2] & (x[w] ^ x[w + 1]));
+        cnt += __popc(sum) + __popc(x[w + 3]) + 2 * __popc(carry);
+      }
+    }
+    d += cnt << b;
   }
   return d;
 }
@@ -629,16 +664,17 @@ struct HamShared {
 // in shared memory. CTA r scores candidates [r*half, (r+1)*half); the histograms and the
 // compaction offsets are combined through distributed shared memory.
 // hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
-template <int NB>
+template <int NB, int CW, int NT>
 __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
                                      const int32_t* kphys, int m, const uint32_t* qcs,
-                                     uint32_t (*planes)[kWords][4], uint32_t* hsm, HamShared& hs) {
+                                     uint32_t (*planes)[CW][4], uint32_t* hsm, HamShared& hs) {
+  constexpr int kBins = (kMaxGroup * 32 * CW + 1 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int b = row / a.G, g = row % a.G;
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.G;
-  const int nbins = gs * 128 + 1;
+  const int nbins = gs * 32 * CW + 1;
   m = min(m, a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                                // [nbins]
   uint16_t* dist = reinterpret_cast<uint16_t*>(hist + ((nbins + 31) & ~31));  // [half], 16B-aligned
@@ -647,62 +683,62 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   const int half = ((ceil_div(C, kHamRanks) + 7) / 8) * 8;
   const int lo = min(C, rank * half), hi = min(C, lo + half);
   const int Cr = hi - lo;
-  for (int i = tid; i < nbins; i += kHamThreads) hist[i] = 0;
+  for (int i = tid; i < nbins; i += NT) hist[i] = 0;
   if (tid == 0) { hs.T = -1; hs.need_eq = 0; }
-  if (tid < 2 * kWords) {
-    const int kind = tid / kWords, w = tid % kWords;
-    build_plane_word<NB>(qcs + w, gs, kind, &planes[kind][w][0]);
+  if (tid < 2 * CW) {
+    const int kind = tid / CW, w = tid % CW;
+    build_plane_word<NB>(qcs + w, CW, gs, kind, &planes[kind][w][0]);
   }
   __syncthreads();  // histogram zeroed, planes built
-  QueryPlanes<NB> qp;
+  QueryPlanes<NB, CW> qp;
 #pragma unroll
-  for (int w = 0; w < kWords; ++w) {
+  for (int w = 0; w < CW; ++w) {
 #pragma unroll
     for (int pb = 0; pb < NB; ++pb) {
       qp.n[w][pb] = planes[0][w][pb];
       qp.z[w][pb] = planes[1][w][pb];
     }
   }
-  // Candidates c = lo + tid + j*1024: consecutive threads read consecutive 16-byte codes of
-  // a page (coalesced); all ham_load() code loads of a thread are issued before any math.
+  // Candidates c = lo + tid + j*NT: consecutive threads read consecutive codes of a page
+  // (coalesced); all ham_load() code loads of a thread are issued before any math.
   // c / P by multiply-high: exact for c < 2^24 with magic = floor(2^32 / P) + 1.
   const uint32_t magic = (uint32_t)(0xffffffffu / (uint32_t)a.P) + 1u;
-  constexpr int kHamLoad = ham_load<NB>();
-  for (int c0 = lo; c0 < hi; c0 += kHamThreads * kHamLoad) {
-    uint4 code[kHamLoad];
+  constexpr int kHamLoad = ham_load<NB, CW>();
+  for (int c0 = lo; c0 < hi; c0 += NT * kHamLoad) {
+    uint32_t code[kHamLoad][CW];
     bool ok[kHamLoad];
 #pragma unroll
     for (int j = 0; j < kHamLoad; ++j) {
-      const int c = c0 + j * kHamThreads + tid;
+      const int c = c0 + j * NT + tid;
       ok[j] = false;
-      code[j] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int w = 0; w < CW; ++w) code[j][w] = 0u;
       if (c < hi) {
         const int i = (a.P == 1) ? c : (int)__umulhi((uint32_t)c, magic);
         const int slot = c - i * a.P;
         const int phys = kphys[i];
         if (phys >= 0 && klp[i] * a.P + slot < n) {
           ok[j] = true;
-          code[j] = __ldcs(reinterpret_cast<const uint4*>(
-              a.codes + (((size_t)phys * a.G + g) * a.P + slot) * kWords));
+          load_code<CW>(a.codes + (((size_t)phys * a.G + g) * a.P + slot) * CW, code[j]);
         }
       }
     }
 #pragma unroll
     for (int j = 0; j < kHamLoad; ++j) {
-      const int c = c0 + j * kHamThreads + tid;
-      const int d = hamming_delta<NB>(qp, code[j]);
+      const int c = c0 + j * NT + tid;
+      const int d = hamming_delta<NB, CW>(qp, code[j]);
       if (ok[j]) atomicAdd(&hist[d], 1);
       if (c < hi) dist[c - lo] = ok[j] ? (uint16_t)d : (uint16_t)0xffff;
     }
   }
   cluster_sync_all();  // every rank's histogram is complete
   // Threshold bucket: smallest T with #(delta <= T) >= k_eff over the summed histograms.
-  // Thread t holds bins [kHamBins t, kHamBins (t + 1)) (fewer past nbins).
+  // Thread t holds bins [kBins t, kBins (t + 1)) (fewer past nbins).
   {
-    int hv[kHamBins], sum = 0;
+    int hv[kBins], sum = 0;
 #pragma unroll
-    for (int q = 0; q < kHamBins; ++q) {
-      const int i = kHamBins * tid + q;
+    for (int q = 0; q < kBins; ++q) {
+      const int i = kBins * tid + q;
       hv[q] = 0;
       if (i < nbins) {
 #pragma unroll
@@ -717,9 +753,9 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
       int run = excl;
       bool found = false;
 #pragma unroll
-      for (int q = 0; q < kHamBins; ++q) {
+      for (int q = 0; q < kBins; ++q) {
         if (!found && keff <= run + hv[q]) {
-          hs.T = kHamBins * tid + q;
+          hs.T = kBins * tid + q;
           hs.need_eq = keff - run;
           found = true;
         }
@@ -728,13 +764,13 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
     }
     if (tid == 0) a.out_count[row] = keff;  // every rank writes the same value
     __syncthreads();
-    for (int i = keff + rank * kHamThreads + tid; i < a.top_k; i += kHamRanks * kHamThreads)
+    for (int i = keff + rank * NT + tid; i < a.top_k; i += kHamRanks * NT)
       a.out_idx[(size_t)row * a.top_k + i] = -1;
   }
   const int T = hs.T, need_eq = hs.need_eq;
   // Ordered compaction of this rank's candidates: thread t owns [t*cpt, (t+1)*cpt), cpt a
   // multiple of 8, read as 16-byte groups of 8 distances.
-  const int cpt = ((ceil_div(Cr, kHamThreads) + 7) / 8) * 8;
+  const int cpt = ((ceil_div(Cr, NT) + 7) / 8) * 8;
   const int ngrp = cpt / 8;
   auto load8 = [&](int i0, uint16_t (&dv)[8]) {
     uint4 raw = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
@@ -801,8 +837,8 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   cluster_wait();  // keep this CTA's shared memory alive until every rank has read it
 }
 
-inline size_t hamming_smem(int gs, int m_max, int P) {
-  const int nbins = gs * 128 + 1;
+inline size_t hamming_smem(int gs, int cw, int m_max, int P) {
+  const int nbins = gs * 32 * cw + 1;
   const size_t ints = (size_t)((nbins + 31) & ~31);
   // This rank's distances, padded so the 16-byte group reads of the last thread stay inside.
   const size_t c = (size_t)m_max * P < (size_t)kMaxCand ? (size_t)m_max * P : (size_t)kMaxCand;
@@ -821,24 +857,29 @@ struct TopmHammingArgs {
   int m_pages, keep_div;
 };
 
-// Per-warp ballots of the kept-page pass of topm_hamming_kernel.
-constexpr int kTopmWarps = kHamThreads / 32;
-constexpr int kTopmChunks = 32;   // 32-page chunks per warp: up to 32 * 32 * 32 = 32768 pages
+// Per-warp ballots of the kept-page pass of topm_hamming_kernel: NT / 32 warps share the
+// 32768 pages a sequence may hold, in 32-page chunks.
+constexpr int kTopmPages = 32768;
 constexpr int kTopmPtPre = 4;     // chunks whose page-table entries are loaded up front
+template <int NT>
 struct TopmShared {
-  uint32_t bal[kTopmWarps][kTopmChunks][2];  // (above, tie) ballots per warp and chunk
-  int cnt[kTopmWarps][2];                    // per-warp counts, then their exclusive prefix
+  static constexpr int kWarps = NT / 32;
+  static constexpr int kChunks = kTopmPages / 32 / kWarps;
+  uint32_t bal[kWarps][kChunks][2];  // (above, tie) ballots per warp and chunk
+  int cnt[kWarps][2];                // per-warp counts, then their exclusive prefix
+  static_assert(kWarps <= 32, "the warp-prefix scan covers the warps with one warp");
 };
-static_assert(kTopmWarps == 32, "the warp-prefix scan covers 32 warps with one warp");
 
-template <int NB>
-__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
+template <int NB, int CW>
+__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(ham_threads<CW>())
     topm_hamming_kernel(TopmHammingArgs a) {
+  constexpr int NT = ham_threads<CW>();
+  constexpr int kTopmWarps = NT / 32;
   __shared__ SelShared sh;
   __shared__ HamShared hs;
-  __shared__ uint32_t qcs[kMaxGroup * kWords];     // the group's query codes
-  __shared__ uint32_t planes[2][kWords][4];         // their bit planes
-  __shared__ TopmShared ts;
+  __shared__ uint32_t qcs[kMaxGroup * CW];     // the group's query codes
+  __shared__ uint32_t planes[2][CW][4];         // their bit planes
+  __shared__ TopmShared<NT> ts;
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint32_t fsm[];
@@ -846,8 +887,8 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
   const int b = row / h.G, g = row % h.G;
   const int gs = h.Hq / h.G;
-  if (threadIdx.x < gs * kWords)  // visible after the selection's first barrier
-    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + g * gs) * kWords + threadIdx.x];
+  if (threadIdx.x < gs * CW)  // visible after the selection's first barrier
+    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + g * gs) * CW + threadIdx.x];
   const int mw = (h.m_max + 3) & ~3;
   int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
   int32_t* kphys_s = kept_s + mw;
@@ -867,7 +908,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
     const int p = wbase + 32 * j + lane;
     pt[j] = (j < J && p < n) ? ptab[p] : -1;
   }
-  const SelCut cut = block_select_cut<kHamThreads>(a.bounds + (size_t)row * h.maxp, n, work, sh,
+  const SelCut cut = block_select_cut<NT>(a.bounds + (size_t)row * h.maxp, n, work, sh,
                                                    true, a.m_pages, a.keep_div, 0);
   int ng = 0, ne = 0;
   for (int j = 0; j < J; ++j) {
@@ -888,18 +929,21 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   }
   __syncthreads();
   if (warp == 0) {  // exclusive prefix over the warps of (above, tie) counts
-    const int xg = ts.cnt[lane][0], xe = ts.cnt[lane][1];
+    const int xg = lane < kTopmWarps ? ts.cnt[lane][0] : 0;
+    const int xe = lane < kTopmWarps ? ts.cnt[lane][1] : 0;
     const int ig = warp_incl_scan(xg, lane), ie = warp_incl_scan(xe, lane);
-    ts.cnt[lane][0] = ig - xg;
-    ts.cnt[lane][1] = ie - xe;
+    if (lane < kTopmWarps) {
+      ts.cnt[lane][0] = ig - xg;
+      ts.cnt[lane][1] = ie - xe;
+    }
   }
   __syncthreads();
   const int m = cut.k;
   int e = ts.cnt[warp][1];                 // ties before this warp's pages
   int pos = ts.cnt[warp][0] + min(e, cut.rem);
   int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
-  const uint32_t* code_g = h.codes + (size_t)g * h.P * kWords;
-  const size_t code_page = (size_t)h.G * h.P * kWords;
+  const uint32_t* code_g = h.codes + (size_t)g * h.P * CW;
+  const size_t code_page = (size_t)h.G * h.P * CW;
   for (int j = 0; j < J; ++j) {
     uint32_t takem = ts.bal[warp][j][0];
     uint32_t be = ts.bal[warp][j][1];
@@ -918,7 +962,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
         flag_status(kStatusBadPage);
         phys = -1;
       } else {
-        prefetch_l2(code_g + (size_t)phys * code_page, (unsigned)(h.P * kWords * 4));
+        prefetch_l2(code_g + (size_t)phys * code_page, (unsigned)(h.P * CW * 4));
       }
       if (kpos < h.m_max) {
         kept_s[kpos] = p;
@@ -930,25 +974,35 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(kHamThreads)
   }
   if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
   __syncthreads();
-  hamming_topk_cluster<NB>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
+  hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
 }
 
-inline size_t topm_hamming_smem(int gs, int m_max, int P, int maxp) {
+inline size_t topm_hamming_smem(int gs, int cw, int m_max, int P, int maxp) {
   const size_t sel = (size_t)maxp * 4;
-  const size_t ham = hamming_smem(gs, m_max, P);
+  const size_t ham = hamming_smem(gs, cw, m_max, P);
   return (size_t)((m_max + 3) & ~3) * 8 + (sel > ham ? sel : ham);
 }
 
 using TopmHammingFn = void (*)(TopmHammingArgs);
 
-// The instantiation for group size gs (1..kMaxGroup).
-inline TopmHammingFn topm_hamming_for(int gs) {
+template <int CW>
+inline TopmHammingFn topm_hamming_for_cw(int gs) {
   switch (hamming_planes(gs)) {
-    case 1: return topm_hamming_kernel<1>;
-    case 2: return topm_hamming_kernel<2>;
-    case 3: return topm_hamming_kernel<3>;
-    default: return topm_hamming_kernel<4>;
+    case 1: return topm_hamming_kernel<1, CW>;
+    case 2: return topm_hamming_kernel<2, CW>;
+    case 3: return topm_hamming_kernel<3, CW>;
+    default: return topm_hamming_kernel<4, CW>;
   }
+}
+
+// The instantiation for group size gs (1..kMaxGroup) and cw code words (2, 4 or 8), with
+// its thread count.
+inline TopmHammingFn topm_hamming_for(int gs, int cw) {
+  return cw == 2 ? topm_hamming_for_cw<2>(gs)
+                 : cw == 8 ? topm_hamming_for_cw<8>(gs) : topm_hamming_for_cw<4>(gs);
+}
+inline int topm_hamming_threads(int cw) {
+  return cw == 8 ? ham_threads<8>() : cw == 2 ? ham_threads<2>() : ham_threads<4>();
 }
 
 // ---------------------------------------------------------------------------- HISA a1'

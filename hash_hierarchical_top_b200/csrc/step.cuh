@@ -29,7 +29,7 @@ struct PrologueArgs {
   void* page_minmax;
   uint32_t* codes;
   float* q_rot;            // [B][Hq][d]
-  uint32_t* q_code;        // [B][Hq][4]
+  uint32_t* q_code;        // [B][Hq][CW]
   float* qpn;              // [B][G][2][d]
   int Hq, G, P, maxp, n_phys, summary_fp16;
 };
@@ -99,23 +99,24 @@ __device__ __forceinline__ void store_bf16x8(const uint4 raw, float* dst) {
 // A cluster of kPrologueRanks CTAs per (group, sequence). CTA r owns rows 32r..32r+31 of R_g
 // and W_g (one row block of row_dot16, 16 threads per row). It rotates all 1 + GS vectors on
 // its rows and sends the results, as 16-byte pieces, into every CTA's copy of the rotated
-// vectors (distributed shared memory); after one cluster barrier it projects them on its rows of W_g, whose 32
-// sign bits are code word r. CTA r also owns summary channels and folded-query channels
-// 32r..32r+31. Every input load is issued at the start; only the key's cache slot (and the
+// vectors (distributed shared memory); after one cluster barrier it projects them on the
+// rows of W_g of code words r, r + 4, ... (below CW), whose 32 sign bits are those words.
+// CTA r also owns summary channels and folded-query channels 32r..32r+31. Every input load is issued at the start; only the key's cache slot (and the
 // key itself when k_new is null) waits for the page table.
 constexpr int kPrologueRanks = kRowBlocks;
 constexpr int kPrologueThreads = kMvThreads;  // 32 rows x 16 threads
 
-template <int GS>
+template <int GS, int CW>
 __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kPrologueThreads)
     step_prologue_cluster_kernel(PrologueArgs a) {
   namespace cg = cooperative_groups;
   constexpr int NV = 1 + GS;  // vector 0: the newest key; 1..GS: the query heads
+  constexpr int kWpr = (CW + kPrologueRanks - 1) / kPrologueRanks;  // code words per rank
   static_assert(16 * (NV + 1) <= kPrologueThreads, "one 16-byte piece per thread");
   __shared__ __align__(16) float xs[NV][kD];  // raw vectors
   __shared__ __align__(16) float xpart[NV][32];  // rotated vectors, this CTA's rows
   __shared__ __align__(16) float xr[NV][kD];     // rotated vectors, every row
-  __shared__ uint32_t cpart[NV][kPrologueThreads / 32];  // sign bits of each warp's rows
+  __shared__ uint32_t cpart[kWpr][NV][kPrologueThreads / 32];  // sign bits of each warp's rows
   pdl_wait();
   pdl_trigger();
   cg::cluster_group cl = cg::this_cluster();
@@ -125,9 +126,13 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   const int row = rank * 32 + lrow;
   const bool row_lead = part == 0;
 
-  float4 rr[2], wr[2];
+  float4 rr[2], wr[kWpr][2];
   load_row16(a.R + (size_t)g * kD * kD, row, rr);
-  load_row16(a.W + (size_t)g * kD * kD, row, wr);
+#pragma unroll
+  for (int i = 0; i < kWpr; ++i) {
+    const int w = rank + kPrologueRanks * i;
+    if (w < CW) load_row16(a.W + (size_t)g * (32 * CW) * kD, w * 32 + lrow, wr[i]);
+  }
   const int len = a.seq_len[b];
   // Threads [16v, 16v + 16) load vector v (k_new, then the queries) as 16-byte pieces of
   // 8 channels; threads [16 NV, 16 NV + 16) load v_new.
@@ -190,31 +195,40 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   }
   cluster_sync_all();  // every rank's rows of every rotated vector have landed
 
-  // LHP codes: the sign of W_g x' on this thread's row is bit lrow of code word `rank`.
-  // Warp w holds rows 2w and 2w + 1: an OR-reduction collects the warp's two bits, and
+  // LHP codes: the sign of W_g x' on this thread's row of word w is bit lrow of code word
+  // w. Warp w holds rows 2w and 2w + 1: an OR-reduction collects the warp's two bits, and
   // warp 0 merges the warps' pieces.
   const int lane = tid & 31, warp = tid >> 5;
-  float pj[NV];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) pj[v] = row_dot16(wr, &xr[v][0]);
+  for (int i = 0; i < kWpr; ++i) {
+    if (rank + kPrologueRanks * i >= CW) continue;  // uniform over the CTA
+    float pj[NV];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const uint32_t bits = __reduce_or_sync(kFull, row_lead && pj[v] > 0.f ? 1u << lrow : 0u);
-    if (lane == 0) cpart[v][warp] = bits;
+    for (int v = 0; v < NV; ++v) pj[v] = row_dot16(wr[i], &xr[v][0]);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const uint32_t bits = __reduce_or_sync(kFull, row_lead && pj[v] > 0.f ? 1u << lrow : 0u);
+      if (lane == 0) cpart[i][v][warp] = bits;
+    }
   }
   __syncthreads();
   if (warp == 0) {
-    uint32_t mine = 0u;
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const uint32_t word =
-          __reduce_or_sync(kFull, lane < kPrologueThreads / 32 ? cpart[v][lane] : 0u);
-      if (lane == v) mine = word;
-    }
-    if (lane == 0) {
-      if (has_key) a.codes[(((size_t)s.phys * a.G + g) * a.P + s.slot) * kWords + rank] = mine;
-    } else if (lane < NV) {
-      a.q_code[((size_t)b * a.Hq + g * GS + (lane - 1)) * kWords + rank] = mine;
+    for (int i = 0; i < kWpr; ++i) {
+      const int w = rank + kPrologueRanks * i;
+      if (w >= CW) continue;
+      uint32_t mine = 0u;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const uint32_t word =
+            __reduce_or_sync(kFull, lane < kPrologueThreads / 32 ? cpart[i][v][lane] : 0u);
+        if (lane == v) mine = word;
+      }
+      if (lane == 0) {
+        if (has_key) a.codes[(((size_t)s.phys * a.G + g) * a.P + s.slot) * CW + w] = mine;
+      } else if (lane < NV) {
+        a.q_code[((size_t)b * a.Hq + g * GS + (lane - 1)) * CW + w] = mine;
+      }
     }
   }
   if (row_lead) {
@@ -227,18 +241,24 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
 
 using PrologueFn = void (*)(PrologueArgs);
 
-// The instantiation for group size gs (1..kMaxGroup).
-inline PrologueFn step_prologue_for(int gs) {
+template <int CW>
+inline PrologueFn step_prologue_for_cw(int gs) {
   switch (gs) {
-    case 1: return step_prologue_cluster_kernel<1>;
-    case 2: return step_prologue_cluster_kernel<2>;
-    case 3: return step_prologue_cluster_kernel<3>;
-    case 4: return step_prologue_cluster_kernel<4>;
-    case 5: return step_prologue_cluster_kernel<5>;
-    case 6: return step_prologue_cluster_kernel<6>;
-    case 7: return step_prologue_cluster_kernel<7>;
-    default: return step_prologue_cluster_kernel<8>;
+    case 1: return step_prologue_cluster_kernel<1, CW>;
+    case 2: return step_prologue_cluster_kernel<2, CW>;
+    case 3: return step_prologue_cluster_kernel<3, CW>;
+    case 4: return step_prologue_cluster_kernel<4, CW>;
+    case 5: return step_prologue_cluster_kernel<5, CW>;
+    case 6: return step_prologue_cluster_kernel<6, CW>;
+    case 7: return step_prologue_cluster_kernel<7, CW>;
+    default: return step_prologue_cluster_kernel<8, CW>;
   }
+}
+
+// The instantiation for group size gs (1..kMaxGroup) and cw code words (2, 4 or 8).
+inline PrologueFn step_prologue_for(int gs, int cw) {
+  return cw == 2 ? step_prologue_for_cw<2>(gs)
+                 : cw == 8 ? step_prologue_for_cw<8>(gs) : step_prologue_for_cw<4>(gs);
 }
 
 }  // namespace hhr

@@ -209,16 +209,14 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0, with_values: bool = 
             del v
 
     gR = _gen("cpu", wl, J_R, layer)
-    gW = _gen("cpu", wl, J_W, layer)
     R = torch.empty(G, d, d, dtype=torch.float32)
-    W = torch.empty(G, wl.code_bits, d, dtype=torch.float32)
     for g in range(G):
         a = torch.randn(d, d, generator=gR, dtype=torch.float64)
         Qm, Rr = torch.linalg.qr(a)
         # Fix the column signs so the factorisation is unique.
         Qm = Qm * torch.sign(torch.diagonal(Rr))[None, :]
         R[g] = Qm.to(torch.float32)
-        W[g] = torch.randn(wl.code_bits, d, generator=gW)
+    W = lhp_projection(wl, layer)
 
     out = dict(
         k_cache=k_cache, v_cache=v_cache, q=q_bf,
@@ -232,6 +230,16 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0, with_values: bool = 
                           dtype=torch.int32)
         out["q_pos"] = qp.to(device)
     return out
+
+
+def lhp_projection(wl: Workload, layer: int = 0) -> torch.Tensor:
+    """The projection W [G][code_bits][d] (float32, CPU) of a layer: N(0, 1) entries drawn
+    group by group from the layer's W stream, the same draws make_inputs uses."""
+    gW = _gen("cpu", wl, J_W, layer)
+    W = torch.empty(wl.n_kv_heads, wl.code_bits, wl.head_dim, dtype=torch.float32)
+    for g in range(wl.n_kv_heads):
+        W[g] = torch.randn(wl.code_bits, wl.head_dim, generator=gW)
+    return W
 
 
 def _scatter(cache, pt_row, k, P):

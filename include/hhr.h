@@ -7,7 +7,8 @@
  *     Geometry-Aware Key Routing (a head-wise orthogonal transform R_h and
  *     page-level logit bounds that prune pages), then Learned Hash Projection
  *     (binary codes of a head-wise projection W_h, ranked by Hamming distance),
- *     then attention over the selected keys. Appendix Table 4 fixes 128-bit codes.
+ *     then attention over the selected keys. Appendix Table 4 fixes 128-bit codes;
+ *     64 and 256 bits are supported as code-length variants.
  *   - "HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse Attention",
  *     Abstract: a block-level coarse filter over pooled block representatives,
  *     then the original token indexer inside the kept blocks, then token top-k.
@@ -24,14 +25,14 @@
  *   - Host-side validation runs first and returns an error before any launch:
  *     HHR_ERR_INVALID_ARG (null or misaligned pointer, negative size,
  *     H % G != 0, ...),
- *     HHR_ERR_UNSUPPORTED (head_dim != 128, code_bits != 128, group > 8, a size
+ *     HHR_ERR_UNSUPPORTED (head_dim != 128, code_bits not 64/128/256, group > 8, a size
  *     beyond a documented limit), HHR_ERR_WORKSPACE (workspace too small).
  *     A failed launch returns HHR_ERR_CUDA.
  *   - Device-side checks never trap: a page id outside [0, n_phys_pages) or a
  *     token index outside the sequence is skipped and recorded in a device status
  *     word that hhr_read_device_status returns and clears.
  *
- * Layouts (row-major; d = head_dim = 128, W = code_bits / 32 = 4 words)
+ * Layouts (row-major; d = head_dim = 128, W = code_bits / 32 = 2, 4 or 8 words)
  *   k_cache, v_cache : bf16 (uint16 bit patterns) [n_phys_pages][G][P][d]
  *   page_table       : int32 [B][max_pages_per_seq], logical page -> physical page
  *   seq_len          : int32 [B], keys currently in each sequence (after appends)
@@ -78,7 +79,7 @@ typedef struct {
   int n_kv_heads;         /* G */
   int head_dim;           /* d; must be 128 */
   int page_size;          /* P keys per page (HISA: keys per block), 1..256 */
-  int code_bits;          /* must be 128 */
+  int code_bits;          /* 64, 128 (the pages' setting) or 256 */
   int max_pages_per_seq;  /* columns of page_table */
   int n_phys_pages;       /* pages in the pool */
   int summary_fp16;       /* page_minmax element type: 0 = f32; 1 = f16 rounded outward
@@ -112,9 +113,9 @@ typedef struct {
  *   max_new      : host int, an upper bound on every n_new[b] (sizes the launch;
  *                  a larger n_new[b] is clipped to it and flagged in the device
  *                  status word)
- * Appends of at least 4096 keys (max_new) with page_size 32 and no block means run
- * on the tensor-core encoder (tcgen05: one GEMM per 128-key tile against [R; W R],
- * fp32 operands split into three bf16 terms); others on the per-page encoder. Both
+ * Appends of at least 4096 keys (max_new) with page_size 32, 128-bit codes and no block
+ * means run on the tensor-core encoder (tcgen05: one GEMM per 128-key tile against
+ * [R; W R], fp32 operands split into three bf16 terms); others on the per-page encoder. Both
  * produce the same layout; their results agree within the code and bound tolerances. */
 int hhr_encode_keys(const hhr_dims* dims, const uint16_t* k_cache, const int32_t* page_table,
                     const int32_t* start, const int32_t* n_new, int max_new, const float* R,

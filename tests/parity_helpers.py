@@ -65,7 +65,8 @@ def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
     rows = d.n_kv_heads if hashing else d.n_q_heads
     tr_t = dict(
         q_rot=torch.empty(B, d.n_q_heads, 128, dtype=torch.float32, device=dev) if hashing else None,
-        q_code=torch.empty(B, d.n_q_heads, 4, dtype=torch.int32, device=dev) if hashing else None,
+        q_code=(torch.empty(B, d.n_q_heads, d.code_bits // 32, dtype=torch.int32, device=dev)
+                if hashing else None),
         bounds=torch.empty(B, rows, d.max_pages_per_seq, dtype=torch.float32, device=dev),
         kept=torch.empty(B, rows, step.m_max, dtype=torch.int32, device=dev),
         kept_count=torch.empty(B, rows, dtype=torch.int32, device=dev),
@@ -97,9 +98,9 @@ def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
 
 
 def gpu_codes_logical(g_out, pt_row, g, n, P):
-    """GPU codes of one sequence/group in logical token order, [n][4]."""
+    """GPU codes of one sequence/group in logical token order, [n][code words]."""
     n_pages = -(-n // P)
-    c = g_out["codes"][np.asarray(pt_row[:n_pages], dtype=np.int64), g]  # [n_pages][P][4]
+    c = g_out["codes"][np.asarray(pt_row[:n_pages], dtype=np.int64), g]  # [n_pages][P][CW]
     return c.reshape(n_pages * P, -1)[:n]
 
 
@@ -117,7 +118,8 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
     gc = gpu_codes_logical(g_out, pt, g, n, P)
     diff = gc ^ enc["codes"]
     bad = 0
-    for w in range(4):
+    CW = wl.code_bits // 32
+    for w in range(CW):
         for bit in range(32):
             flips = ((diff[:, w] >> np.uint32(bit)) & 1).astype(bool)
             bad += int(np.count_nonzero(flips & ~enc["fragile"][:, 32 * w + bit]))
@@ -144,7 +146,7 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
     gq = g_out["q_code"][b, g * gs:(g + 1) * gs]
     qd = gq ^ qcodes
     for h in range(gs):
-        for w in range(4):
+        for w in range(CW):
             for bit in range(32):
                 if (int(qd[h, w]) >> bit) & 1:
                     assert qfrag[h, 32 * w + bit], "non-fragile query code bit differs"

@@ -61,7 +61,8 @@ def test_workspace_and_kept_sizes(L):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(head_dim=64), dict(code_bits=64), dict(n_q_heads=30), dict(n_q_heads=72),
+    dict(head_dim=64), dict(code_bits=96), dict(code_bits=512), dict(code_bits=32),
+    dict(n_q_heads=30), dict(n_q_heads=72),
     dict(page_size=0), dict(page_size=512), dict(batch=0), dict(max_pages_per_seq=40000),
 ])
 def test_bad_dims_rejected(L, bad):
@@ -70,6 +71,19 @@ def test_bad_dims_rejected(L, bad):
     st = L.hhr_select(ctypes.byref(d), 0, *([None] * 10), 0, 16, 2048, None, None, None, 0,
                       None, None)
     assert st in (hhr.HHR_ERR_INVALID_ARG, hhr.HHR_ERR_UNSUPPORTED)
+
+
+@pytest.mark.parametrize("bits", [64, 128, 256])
+def test_code_lengths_accepted(L, bits):
+    # 64-, 128- and 256-bit codes: the workspace holds B * Hq query codes of bits / 8 bytes.
+    d = _d(code_bits=bits)
+    ws = hhr.hhr_select_workspace_bytes(d, hhr.HHR_MODE_HASH, 0, 16, 2048)
+    assert ws > 0
+    assert hhr.hhr_decode_step_workspace_bytes(d, 0, 16, 2048) > 0
+    base = hhr.hhr_select_workspace_bytes(_d(code_bits=64), hhr.HHR_MODE_HASH, 0, 16, 2048)
+    q_code_64 = -(-d.batch * d.n_q_heads * 8 // 256) * 256
+    q_code = -(-d.batch * d.n_q_heads * bits // 8 // 256) * 256
+    assert ws - base == q_code - q_code_64
 
 
 def test_select_validation_order(L):

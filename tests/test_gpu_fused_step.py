@@ -38,6 +38,17 @@ def test_fused_step_group_shapes(heads):
     _fused_vs_separate(wl, 1, True)
 
 
+@pytest.mark.parametrize("bits", [64, 256])
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1), (14, 2)])
+def test_fused_step_code_lengths(bits, heads):
+    """64- and 256-bit codes: the prologue projects 2 words on ranks 0-1, or 2 words on
+    every rank, and must match the separate encoder and query prep bit for bit."""
+    hq, g = heads
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=3, ragged=(33, 4000), top_k=200,
+                  n_q_heads=hq, n_kv_heads=g, code_bits=bits)
+    _fused_vs_separate(wl, 1, True)
+
+
 def _fused_vs_separate(wl, f16, with_new_rows):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
@@ -89,7 +100,7 @@ def test_fused_step_against_oracle():
     fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
     B, Hq = wl.batch, wl.n_q_heads
     tr = dict(q_rot=torch.empty(B, Hq, 128, device="cuda"),
-              q_code=torch.empty(B, Hq, 4, dtype=torch.int32, device="cuda"))
+              q_code=torch.empty(B, Hq, wl.code_bits // 32, dtype=torch.int32, device="cuda"))
     fs.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_len"],
                   inp["R"], inp["W"], cache)
     torch.cuda.synchronize()

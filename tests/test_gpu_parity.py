@@ -116,6 +116,34 @@ def test_group_shapes(heads):
     _check_all_groups(wl, inp_np, run_gpu(wl, inp))
 
 
+@pytest.mark.parametrize("bits", [64, 256])
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1), (6, 2)])
+def test_code_lengths(bits, heads):
+    """64- and 256-bit codes (their own encoder, query-prep and Hamming instantiations; the
+    256-bit Hamming stage runs 512 threads): every layered check, for a whole-sequence
+    append and for appends in pieces of 37 keys."""
+    hq, g = heads
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], code_bits=bits, n_q_heads=hq, n_kv_heads=g,
+                  seq_lens=(5000, 2345), batch=2, top_k=400)
+    inp, inp_np = _inputs(wl)
+    a = run_gpu(wl, inp, summary_fp16=1)
+    assert a["codes"].shape[-1] == bits // 32 and a["q_code"].shape[-1] == bits // 32
+    _check_all_groups(wl, inp_np, a)
+    c = run_gpu(wl, inp, encode_chunks=37)
+    _check_all_groups(wl, inp_np, c)
+    assert np.bitwise_count(a["codes"] ^ c["codes"]).sum() <= 16
+
+
+@pytest.mark.parametrize("bits", [64, 256])
+def test_code_lengths_128k_sampled(bits):
+    """Full 128K context with 64- and 256-bit codes: 65536 candidates per group."""
+    wl = S.scaled(S.WORKLOADS["llama8b_128k_b1"], code_bits=bits)
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp, summary_fp16=1)
+    assert np.all(out["count"] == wl.top_k)
+    _check_all_groups(wl, inp_np, out, groups={(0, 1), (0, 6)})
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
