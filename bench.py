@@ -67,14 +67,16 @@ def measured_peaks():
 
 
 def required_bytes(wl, lens, m_of, sbytes=4):
-    """Algorithmic bytes of one step: summaries + kept-page codes + selected K/V rows."""
+    """Algorithmic bytes of one step: summaries (unless every page is kept: a flat top-k
+    needs no bounds) + kept-page codes + selected K/V rows."""
     G, P, d = wl.n_kv_heads, wl.page_size, wl.head_dim
     summ = codes = kv = 0
     for n in lens:
         npg = -(-n // P)
         m = m_of(npg)
         cand = min(n, m * P)
-        summ += G * npg * 2 * d * sbytes
+        if m < npg:
+            summ += G * npg * 2 * d * sbytes
         codes += G * cand * (wl.code_bits // 8)
         kv += G * min(wl.top_k, cand) * 2 * d * 2
     return summ, codes, kv
@@ -354,6 +356,7 @@ def selection_quality(dev):
     sweep = {"quest_R_identity_keep_1/16": hhr_quality(wl, inp, dev, eye, 0, 16, full=False)}
     for kd in (8, 32):
         sweep[f"gkr_keep_1/{kd}"] = hhr_quality(wl, inp, dev, inp["R"], 0, kd, full=False)
+    sweep["flat_all_4096_pages"] = hhr_quality(wl, inp, dev, inp["R"], 4096, 0, full=False)
     for bits in (64, 256):
         wb = S.scaled(wl, code_bits=bits)
         Wb = S.lhp_projection(wb, layer=0).to(dev)
@@ -406,7 +409,8 @@ def selection_quality(dev):
 # ----------------------------------------------------------------------------- other workloads
 
 SECONDARY = ("llama8b_128k_b1", "ragged_b32", "llama8b_32k", "tiny_1h_4k", "hisa_128k_t1",
-             "hisa_128k_t64")
+             "hisa_128k_t64", "llama8b_128k_b8_codes64", "llama8b_128k_b8_codes256",
+             "llama8b_128k_b8_flat")
 
 
 def indexer_required_bytes(wl, lens):
@@ -446,7 +450,7 @@ def measure_secondary(name, dev, l2, f16, steps, stream, mem_cap):
         inp = S.make_inputs(wl, device=dev, layer=l, with_values=hashing)
         d = hhr.make_dims(wl.batch, wl.n_q_heads if hashing else wl.n_queries, wl.n_kv_heads,
                           wl.page_size, inp["max_pages"], inp["n_phys"],
-                          summary_fp16=f16 if hashing else 0)
+                          summary_fp16=f16 if hashing else 0, code_bits=wl.code_bits)
         cache = LayerCache(d, dev, hashing=hashing, block_means=not hashing)
         zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
         hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],

@@ -337,25 +337,27 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
         QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
     prof_end(HHR_KERNEL_QPREP, s);
     if ((st = launch_status()) != HHR_OK) return st;
-    prof_begin(HHR_KERNEL_BOUND, s);
-    {
+    // Every page kept (flat hash top-k): the bounds are computed only for a trace.
+    const bool flat = m_max >= maxp;
+    if (!flat || (trace != nullptr && trace->bounds != nullptr)) {
       const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                          d->n_phys_pages};
       const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
       const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
+      prof_begin(HHR_KERNEL_BOUND, s);
       if (d->summary_fp16)
         page_bound_kernel<true><<<grid, kBoundWarps * 32, 0, s>>>(ba);
       else
         page_bound_kernel<false><<<grid, kBoundWarps * 32, 0, s>>>(ba);
+      prof_end(HHR_KERNEL_BOUND, s);
+      if ((st = launch_status()) != HHR_OK) return st;
     }
-    prof_end(HHR_KERNEL_BOUND, s);
-    if ((st = launch_status()) != HHR_OK) return st;
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
     const size_t fsm = topm_hamming_smem(Hq / G, cw, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
     topm_hamming_for(Hq / G, cw)<<<B * G * kHamRanks, topm_hamming_threads(cw), fsm, s>>>(
-        TopmHammingArgs{ha, bounds, m_pages, keep_div});
+        TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
     if (trace != nullptr) {
@@ -538,8 +540,9 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
                    d->summary_fp16});
   prof_end(HHR_KERNEL_ENCODE, s);
   if ((st = launch_status()) != HHR_OK) return st;
-  // a2: page bounds.
-  {
+  // a2: page bounds (none when every page is kept: a flat hash top-k).
+  const bool flat = m_max >= maxp;
+  if (!flat) {
     const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                        d->n_phys_pages};
     const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
@@ -557,7 +560,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     prof_begin(HHR_KERNEL_HAMMING, s);
     e = launch_pdl(topm_hamming_for(gs, cw), dim3(B * G * kHamRanks),
                    dim3(topm_hamming_threads(cw)), fsm, s,
-                   TopmHammingArgs{ha, bounds, m_pages, keep_div});
+                   TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   }

@@ -551,7 +551,7 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 // gives the contributions' bits, and a carry-save step over the 4 words leaves 3
 // popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
 constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
-constexpr int kMaxCand = 65536;
+constexpr int kMaxCand = 131072;  // a flat top-k over 4096 pages of 32 keys
 constexpr int kMaxCodeWords = 8;  // 256-bit codes
 
 // Threads of a top-m + Hamming CTA: 1024, or 512 for 8-word codes (whose query bit planes
@@ -853,8 +853,9 @@ inline size_t hamming_smem(int gs, int cw, int m_max, int P) {
 // physical pages: m_max words][union of: top-m keys (maxp words) | Hamming scratch].
 struct TopmHammingArgs {
   HammingArgs h;
-  const float* bounds;  // [B][G][maxp]
+  const float* bounds;  // [B][G][maxp]; not read when flat
   int m_pages, keep_div;
+  int flat;             // every page is kept (flat hash top-k): no bounds, no top-m
 };
 
 // Per-warp ballots of the kept-page pass of topm_hamming_kernel: NT / 32 warps share the
@@ -902,6 +903,26 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(ham_threads<
   const int J = R / 32;
   const int wbase = warp * R;
   const int32_t* ptab = h.page_table + (size_t)b * h.maxp;
+  int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
+  const uint32_t* code_g = h.codes + (size_t)g * h.P * CW;
+  const size_t code_page = (size_t)h.G * h.P * CW;
+  if (a.flat) {  // flat hash top-k: the kept list is every page of the sequence
+    const int m = min(n, h.m_max);
+    for (int p = threadIdx.x; p < m; p += NT) {
+      int phys = ptab[p];
+      if (phys < 0 || phys >= h.n_phys) {
+        flag_status(kStatusBadPage);
+        phys = -1;
+      }
+      kept_s[p] = p;
+      kphys_s[p] = phys;
+      if (rank == 0) kept_g[p] = p;
+    }
+    if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
+    __syncthreads();
+    hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
+    return;
+  }
   int pt[kTopmPtPre];  // page-table entries of the first chunks, loaded with the bounds
 #pragma unroll
   for (int j = 0; j < kTopmPtPre; ++j) {
@@ -941,9 +962,6 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(ham_threads<
   const int m = cut.k;
   int e = ts.cnt[warp][1];                 // ties before this warp's pages
   int pos = ts.cnt[warp][0] + min(e, cut.rem);
-  int32_t* kept_g = const_cast<int32_t*>(h.kept) + (size_t)row * h.m_max;
-  const uint32_t* code_g = h.codes + (size_t)g * h.P * CW;
-  const size_t code_page = (size_t)h.G * h.P * CW;
   for (int j = 0; j < J; ++j) {
     uint32_t takem = ts.bal[warp][j][0];
     uint32_t be = ts.bal[warp][j][1];

@@ -108,6 +108,15 @@ WORKLOADS = {
 }
 
 
+# Variants of the 128K batch-8 decode (same keys, queries and rotations): a flat hash top-k
+# (every page kept), and codes of 64 or 256 bits (W has 64 or 256 rows).
+WORKLOADS["llama8b_128k_b8_flat"] = dataclasses.replace(
+    WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_b8_flat", m_pages=4096, keep_div=0)
+for _bits in (64, 256):
+    _n = f"llama8b_128k_b8_codes{_bits}"
+    WORKLOADS[_n] = dataclasses.replace(WORKLOADS["llama8b_128k_b8"], name=_n, code_bits=_bits)
+
+
 def scaled(wl: Workload, **changes) -> Workload:
     """A copy of ``wl`` with some fields replaced (e.g. shorter contexts for parity tests)."""
     return dataclasses.replace(wl, **changes)

@@ -153,7 +153,9 @@ size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, i
  *   a4  out_idx[b][i][0..k_eff) = the k_eff best by (sigma desc, t asc), ascending.
  *   Uses q, seq_len, q_pos, page_table, block_mean, k_cache; R, W, page_minmax and
  *   codes may be NULL. keep_div must be 0.
- * Limits: ceil(seq_len/P) <= 32768 pages per sequence; m_b * P <= 65536 candidates.
+ * Limits: ceil(seq_len/P) <= 32768 pages per sequence; m_b * P <= 131072 candidates
+ * (hash mode: every page of a 128K-key sequence, a flat hash top-k) or <= 32768
+ * (indexer mode).
  * out_idx: int32 [B][rows][top_k]; out_count: int32 [B][rows] (rows = G or T).
  * trace: may be NULL. workspace: at least hhr_select_workspace_bytes(). */
 int hhr_select(const hhr_dims* dims, int mode, const uint16_t* q, const int32_t* seq_len,

@@ -74,6 +74,15 @@ def test_bad_dims_rejected(L, bad):
 
 
 @pytest.mark.parametrize("bits", [64, 128, 256])
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1)])
+def test_flat_top_k_at_128k_accepted(L, bits, heads):
+    # Every page of a 128K-key sequence kept (131072 candidates), for every code length.
+    d = _d(code_bits=bits, n_q_heads=heads[0], n_kv_heads=heads[1])
+    assert hhr.hhr_select_workspace_bytes(d, hhr.HHR_MODE_HASH, 4096, 0, 2048) > 0
+    assert hhr.hhr_decode_step_workspace_bytes(d, 4096, 0, 2048) > 0
+
+
+@pytest.mark.parametrize("bits", [64, 128, 256])
 def test_code_lengths_accepted(L, bits):
     # 64-, 128- and 256-bit codes: the workspace holds B * Hq query codes of bits / 8 bytes.
     d = _d(code_bits=bits)
@@ -102,8 +111,8 @@ def test_select_validation_order(L):
     # workspace too small
     assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 2048, p, p, p, 16, None,
                         None) == hhr.HHR_ERR_WORKSPACE
-    # too many candidates per row (m * P > 65536)
-    assert L.hhr_select(ctypes.byref(_d(page_size=256)), 0, *args, 512, 0, 2048, p, p, p,
+    # too many candidates per row (m * P > 131072)
+    assert L.hhr_select(ctypes.byref(_d(page_size=256)), 0, *args, 1024, 0, 2048, p, p, p,
                         1 << 30, None, None) == hhr.HHR_ERR_UNSUPPORTED
     # indexer mode needs a single KV head and m_pages
     assert L.hhr_select(ctypes.byref(d), 1, *args, 64, 0, 2048, p, p, p, 1 << 30, None,

@@ -49,6 +49,14 @@ def test_fused_step_code_lengths(bits, heads):
     _fused_vs_separate(wl, 1, True)
 
 
+@pytest.mark.parametrize("bits", [64, 128])
+def test_fused_step_flat(bits):
+    """Flat hash top-k (every page kept): no page-bound kernel in either path."""
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=3, ragged=(33, 6000), top_k=300,
+                  m_pages=4096, keep_div=0, code_bits=bits)
+    _fused_vs_separate(wl, 1, True)
+
+
 def _fused_vs_separate(wl, f16, with_new_rows):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
@@ -89,10 +97,13 @@ def _fused_vs_separate(wl, f16, with_new_rows):
     assert torch.equal(fs.out.view(torch.int32), ref.out.view(torch.int32))
 
 
-def test_fused_step_against_oracle():
+@pytest.mark.parametrize("flat", [False, True], ids=["hierarchical", "flat"])
+def test_fused_step_against_oracle(flat):
     """The fused call's outputs through the layered oracle checks (selection + attention)."""
     build.build()
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(7777,), top_k=700)
+    if flat:
+        wl = S.scaled(wl, m_pages=4096, keep_div=0)
     inp = S.make_inputs(wl, device="cuda")
     inp_np = S.to_numpy_inputs(inp)
     d = dims_of(wl, inp, 1)

@@ -144,6 +144,17 @@ def test_code_lengths_128k_sampled(bits):
     _check_all_groups(wl, inp_np, out, groups={(0, 1), (0, 6)})
 
 
+@pytest.mark.parametrize("bits", [128, 256])
+def test_flat_hash_topk_128k(bits):
+    """Flat hash top-k (every page kept, HATA-style) at 128K: 131072 candidates per group."""
+    wl = S.scaled(S.WORKLOADS["llama8b_128k_b1"], m_pages=4096, keep_div=0, code_bits=bits)
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp, summary_fp16=1)
+    assert np.all(out["count"] == wl.top_k)
+    assert np.all(out["kept_count"] == 4096)
+    _check_all_groups(wl, inp_np, out, groups={(0, 2), (0, 5)})
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
