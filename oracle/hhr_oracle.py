@@ -193,6 +193,37 @@ def candidates_of(kept_pages, n, P):
     return t[t < n]
 
 
+# --------------------------------------------------------------------------- forced pages
+# Variant: sink and local-window pages. Neither HHR nor HISA forces any page; the HHR page's
+# MagicPIG baseline attends to sink tokens and a local window (HHR appendix, baseline
+# settings). Reading taken: the first `sink` and the last `local` logical pages of a sequence
+# are always kept, inside the page budget (which grows only when it is smaller than the forced
+# set), and their keys are selected ahead of the Hamming ranking, in token order.
+
+def forced_pages(n_pages, sink, local):
+    """Logical pages [0, sink) and [n_pages - local, n_pages), ascending."""
+    p = np.arange(n_pages)
+    return p[(p < sink) | (p >= n_pages - local)]
+
+
+def top_m_forced(scores, m, forced):
+    """The forced pages plus the m' - |forced| largest other scores (ties to the lower index),
+    m' = max(m, |forced|); returned ascending. No forced pages: top_m."""
+    forced = np.asarray(forced, dtype=np.int64)
+    rest = np.setdiff1d(np.arange(len(scores)), forced)
+    m_eff = max(m, len(forced))
+    pick = rest[top_m(np.asarray(scores)[rest], m_eff - len(forced))]
+    return np.sort(np.concatenate([forced, pick]))
+
+
+def top_k_forced(dist, tok, k, is_forced):
+    """k candidates: the forced ones first (in token order), then the smallest (dist, token)
+    pairs of the rest; returned as tokens ascending. No forced candidates: top_k_smallest."""
+    primary = np.where(np.asarray(is_forced, dtype=bool), -1, np.asarray(dist, dtype=np.int64))
+    order = np.lexsort((tok, primary))
+    return np.sort(np.asarray(tok)[order[:k]])
+
+
 # --------------------------------------------------------------------------- step a5
 # Attention over the selected subset only (HISA page, Abstract: "computing attention only
 # over the selected subset"; GQA layout from HHR appendix Table 3: 32 heads, 8 KV heads).
@@ -209,23 +240,33 @@ def sparse_attention(Qg, Ksel, Vsel, scale):
 
 # --------------------------------------------------------------------------- composites
 
-def select_group(Qg, R_g, W_g, kmin, kmax, codes, n, P, m, k):
+def select_group(Qg, R_g, W_g, kmin, kmax, codes, n, P, m, k, sink=0, local=0):
     """Steps a1-a4 for one (sequence, KV group) in the HHR order: bound, prune, Hamming, top-k.
 
-    codes are indexed by logical token. Returns a dict of every intermediate.
+    codes are indexed by logical token; sink/local: forced pages (variant, see forced_pages).
+    Returns a dict of every intermediate.
     """
     Qrot, qcodes, qfragile = query_prep(R_g, W_g, Qg)
     beta = page_bounds(Qrot, kmin, kmax)
-    kept = top_m(beta, m)
+    forced = forced_pages(len(beta), sink, local)
+    if len(forced):
+        kept = top_m_forced(beta, m, forced)
+    else:
+        kept = top_m(beta, m)
     cand = candidates_of(kept, n, P)
     delta = hamming(qcodes, codes[cand])
-    S = top_k_smallest(delta, cand, min(k, len(cand)))
+    if len(forced):
+        S = top_k_forced(delta, cand, min(k, len(cand)), np.isin(cand // P, forced))
+    else:
+        S = top_k_smallest(delta, cand, min(k, len(cand)))
     return dict(q_rot=Qrot, qcodes=qcodes, qfragile=qfragile, bounds=beta, kept=kept,
                 cand=cand, delta=delta, idx=S)
 
 
-def decode_step_hash(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=None):
-    """Whole HHR decode step (a0-a5) for every (sequence, KV group), or for ``groups`` only.
+def decode_step_hash(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=None, sink=0,
+                     local=0):
+    """Whole HHR decode step (a0-a5) for every (sequence, KV group), or for ``groups`` only;
+    sink/local: forced pages (variant).
 
     inp: numpy dict from hhr_synth.to_numpy_inputs. Returns {(b, g): dict}.
     """
@@ -247,12 +288,12 @@ def decode_step_hash(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=Non
             enc = encode_group(k_bits, pt[b], g, n, P, R[g], W[g])
             Qg = bf16_to_f64(q_bits[b, g * gs:(g + 1) * gs])
             r = select_group(Qg, R[g], W[g], enc["kmin"], enc["kmax"], enc["codes"], n, P, m,
-                             top_k)
+                             top_k, sink, local)
             K = logical_rows(k_bits, pt[b], g, n, P)
             V = logical_rows(v_bits, pt[b], g, n, P)
             r["out"] = sparse_attention(Qg, K[r["idx"]], V[r["idx"]], scale)
             r.update(enc)
-            r["m"] = m
+            r["m"] = max(m, len(forced_pages(n_pages, sink, local)))
             out[(b, g)] = r
     return out
 

@@ -16,7 +16,10 @@ routine):
   * top-k equals a full stable sort of (distance, token);
   * k = all keys and m = all pages gives dense softmax attention (library SDPA);
   * HISA: block size 1 makes block scores the token scores; keeping all blocks
-    gives the flat indexer top-k; the causal rule by brute force.
+    gives the flat indexer top-k; the causal rule by brute force;
+  * forced sink/local pages: closed forms of the forced set, the kept set as the best
+    subset by brute force over all subsets that hold the forced pages, and the token
+    top-k decomposed into the forced keys plus a plain top-k of the others.
 """
 from __future__ import annotations
 
@@ -349,10 +352,76 @@ def check_hisa_all_blocks_and_causal(O, seed=11):
                     1 + abs(mu[b, c]))
 
 
+def check_forced_pages(O, seed=12):
+    """Forced sink/local pages: closed forms, subset brute force and decomposition."""
+    import itertools
+    assert list(O.forced_pages(10, 2, 3)) == [0, 1, 7, 8, 9]
+    assert list(O.forced_pages(4, 3, 3)) == [0, 1, 2, 3]
+    assert list(O.forced_pages(5, 0, 0)) == []
+    assert list(O.forced_pages(5, 0, 1)) == [4]
+    assert list(O.forced_pages(5, 1, 0)) == [0]
+    assert list(O.forced_pages(1, 1, 1)) == [0]
+    rng = np.random.default_rng(seed)
+    # Kept set = the subset of size max(m, |forced|) that holds the forced pages and has the
+    # largest score sum (distinct scores: unique), by enumeration.
+    for trial in range(40):
+        n = int(rng.integers(1, 9))
+        sink, local = int(rng.integers(0, 3)), int(rng.integers(0, 3))
+        m = int(rng.integers(1, n + 1))
+        scores = rng.permutation(n).astype(np.float64) - 3.5
+        forced = [p for p in range(n) if p < sink or p >= n - local]
+        size = max(m, len(forced))
+        best = max((c for c in itertools.combinations(range(n), size) if set(forced) <= set(c)),
+                   key=lambda c: sum(scores[list(c)]))
+        assert list(O.top_m_forced(scores, m, forced)) == list(best), (n, sink, local, m)
+    # Equal scores: the forced pages, then the lowest other indices.
+    assert list(O.top_m_forced(np.zeros(8), 4, [0, 7])) == [0, 1, 2, 7]
+    assert list(O.top_m_forced(np.zeros(8), 4, [])) == [0, 1, 2, 3]
+    # Token top-k: forced keys first in token order, the rest a plain top-k of the others.
+    for trial in range(30):
+        n = int(rng.integers(1, 120))
+        tok = np.sort(rng.choice(3000, size=n, replace=False))
+        dist = rng.integers(0, 5, size=n)
+        isf = rng.random(n) < 0.3
+        k = int(rng.integers(1, n + 1))
+        ftok = sorted(tok[isf].tolist())
+        if k <= len(ftok):
+            want = ftok[:k]
+        else:
+            rest = sorted(zip(dist[~isf].tolist(), tok[~isf].tolist()))[:k - len(ftok)]
+            want = sorted(ftok + [t for _, t in rest])
+        assert list(O.top_k_forced(dist, tok, k, isf)) == want
+    # Through the selection: the forced pages are kept and all their keys selected; the
+    # other keys are the Hamming top-k (brute force) of the other kept pages' keys.
+    n, P, d, gs, bits, k = 70, 8, 32, 2, 64, 30
+    kc, vc, pt = tiny_cache(rng, n, P, 1, d)
+    R = orthogonal(rng, d)
+    W = rng.standard_normal((bits, d)).astype(np.float32)
+    enc = O.encode_group(kc, pt, 0, n, P, R, W)
+    Q = bf(rand_bf16_bits(rng, (gs, d)))
+    r = O.select_group(Q, R, W, enc["kmin"], enc["kmax"], enc["codes"], n, P, 4, k, 1, 1)
+    n_pages = -(-n // P)
+    assert 0 in r["kept"] and n_pages - 1 in r["kept"] and len(r["kept"]) == 4
+    forced_keys = [t for t in range(n) if t // P in (0, n_pages - 1)]
+    assert set(forced_keys) <= set(r["idx"].tolist())
+    Kb = brute_logical(kc, pt, 0, n, P)
+    kbits = [brute_code_bits(R, W, list(x)) for x in Kb]
+    qbits = [brute_code_bits(R, W, list(q)) for q in Q]
+    others = [t for t in range(n) if t // P in r["kept"] and t not in forced_keys]
+    dist = [sum(qbits[h][j] != kbits[t][j] for h in range(gs) for j in range(bits))
+            for t in others]
+    want = sorted(forced_keys + [t for _, t in sorted(zip(dist, others))[:k - len(forced_keys)]])
+    assert list(r["idx"]) == want
+    # Every page forced: the flat top-k of the forced keys in token order.
+    r = O.select_group(Q, R, W, enc["kmin"], enc["kmax"], enc["codes"], n, P, 2, k, 9, 0)
+    assert list(r["kept"]) == list(range(n_pages)) and list(r["idx"]) == list(range(k))
+
+
 ALL_CHECKS = [
     check_bound_invariant, check_page_size_one, check_rotation_preserves_logits,
     check_identity_rotation_summaries, check_codes_bruteforce,
     check_codes_identity_projection, check_topk_bruteforce, check_kept_count,
     check_flat_hash_topk, check_dense_attention, check_single_key_attention,
     check_hand_example, check_hisa_block_size_one, check_hisa_all_blocks_and_causal,
+    check_forced_pages,
 ]

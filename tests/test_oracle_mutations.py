@@ -85,6 +85,22 @@ def _topk_largest_ascending(score, tok, k):
     return np.sort(np.asarray(tok)[order[:k]])
 
 
+def _forced_local_one_early(n_pages, sink, local):
+    p = np.arange(n_pages)
+    return p[(p < sink) | (p >= n_pages - local - 1)]
+
+
+def _forced_budget_fixed(scores, m, forced):
+    forced = np.asarray(forced, dtype=np.int64)
+    rest = np.setdiff1d(np.arange(len(scores)), forced)
+    pick = rest[_orig["top_m"](np.asarray(scores)[rest], max(m - len(forced), 0))]
+    return np.sort(np.concatenate([forced, pick]))[:m]
+
+
+def _forced_keys_not_first(dist, tok, k, is_forced):
+    return _orig["top_k_smallest"](dist, tok, k)
+
+
 MUTATIONS = {
     "rotate_transposed": ("rotate", _rotate_transposed),
     "bound_min_not_max": ("page_bounds", _bounds_min),
@@ -101,6 +117,9 @@ MUTATIONS = {
     "kept_floor": ("kept_count", _kept_floor),
     "candidates_past_end": ("candidates_of", _cands_include_tail),
     "indexer_smallest_scores": ("top_k_largest", _topk_largest_ascending),
+    "forced_local_one_early": ("forced_pages", _forced_local_one_early),
+    "forced_budget_not_grown": ("top_m_forced", _forced_budget_fixed),
+    "forced_keys_not_first": ("top_k_forced", _forced_keys_not_first),
 }
 
 
