@@ -289,7 +289,8 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None):
     hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
                         int(inp["seq_len"].max()), R, W, cache.page_minmax, cache.codes,
                         None)
-    st = DecodeStep(d, hhr.HHR_MODE_HASH, m_pages, keep_div, wl.top_k, dev, attention=False)
+    st = DecodeStep(d, hhr.HHR_MODE_HASH, m_pages, keep_div, wl.top_k, dev, attention=False,
+                    sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     B, G, gs, P = wl.batch, wl.n_kv_heads, wl.n_q_heads // wl.n_kv_heads, wl.page_size
     qcode = torch.empty(B, wl.n_q_heads, CW, dtype=torch.int32, device=dev)
     kept = torch.empty(B, G, st.m_max, dtype=torch.int32, device=dev)
@@ -357,6 +358,8 @@ def selection_quality(dev):
     for kd in (8, 32):
         sweep[f"gkr_keep_1/{kd}"] = hhr_quality(wl, inp, dev, inp["R"], 0, kd, full=False)
     sweep["flat_all_4096_pages"] = hhr_quality(wl, inp, dev, inp["R"], 4096, 0, full=False)
+    sweep["sink_1_local_2_pages_keep_1/16"] = hhr_quality(
+        S.scaled(wl, sink_pages=1, local_pages=2), inp, dev, inp["R"], 0, 16, full=False)
     for bits in (64, 256):
         wb = S.scaled(wl, code_bits=bits)
         Wb = S.lhp_projection(wb, layer=0).to(dev)
@@ -410,7 +413,7 @@ def selection_quality(dev):
 
 SECONDARY = ("llama8b_128k_b1", "ragged_b32", "llama8b_32k", "tiny_1h_4k", "hisa_128k_t1",
              "hisa_128k_t64", "llama8b_128k_b8_codes64", "llama8b_128k_b8_codes256",
-             "llama8b_128k_b8_flat")
+             "llama8b_128k_b8_flat", "llama8b_128k_b8_sink1_local2")
 
 
 def indexer_required_bytes(wl, lens):
@@ -460,7 +463,8 @@ def measure_secondary(name, dev, l2, f16, steps, stream, mem_cap):
                             cache.codes if hashing else None,
                             None if hashing else cache.block_mean)
         mode = hhr.HHR_MODE_HASH if hashing else hhr.HHR_MODE_INDEXER
-        st = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev, attention=hashing)
+        st = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev, attention=hashing,
+                        sink_pages=wl.sink_pages, local_pages=wl.local_pages)
         if hashing:
             t = (inp["seq_len"] - 1).long()
             phys = inp["page_table"][torch.arange(wl.batch, device=dev), t // wl.page_size].long()

@@ -143,6 +143,21 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
   return HHR_OK;
 }
 
+// Forced sink/local pages of the options (zero without options), validated.
+int read_opts(const hhr_dims* d, int mode, const hhr_select_opts* o, int m_pages, int keep_div,
+              int* sink, int* local) {
+  *sink = *local = 0;
+  if (o == nullptr) return HHR_OK;
+  if (o->sink_pages < 0 || o->local_pages < 0) return HHR_ERR_INVALID_ARG;
+  if (o->sink_pages == 0 && o->local_pages == 0) return HHR_OK;
+  if (mode != HHR_MODE_HASH) return HHR_ERR_UNSUPPORTED;
+  if ((long long)o->sink_pages + o->local_pages > kept_max(d, m_pages, keep_div))
+    return HHR_ERR_INVALID_ARG;
+  *sink = o->sink_pages;
+  *local = o->local_pages;
+  return HHR_OK;
+}
+
 // One-shot event pairs of hhr_profile_next, per host thread.
 struct ProfPair {
   cudaEvent_t start, stop;
@@ -291,11 +306,13 @@ size_t hhr_select_workspace_bytes(const hhr_dims* d, int mode, int m_pages, int 
 int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* seq_len,
                const int32_t* q_pos, const int32_t* page_table, const float* R, const float* W,
                const void* page_minmax, const uint32_t* codes, const float* block_mean,
-               const uint16_t* k_cache, int m_pages, int keep_div, int top_k, int32_t* out_idx,
-               int32_t* out_count, void* workspace, size_t ws_bytes, hhr_trace* trace,
-               void* stream) {
+               const uint16_t* k_cache, int m_pages, int keep_div, int top_k,
+               const hhr_select_opts* opts, int32_t* out_idx, int32_t* out_count,
+               void* workspace, size_t ws_bytes, hhr_trace* trace, void* stream) {
   int st = check_select_params(d, mode, m_pages, keep_div, top_k);
   if (st != HHR_OK) return st;
+  int sink = 0, local = 0;
+  if ((st = read_opts(d, mode, opts, m_pages, keep_div, &sink, &local)) != HHR_OK) return st;
   if (q == nullptr || seq_len == nullptr || page_table == nullptr || out_idx == nullptr ||
       out_count == nullptr || workspace == nullptr)
     return HHR_ERR_INVALID_ARG;
@@ -353,7 +370,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
       if ((st = launch_status()) != HHR_OK) return st;
     }
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k};
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, nullptr, sink, local};
     const size_t fsm = topm_hamming_smem(Hq / G, cw, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
     topm_hamming_for(Hq / G, cw)<<<B * G * kHamRanks, topm_hamming_threads(cw), fsm, s>>>(
@@ -484,10 +501,14 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
                     const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
                     const int32_t* page_table, const int32_t* seq_len, const float* R,
                     const float* W, void* page_minmax, uint32_t* codes, int m_pages,
-                    int keep_div, int top_k, float scale, int32_t* out_idx, int32_t* out_count,
-                    float* out, void* workspace, size_t ws_bytes, void* stream) {
+                    int keep_div, int top_k, const hhr_select_opts* opts, float scale,
+                    int32_t* out_idx, int32_t* out_count, float* out, void* workspace,
+                    size_t ws_bytes, void* stream) {
   int st = check_select_params(d, HHR_MODE_HASH, m_pages, keep_div, top_k);
   if (st != HHR_OK) return st;
+  int sink = 0, local = 0;
+  if ((st = read_opts(d, HHR_MODE_HASH, opts, m_pages, keep_div, &sink, &local)) != HHR_OK)
+    return st;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || page_table == nullptr ||
       seq_len == nullptr || R == nullptr || W == nullptr || page_minmax == nullptr ||
       codes == nullptr || out_idx == nullptr || out_count == nullptr || out == nullptr ||
@@ -556,7 +577,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   // a2 top-m + a3 + a4: kept pages, Hamming distances, deterministic top-k.
   {
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows};
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows, sink, local};
     prof_begin(HHR_KERNEL_HAMMING, s);
     e = launch_pdl(topm_hamming_for(gs, cw), dim3(B * G * kHamRanks),
                    dim3(topm_hamming_threads(cw)), fsm, s,

@@ -355,11 +355,14 @@ struct SelCut {
 // Threshold search of a block-wide selection (NT threads, call uniformly) of the k largest
 // finite scores of sc[0..n), ties to the lower index. k = kept_for(#finite, m_pages,
 // keep_div) when by_kept, else min(top_k, #finite). Leaves the order-preserving keys of
-// the scores in keys[0..n) (shared memory, 16-byte aligned).
+// the scores in keys[0..n) (shared memory, 16-byte aligned). Forced entries i < sink and
+// i >= n - local take the largest key (above every finite score) and, when by_kept, k is at
+// least their number.
 template <int NT>
 __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint32_t* keys,
                                                    SelShared& sh, bool by_kept, int m_pages,
-                                                   int keep_div, int top_k) {
+                                                   int keep_div, int top_k, int sink = 0,
+                                                   int local = 0) {
   const int tid = threadIdx.x;
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
@@ -373,17 +376,19 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
 #pragma unroll
     for (int j = 0; j < kSelLoadUnroll; ++j) {
       const int i = base + j * NT + tid;
-      const bool fin = f[j] > -INFINITY;
-      const uint32_t kk = fin ? f2key(f[j]) : 0u;
+      const bool forced = i < n && (i < sink || i >= n - local);
+      const bool live = forced || f[j] > -INFINITY;
+      const uint32_t kk = forced ? 0xffffffffu : live ? f2key(f[j]) : 0u;
       if (i < n) keys[i] = kk;
-      nfin += fin;
-      if (fin) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
+      nfin += live;
+      if (live) { kmin = min(kmin, kk); kmax = max(kmax, kk); }
     }
   }
   // Also orders the key stores before any read (sh.mm is not reused: no tail barrier).
   block_count_minmax<false>(nfin, kmin, kmax, sh.mm, &nfin, &kmin, &kmax);
   SelCut c;
-  c.k = by_kept ? kept_for(nfin, m_pages, keep_div) : min(top_k, nfin);
+  c.k = by_kept ? max(kept_for(nfin, m_pages, keep_div), min(n, max(sink + local, 0)))
+                : min(top_k, nfin);
   // Selection rule after the search: key >> sel_shift > thr >> sel_shift selects; equal
   // keys at sel_shift == 0 are taken in index order until `rem` of them are taken; at
   // sel_shift > 0 the whole bin is taken (>=).
@@ -574,6 +579,7 @@ struct HammingArgs {
   int Hq, G, P, maxp, n_phys, m_max, top_k;
   uint32_t* out_rows;        // [B][G][top_k] cache row (phys*G + g)*P + slot of each selected
                              // key, for the attention of the fused step; or null
+  int sink, local;           // forced pages [0, sink) and the last `local` of each sequence
 };
 
 inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
@@ -668,17 +674,19 @@ template <int NB, int CW, int NT>
 __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
                                      const int32_t* kphys, int m, const uint32_t* qcs,
                                      uint32_t (*planes)[CW][4], uint32_t* hsm, HamShared& hs) {
-  constexpr int kBins = (kMaxGroup * 32 * CW + 1 + NT - 1) / NT;  // threshold bins per thread
+  // Ranked distance: 0 for a key of a forced page, else 1 + delta (bins 0 .. gs*32*CW + 1).
+  constexpr int kBins = (kMaxGroup * 32 * CW + 2 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int b = row / a.G, g = row % a.G;
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.G;
-  const int nbins = gs * 32 * CW + 1;
+  const int nbins = gs * 32 * CW + 2;
   m = min(m, a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                                // [nbins]
   uint16_t* dist = reinterpret_cast<uint16_t*>(hist + ((nbins + 31) & ~31));  // [half], 16B-aligned
   const int n = a.seq_len[b];
+  const int npg = min(ceil_div(max(n, 0), a.P), a.maxp);  // pages of the sequence
   const int C = min(m * a.P, kMaxCand);
   const int half = ((ceil_div(C, kHamRanks) + 7) / 8) * 8;
   const int lo = min(C, rank * half), hi = min(C, lo + half);
@@ -706,18 +714,21 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   constexpr int kHamLoad = ham_load<NB, CW>();
   for (int c0 = lo; c0 < hi; c0 += NT * kHamLoad) {
     uint32_t code[kHamLoad][CW];
-    bool ok[kHamLoad];
+    bool ok[kHamLoad], fr[kHamLoad];
 #pragma unroll
     for (int j = 0; j < kHamLoad; ++j) {
       const int c = c0 + j * NT + tid;
       ok[j] = false;
+      fr[j] = false;
 #pragma unroll
       for (int w = 0; w < CW; ++w) code[j][w] = 0u;
       if (c < hi) {
         const int i = (a.P == 1) ? c : (int)__umulhi((uint32_t)c, magic);
         const int slot = c - i * a.P;
         const int phys = kphys[i];
-        if (phys >= 0 && klp[i] * a.P + slot < n) {
+        const int lp = klp[i];
+        fr[j] = lp < a.sink || lp >= npg - a.local;
+        if (phys >= 0 && lp * a.P + slot < n) {
           ok[j] = true;
           load_code<CW>(a.codes + (((size_t)phys * a.G + g) * a.P + slot) * CW, code[j]);
         }
@@ -726,7 +737,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
 #pragma unroll
     for (int j = 0; j < kHamLoad; ++j) {
       const int c = c0 + j * NT + tid;
-      const int d = hamming_delta<NB, CW>(qp, code[j]);
+      const int d = fr[j] ? 0 : 1 + hamming_delta<NB, CW>(qp, code[j]);
       if (ok[j]) atomicAdd(&hist[d], 1);
       if (c < hi) dist[c - lo] = ok[j] ? (uint16_t)d : (uint16_t)0xffff;
     }
@@ -838,7 +849,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
 }
 
 inline size_t hamming_smem(int gs, int cw, int m_max, int P) {
-  const int nbins = gs * 32 * cw + 1;
+  const int nbins = gs * 32 * cw + 2;
   const size_t ints = (size_t)((nbins + 31) & ~31);
   // This rank's distances, padded so the 16-byte group reads of the last thread stay inside.
   const size_t c = (size_t)m_max * P < (size_t)kMaxCand ? (size_t)m_max * P : (size_t)kMaxCand;
@@ -930,7 +941,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(ham_threads<
     pt[j] = (j < J && p < n) ? ptab[p] : -1;
   }
   const SelCut cut = block_select_cut<NT>(a.bounds + (size_t)row * h.maxp, n, work, sh,
-                                                   true, a.m_pages, a.keep_div, 0);
+                                          true, a.m_pages, a.keep_div, 0, h.sink, h.local);
   int ng = 0, ne = 0;
   for (int j = 0; j < J; ++j) {
     const int p = wbase + 32 * j + lane;

@@ -52,6 +52,18 @@ class Dims(ctypes.Structure):
         "max_pages_per_seq", "n_phys_pages", "summary_fp16")]
 
 
+class SelectOpts(ctypes.Structure):
+    """hhr_select_opts: forced sink and local-window pages (0 = none)."""
+    _fields_ = [("sink_pages", ctypes.c_int), ("local_pages", ctypes.c_int)]
+
+
+def make_opts(sink_pages=0, local_pages=0):
+    """Options for hhr_select / hhr_decode_step, or None when nothing is forced."""
+    if not sink_pages and not local_pages:
+        return None
+    return SelectOpts(int(sink_pages), int(local_pages))
+
+
 class Trace(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("q_rot", "q_code", "bounds", "kept", "kept_count")]
 
@@ -75,8 +87,9 @@ def lib():
         L.hhr_kept_max.restype = i32
         L.hhr_select_workspace_bytes.argtypes = [pd, i32, i32, i32, i32]
         L.hhr_select_workspace_bytes.restype = sz
+        po = ctypes.POINTER(SelectOpts)
         L.hhr_select.argtypes = [pd, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
-                                 vp, vp, vp, sz, ctypes.POINTER(Trace), vp]
+                                 po, vp, vp, vp, sz, ctypes.POINTER(Trace), vp]
         L.hhr_select.restype = i32
         L.hhr_attn_workspace_bytes.argtypes = [pd, i32]
         L.hhr_attn_workspace_bytes.restype = sz
@@ -90,7 +103,7 @@ def lib():
         L.hhr_decode_step_workspace_bytes.argtypes = [pd, i32, i32, i32]
         L.hhr_decode_step_workspace_bytes.restype = sz
         L.hhr_decode_step.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
-                                      i32, ctypes.c_float, vp, vp, vp, vp, sz, vp]
+                                      i32, po, ctypes.c_float, vp, vp, vp, vp, sz, vp]
         L.hhr_decode_step.restype = i32
         L.hhr_sparse_attn_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, i32,
                                               ctypes.c_float, vp, vp]
@@ -182,14 +195,16 @@ def make_trace(q_rot=None, q_code=None, bounds=None, kept=None, kept_count=None)
 
 def hhr_select(d, mode, q, seq_len, q_pos, page_table, R, W, page_minmax, codes, block_mean,
                k_cache, m_pages, keep_div, top_k, out_idx, out_count, workspace, trace=None,
-               stream=None):
+               stream=None, opts=None):
     tr = ctypes.byref(trace) if trace is not None else None
+    op = ctypes.byref(opts) if opts is not None else None
     _check("hhr_select", lib().hhr_select(
         ctypes.byref(d), int(mode), _p(q, _BF16, "q"), _p(seq_len, I32, "seq_len"),
         _p(q_pos, I32, "q_pos"), _p(page_table, I32, "page_table"), _p(R, F32, "R"),
         _p(W, F32, "W"), _p(page_minmax, SUMMARY, "page_minmax"), _p(codes, U32, "codes"),
         _p(block_mean, F32, "block_mean"), _p(k_cache, _BF16, "k_cache"), int(m_pages),
-        int(keep_div), int(top_k), _p(out_idx, I32, "out_idx"), _p(out_count, I32, "out_count"),
+        int(keep_div), int(top_k), op, _p(out_idx, I32, "out_idx"),
+        _p(out_count, I32, "out_count"),
         _p(workspace, (torch.uint8,), "workspace"), workspace.numel(), tr, _s(stream)))
 
 
@@ -237,12 +252,13 @@ def hhr_decode_step_workspace_bytes(d, m_pages, keep_div, top_k) -> int:
 
 def hhr_decode_step(d, q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W,
                     page_minmax, codes, m_pages, keep_div, top_k, scale, out_idx, out_count, out,
-                    workspace, stream=None):
+                    workspace, stream=None, opts=None):
+    op = ctypes.byref(opts) if opts is not None else None
     _check("hhr_decode_step", lib().hhr_decode_step(
         ctypes.byref(d), _p(q, _BF16, "q"), _p(k_new, _BF16, "k_new"), _p(v_new, _BF16, "v_new"),
         _p(k_cache, _BF16, "k_cache"), _p(v_cache, _BF16, "v_cache"),
         _p(page_table, I32, "page_table"), _p(seq_len, I32, "seq_len"), _p(R, F32, "R"),
         _p(W, F32, "W"), _p(page_minmax, SUMMARY, "page_minmax"), _p(codes, U32, "codes"),
-        int(m_pages), int(keep_div), int(top_k), float(scale), _p(out_idx, I32, "out_idx"),
+        int(m_pages), int(keep_div), int(top_k), op, float(scale), _p(out_idx, I32, "out_idx"),
         _p(out_count, I32, "out_count"), _p(out, F32, "out"),
         _p(workspace, (torch.uint8,), "workspace"), workspace.numel(), _s(stream)))

@@ -34,8 +34,9 @@ class DecodeStep:
     """Workspaces and outputs of one decode step (hash mode) or one selection (indexer)."""
 
     def __init__(self, d: hhr.Dims, mode: int, m_pages: int, keep_div: int, top_k: int, device,
-                 attention: bool = True):
+                 attention: bool = True, sink_pages: int = 0, local_pages: int = 0):
         self.d, self.mode, self.m_pages, self.keep_div, self.top_k = d, mode, m_pages, keep_div, top_k
+        self.opts = hhr.make_opts(sink_pages, local_pages)  # forced pages (hash mode variant)
         rows = d.n_kv_heads if mode == hhr.HHR_MODE_HASH else d.n_q_heads
         ws = hhr.hhr_select_workspace_bytes(d, mode, m_pages, keep_div, top_k)
         if ws == 0:
@@ -61,7 +62,7 @@ class DecodeStep:
                q_pos=None, trace=None, stream=None):
         hhr.hhr_select(self.d, self.mode, q, seq_len, q_pos, page_table, R, W, cache.page_minmax,
                        cache.codes, cache.block_mean, k_cache, self.m_pages, self.keep_div,
-                       self.top_k, self.idx, self.count, self.sel_ws, trace, stream)
+                       self.top_k, self.idx, self.count, self.sel_ws, trace, stream, self.opts)
 
     def attend(self, q, k_cache, v_cache, page_table, seq_len, scale=None, stream=None):
         if scale is None:
@@ -81,7 +82,7 @@ class DecodeStep:
         hhr.hhr_decode_step(self.d, q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W,
                             cache.page_minmax, cache.codes, self.m_pages, self.keep_div,
                             self.top_k, scale, self.idx, self.count, self.out, self.fused_ws,
-                            stream)
+                            stream, self.opts)
         return self.out
 
     def step(self, q, k_cache, v_cache, page_table, seq_len, R, W, cache: LayerCache,

@@ -59,6 +59,8 @@ class Workload:
     needle_scale: float = 4.0
     ragged: Optional[tuple] = None   # (lo, hi) inclusive bounds of per-sequence lengths
     permute_pages: bool = False      # page table = random permutation of the pool
+    sink_pages: int = 0              # selection variant: forced first pages of a sequence
+    local_pages: int = 0             # selection variant: forced last pages of a sequence
 
     @property
     def group_size(self):
@@ -109,9 +111,13 @@ WORKLOADS = {
 
 
 # Variants of the 128K batch-8 decode (same keys, queries and rotations): a flat hash top-k
-# (every page kept), and codes of 64 or 256 bits (W has 64 or 256 rows).
+# (every page kept), forced sink and local pages, and codes of 64 or 256 bits (W has 64 or
+# 256 rows).
 WORKLOADS["llama8b_128k_b8_flat"] = dataclasses.replace(
     WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_b8_flat", m_pages=4096, keep_div=0)
+WORKLOADS["llama8b_128k_b8_sink1_local2"] = dataclasses.replace(
+    WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_b8_sink1_local2", sink_pages=1,
+    local_pages=2)
 for _bits in (64, 256):
     _n = f"llama8b_128k_b8_codes{_bits}"
     WORKLOADS[_n] = dataclasses.replace(WORKLOADS["llama8b_128k_b8"], name=_n, code_bits=_bits)

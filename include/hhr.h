@@ -127,6 +127,23 @@ int hhr_encode_keys(const hhr_dims* dims, const uint16_t* k_cache, const int32_t
  * sequence of at most max_pages_per_seq pages (the row stride of trace->kept). */
 int hhr_kept_max(const hhr_dims* dims, int m_pages, int keep_div);
 
+/* Optional selection settings of hhr_select / hhr_decode_step (hash mode); a NULL pointer
+ * means all zero. Forced sink and local pages are a variant: neither HHR nor HISA forces
+ * any page (the HHR page's MagicPIG baseline attends to sink tokens and a local window).
+ *   sink_pages  : logical pages [0, sink_pages) of every sequence are always kept, and
+ *                 their keys are always selected;
+ *   local_pages : likewise the last local_pages pages [n_pages - local_pages, n_pages)
+ *                 (the local window, which holds the newest key).
+ * Forced pages count toward the page budget: m_b' = max(m_b, #forced pages), the rest
+ * chosen by the bound. Forced keys come first in the top-k, in token order (if there are
+ * more than top_k of them, the top_k lowest), the others by (delta, t).
+ * Both must be >= 0, with sink_pages + local_pages <= hhr_kept_max() (else
+ * HHR_ERR_INVALID_ARG); indexer mode accepts only zeros (else HHR_ERR_UNSUPPORTED). */
+typedef struct {
+  int sink_pages;
+  int local_pages;
+} hhr_select_opts;
+
 /* Workspace needed by hhr_select (bytes, 256-byte multiple); 0 on invalid input. */
 size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, int keep_div,
                                   int top_k);
@@ -157,13 +174,14 @@ size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, i
  * (hash mode: every page of a 128K-key sequence, a flat hash top-k) or <= 32768
  * (indexer mode).
  * out_idx: int32 [B][rows][top_k]; out_count: int32 [B][rows] (rows = G or T).
+ * opts: may be NULL (see hhr_select_opts).
  * trace: may be NULL. workspace: at least hhr_select_workspace_bytes(). */
 int hhr_select(const hhr_dims* dims, int mode, const uint16_t* q, const int32_t* seq_len,
                const int32_t* q_pos, const int32_t* page_table, const float* R, const float* W,
                const void* page_minmax, const uint32_t* codes, const float* block_mean,
-               const uint16_t* k_cache, int m_pages, int keep_div, int top_k, int32_t* out_idx,
-               int32_t* out_count, void* workspace, size_t ws_bytes, hhr_trace* trace,
-               void* stream);
+               const uint16_t* k_cache, int m_pages, int keep_div, int top_k,
+               const hhr_select_opts* opts, int32_t* out_idx, int32_t* out_count,
+               void* workspace, size_t ws_bytes, hhr_trace* trace, void* stream);
 
 /* Workspace needed by hhr_sparse_attn (bytes, 256-byte multiple); 0 on invalid input. */
 size_t hhr_attn_workspace_bytes(const hhr_dims* dims, int top_k);
@@ -198,14 +216,15 @@ size_t hhr_decode_step_workspace_bytes(const hhr_dims* dims, int m_pages, int ke
  *             seq_len[b] - 1 (its page must be mapped in page_table).
  *   k_new, v_new : bf16 [B][G][d] newest rows, written into k_cache/v_cache at that
  *             position before encoding; both NULL when the caller already wrote them.
- *   out_idx, out_count, out, scale : as in hhr_select / hhr_sparse_attn.
+ *   opts, out_idx, out_count, out, scale : as in hhr_select / hhr_sparse_attn.
  * workspace: at least hhr_decode_step_workspace_bytes(). Errors as in the separate calls. */
 int hhr_decode_step(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_new,
                     const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
                     const int32_t* page_table, const int32_t* seq_len, const float* R,
                     const float* W, void* page_minmax, uint32_t* codes, int m_pages,
-                    int keep_div, int top_k, float scale, int32_t* out_idx, int32_t* out_count,
-                    float* out, void* workspace, size_t ws_bytes, void* stream);
+                    int keep_div, int top_k, const hhr_select_opts* opts, float scale,
+                    int32_t* out_idx, int32_t* out_count, float* out, void* workspace,
+                    size_t ws_bytes, void* stream);
 
 /* hhr_sparse_attn without a workspace argument, for callers that cannot allocate
  * device memory themselves: runtimes without a device allocator, code running

@@ -50,12 +50,14 @@ def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
     lens = inp["seq_len"]
     if encode_chunks is None:
         start = torch.zeros(B, dtype=torch.int32, device=dev)
-        step = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev)
+        step = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev,
+                          sink_pages=wl.sink_pages, local_pages=wl.local_pages)
         step.encode(inp["k_cache"], inp["page_table"], start, lens, int(lens.max()),
                     inp["R"] if hashing else None, inp["W"] if hashing else None, cache)
     else:
         # Append in pieces of at most `encode_chunks` keys, as a decode loop would.
-        step = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev)
+        step = DecodeStep(d, mode, wl.m_pages, wl.keep_div, wl.top_k, dev,
+                          sink_pages=wl.sink_pages, local_pages=wl.local_pages)
         done = torch.zeros(B, dtype=torch.int32, device=dev)
         while bool((done < lens).any()):
             n_new = torch.clamp(lens - done, max=encode_chunks).to(torch.int32)
@@ -163,30 +165,41 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
     page_max = np.full(n_pages, -np.inf)
     np.maximum.at(page_max, np.arange(n) // P, summed)
     assert np.all(beta_gpu >= page_max - 1e-5 * scale), "bound below a true logit"
-    m = O.kept_count(n_pages, wl.m_pages, wl.keep_div)
+    forced = O.forced_pages(n_pages, wl.sink_pages, wl.local_pages)
+    m = max(O.kept_count(n_pages, wl.m_pages, wl.keep_div), len(forced))
     kc = int(g_out["kept_count"][b, g])
     assert kc == m
     kept_gpu = g_out["kept"][b, g, :kc]
     # Same-precision decision: the oracle's top-m of the GPU's own fp32 bounds.
-    assert np.array_equal(kept_gpu, O.top_m(g_out["bounds"][b, g, :n_pages], m)), "top-m differs"
-    # Against the full fp64 oracle bounds: exact unless the cut is within tolerance.
+    beta_gpu32 = g_out["bounds"][b, g, :n_pages]
+    want = O.top_m_forced(beta_gpu32, m, forced) if len(forced) else O.top_m(beta_gpu32, m)
+    assert np.array_equal(kept_gpu, want), "top-m differs"
+    # Against the full fp64 oracle bounds (over the pages that are not forced): exact unless
+    # the cut is within tolerance.
     beta_full = O.page_bounds(Qrot, enc["kmin"], enc["kmax"])
-    order = np.sort(beta_full)[::-1]
+    rest = np.setdiff1d(np.arange(n_pages), forced)
+    mr = m - len(forced)
+    order = np.sort(beta_full[rest])[::-1]
     tol_cut = BOUND_TOL * float(scale.max())
-    if m < n_pages:
-        margin = order[m - 1] - order[m]
+    if 0 < mr < len(rest):
+        margin = order[mr - 1] - order[mr]
         if margin > 2 * tol_cut:
-            assert np.array_equal(kept_gpu, O.top_m(beta_full, m))
+            assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
         else:
             report["near_tie_cuts"] = report.get("near_tie_cuts", 0) + 1
-            sure_in = np.nonzero(beta_full > order[m - 1] + 2 * tol_cut)[0]
-            maybe = np.nonzero(beta_full >= order[m - 1] - 2 * tol_cut)[0]
-            assert set(sure_in) <= set(kept_gpu) <= set(maybe)
+            sure_in = set(rest[beta_full[rest] > order[mr - 1] + 2 * tol_cut]) | set(forced)
+            maybe = set(rest[beta_full[rest] >= order[mr - 1] - 2 * tol_cut]) | set(forced)
+            assert sure_in <= set(kept_gpu) <= maybe
+    else:
+        assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
 
     # a3 + a4: Hamming top-k on the GPU's codes and kept pages, bit-exact.
     cand = O.candidates_of(kept_gpu, n, P)
     delta = O.hamming(gq, gc[cand])
-    S_ref = O.top_k_smallest(delta, cand, min(wl.top_k, len(cand)))
+    if len(forced):
+        S_ref = O.top_k_forced(delta, cand, min(wl.top_k, len(cand)), np.isin(cand // P, forced))
+    else:
+        S_ref = O.top_k_smallest(delta, cand, min(wl.top_k, len(cand)))
     cnt = int(g_out["count"][b, g])
     assert cnt == len(S_ref)
     assert np.array_equal(g_out["idx"][b, g, :cnt], S_ref), "Hamming top-k differs"

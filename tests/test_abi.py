@@ -68,7 +68,7 @@ def test_workspace_and_kept_sizes(L):
 def test_bad_dims_rejected(L, bad):
     d = _d(**bad)
     assert hhr.hhr_select_workspace_bytes(d, hhr.HHR_MODE_HASH, 0, 16, 2048) == 0
-    st = L.hhr_select(ctypes.byref(d), 0, *([None] * 10), 0, 16, 2048, None, None, None, 0,
+    st = L.hhr_select(ctypes.byref(d), 0, *([None] * 10), 0, 16, 2048, None, None, None, None, 0,
                       None, None)
     assert st in (hhr.HHR_ERR_INVALID_ARG, hhr.HHR_ERR_UNSUPPORTED)
 
@@ -95,30 +95,55 @@ def test_code_lengths_accepted(L, bits):
     assert ws - base == q_code - q_code_64
 
 
+def test_select_opts_validated(L):
+    """Forced sink/local pages: non-negative, within the page budget, hash mode only."""
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    args = [p] * 10
+    d = _d()  # 4096 pages, keep 1/16 -> at most 256 kept pages
+
+    def sel(dd, mode, m_pages, keep_div, opts):
+        return L.hhr_select(ctypes.byref(dd), mode, *args, m_pages, keep_div, 2048,
+                            ctypes.byref(opts), p, p, p, 1 << 30, None, None)
+
+    assert sel(d, 0, 0, 16, hhr.SelectOpts(-1, 0)) == hhr.HHR_ERR_INVALID_ARG
+    assert sel(d, 0, 0, 16, hhr.SelectOpts(0, -2)) == hhr.HHR_ERR_INVALID_ARG
+    assert sel(d, 0, 0, 16, hhr.SelectOpts(200, 57)) == hhr.HHR_ERR_INVALID_ARG
+    assert sel(d, 0, 64, 0, hhr.SelectOpts(60, 5)) == hhr.HHR_ERR_INVALID_ARG
+    di = _d(n_q_heads=64, n_kv_heads=1, page_size=128, max_pages_per_seq=1024)
+    assert sel(di, 1, 64, 0, hhr.SelectOpts(1, 0)) == hhr.HHR_ERR_UNSUPPORTED
+    step = [p] * 11
+    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048,
+                             ctypes.byref(hhr.SelectOpts(0, 300)), ctypes.c_float(0.1),
+                             p, p, p, p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    assert hhr.make_opts() is None
+    o = hhr.make_opts(1, 2)
+    assert (o.sink_pages, o.local_pages) == (1, 2)
+
+
 def test_select_validation_order(L):
     d = _d()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
     args = [p] * 10
     # both m_pages and keep_div given
-    assert L.hhr_select(ctypes.byref(d), 0, *args, 16, 16, 2048, p, p, p, 1 << 30, None,
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 16, 16, 2048, None, p, p, p, 1 << 30, None,
                         None) == hhr.HHR_ERR_INVALID_ARG
     # top_k < 1
-    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 0, p, p, p, 1 << 30, None,
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 0, None, p, p, p, 1 << 30, None,
                         None) == hhr.HHR_ERR_INVALID_ARG
     # null query
-    assert L.hhr_select(ctypes.byref(d), 0, None, *args[1:], 0, 16, 2048, p, p, p, 1 << 30, None,
+    assert L.hhr_select(ctypes.byref(d), 0, None, *args[1:], 0, 16, 2048, None, p, p, p, 1 << 30, None,
                         None) == hhr.HHR_ERR_INVALID_ARG
     # workspace too small
-    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 2048, p, p, p, 16, None,
+    assert L.hhr_select(ctypes.byref(d), 0, *args, 0, 16, 2048, None, p, p, p, 16, None,
                         None) == hhr.HHR_ERR_WORKSPACE
     # too many candidates per row (m * P > 131072)
-    assert L.hhr_select(ctypes.byref(_d(page_size=256)), 0, *args, 1024, 0, 2048, p, p, p,
+    assert L.hhr_select(ctypes.byref(_d(page_size=256)), 0, *args, 1024, 0, 2048, None, p, p, p,
                         1 << 30, None, None) == hhr.HHR_ERR_UNSUPPORTED
     # indexer mode needs a single KV head and m_pages
-    assert L.hhr_select(ctypes.byref(d), 1, *args, 64, 0, 2048, p, p, p, 1 << 30, None,
+    assert L.hhr_select(ctypes.byref(d), 1, *args, 64, 0, 2048, None, p, p, p, 1 << 30, None,
                         None) == hhr.HHR_ERR_INVALID_ARG
     # unknown mode
-    assert L.hhr_select(ctypes.byref(d), 7, *args, 0, 16, 2048, p, p, p, 1 << 30, None,
+    assert L.hhr_select(ctypes.byref(d), 7, *args, 0, 16, 2048, None, p, p, p, 1 << 30, None,
                         None) == hhr.HHR_ERR_INVALID_ARG
 
 
@@ -164,9 +189,9 @@ def test_misaligned_pointers_rejected(L):
     assert L.hhr_encode_keys(ctypes.byref(d), p, p, p, p, 1, p, bad, p, p, None,
                              None) == hhr.HHR_ERR_INVALID_ARG
     step = [p, bad, bad, p, p, p, p, p, p, p, p]  # q, k_new, v_new, k/v cache, ..., codes
-    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, ctypes.c_float(0.1), p, p, p,
-                             p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, None, ctypes.c_float(0.1),
+                             p, p, p, p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
     step = [p] * 11
     step[7] = bad  # R
-    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, ctypes.c_float(0.1), p, p, p,
-                             p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+    assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, None, ctypes.c_float(0.1),
+                             p, p, p, p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG

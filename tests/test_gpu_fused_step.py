@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 def _prefill(wl, inp, d, upto):
     """Encode positions [0, upto[b]) of every sequence; returns the cache."""
     cache = LayerCache(d, "cuda")
-    step = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    step = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
+                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     z = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
     step.encode(inp["k_cache"], inp["page_table"], z, upto, int(upto.max()), inp["R"], inp["W"],
                 cache)
@@ -57,6 +58,14 @@ def test_fused_step_flat(bits):
     _fused_vs_separate(wl, 1, True)
 
 
+@pytest.mark.parametrize("forced", [(1, 2), (0, 3)])
+def test_fused_step_forced_pages(forced):
+    """Forced sink/local pages: the fused call equals the separate calls."""
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=4, ragged=(33, 6000), top_k=300,
+                  sink_pages=forced[0], local_pages=forced[1])
+    _fused_vs_separate(wl, 1, True)
+
+
 def _fused_vs_separate(wl, f16, with_new_rows):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
@@ -73,7 +82,8 @@ def _fused_vs_separate(wl, f16, with_new_rows):
 
     # Reference: separate calls.
     ref_cache = _prefill(wl, inp, d, lens - 1)
-    ref = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    ref = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
+                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     one = torch.ones(wl.batch, dtype=torch.int32, device="cuda")
     ref.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], lens, inp["R"],
              inp["W"], ref_cache, (lens - 1).to(torch.int32), one)
@@ -84,7 +94,8 @@ def _fused_vs_separate(wl, f16, with_new_rows):
     if with_new_rows:
         kc[phys, :, t % P] = 0
         vc[phys, :, t % P] = 0
-    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
+                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     fs.fused_step(inp["q"], kc, vc, inp["page_table"], lens, inp["R"], inp["W"], cache,
                   k_new=k_new if with_new_rows else None, v_new=v_new if with_new_rows else None)
     torch.cuda.synchronize()
@@ -97,18 +108,21 @@ def _fused_vs_separate(wl, f16, with_new_rows):
     assert torch.equal(fs.out.view(torch.int32), ref.out.view(torch.int32))
 
 
-@pytest.mark.parametrize("flat", [False, True], ids=["hierarchical", "flat"])
-def test_fused_step_against_oracle(flat):
+@pytest.mark.parametrize("variant", ["hierarchical", "flat", "forced"])
+def test_fused_step_against_oracle(variant):
     """The fused call's outputs through the layered oracle checks (selection + attention)."""
     build.build()
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(7777,), top_k=700)
-    if flat:
+    if variant == "flat":
         wl = S.scaled(wl, m_pages=4096, keep_div=0)
+    elif variant == "forced":
+        wl = S.scaled(wl, sink_pages=2, local_pages=4)
     inp = S.make_inputs(wl, device="cuda")
     inp_np = S.to_numpy_inputs(inp)
     d = dims_of(wl, inp, 1)
     cache = _prefill(wl, inp, d, inp["seq_len"] - 1)
-    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    fs = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
+                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     B, Hq = wl.batch, wl.n_q_heads
     tr = dict(q_rot=torch.empty(B, Hq, 128, device="cuda"),
               q_code=torch.empty(B, Hq, wl.code_bits // 32, dtype=torch.int32, device="cuda"))
@@ -117,7 +131,8 @@ def test_fused_step_against_oracle(flat):
     torch.cuda.synchronize()
     # Intermediates live in the fused workspace; recompute them with the select call to
     # feed the layered checks (the fused selection must equal it).
-    sel = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
+    sel = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
+                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     bounds = torch.empty(B, wl.n_kv_heads, d.max_pages_per_seq, device="cuda")
     kept = torch.empty(B, wl.n_kv_heads, sel.m_max, dtype=torch.int32, device="cuda")
     kc = torch.empty(B, wl.n_kv_heads, dtype=torch.int32, device="cuda")

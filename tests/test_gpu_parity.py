@@ -155,6 +155,26 @@ def test_flat_hash_topk_128k(bits):
     _check_all_groups(wl, inp_np, out, groups={(0, 2), (0, 5)})
 
 
+@pytest.mark.parametrize("forced", [(1, 2), (4, 0), (0, 8), (3, 3)])
+def test_forced_sink_local_pages(forced):
+    """Forced sink/local pages (variant): kept inside the budget, their keys selected first.
+    Short sequences (n = 300: 10 pages, keep 1/16 = 1) grow the budget to the forced set;
+    (3, 3) on 2 pages forces every page."""
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(5000, 300, 40), batch=3, top_k=400,
+                  keep_div=16, sink_pages=forced[0], local_pages=forced[1])
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp, summary_fp16=1)
+    _check_all_groups(wl, inp_np, out)
+    # Every key of a forced page is selected while top_k leaves room for them.
+    P = wl.page_size
+    for b, n in enumerate(wl.seq_lens):
+        npg = -(-n // P)
+        fk = [t for t in range(n) if t // P < forced[0] or t // P >= npg - forced[1]]
+        if len(fk) <= wl.top_k:
+            for g in range(wl.n_kv_heads):
+                assert set(fk) <= set(out["idx"][b, g, :out["count"][b, g]].tolist())
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
