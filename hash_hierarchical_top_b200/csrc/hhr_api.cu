@@ -61,6 +61,20 @@ int check_group(const hhr_dims* d) {
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
 
+// SMs of the current device (cached per device; 148 on B200 if the query fails).
+int sm_count() {
+  static int cached[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // Raise a kernel's dynamic shared-memory limit (opt-in maximum minus the kernel's
 // static shared memory) once per device, and check that `bytes` fits under it.
 template <typename K>
@@ -358,7 +372,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     const bool flat = m_max >= maxp;
     if (!flat || (trace != nullptr && trace->bounds != nullptr)) {
       const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                         d->n_phys_pages};
+                         d->n_phys_pages, 0};
       const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
       const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
       prof_begin(HHR_KERNEL_BOUND, s);
@@ -564,8 +578,11 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   // a2: page bounds (none when every page is kept: a flat hash top-k).
   const bool flat = m_max >= maxp;
   if (!flat) {
+    // Launched behind the prologue: its first CTAs warm L2 while the prologue runs, unless
+    // an event is recorded between the two (profiling), which leaves no overlap to use.
+    const int early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
     const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                       d->n_phys_pages};
+                       d->n_phys_pages, early};
     const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
     const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
     prof_begin(HHR_KERNEL_BOUND, s);

@@ -96,6 +96,11 @@ inline size_t qprep_smem() { return 0; }
 // path, so this kernel is a pure streaming GEMV.
 // Tuned on B200 at 128K context, batch 8 (4096 pages x 8 groups x 8 sequences); the
 // macros below exist for such sweeps.
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
 #ifndef HHR_BOUND_WARPS
 #define HHR_BOUND_WARPS 4
 #endif
@@ -110,13 +115,25 @@ constexpr int kBoundWarps = HHR_BOUND_WARPS;
 // Grid of the bound kernels: (page chunk, group, sequence), or (group, page chunk,
 // sequence) when HHR_BOUND_GROUP_FAST is set.
 #ifdef HHR_BOUND_GROUP_FAST
-__device__ __forceinline__ int bound_group() { return blockIdx.x; }
-__device__ __forceinline__ int bound_chunk() { return blockIdx.y; }
+__device__ __forceinline__ int bound_group_of(int x, int y) { return x; }
+__device__ __forceinline__ int bound_chunk_of(int x, int y) { return y; }
 inline dim3 bound_grid(int G, int chunks, int B) { return dim3(G, chunks, B); }
 #else
-__device__ __forceinline__ int bound_group() { return blockIdx.y; }
-__device__ __forceinline__ int bound_chunk() { return blockIdx.x; }
+__device__ __forceinline__ int bound_group_of(int x, int y) { return y; }
+__device__ __forceinline__ int bound_chunk_of(int x, int y) { return x; }
 inline dim3 bound_grid(int G, int chunks, int B) { return dim3(chunks, G, B); }
+#endif
+__device__ __forceinline__ int bound_group() { return bound_group_of(blockIdx.x, blockIdx.y); }
+__device__ __forceinline__ int bound_chunk() { return bound_chunk_of(blockIdx.x, blockIdx.y); }
+
+// L2 warm-up before the dependency wait: with programmatic launch the first CTAs of the
+// bound kernel are resident while the previous kernel (the fused step's prologue) still
+// runs and HBM idles. The first E = BoundArgs::early CTAs (by linear index) prefetch the
+// summaries of CTAs lin, lin + E, ..., lin + (HHR_BOUND_LOOKAHEAD - 1) E into L2. Measured
+// on B200 (128K context, batch 8, f16): E = 3 x 148 SMs and 3 strides (about 44 MB, what
+// HBM can move during the prologue) take 2 us off the step; more lookahead is slower.
+#ifndef HHR_BOUND_LOOKAHEAD
+#define HHR_BOUND_LOOKAHEAD 3
 #endif
 
 struct BoundArgs {
@@ -126,6 +143,7 @@ struct BoundArgs {
   const int32_t* seq_len;
   float* bounds;  // [B][G][maxp]
   int G, P, maxp, n_phys;
+  int early;      // CTAs that warm L2 before the dependency wait (0: none)
 };
 
 // Sum over the warp of 8 per-lane partials (one per page): a butterfly over lane bits 4
@@ -192,10 +210,38 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
   // summary pieces), so that each warp keeps kSets * 8 page summaries in flight.
   constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
   constexpr int kPagesPerWarp = 8 * kSets;
+  // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
+  constexpr int kPieces = F16 ? 32 : 64;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if constexpr (HHR_BOUND_LOOKAHEAD > 0) {
+    // Reads only inputs no earlier kernel of the step writes (page table, lengths); a
+    // prefetch of a summary that the previous kernel is updating is coherent in L2.
+    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int total = gridDim.x * gridDim.y * gridDim.z;
+    if (lin < a.early && lane < kPagesPerWarp) {
+#pragma unroll
+      for (int j = 0; j < HHR_BOUND_LOOKAHEAD; ++j) {
+        const int t = lin + j * a.early;
+        if (t < total) {
+          const int tx = t % gridDim.x, ty = (t / gridDim.x) % gridDim.y;
+          const int tb = t / (gridDim.x * gridDim.y);
+          const int tg = bound_group_of(tx, ty);
+          const int p = bound_chunk_of(tx, ty) * kBoundWarps * kPagesPerWarp +
+                        warp * kPagesPerWarp + lane;
+          if (p < min(ceil_div(a.seq_len[tb], a.P), a.maxp)) {
+            const int phys = a.page_table[(size_t)tb * a.maxp + p];
+            if (phys >= 0 && phys < a.n_phys)
+              prefetch_l2(reinterpret_cast<const uint4*>(a.page_minmax) +
+                              ((size_t)phys * a.G + tg) * kPieces,
+                          kPieces * 16);
+          }
+        }
+      }
+    }
+  }
   pdl_wait();
   pdl_trigger();
   const int g = bound_group(), b = blockIdx.z;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
   const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
   if (p0 >= npg) return;
@@ -209,8 +255,6 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
     q0 = reinterpret_cast<const float4*>(qb)[lane];
     q1 = reinterpret_cast<const float4*>(qb + kD)[lane];
   }
-  // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
-  constexpr int kPieces = F16 ? 32 : 64;
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
   int my_phys = -1;  // lane i < kPagesPerWarp resolves page p0 + i
   if (lane < kPagesPerWarp && p0 + lane < npg)
@@ -328,10 +372,6 @@ struct SelShared {
   uint32_t mm[96];
   int res[2][3];     // per pass (alternating): digit, rem, cnt
 };
-
-__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
-}
 
 constexpr int kSelLoadUnroll = 4;  // score loads in flight per thread
 
