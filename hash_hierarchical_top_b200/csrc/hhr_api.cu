@@ -99,7 +99,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
 }
 
 bool g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
-    g_smem_sel[kMaxDevices], g_smem_ham[3][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
+    g_smem_sel[kMaxDevices], g_smem_ham[3][2][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
     g_smem_attn_cl[kMaxDevices];
 
 struct SelectLayout {
@@ -360,8 +360,9 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     void (*qp)(QPrepArgs) =
         cw == 2 ? qprep_kernel<2> : cw == 8 ? qprep_kernel<8> : qprep_kernel<4>;
     if (allow_smem(qp, qprep_smem(), g_smem_qprep[cw_index(cw)]) != cudaSuccess) return HHR_ERR_CUDA;
-    if (allow_smem(topm_hamming_for(Hq / G, cw), topm_hamming_smem(Hq / G, cw, m_max, P, maxp),
-                   g_smem_ham[cw_index(cw)][hamming_planes(Hq / G) - 1]) != cudaSuccess)
+    const int nt = topm_hamming_threads(cw, (long long)B * G * kHamRanks, sm_count());
+    if (allow_smem(topm_hamming_for(Hq / G, cw, nt), topm_hamming_smem(Hq / G, cw, m_max, P, maxp),
+                   g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(Hq / G) - 1]) != cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qp<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
@@ -387,7 +388,7 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, nullptr, sink, local};
     const size_t fsm = topm_hamming_smem(Hq / G, cw, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
-    topm_hamming_for(Hq / G, cw)<<<B * G * kHamRanks, topm_hamming_threads(cw), fsm, s>>>(
+    topm_hamming_for(Hq / G, cw, nt)<<<B * G * kHamRanks, nt, fsm, s>>>(
         TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
@@ -558,8 +559,9 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   uint32_t* sel_rows = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
   const int cw = code_words(d);
   const size_t fsm = topm_hamming_smem(gs, cw, m_max, P, maxp);
-  if (allow_smem(topm_hamming_for(gs, cw), fsm, g_smem_ham[cw_index(cw)][hamming_planes(gs) - 1]) !=
-      cudaSuccess)
+  const int nt = topm_hamming_threads(cw, (long long)B * G * kHamRanks, sm_count());
+  if (allow_smem(topm_hamming_for(gs, cw, nt), fsm,
+                 g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(gs) - 1]) != cudaSuccess)
     return HHR_ERR_CUDA;
   if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
@@ -596,8 +598,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows, sink, local};
     prof_begin(HHR_KERNEL_HAMMING, s);
-    e = launch_pdl(topm_hamming_for(gs, cw), dim3(B * G * kHamRanks),
-                   dim3(topm_hamming_threads(cw)), fsm, s,
+    e = launch_pdl(topm_hamming_for(gs, cw, nt), dim3(B * G * kHamRanks), dim3(nt), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }

@@ -599,10 +599,12 @@ constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
 constexpr int kMaxCand = 131072;  // a flat top-k over 4096 pages of 32 keys
 constexpr int kMaxCodeWords = 8;  // 256-bit codes
 
-// Threads of a top-m + Hamming CTA: 1024, or 512 for 8-word codes (whose query bit planes
-// need the larger register budget).
-template <int CW>
-constexpr int ham_threads() { return CW >= 8 ? 512 : 1024; }
+// Threads of a top-m + Hamming CTA: 1024 (one CTA per SM, at most 64 registers), or 512 with
+// two CTAs per SM, for grids larger than the SM count (a latency-bound chain per CTA, so two
+// co-resident CTAs halve the waves). 8-word codes always take 512 threads and one CTA per SM
+// (their query bit planes need the larger register budget).
+template <int CW, int NT>
+constexpr int ham_min_blocks() { return (NT == 512 && CW <= 4) ? 2 : 1; }
 // Code loads in flight per thread (fewer when the plane words fill the registers).
 template <int NB, int CW>
 constexpr int ham_load() { return NB * CW >= 16 ? 2 : 4; }
@@ -922,10 +924,10 @@ struct TopmShared {
   static_assert(kWarps <= 32, "the warp-prefix scan covers the warps with one warp");
 };
 
-template <int NB, int CW>
-__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(ham_threads<CW>())
+template <int NB, int CW, int NT>
+__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_blocks<CW, NT>())
     topm_hamming_kernel(TopmHammingArgs a) {
-  constexpr int NT = ham_threads<CW>();
+  static_assert(NT == 512 || (NT == 1024 && CW <= 4), "512 threads, or 1024 up to 4 words");
   constexpr int kTopmWarps = NT / 32;
   __shared__ SelShared sh;
   __shared__ HamShared hs;
@@ -1054,24 +1056,33 @@ inline size_t topm_hamming_smem(int gs, int cw, int m_max, int P, int maxp) {
 
 using TopmHammingFn = void (*)(TopmHammingArgs);
 
-template <int CW>
+template <int CW, int NT>
 inline TopmHammingFn topm_hamming_for_cw(int gs) {
   switch (hamming_planes(gs)) {
-    case 1: return topm_hamming_kernel<1, CW>;
-    case 2: return topm_hamming_kernel<2, CW>;
-    case 3: return topm_hamming_kernel<3, CW>;
-    default: return topm_hamming_kernel<4, CW>;
+    case 1: return topm_hamming_kernel<1, CW, NT>;
+    case 2: return topm_hamming_kernel<2, CW, NT>;
+    case 3: return topm_hamming_kernel<3, CW, NT>;
+    default: return topm_hamming_kernel<4, CW, NT>;
   }
 }
 
-// The instantiation for group size gs (1..kMaxGroup) and cw code words (2, 4 or 8), with
-// its thread count.
-inline TopmHammingFn topm_hamming_for(int gs, int cw) {
-  return cw == 2 ? topm_hamming_for_cw<2>(gs)
-                 : cw == 8 ? topm_hamming_for_cw<8>(gs) : topm_hamming_for_cw<4>(gs);
+// Threads per CTA for cw code words and a grid of `ctas` CTAs on `sms` SMs (see
+// ham_min_blocks). HHR_HAM_THREADS fixes the choice (512 or 1024) for sweeps.
+#ifndef HHR_HAM_THREADS
+#define HHR_HAM_THREADS 0
+#endif
+inline int topm_hamming_threads(int cw, long long ctas, int sms) {
+  if (cw == 8) return 512;
+  if (HHR_HAM_THREADS == 512 || HHR_HAM_THREADS == 1024) return HHR_HAM_THREADS;
+  return ctas > sms ? 512 : 1024;
 }
-inline int topm_hamming_threads(int cw) {
-  return cw == 8 ? ham_threads<8>() : cw == 2 ? ham_threads<2>() : ham_threads<4>();
+
+// The instantiation for group size gs (1..kMaxGroup), cw code words (2, 4 or 8) and nt
+// threads (topm_hamming_threads).
+inline TopmHammingFn topm_hamming_for(int gs, int cw, int nt) {
+  if (cw == 8) return topm_hamming_for_cw<8, 512>(gs);
+  if (cw == 2) return nt == 512 ? topm_hamming_for_cw<2, 512>(gs) : topm_hamming_for_cw<2, 1024>(gs);
+  return nt == 512 ? topm_hamming_for_cw<4, 512>(gs) : topm_hamming_for_cw<4, 1024>(gs);
 }
 
 // ---------------------------------------------------------------------------- HISA a1'

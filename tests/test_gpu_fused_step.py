@@ -66,6 +66,12 @@ def test_fused_step_forced_pages(forced):
     _fused_vs_separate(wl, 1, True)
 
 
+def test_fused_step_many_rows():
+    """192 top-m + Hamming CTAs (more than the SMs): the 512-thread instantiation."""
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=12, ragged=(33, 3000), top_k=200)
+    _fused_vs_separate(wl, 1, True)
+
+
 def _fused_vs_separate(wl, f16, with_new_rows):
     build.build()
     inp = S.make_inputs(wl, device="cuda")

@@ -175,6 +175,16 @@ def test_forced_sink_local_pages(forced):
                 assert set(fk) <= set(out["idx"][b, g, :out["count"][b, g]].tolist())
 
 
+@pytest.mark.parametrize("bits", [64, 128])
+def test_many_rows_two_ctas_per_sm(bits):
+    """More (sequence, group) rows than SMs: the top-m + Hamming kernel runs 512 threads per
+    CTA, two CTAs per SM. 12 sequences x 8 groups x 2 ranks = 192 CTAs."""
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=12, ragged=(33, 3000), top_k=200,
+                  code_bits=bits)
+    inp, inp_np = _inputs(wl)
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=1))
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
