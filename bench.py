@@ -272,10 +272,11 @@ def popcount32(x):
     return ((x * 0x01010101) & 0xFFFFFFFF) >> 24
 
 
-def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None):
+def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=None):
     """Encode layer inputs `inp` with rotation R (and projection W, default inp["W"], of
-    wl.code_bits rows), select with the given page budget and score the selection against
-    the exact group logits (see selection_quality)."""
+    wl.code_bits rows), select wl.top_k keys with the given page budget and score the
+    selection against the exact group logits' top-k_true (default wl.top_k; see
+    selection_quality)."""
     import statistics
     import torch
     from hash_hierarchical_top_b200 import hhr
@@ -309,7 +310,7 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None):
             K = inp["k_cache"][pages, g].reshape(npg * P, -1)[:n].float()
             lg = inp["q"][b, g * gs:(g + 1) * gs].float() @ K.T          # [gs][n]
             grp = lg.sum(0)
-            true = torch.topk(grp, min(wl.top_k, n)).indices
+            true = torch.topk(grp, min(k_true or wl.top_k, n)).indices
             sel = st.idx[b, g, :int(st.count[b, g])].long()
             rec.append(recall_at_k(sel, true))
             mass.append(mass_recall(lg, sel, scale))
@@ -328,7 +329,7 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None):
            "attention_mass_recall": statistics.mean(mass),
            "true_topk_in_kept_pages": statistics.mean(page_rec),
            "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
-           "k": wl.top_k, "kept_pages": st.m_max, "rows": B * G}
+           "k": wl.top_k, "k_true": k_true or wl.top_k, "kept_pages": st.m_max, "rows": B * G}
     if full:
         res["spearman_minus_hamming_vs_logit"] = statistics.mean(rho)
         res["random_selection_mass"] = wl.top_k / float(inp["seq_len"].float().mean())
@@ -358,6 +359,16 @@ def selection_quality(dev):
     for kd in (8, 32):
         sweep[f"gkr_keep_1/{kd}"] = hhr_quality(wl, inp, dev, inp["R"], 0, kd, full=False)
     sweep["flat_all_4096_pages"] = hhr_quality(wl, inp, dev, inp["R"], 4096, 0, full=False)
+    # Page stage only (every key of the 256 kept pages attended, no Hamming ranking), with
+    # GKR bounds and with QUEST-style bounds; recall against the true top-2048.
+    every = S.scaled(wl, top_k=256 * wl.page_size)
+    sweep["gkr_only_keep_1/16_attend_kept_pages"] = hhr_quality(
+        every, inp, dev, inp["R"], 0, 16, full=False, k_true=wl.top_k)
+    sweep["quest_R_identity_keep_1/16_attend_kept_pages"] = hhr_quality(
+        every, inp, dev, eye, 0, 16, full=False, k_true=wl.top_k)
+    for k in (1024, 4096):
+        sweep[f"gkr_keep_1/16_k{k}"] = hhr_quality(S.scaled(wl, top_k=k), inp, dev, inp["R"], 0,
+                                                   16, full=False)
     sweep["sink_1_local_2_pages_keep_1/16"] = hhr_quality(
         S.scaled(wl, sink_pages=1, local_pages=2), inp, dev, inp["R"], 0, 16, full=False)
     for bits in (64, 256):

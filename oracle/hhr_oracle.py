@@ -264,9 +264,12 @@ def select_group(Qg, R_g, W_g, kmin, kmax, codes, n, P, m, k, sink=0, local=0):
 
 
 def decode_step_hash(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=None, sink=0,
-                     local=0):
+                     local=0, per_head=False):
     """Whole HHR decode step (a0-a5) for every (sequence, KV group), or for ``groups`` only;
-    sink/local: forced pages (variant).
+    sink/local: forced pages (variant). per_head (variant): one selection per query head
+    instead of per KV group -- head h of group g scores the group's summaries and codes
+    with its own query alone and attends its own selection; the result for (b, g) is then
+    a list of per-head dicts.
 
     inp: numpy dict from hhr_synth.to_numpy_inputs. Returns {(b, g): dict}.
     """
@@ -287,14 +290,19 @@ def decode_step_hash(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=Non
                 continue
             enc = encode_group(k_bits, pt[b], g, n, P, R[g], W[g])
             Qg = bf16_to_f64(q_bits[b, g * gs:(g + 1) * gs])
-            r = select_group(Qg, R[g], W[g], enc["kmin"], enc["kmax"], enc["codes"], n, P, m,
-                             top_k, sink, local)
             K = logical_rows(k_bits, pt[b], g, n, P)
             V = logical_rows(v_bits, pt[b], g, n, P)
-            r["out"] = sparse_attention(Qg, K[r["idx"]], V[r["idx"]], scale)
-            r.update(enc)
-            r["m"] = max(m, len(forced_pages(n_pages, sink, local)))
-            out[(b, g)] = r
+            m_eff = max(m, len(forced_pages(n_pages, sink, local)))
+            heads = [Qg[h:h + 1] for h in range(gs)] if per_head else [Qg]
+            res = []
+            for Qs in heads:
+                r = select_group(Qs, R[g], W[g], enc["kmin"], enc["kmax"], enc["codes"], n, P,
+                                 m, top_k, sink, local)
+                r["out"] = sparse_attention(Qs, K[r["idx"]], V[r["idx"]], scale)
+                r.update(enc)
+                r["m"] = m_eff
+                res.append(r)
+            out[(b, g)] = res if per_head else res[0]
     return out
 
 

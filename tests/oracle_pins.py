@@ -417,11 +417,58 @@ def check_forced_pages(O, seed=12):
     assert list(r["kept"]) == list(range(n_pages)) and list(r["idx"]) == list(range(k))
 
 
+def check_per_head_selection(O, seed=13):
+    """One selection per query head: identical heads reproduce the group selection (the
+    group's bounds and distances are then gs times one head's), a group of one head is the
+    group path, and with every page kept each head's set is its own brute-force Hamming
+    top-k and its output its own dense attention over that set."""
+    rng = np.random.default_rng(seed)
+    n, P, d, G, gs, bits, k = 60, 8, 32, 1, 3, 64, 17
+    kc, vc, pt = tiny_cache(rng, n, P, G, d)
+    R = np.stack([orthogonal(rng, d) for _ in range(G)])
+    W = rng.standard_normal((G, bits, d)).astype(np.float32)
+    base = dict(k_cache=kc, v_cache=vc, page_table=pt[None, :],
+                seq_len=np.array([n], dtype=np.int32), R=R, W=W)
+    one = rand_bf16_bits(rng, (1, 1, d))
+    same = dict(base, q=np.repeat(one, gs, axis=1))
+    grp = O.decode_step_hash(same, P=P, m_pages=3, keep_div=0, top_k=k)[(0, 0)]
+    per = O.decode_step_hash(same, P=P, m_pages=3, keep_div=0, top_k=k, per_head=True)[(0, 0)]
+    assert len(per) == gs
+    for r in per:
+        assert list(r["kept"]) == list(grp["kept"]) and list(r["idx"]) == list(grp["idx"])
+        np.testing.assert_allclose(r["out"][0], grp["out"][0], rtol=1e-12, atol=1e-12)
+    solo = dict(base, q=one)
+    a = O.decode_step_hash(solo, P=P, m_pages=3, keep_div=0, top_k=k)[(0, 0)]
+    b = O.decode_step_hash(solo, P=P, m_pages=3, keep_div=0, top_k=k, per_head=True)[(0, 0)]
+    assert list(a["idx"]) == list(b[0]["idx"])
+    q = rand_bf16_bits(rng, (1, gs, d))
+    per = O.decode_step_hash(dict(base, q=q), P=P, m_pages=10 ** 6, keep_div=0, top_k=k,
+                             per_head=True)[(0, 0)]
+    Kb = brute_logical(kc, pt, 0, n, P)
+    Vb = brute_logical(vc, pt, 0, n, P)
+    kbits = [brute_code_bits(R[0], W[0], list(x)) for x in Kb]
+    sets = []
+    for h in range(gs):
+        qh = bf(q[0, h])
+        qb = brute_code_bits(R[0], W[0], list(qh))
+        dist = [sum(qb[j] != kbits[t][j] for j in range(bits)) for t in range(n)]
+        want = sorted(t for _, t in sorted(zip(dist, range(n)))[:k])
+        assert list(per[h]["idx"]) == want, h
+        lg = [math.fsum(qh[c] * Kb[t][c] for c in range(d)) / math.sqrt(d) for t in want]
+        mx = max(lg)
+        w = [math.exp(x - mx) for x in lg]
+        ref = [math.fsum(w[i] * Vb[t][c] for i, t in enumerate(want)) / math.fsum(w)
+               for c in range(d)]
+        np.testing.assert_allclose(per[h]["out"][0], ref, rtol=1e-10, atol=1e-12)
+        sets.append(tuple(want))
+    assert len(set(sets)) > 1  # distinct heads select differently on this input
+
+
 ALL_CHECKS = [
     check_bound_invariant, check_page_size_one, check_rotation_preserves_logits,
     check_identity_rotation_summaries, check_codes_bruteforce,
     check_codes_identity_projection, check_topk_bruteforce, check_kept_count,
     check_flat_hash_topk, check_dense_attention, check_single_key_attention,
     check_hand_example, check_hisa_block_size_one, check_hisa_all_blocks_and_causal,
-    check_forced_pages,
+    check_forced_pages, check_per_head_selection,
 ]

@@ -101,6 +101,16 @@ def _forced_keys_not_first(dist, tok, k, is_forced):
     return _orig["top_k_smallest"](dist, tok, k)
 
 
+def _per_head_uses_group(inp, *, P, m_pages, keep_div, top_k, scale=None, groups=None, sink=0,
+                         local=0, per_head=False):
+    res = _orig["decode_step_hash"](inp, P=P, m_pages=m_pages, keep_div=keep_div, top_k=top_k,
+                                    scale=scale, groups=groups, sink=sink, local=local)
+    if not per_head:
+        return res
+    gs = inp["q"].shape[1] // inp["k_cache"].shape[1]
+    return {key: [r] * gs for key, r in res.items()}
+
+
 MUTATIONS = {
     "rotate_transposed": ("rotate", _rotate_transposed),
     "bound_min_not_max": ("page_bounds", _bounds_min),
@@ -120,6 +130,7 @@ MUTATIONS = {
     "forced_local_one_early": ("forced_pages", _forced_local_one_early),
     "forced_budget_not_grown": ("top_m_forced", _forced_budget_fixed),
     "forced_keys_not_first": ("top_k_forced", _forced_keys_not_first),
+    "per_head_uses_group": ("decode_step_hash", _per_head_uses_group),
 }
 
 
