@@ -68,8 +68,10 @@ def measured_peaks():
 
 def required_bytes(wl, lens, m_of, sbytes=4):
     """Algorithmic bytes of one step: summaries (unless every page is kept: a flat top-k
-    needs no bounds) + kept-page codes + selected K/V rows."""
+    needs no bounds) + kept-page codes + selected K/V rows, for every selection row (KV
+    group, or query head with per-head selection, whose sets are read separately)."""
     G, P, d = wl.n_kv_heads, wl.page_size, wl.head_dim
+    rows = wl.n_q_heads if wl.select_per_head else G
     summ = codes = kv = 0
     for n in lens:
         npg = -(-n // P)
@@ -77,8 +79,8 @@ def required_bytes(wl, lens, m_of, sbytes=4):
         cand = min(n, m * P)
         if m < npg:
             summ += G * npg * 2 * d * sbytes
-        codes += G * cand * (wl.code_bits // 8)
-        kv += G * min(wl.top_k, cand) * 2 * d * 2
+        codes += rows * cand * (wl.code_bits // 8)
+        kv += rows * min(wl.top_k, cand) * 2 * d * 2
     return summ, codes, kv
 
 
@@ -284,7 +286,8 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
     W = inp["W"] if W is None else W
     CW = wl.code_bits // 32
     d = hhr.make_dims(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.page_size, inp["max_pages"],
-                      inp["n_phys"], summary_fp16=1, code_bits=wl.code_bits)
+                      inp["n_phys"], summary_fp16=1, code_bits=wl.code_bits,
+                      select_per_head=int(wl.select_per_head))
     cache = LayerCache(d, dev)
     zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
     hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],
@@ -294,8 +297,9 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
                     sink_pages=wl.sink_pages, local_pages=wl.local_pages)
     B, G, gs, P = wl.batch, wl.n_kv_heads, wl.n_q_heads // wl.n_kv_heads, wl.page_size
     qcode = torch.empty(B, wl.n_q_heads, CW, dtype=torch.int32, device=dev)
-    kept = torch.empty(B, G, st.m_max, dtype=torch.int32, device=dev)
-    kcnt = torch.empty(B, G, dtype=torch.int32, device=dev)
+    rows = hhr.sel_rows(d)
+    kept = torch.empty(B, rows, st.m_max, dtype=torch.int32, device=dev)
+    kcnt = torch.empty(B, rows, dtype=torch.int32, device=dev)
     st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=R, W=W,
               trace=hhr.make_trace(q_code=qcode, kept=kept, kept_count=kcnt))
     torch.cuda.synchronize()
@@ -309,6 +313,19 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
         for g in range(G):
             K = inp["k_cache"][pages, g].reshape(npg * P, -1)[:n].float()
             lg = inp["q"][b, g * gs:(g + 1) * gs].float() @ K.T          # [gs][n]
+            if wl.select_per_head:  # each head against its own logits' top-k
+                for h in range(gs):
+                    r = g * gs + h
+                    true = torch.topk(lg[h], min(k_true or wl.top_k, n)).indices
+                    sel = st.idx[b, r, :int(st.count[b, r])].long()
+                    rec.append(recall_at_k(sel, true))
+                    mass.append(mass_recall(lg[h:h + 1], sel, scale))
+                    kp = kept[b, r, :int(kcnt[b, r])].long()
+                    in_kept = torch.isin(true // P, kp)
+                    page_rec.append(float(in_kept.float().mean().item()))
+                    if bool(in_kept.any()):
+                        ham_rec.append(recall_at_k(sel, true[in_kept]))
+                continue
             grp = lg.sum(0)
             true = torch.topk(grp, min(k_true or wl.top_k, n)).indices
             sel = st.idx[b, g, :int(st.count[b, g])].long()
@@ -329,7 +346,8 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
            "attention_mass_recall": statistics.mean(mass),
            "true_topk_in_kept_pages": statistics.mean(page_rec),
            "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
-           "k": wl.top_k, "k_true": k_true or wl.top_k, "kept_pages": st.m_max, "rows": B * G}
+           "k": wl.top_k, "k_true": k_true or wl.top_k, "kept_pages": st.m_max,
+           "rows": B * rows}
     if full:
         res["spearman_minus_hamming_vs_logit"] = statistics.mean(rho)
         res["random_selection_mass"] = wl.top_k / float(inp["seq_len"].float().mean())
@@ -369,6 +387,8 @@ def selection_quality(dev):
     for k in (1024, 4096):
         sweep[f"gkr_keep_1/16_k{k}"] = hhr_quality(S.scaled(wl, top_k=k), inp, dev, inp["R"], 0,
                                                    16, full=False)
+    sweep["per_query_head_keep_1/16"] = hhr_quality(
+        S.scaled(wl, select_per_head=True), inp, dev, inp["R"], 0, 16, full=False)
     sweep["sink_1_local_2_pages_keep_1/16"] = hhr_quality(
         S.scaled(wl, sink_pages=1, local_pages=2), inp, dev, inp["R"], 0, 16, full=False)
     for bits in (64, 256):
@@ -424,7 +444,7 @@ def selection_quality(dev):
 
 SECONDARY = ("llama8b_128k_b1", "ragged_b32", "llama8b_32k", "tiny_1h_4k", "hisa_128k_t1",
              "hisa_128k_t64", "llama8b_128k_b8_codes64", "llama8b_128k_b8_codes256",
-             "llama8b_128k_b8_flat", "llama8b_128k_b8_sink1_local2")
+             "llama8b_128k_b8_flat", "llama8b_128k_b8_sink1_local2", "llama8b_128k_b8_per_head")
 
 
 def indexer_required_bytes(wl, lens):
@@ -464,7 +484,8 @@ def measure_secondary(name, dev, l2, f16, steps, stream, mem_cap):
         inp = S.make_inputs(wl, device=dev, layer=l, with_values=hashing)
         d = hhr.make_dims(wl.batch, wl.n_q_heads if hashing else wl.n_queries, wl.n_kv_heads,
                           wl.page_size, inp["max_pages"], inp["n_phys"],
-                          summary_fp16=f16 if hashing else 0, code_bits=wl.code_bits)
+                          summary_fp16=f16 if hashing else 0, code_bits=wl.code_bits,
+                          select_per_head=int(wl.select_per_head))
         cache = LayerCache(d, dev, hashing=hashing, block_means=not hashing)
         zero = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
         hhr.hhr_encode_keys(d, inp["k_cache"], inp["page_table"], zero, inp["seq_len"],

@@ -40,15 +40,18 @@ struct AttnArgs {
   const uint16_t* v_cache;
   const int32_t* page_table;
   const int32_t* seq_len;
-  const int32_t* idx;       // [B][G][top_k]
-  const int32_t* count;     // [B][G]
-  float* part_o;            // [B][G][n_splits][gs][d]   (n_splits > 1)
-  float* part_ml;           // [B][G][n_splits][gs][2]
+  const int32_t* idx;       // [B][Gs][top_k]
+  const int32_t* count;     // [B][Gs]
+  float* part_o;            // [B][Gs][n_splits][gs][d]   (n_splits > 1)
+  float* part_ml;           // [B][Gs][n_splits][gs][2]
   float* out;               // [B][Hq][d]                 (n_splits == 1)
   float scale_log2;
   int Hq, G, P, maxp, n_phys, top_k, n_splits, split_rows;
-  const uint32_t* rows;     // [B][G][top_k] cache rows of the selected keys, already
+  const uint32_t* rows;     // [B][Gs][top_k] cache rows of the selected keys, already
                             // resolved and checked (fused step); null: resolve from idx
+  int Gs, kv_div;           // selection rows per sequence (G, or Hq per head): row r holds
+                            // query heads [r gs, (r + 1) gs), gs = Hq / Gs, and reads the
+                            // K/V of head r / kv_div
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -123,11 +126,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   uint16_t* stage_base = reinterpret_cast<uint16_t*>(at_smem);             // [kStages][2][kTile][d]
   uint32_t* offs = reinterpret_cast<uint32_t*>(stage_base + (size_t)kStages * 2 * kTile * kD);
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;  // g: selection row
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;   // fragment coordinates
-  const int gs = a.Hq / a.G;
-  const int row = b * a.G + g;
+  const int gs = a.Hq / a.Gs;
+  const int row = b * a.Gs + g;
   const int cnt = min(a.count[row], a.top_k);
   const int base = split * a.split_rows;
   // A split past the selection does no work (in a cluster it still joins the merge).
@@ -147,7 +150,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
       if (t >= 0 && t < n && lp < a.maxp) {
         const int phys = a.page_table[(size_t)b * a.maxp + lp];
         if (phys >= 0 && phys < a.n_phys)
-          o = ((uint32_t)phys * (uint32_t)a.G + (uint32_t)g) * (uint32_t)a.P + (uint32_t)(t % a.P);
+          o = ((uint32_t)phys * (uint32_t)a.G + (uint32_t)(g / a.kv_div)) * (uint32_t)a.P +
+              (uint32_t)(t % a.P);
         else
           flag_status(kStatusBadPage);
       } else {
@@ -379,7 +383,7 @@ struct CombineArgs {
   const float* part_ml;
   const int32_t* count;
   float* out;  // [B][Hq][d]
-  int Hq, G, top_k, n_splits, split_rows;
+  int Hq, G, top_k, n_splits, split_rows;  // G: selection rows per sequence (Gs)
 };
 
 __global__ void __launch_bounds__(kD) attn_combine_kernel(CombineArgs a) {

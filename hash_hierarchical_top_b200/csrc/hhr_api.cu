@@ -48,8 +48,14 @@ int check_dims(const hhr_dims* d) {
     return HHR_ERR_UNSUPPORTED;
   if (d->max_pages_per_seq > kMaxPagesPerSeq) return HHR_ERR_UNSUPPORTED;
   if (d->summary_fp16 != 0 && d->summary_fp16 != 1) return HHR_ERR_INVALID_ARG;
+  if (d->select_per_head != 0 && d->select_per_head != 1) return HHR_ERR_INVALID_ARG;
   return HHR_OK;
 }
+
+// Selection rows per sequence (KV groups, or query heads with select_per_head) and the
+// number of rows that share one KV head.
+inline int sel_rows(const hhr_dims* d) { return d->select_per_head ? d->n_q_heads : d->n_kv_heads; }
+inline int kv_div(const hhr_dims* d) { return sel_rows(d) / d->n_kv_heads; }
 
 // 32-bit code words per key and its index among the supported lengths (2, 4, 8 words).
 inline int code_words(const hhr_dims* d) { return d->code_bits / 32; }
@@ -112,15 +118,15 @@ int kept_max(const hhr_dims* d, int m_pages, int keep_div) {
 
 SelectLayout select_layout(const hhr_dims* d, int mode, int m_max) {
   SelectLayout L{};
-  const size_t B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, maxp = d->max_pages_per_seq;
+  const size_t B = d->batch, Gs = sel_rows(d), Hq = d->n_q_heads, maxp = d->max_pages_per_seq;
   size_t off = 0;
   if (mode == HHR_MODE_HASH) {
-    L.qpn = off;    off += align256(B * G * 2 * kD * 4);
+    L.qpn = off;    off += align256(B * Gs * 2 * kD * 4);
     L.q_rot = off;  off += align256(B * Hq * kD * 4);
     L.q_code = off; off += align256(B * Hq * code_words(d) * 4);
-    L.bounds = off; off += align256(B * G * maxp * 4);
-    L.kept = off;   off += align256(B * G * (size_t)m_max * 4);
-    L.kept_count = off; off += align256(B * G * 4);
+    L.bounds = off; off += align256(B * Gs * maxp * 4);
+    L.kept = off;   off += align256(B * Gs * (size_t)m_max * 4);
+    L.kept_count = off; off += align256(B * Gs * 4);
   } else {
     const size_t T = Hq;
     L.bounds = off; off += align256(B * T * maxp * 4);
@@ -141,12 +147,13 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
     if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
     if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
       return HHR_ERR_UNSUPPORTED;
-    if (topm_hamming_smem(d->n_q_heads / d->n_kv_heads, code_words(d),
+    if (topm_hamming_smem(d->n_q_heads / sel_rows(d), code_words(d),
                           kept_max(d, m_pages, keep_div), d->page_size,
                           d->max_pages_per_seq) > kMaxKernelSmem)
       return HHR_ERR_UNSUPPORTED;
   } else if (mode == HHR_MODE_INDEXER) {
     if (m_pages < 1 || keep_div != 0) return HHR_ERR_INVALID_ARG;
+    if (d->select_per_head) return HHR_ERR_INVALID_ARG;  // indexer rows are queries already
     if (d->n_kv_heads != 1) return HHR_ERR_INVALID_ARG;
     if ((long long)kept_max(d, m_pages, 0) * d->page_size > kMaxTokCand)
       return HHR_ERR_UNSUPPORTED;
@@ -360,22 +367,23 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     void (*qp)(QPrepArgs) =
         cw == 2 ? qprep_kernel<2> : cw == 8 ? qprep_kernel<8> : qprep_kernel<4>;
     if (allow_smem(qp, qprep_smem(), g_smem_qprep[cw_index(cw)]) != cudaSuccess) return HHR_ERR_CUDA;
-    const int nt = topm_hamming_threads(cw, (long long)B * G * kHamRanks, sm_count());
-    if (allow_smem(topm_hamming_for(Hq / G, cw, nt), topm_hamming_smem(Hq / G, cw, m_max, P, maxp),
-                   g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(Hq / G) - 1]) != cudaSuccess)
+    const int Gs = sel_rows(d), rh = Hq / Gs;  // selection rows and their query heads
+    const int nt = topm_hamming_threads(cw, (long long)B * Gs * kHamRanks, sm_count());
+    if (allow_smem(topm_hamming_for(rh, cw, nt), topm_hamming_smem(rh, cw, m_max, P, maxp),
+                   g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(rh) - 1]) != cudaSuccess)
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qp<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
-        QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
+        QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G, d->select_per_head});
     prof_end(HHR_KERNEL_QPREP, s);
     if ((st = launch_status()) != HHR_OK) return st;
     // Every page kept (flat hash top-k): the bounds are computed only for a trace.
     const bool flat = m_max >= maxp;
     if (!flat || (trace != nullptr && trace->bounds != nullptr)) {
       const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                         d->n_phys_pages, 0};
+                         d->n_phys_pages, 0, Gs, kv_div(d)};
       const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
-      const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
+      const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
       prof_begin(HHR_KERNEL_BOUND, s);
       if (d->summary_fp16)
         page_bound_kernel<true><<<grid, kBoundWarps * 32, 0, s>>>(ba);
@@ -385,19 +393,20 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
       if ((st = launch_status()) != HHR_OK) return st;
     }
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, nullptr, sink, local};
-    const size_t fsm = topm_hamming_smem(Hq / G, cw, m_max, P, maxp);
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, nullptr, sink, local,
+                   Gs, kv_div(d)};
+    const size_t fsm = topm_hamming_smem(rh, cw, m_max, P, maxp);
     prof_begin(HHR_KERNEL_HAMMING, s);
-    topm_hamming_for(Hq / G, cw, nt)<<<B * G * kHamRanks, nt, fsm, s>>>(
+    topm_hamming_for(rh, cw, nt)<<<B * Gs * kHamRanks, nt, fsm, s>>>(
         TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if ((st = launch_status()) != HHR_OK) return st;
     if (trace != nullptr) {
       if ((st = copy_trace(trace->q_rot, ws, L.q_rot, (size_t)B * Hq * kD * 4, s))) return st;
       if ((st = copy_trace(trace->q_code, ws, L.q_code, (size_t)B * Hq * cw * 4, s))) return st;
-      if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * G * maxp * 4, s))) return st;
-      if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * G * m_max * 4, s))) return st;
-      if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * G * 4, s))) return st;
+      if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * Gs * maxp * 4, s))) return st;
+      if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * Gs * m_max * 4, s))) return st;
+      if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * Gs * 4, s))) return st;
     }
     return HHR_OK;
   }
@@ -451,10 +460,10 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
 
 size_t hhr_attn_workspace_bytes(const hhr_dims* d, int top_k) {
   if (check_dims(d) != HHR_OK || check_group(d) != HHR_OK || top_k < 1) return 0;
-  const AttnPlan plan = attn_plan(d->batch, d->n_kv_heads, top_k);
+  const AttnPlan plan = attn_plan(d->batch, sel_rows(d), top_k);
   const size_t ns = plan.n_splits;
-  const size_t rows = (size_t)d->batch * d->n_kv_heads;
-  const size_t gs = d->n_q_heads / d->n_kv_heads;
+  const size_t rows = (size_t)d->batch * sel_rows(d);
+  const size_t gs = d->n_q_heads / sel_rows(d);
   return align256(rows * ns * gs * kD * 4) + align256(rows * ns * gs * 2 * 4);
 }
 
@@ -478,26 +487,26 @@ int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cach
   if (ws_bytes < need) return HHR_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads;
-  const AttnPlan plan = attn_plan(B, G, top_k);
+  const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, Gs = sel_rows(d);
+  const AttnPlan plan = attn_plan(B, Gs, top_k);
   const int ns = plan.n_splits;
-  const int gs = Hq / G;
+  const int gs = Hq / Gs;
   char* ws = static_cast<char*>(workspace);
   float* part_o = reinterpret_cast<float*>(ws);
-  float* part_ml = reinterpret_cast<float*>(ws + align256((size_t)B * G * ns * gs * kD * 4));
+  float* part_ml = reinterpret_cast<float*>(ws + align256((size_t)B * Gs * ns * gs * kD * 4));
   AttnArgs a{q, k_cache, v_cache, page_table, seq_len, idx, count, part_o, part_ml, out,
              scale * 1.4426950408889634f, Hq, G, d->page_size, d->max_pages_per_seq,
-             d->n_phys_pages, top_k, ns, plan.split_rows};
+             d->n_phys_pages, top_k, ns, plan.split_rows, nullptr, Gs, kv_div(d)};
   prof_begin(HHR_KERNEL_ATTN, s);
   if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
-  sparse_attn_kernel<false><<<dim3(ns, G, B), kAttnThreads, attn_smem(), s>>>(a);
+  sparse_attn_kernel<false><<<dim3(ns, Gs, B), kAttnThreads, attn_smem(), s>>>(a);
   prof_end(HHR_KERNEL_ATTN, s);
   if ((st = launch_status()) != HHR_OK) return st;
   if (ns > 1) {
     prof_begin(HHR_KERNEL_COMBINE, s);
     attn_combine_kernel<<<dim3(Hq, B), kD, 0, s>>>(
-        CombineArgs{part_o, part_ml, count, out, Hq, G, top_k, ns, plan.split_rows});
+        CombineArgs{part_o, part_ml, count, out, Hq, Gs, top_k, ns, plan.split_rows});
     prof_end(HHR_KERNEL_COMBINE, s);
   }
   return launch_status();
@@ -509,7 +518,7 @@ size_t hhr_decode_step_workspace_bytes(const hhr_dims* d, int m_pages, int keep_
   const size_t att = hhr_attn_workspace_bytes(d, top_k);
   if (sel == 0 || att == 0) return 0;
   // + the cache row of every selected key, handed from the selection to the attention.
-  return sel + att + align256((size_t)d->batch * d->n_kv_heads * top_k * 4);
+  return sel + att + align256((size_t)d->batch * sel_rows(d) * top_k * 4);
 }
 
 int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
@@ -541,6 +550,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   const int B = d->batch, G = d->n_kv_heads, Hq = d->n_q_heads, P = d->page_size;
+  const int Gs = sel_rows(d), rh = Hq / Gs;  // selection rows and their query heads
   const int maxp = d->max_pages_per_seq, gs = Hq / G;
   const int m_max = kept_max(d, m_pages, keep_div);
   const SelectLayout L = select_layout(d, HHR_MODE_HASH, m_max);
@@ -552,16 +562,16 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
   int32_t* kept_count = reinterpret_cast<int32_t*>(ws + L.kept_count);
   char* aws = ws + L.total;
-  const AttnPlan plan = attn_plan(B, G, top_k);
+  const AttnPlan plan = attn_plan(B, Gs, top_k);
   const int ns = plan.n_splits;
   float* part_o = reinterpret_cast<float*>(aws);
-  float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * G * ns * gs * kD * 4));
-  uint32_t* sel_rows = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
+  float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * Gs * ns * rh * kD * 4));
+  uint32_t* row_buf = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
   const int cw = code_words(d);
-  const size_t fsm = topm_hamming_smem(gs, cw, m_max, P, maxp);
-  const int nt = topm_hamming_threads(cw, (long long)B * G * kHamRanks, sm_count());
-  if (allow_smem(topm_hamming_for(gs, cw, nt), fsm,
-                 g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(gs) - 1]) != cudaSuccess)
+  const size_t fsm = topm_hamming_smem(rh, cw, m_max, P, maxp);
+  const int nt = topm_hamming_threads(cw, (long long)B * Gs * kHamRanks, sm_count());
+  if (allow_smem(topm_hamming_for(rh, cw, nt), fsm,
+                 g_smem_ham[cw_index(cw)][nt == 512][hamming_planes(rh) - 1]) != cudaSuccess)
     return HHR_ERR_CUDA;
   if (allow_smem(sparse_attn_kernel<false>, attn_smem(), g_smem_attn) != cudaSuccess)
     return HHR_ERR_CUDA;
@@ -574,7 +584,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   step_prologue_for(gs, cw)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
-                   d->summary_fp16});
+                   d->summary_fp16, d->select_per_head});
   prof_end(HHR_KERNEL_ENCODE, s);
   if ((st = launch_status()) != HHR_OK) return st;
   // a2: page bounds (none when every page is kept: a flat hash top-k).
@@ -584,9 +594,9 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     // an event is recorded between the two (profiling), which leaves no overlap to use.
     const int early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
     const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                       d->n_phys_pages, early};
+                       d->n_phys_pages, early, Gs, kv_div(d)};
     const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
-    const dim3 grid = bound_grid(G, (maxp + ppc - 1) / ppc, B);
+    const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
     prof_begin(HHR_KERNEL_BOUND, s);
     e = d->summary_fp16 ? launch_pdl(page_bound_kernel<true>, grid, dim3(kBoundWarps * 32), 0, s, ba)
                         : launch_pdl(page_bound_kernel<false>, grid, dim3(kBoundWarps * 32), 0, s, ba);
@@ -596,9 +606,10 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   // a2 top-m + a3 + a4: kept pages, Hamming distances, deterministic top-k.
   {
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, sel_rows, sink, local};
+                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, row_buf, sink, local,
+                   Gs, kv_div(d)};
     prof_begin(HHR_KERNEL_HAMMING, s);
-    e = launch_pdl(topm_hamming_for(gs, cw, nt), dim3(B * G * kHamRanks), dim3(nt), fsm, s,
+    e = launch_pdl(topm_hamming_for(rh, cw, nt), dim3(B * Gs * kHamRanks), dim3(nt), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
     prof_end(HHR_KERNEL_HAMMING, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
@@ -606,13 +617,13 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   // a5: sparse attention over the selected rows. The splits of a group form a cluster
   // merged through distributed shared memory when they fit one (at most 8 splits).
   {
-    const AttnPlan cp = attn_plan(B, G, top_k, kMaxClusterSplits);
+    const AttnPlan cp = attn_plan(B, Gs, top_k, kMaxClusterSplits);
     if (cp.n_splits <= kMaxClusterSplits) {
       AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, nullptr, nullptr,
                   out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k,
-                  cp.n_splits, cp.split_rows, sel_rows};
+                  cp.n_splits, cp.split_rows, row_buf, Gs, kv_div(d)};
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(cp.n_splits, G, B);
+      cfg.gridDim = dim3(cp.n_splits, Gs, B);
       cfg.blockDim = dim3(kAttnThreads);
       cfg.dynamicSmemBytes = attn_smem();
       cfg.stream = s;
@@ -632,16 +643,16 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     } else {
       AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, part_o, part_ml,
                   out, scale * 1.4426950408889634f, Hq, G, P, maxp, d->n_phys_pages, top_k, ns,
-                  plan.split_rows, sel_rows};
+                  plan.split_rows, row_buf, Gs, kv_div(d)};
       prof_begin(HHR_KERNEL_ATTN, s);
-      e = launch_pdl(sparse_attn_kernel<false>, dim3(ns, G, B), dim3(kAttnThreads), attn_smem(),
+      e = launch_pdl(sparse_attn_kernel<false>, dim3(ns, Gs, B), dim3(kAttnThreads), attn_smem(),
                      s, aa);
       prof_end(HHR_KERNEL_ATTN, s);
       if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
       if (ns > 1) {
         prof_begin(HHR_KERNEL_COMBINE, s);
         e = launch_pdl(attn_combine_kernel, dim3(Hq, B), dim3(kD), 0, s,
-                       CombineArgs{part_o, part_ml, out_count, out, Hq, G, top_k, ns,
+                       CombineArgs{part_o, part_ml, out_count, out, Hq, Gs, top_k, ns,
                                    plan.split_rows});
         prof_end(HHR_KERNEL_COMBINE, s);
         if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }

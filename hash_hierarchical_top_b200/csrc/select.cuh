@@ -23,8 +23,9 @@ struct QPrepArgs {
   const float* W;
   float* q_rot;      // [B][Hq][d]
   uint32_t* q_code;  // [B][Hq][CW]
-  float* qpn;        // [B][G][2][d]: [0] = qneg, [1] = qpos
+  float* qpn;        // [B][G][2][d] ([B][Hq][2][d] per head): [0] = qneg, [1] = qpos
   int Hq, G;
+  int per_head;      // one folded query per query head instead of per KV group
 };
 
 template <int CW>
@@ -77,12 +78,22 @@ __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
     const int h = tid / CW, w = tid % CW;
     a.q_code[((size_t)b * a.Hq + g * gs + h) * CW + w] = cword[h][w];
   }
-  if (row_lead) {
+  if (row_lead && !a.per_head) {
     float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
 #pragma unroll
     for (int rb = 0; rb < kRowBlocks; ++rb) {
       o[rb * 32 + lrow] = qneg[rb];
       o[kD + rb * 32 + lrow] = qpos[rb];
+    }
+  } else if (row_lead) {  // each head's own folding of its rotated query
+    for (int h = 0; h < gs; ++h) {
+      float* o = a.qpn + ((size_t)b * a.Hq + g * gs + h) * 2 * kD;
+#pragma unroll
+      for (int rb = 0; rb < kRowBlocks; ++rb) {
+        const float y = qr[h][rb * 32 + lrow];
+        o[rb * 32 + lrow] = fminf(y, 0.f);
+        o[kD + rb * 32 + lrow] = fmaxf(y, 0.f);
+      }
     }
   }
 }
@@ -137,13 +148,14 @@ __device__ __forceinline__ int bound_chunk() { return bound_chunk_of(blockIdx.x,
 #endif
 
 struct BoundArgs {
-  const float* qpn;
+  const float* qpn;         // [B][Gs][2][d]
   const void* page_minmax;  // f32 or f16 [n_phys][G][2][d]
   const int32_t* page_table;
   const int32_t* seq_len;
-  float* bounds;  // [B][G][maxp]
+  float* bounds;  // [B][Gs][maxp]
   int G, P, maxp, n_phys;
   int early;      // CTAs that warm L2 before the dependency wait (0: none)
+  int Gs, kv_div; // selection rows per sequence (G, or Hq per head); row r uses KV head r / kv_div
 };
 
 // Sum over the warp of 8 per-lane partials (one per page): a butterfly over lane bits 4
@@ -232,7 +244,7 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
             const int phys = a.page_table[(size_t)tb * a.maxp + p];
             if (phys >= 0 && phys < a.n_phys)
               prefetch_l2(reinterpret_cast<const uint4*>(a.page_minmax) +
-                              ((size_t)phys * a.G + tg) * kPieces,
+                              ((size_t)phys * a.G + tg / a.kv_div) * kPieces,
                           kPieces * 16);
           }
         }
@@ -241,11 +253,12 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
   }
   pdl_wait();
   pdl_trigger();
-  const int g = bound_group(), b = blockIdx.z;
+  const int r = bound_group(), b = blockIdx.z;  // selection row r reads KV head r / kv_div
+  const int g = r / a.kv_div;
   const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
   const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
   if (p0 >= npg) return;
-  const float* qb = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
+  const float* qb = a.qpn + ((size_t)b * a.Gs + r) * 2 * kD;
   float4 q0, q1;
   if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
     const float4* qv = reinterpret_cast<const float4*>(qb + (lane >> 4) * kD + 8 * (lane & 15));
@@ -271,7 +284,7 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
       if constexpr (!F16) y[i] = load_summary16(src + 32);
     }
   }
-  float* out = a.bounds + ((size_t)b * a.G + g) * a.maxp;
+  float* out = a.bounds + ((size_t)b * a.Gs + r) * a.maxp;
 #pragma unroll
   for (int st = 0; st < kSets; ++st) {
     float v[8];
@@ -622,6 +635,10 @@ struct HammingArgs {
   uint32_t* out_rows;        // [B][G][top_k] cache row (phys*G + g)*P + slot of each selected
                              // key, for the attention of the fused step; or null
   int sink, local;           // forced pages [0, sink) and the last `local` of each sequence
+  int Gs, kv_div;            // selection rows per sequence (G, or Hq per head); row r of a
+                             // sequence uses the KV head r / kv_div and query heads
+                             // [r Hq/Gs, (r + 1) Hq/Gs); bounds, kept lists and outputs are
+                             // indexed by (sequence, row)
 };
 
 inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
@@ -720,9 +737,9 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   constexpr int kBins = (kMaxGroup * 32 * CW + 2 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
-  const int b = row / a.G, g = row % a.G;
+  const int b = row / a.Gs, g = (row % a.Gs) / a.kv_div;
   const int tid = threadIdx.x;
-  const int gs = a.Hq / a.G;
+  const int gs = a.Hq / a.Gs;  // query heads of the row
   const int nbins = gs * 32 * CW + 2;
   m = min(m, a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                                // [nbins]
@@ -939,10 +956,10 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
   extern __shared__ uint32_t fsm[];
   const HammingArgs& h = a.h;
   const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
-  const int b = row / h.G, g = row % h.G;
-  const int gs = h.Hq / h.G;
+  const int b = row / h.Gs, r = row % h.Gs, g = r / h.kv_div;
+  const int gs = h.Hq / h.Gs;  // query heads of the row
   if (threadIdx.x < gs * CW)  // visible after the selection's first barrier
-    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + g * gs) * CW + threadIdx.x];
+    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + r * gs) * CW + threadIdx.x];
   const int mw = (h.m_max + 3) & ~3;
   int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
   int32_t* kphys_s = kept_s + mw;

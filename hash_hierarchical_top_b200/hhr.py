@@ -49,7 +49,7 @@ class HHRError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "head_dim", "page_size", "code_bits",
-        "max_pages_per_seq", "n_phys_pages", "summary_fp16")]
+        "max_pages_per_seq", "n_phys_pages", "summary_fp16", "select_per_head")]
 
 
 class SelectOpts(ctypes.Structure):
@@ -121,9 +121,14 @@ def status_string(status: int) -> str:
 
 
 def make_dims(batch, n_q_heads, n_kv_heads, page_size, max_pages_per_seq, n_phys_pages,
-              head_dim=128, code_bits=128, summary_fp16=0) -> Dims:
+              head_dim=128, code_bits=128, summary_fp16=0, select_per_head=0) -> Dims:
     return Dims(batch, n_q_heads, n_kv_heads, head_dim, page_size, code_bits,
-                max_pages_per_seq, n_phys_pages, int(summary_fp16))
+                max_pages_per_seq, n_phys_pages, int(summary_fp16), int(select_per_head))
+
+
+def sel_rows(d: Dims) -> int:
+    """Selection rows per sequence: KV groups, or query heads with select_per_head."""
+    return d.n_q_heads if d.select_per_head else d.n_kv_heads
 
 
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)

@@ -37,7 +37,7 @@ class DecodeStep:
                  attention: bool = True, sink_pages: int = 0, local_pages: int = 0):
         self.d, self.mode, self.m_pages, self.keep_div, self.top_k = d, mode, m_pages, keep_div, top_k
         self.opts = hhr.make_opts(sink_pages, local_pages)  # forced pages (hash mode variant)
-        rows = d.n_kv_heads if mode == hhr.HHR_MODE_HASH else d.n_q_heads
+        rows = hhr.sel_rows(d) if mode == hhr.HHR_MODE_HASH else d.n_q_heads
         ws = hhr.hhr_select_workspace_bytes(d, mode, m_pages, keep_div, top_k)
         if ws == 0:
             raise ValueError("unsupported selection parameters")

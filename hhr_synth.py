@@ -61,6 +61,7 @@ class Workload:
     permute_pages: bool = False      # page table = random permutation of the pool
     sink_pages: int = 0              # selection variant: forced first pages of a sequence
     local_pages: int = 0             # selection variant: forced last pages of a sequence
+    select_per_head: bool = False    # selection variant: one selection per query head
 
     @property
     def group_size(self):
@@ -118,6 +119,8 @@ WORKLOADS["llama8b_128k_b8_flat"] = dataclasses.replace(
 WORKLOADS["llama8b_128k_b8_sink1_local2"] = dataclasses.replace(
     WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_b8_sink1_local2", sink_pages=1,
     local_pages=2)
+WORKLOADS["llama8b_128k_b8_per_head"] = dataclasses.replace(
+    WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_b8_per_head", select_per_head=True)
 for _bits in (64, 256):
     _n = f"llama8b_128k_b8_codes{_bits}"
     WORKLOADS[_n] = dataclasses.replace(WORKLOADS["llama8b_128k_b8"], name=_n, code_bits=_bits)

@@ -85,6 +85,12 @@ typedef struct {
   int summary_fp16;       /* page_minmax element type: 0 = f32; 1 = f16 rounded outward
                              (min toward -inf, max toward +inf), so the page bound stays an
                              upper bound; values beyond the f16 range saturate to -inf/+inf */
+  int select_per_head;    /* hash mode: 0 = one selection per KV group (the default reading:
+                             bounds and distances summed over the group's query heads);
+                             1 = one per query head (a variant): head h scores the summaries
+                             and codes of KV group h / (Hq/G) with its own query alone and
+                             attends its own set. Selection rows per sequence ("rows" below)
+                             are G, or Hq with 1. Indexer mode: must be 0. */
 } hhr_dims;
 
 /* Optional copies of the intermediates of hhr_select, for inspection and layered
@@ -173,7 +179,8 @@ size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, i
  * Limits: ceil(seq_len/P) <= 32768 pages per sequence; m_b * P <= 131072 candidates
  * (hash mode: every page of a 128K-key sequence, a flat hash top-k) or <= 32768
  * (indexer mode).
- * out_idx: int32 [B][rows][top_k]; out_count: int32 [B][rows] (rows = G or T).
+ * out_idx: int32 [B][rows][top_k]; out_count: int32 [B][rows] (rows = G, Hq with
+ * dims.select_per_head, or T in indexer mode; trace->bounds/kept/kept_count likewise).
  * opts: may be NULL (see hhr_select_opts).
  * trace: may be NULL. workspace: at least hhr_select_workspace_bytes(). */
 int hhr_select(const hhr_dims* dims, int mode, const uint16_t* q, const int32_t* seq_len,
@@ -193,7 +200,8 @@ size_t hhr_attn_workspace_bytes(const hhr_dims* dims, int top_k);
  *   S = idx[b][g][0..count[b][g]) and g = h / (Hq / G). Every selected K/V row is
  *   read once per group and shared by the group's query heads. An empty set gives
  *   a zero output.
- *   idx: int32 [B][G][top_k] logical tokens; count: int32 [B][G] (clipped to
+ *   With dims.select_per_head, each query head h attends its own set S = idx[b][h].
+ *   idx: int32 [B][rows][top_k] logical tokens; count: int32 [B][rows] (clipped to
  *   top_k); an index outside [0, seq_len[b]) is skipped and flagged.
  *   out: f32 [B][Hq][d]. workspace: at least hhr_attn_workspace_bytes(). */
 int hhr_sparse_attn(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_cache,

@@ -36,7 +36,8 @@ def dims_of(wl, inp, summary_fp16=0):
     return hhr.make_dims(wl.batch, wl.n_queries if wl.mode == "indexer" else wl.n_q_heads,
                          wl.n_kv_heads, wl.page_size, inp["max_pages"], inp["n_phys"],
                          head_dim=wl.head_dim, code_bits=wl.code_bits,
-                         summary_fp16=summary_fp16)
+                         summary_fp16=summary_fp16,
+                         select_per_head=int(getattr(wl, "select_per_head", False)))
 
 
 def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
@@ -64,7 +65,7 @@ def run_gpu(wl, inp, bulk=True, trace=True, encode_chunks=None, summary_fp16=0):
             step.encode(inp["k_cache"], inp["page_table"], done, n_new, encode_chunks,
                         inp["R"] if hashing else None, inp["W"] if hashing else None, cache)
             done = (done + n_new).to(torch.int32)
-    rows = d.n_kv_heads if hashing else d.n_q_heads
+    rows = hhr.sel_rows(d) if hashing else d.n_q_heads
     tr_t = dict(
         q_rot=torch.empty(B, d.n_q_heads, 128, dtype=torch.float32, device=dev) if hashing else None,
         q_code=(torch.empty(B, d.n_q_heads, d.code_bits // 32, dtype=torch.int32, device=dev)
@@ -153,70 +154,77 @@ def check_hash_group(wl, inp_np, g_out, b, g, report):
                 if (int(qd[h, w]) >> bit) & 1:
                     assert qfrag[h, 32 * w + bit], "non-fragile query code bit differs"
 
-    # a2: bounds (oracle on the GPU's summaries) and kept pages.
-    kmin_g, kmax_g = gmm[:, 0], gmm[:, 1]
-    beta_ref = O.page_bounds(qr, kmin_g, kmax_g)
-    beta_gpu = g_out["bounds"][b, g, :n_pages].astype(np.float64)
-    scale = (np.abs(qr)[:, None, :] * np.maximum(np.abs(kmin_g), np.abs(kmax_g))[None]).sum(axis=(0, 2))
-    assert np.all(np.abs(beta_gpu - beta_ref) <= BOUND_TOL * scale), "page bound out of tolerance"
-    # Invariant at any size: the GPU's bound dominates every true summed logit of its page.
-    Krot = O.rotate(R, O.logical_rows(inp_np["k_cache"], pt, g, n, P))
-    summed = (Krot @ Qrot.T).sum(axis=1)
-    page_max = np.full(n_pages, -np.inf)
-    np.maximum.at(page_max, np.arange(n) // P, summed)
-    assert np.all(beta_gpu >= page_max - 1e-5 * scale), "bound below a true logit"
-    forced = O.forced_pages(n_pages, wl.sink_pages, wl.local_pages)
-    m = max(O.kept_count(n_pages, wl.m_pages, wl.keep_div), len(forced))
-    kc = int(g_out["kept_count"][b, g])
-    assert kc == m
-    kept_gpu = g_out["kept"][b, g, :kc]
-    # Same-precision decision: the oracle's top-m of the GPU's own fp32 bounds.
-    beta_gpu32 = g_out["bounds"][b, g, :n_pages]
-    want = O.top_m_forced(beta_gpu32, m, forced) if len(forced) else O.top_m(beta_gpu32, m)
-    assert np.array_equal(kept_gpu, want), "top-m differs"
-    # Against the full fp64 oracle bounds (over the pages that are not forced): exact unless
-    # the cut is within tolerance.
-    beta_full = O.page_bounds(Qrot, enc["kmin"], enc["kmax"])
-    rest = np.setdiff1d(np.arange(n_pages), forced)
-    mr = m - len(forced)
-    order = np.sort(beta_full[rest])[::-1]
-    tol_cut = BOUND_TOL * float(scale.max())
-    if 0 < mr < len(rest):
-        margin = order[mr - 1] - order[mr]
-        if margin > 2 * tol_cut:
-            assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
+    # a2-a5 per selection row: the whole group, or each of its query heads on its own.
+    def select_row(row, hs):
+        qr_r, Qrot_r, Qg_r, gq_r = qr[hs], Qrot[hs], Qg[hs], gq[hs]
+        # a2: bounds (oracle on the GPU's summaries) and kept pages.
+        kmin_g, kmax_g = gmm[:, 0], gmm[:, 1]
+        beta_ref = O.page_bounds(qr_r, kmin_g, kmax_g)
+        beta_gpu = g_out["bounds"][b, row, :n_pages].astype(np.float64)
+        scale = (np.abs(qr_r)[:, None, :] * np.maximum(np.abs(kmin_g), np.abs(kmax_g))[None]).sum(axis=(0, 2))
+        assert np.all(np.abs(beta_gpu - beta_ref) <= BOUND_TOL * scale), "page bound out of tolerance"
+        # Invariant at any size: the GPU's bound dominates every true summed logit of its page.
+        Krot = O.rotate(R, O.logical_rows(inp_np["k_cache"], pt, g, n, P))
+        summed = (Krot @ Qrot_r.T).sum(axis=1)
+        page_max = np.full(n_pages, -np.inf)
+        np.maximum.at(page_max, np.arange(n) // P, summed)
+        assert np.all(beta_gpu >= page_max - 1e-5 * scale), "bound below a true logit"
+        forced = O.forced_pages(n_pages, wl.sink_pages, wl.local_pages)
+        m = max(O.kept_count(n_pages, wl.m_pages, wl.keep_div), len(forced))
+        kc = int(g_out["kept_count"][b, row])
+        assert kc == m
+        kept_gpu = g_out["kept"][b, row, :kc]
+        # Same-precision decision: the oracle's top-m of the GPU's own fp32 bounds.
+        beta_gpu32 = g_out["bounds"][b, row, :n_pages]
+        want = O.top_m_forced(beta_gpu32, m, forced) if len(forced) else O.top_m(beta_gpu32, m)
+        assert np.array_equal(kept_gpu, want), "top-m differs"
+        # Against the full fp64 oracle bounds (over the pages that are not forced): exact unless
+        # the cut is within tolerance.
+        beta_full = O.page_bounds(Qrot_r, enc["kmin"], enc["kmax"])
+        rest = np.setdiff1d(np.arange(n_pages), forced)
+        mr = m - len(forced)
+        order = np.sort(beta_full[rest])[::-1]
+        tol_cut = BOUND_TOL * float(scale.max())
+        if 0 < mr < len(rest):
+            margin = order[mr - 1] - order[mr]
+            if margin > 2 * tol_cut:
+                assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
+            else:
+                report["near_tie_cuts"] = report.get("near_tie_cuts", 0) + 1
+                sure_in = set(rest[beta_full[rest] > order[mr - 1] + 2 * tol_cut]) | set(forced)
+                maybe = set(rest[beta_full[rest] >= order[mr - 1] - 2 * tol_cut]) | set(forced)
+                assert sure_in <= set(kept_gpu) <= maybe
         else:
-            report["near_tie_cuts"] = report.get("near_tie_cuts", 0) + 1
-            sure_in = set(rest[beta_full[rest] > order[mr - 1] + 2 * tol_cut]) | set(forced)
-            maybe = set(rest[beta_full[rest] >= order[mr - 1] - 2 * tol_cut]) | set(forced)
-            assert sure_in <= set(kept_gpu) <= maybe
-    else:
-        assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
+            assert np.array_equal(kept_gpu, O.top_m_forced(beta_full, m, forced))
 
-    # a3 + a4: Hamming top-k on the GPU's codes and kept pages, bit-exact.
-    cand = O.candidates_of(kept_gpu, n, P)
-    delta = O.hamming(gq, gc[cand])
-    if len(forced):
-        S_ref = O.top_k_forced(delta, cand, min(wl.top_k, len(cand)), np.isin(cand // P, forced))
-    else:
-        S_ref = O.top_k_smallest(delta, cand, min(wl.top_k, len(cand)))
-    cnt = int(g_out["count"][b, g])
-    assert cnt == len(S_ref)
-    assert np.array_equal(g_out["idx"][b, g, :cnt], S_ref), "Hamming top-k differs"
-    assert np.all(g_out["idx"][b, g, cnt:] == -1)
+        # a3 + a4: Hamming top-k on the GPU's codes and kept pages, bit-exact.
+        cand = O.candidates_of(kept_gpu, n, P)
+        delta = O.hamming(gq_r, gc[cand])
+        if len(forced):
+            S_ref = O.top_k_forced(delta, cand, min(wl.top_k, len(cand)), np.isin(cand // P, forced))
+        else:
+            S_ref = O.top_k_smallest(delta, cand, min(wl.top_k, len(cand)))
+        cnt = int(g_out["count"][b, row])
+        assert cnt == len(S_ref)
+        assert np.array_equal(g_out["idx"][b, row, :cnt], S_ref), "Hamming top-k differs"
+        assert np.all(g_out["idx"][b, row, cnt:] == -1)
 
-    # a5: attention on the GPU's selected set.
-    K = O.logical_rows(inp_np["k_cache"], pt, g, n, P)
-    V = O.logical_rows(inp_np["v_cache"], pt, g, n, P)
-    ref = O.sparse_attention(Qg, K[S_ref], V[S_ref], 1.0 / math.sqrt(wl.head_dim))
-    got = g_out["out"][b, g * gs:(g + 1) * gs].astype(np.float64)
-    for h in range(gs):
-        den = max(np.abs(ref[h]).max(), 1e-30)
-        rel = np.abs(got[h] - ref[h]).max() / den
-        report["attn_max_rel"] = max(report.get("attn_max_rel", 0.0), float(rel))
-        assert rel <= ATTN_TOL, f"attention rel err {rel} (b={b}, h={g * gs + h})"
-    return dict(kept_oracle=O.top_m(beta_full, m), kept_gpu=kept_gpu, idx=S_ref)
+        # a5: attention on the GPU's selected set.
+        K = O.logical_rows(inp_np["k_cache"], pt, g, n, P)
+        V = O.logical_rows(inp_np["v_cache"], pt, g, n, P)
+        ref = O.sparse_attention(Qg_r, K[S_ref], V[S_ref], 1.0 / math.sqrt(wl.head_dim))
+        got = g_out["out"][b, [g * gs + h for h in hs]].astype(np.float64)
+        for j, h in enumerate(hs):
+            den = max(np.abs(ref[j]).max(), 1e-30)
+            rel = np.abs(got[j] - ref[j]).max() / den
+            report["attn_max_rel"] = max(report.get("attn_max_rel", 0.0), float(rel))
+            assert rel <= ATTN_TOL, f"attention rel err {rel} (b={b}, h={g * gs + h})"
+        return dict(kept_oracle=O.top_m(beta_full, m), kept_gpu=kept_gpu, idx=S_ref)
 
+
+    if getattr(wl, "select_per_head", False):
+        return [select_row(g * gs + h, [h]) for h in range(gs)]
+    return select_row(g, list(range(gs)))
 
 def check_indexer_query(wl, inp_np, g_out, b, i, report):
     """Layered checks of the HISA indexer for one (sequence, chunk query)."""

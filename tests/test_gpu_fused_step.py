@@ -72,6 +72,14 @@ def test_fused_step_many_rows():
     _fused_vs_separate(wl, 1, True)
 
 
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1)])
+def test_fused_step_per_head(heads):
+    """One selection per query head: the fused call equals the separate calls."""
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], batch=3, ragged=(33, 4000), top_k=200,
+                  n_q_heads=heads[0], n_kv_heads=heads[1], select_per_head=True)
+    _fused_vs_separate(wl, 1, True)
+
+
 def _fused_vs_separate(wl, f16, with_new_rows):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
@@ -114,7 +122,7 @@ def _fused_vs_separate(wl, f16, with_new_rows):
     assert torch.equal(fs.out.view(torch.int32), ref.out.view(torch.int32))
 
 
-@pytest.mark.parametrize("variant", ["hierarchical", "flat", "forced"])
+@pytest.mark.parametrize("variant", ["hierarchical", "flat", "forced", "per_head"])
 def test_fused_step_against_oracle(variant):
     """The fused call's outputs through the layered oracle checks (selection + attention)."""
     build.build()
@@ -123,6 +131,8 @@ def test_fused_step_against_oracle(variant):
         wl = S.scaled(wl, m_pages=4096, keep_div=0)
     elif variant == "forced":
         wl = S.scaled(wl, sink_pages=2, local_pages=4)
+    elif variant == "per_head":
+        wl = S.scaled(wl, select_per_head=True)
     inp = S.make_inputs(wl, device="cuda")
     inp_np = S.to_numpy_inputs(inp)
     d = dims_of(wl, inp, 1)
@@ -139,9 +149,10 @@ def test_fused_step_against_oracle(variant):
     # feed the layered checks (the fused selection must equal it).
     sel = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda",
                      sink_pages=wl.sink_pages, local_pages=wl.local_pages)
-    bounds = torch.empty(B, wl.n_kv_heads, d.max_pages_per_seq, device="cuda")
-    kept = torch.empty(B, wl.n_kv_heads, sel.m_max, dtype=torch.int32, device="cuda")
-    kc = torch.empty(B, wl.n_kv_heads, dtype=torch.int32, device="cuda")
+    rows = hhr.sel_rows(d)
+    bounds = torch.empty(B, rows, d.max_pages_per_seq, device="cuda")
+    kept = torch.empty(B, rows, sel.m_max, dtype=torch.int32, device="cuda")
+    kc = torch.empty(B, rows, dtype=torch.int32, device="cuda")
     trace = hhr.make_trace(q_rot=tr["q_rot"], q_code=tr["q_code"], bounds=bounds, kept=kept,
                            kept_count=kc)
     sel.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=inp["R"], W=inp["W"],

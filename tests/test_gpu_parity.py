@@ -185,6 +185,19 @@ def test_many_rows_two_ctas_per_sm(bits):
     _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=1))
 
 
+@pytest.mark.parametrize("heads", [(32, 8), (8, 1), (6, 2)])
+def test_per_query_head_selection(heads):
+    """One selection per query head (variant): bounds, Hamming top-k and attention of every
+    head on its own, each against the oracle."""
+    hq, g = heads
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], n_q_heads=hq, n_kv_heads=g, seq_lens=(3000, 1234),
+                  batch=2, top_k=300, select_per_head=True)
+    inp, inp_np = _inputs(wl)
+    out = run_gpu(wl, inp, summary_fp16=1)
+    assert out["idx"].shape[1] == hq
+    _check_all_groups(wl, inp_np, out)
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
