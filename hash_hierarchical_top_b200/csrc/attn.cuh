@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   const int gq = lane >> 2, tq = lane & 3;   // fragment coordinates
   const int gs = a.Hq / a.Gs;
   const int row = b * a.Gs + g;
+  const uint32_t gkv = (uint32_t)(a.kv_div == 1 ? g : g / a.kv_div);  // KV head of the row
   const int cnt = min(a.count[row], a.top_k);
   const int base = split * a.split_rows;
   // A split past the selection does no work (in a cluster it still joins the merge).
@@ -150,8 +151,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
       if (t >= 0 && t < n && lp < a.maxp) {
         const int phys = a.page_table[(size_t)b * a.maxp + lp];
         if (phys >= 0 && phys < a.n_phys)
-          o = ((uint32_t)phys * (uint32_t)a.G + (uint32_t)(g / a.kv_div)) * (uint32_t)a.P +
-              (uint32_t)(t % a.P);
+          o = ((uint32_t)phys * (uint32_t)a.G + gkv) * (uint32_t)a.P + (uint32_t)(t % a.P);
         else
           flag_status(kStatusBadPage);
       } else {

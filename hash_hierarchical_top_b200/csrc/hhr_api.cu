@@ -121,7 +121,7 @@ SelectLayout select_layout(const hhr_dims* d, int mode, int m_max) {
   const size_t B = d->batch, Gs = sel_rows(d), Hq = d->n_q_heads, maxp = d->max_pages_per_seq;
   size_t off = 0;
   if (mode == HHR_MODE_HASH) {
-    L.qpn = off;    off += align256(B * Gs * 2 * kD * 4);
+    L.qpn = off;    off += align256(B * (size_t)d->n_kv_heads * 2 * kD * 4);
     L.q_rot = off;  off += align256(B * Hq * kD * 4);
     L.q_code = off; off += align256(B * Hq * code_words(d) * 4);
     L.bounds = off; off += align256(B * Gs * maxp * 4);
@@ -374,21 +374,24 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
       return HHR_ERR_CUDA;
     prof_begin(HHR_KERNEL_QPREP, s);
     qp<<<dim3(G, B), kMvThreads, qprep_smem(), s>>>(
-        QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G, d->select_per_head});
+        QPrepArgs{q, R, W, q_rot, q_code, qpn, Hq, G});
     prof_end(HHR_KERNEL_QPREP, s);
     if ((st = launch_status()) != HHR_OK) return st;
     // Every page kept (flat hash top-k): the bounds are computed only for a trace.
     const bool flat = m_max >= maxp;
     if (!flat || (trace != nullptr && trace->bounds != nullptr)) {
-      const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
+      const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                          d->n_phys_pages, 0, Gs, kv_div(d)};
       const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
       const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
       prof_begin(HHR_KERNEL_BOUND, s);
+      const dim3 blk(kBoundWarps * 32);
       if (d->summary_fp16)
-        page_bound_kernel<true><<<grid, kBoundWarps * 32, 0, s>>>(ba);
+        (kv_div(d) > 1 ? page_bound_kernel<true, true> : page_bound_kernel<true, false>)
+            <<<grid, blk, 0, s>>>(ba);
       else
-        page_bound_kernel<false><<<grid, kBoundWarps * 32, 0, s>>>(ba);
+        (kv_div(d) > 1 ? page_bound_kernel<false, true> : page_bound_kernel<false, false>)
+            <<<grid, blk, 0, s>>>(ba);
       prof_end(HHR_KERNEL_BOUND, s);
       if ((st = launch_status()) != HHR_OK) return st;
     }
@@ -584,7 +587,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   step_prologue_for(gs, cw)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
-                   d->summary_fp16, d->select_per_head});
+                   d->summary_fp16});
   prof_end(HHR_KERNEL_ENCODE, s);
   if ((st = launch_status()) != HHR_OK) return st;
   // a2: page bounds (none when every page is kept: a flat hash top-k).
@@ -593,13 +596,15 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     // Launched behind the prologue: its first CTAs warm L2 while the prologue runs, unless
     // an event is recorded between the two (profiling), which leaves no overlap to use.
     const int early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
-    const BoundArgs ba{qpn, page_minmax, page_table, seq_len, bounds, G, P, maxp,
+    const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
                        d->n_phys_pages, early, Gs, kv_div(d)};
     const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
     const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
     prof_begin(HHR_KERNEL_BOUND, s);
-    e = d->summary_fp16 ? launch_pdl(page_bound_kernel<true>, grid, dim3(kBoundWarps * 32), 0, s, ba)
-                        : launch_pdl(page_bound_kernel<false>, grid, dim3(kBoundWarps * 32), 0, s, ba);
+    void (*bk)(BoundArgs) =
+        d->summary_fp16 ? (kv_div(d) > 1 ? page_bound_kernel<true, true> : page_bound_kernel<true, false>)
+                        : (kv_div(d) > 1 ? page_bound_kernel<false, true> : page_bound_kernel<false, false>);
+    e = launch_pdl(bk, grid, dim3(kBoundWarps * 32), 0, s, ba);
     prof_end(HHR_KERNEL_BOUND, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   }

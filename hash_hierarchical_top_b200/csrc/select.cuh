@@ -23,9 +23,8 @@ struct QPrepArgs {
   const float* W;
   float* q_rot;      // [B][Hq][d]
   uint32_t* q_code;  // [B][Hq][CW]
-  float* qpn;        // [B][G][2][d] ([B][Hq][2][d] per head): [0] = qneg, [1] = qpos
+  float* qpn;        // [B][G][2][d]: [0] = qneg, [1] = qpos
   int Hq, G;
-  int per_head;      // one folded query per query head instead of per KV group
 };
 
 template <int CW>
@@ -78,22 +77,12 @@ __global__ void __launch_bounds__(kMvThreads) qprep_kernel(QPrepArgs a) {
     const int h = tid / CW, w = tid % CW;
     a.q_code[((size_t)b * a.Hq + g * gs + h) * CW + w] = cword[h][w];
   }
-  if (row_lead && !a.per_head) {
+  if (row_lead) {
     float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
 #pragma unroll
     for (int rb = 0; rb < kRowBlocks; ++rb) {
       o[rb * 32 + lrow] = qneg[rb];
       o[kD + rb * 32 + lrow] = qpos[rb];
-    }
-  } else if (row_lead) {  // each head's own folding of its rotated query
-    for (int h = 0; h < gs; ++h) {
-      float* o = a.qpn + ((size_t)b * a.Hq + g * gs + h) * 2 * kD;
-#pragma unroll
-      for (int rb = 0; rb < kRowBlocks; ++rb) {
-        const float y = qr[h][rb * 32 + lrow];
-        o[rb * 32 + lrow] = fminf(y, 0.f);
-        o[kD + rb * 32 + lrow] = fmaxf(y, 0.f);
-      }
     }
   }
 }
@@ -148,7 +137,8 @@ __device__ __forceinline__ int bound_chunk() { return bound_chunk_of(blockIdx.x,
 #endif
 
 struct BoundArgs {
-  const float* qpn;         // [B][Gs][2][d]
+  const float* qpn;         // [B][G][2][d] folded group queries (rows are KV groups)
+  const float* q_rot;       // [B][Hq][d] rotated queries (rows are query heads: folded here)
   const void* page_minmax;  // f32 or f16 [n_phys][G][2][d]
   const int32_t* page_table;
   const int32_t* seq_len;
@@ -216,7 +206,8 @@ __device__ __forceinline__ uint4 load_summary16(const uint4* p) {
 #endif
 }
 
-template <bool F16>
+// PH: one query head per selection row (per-head selection), folded here from q_rot.
+template <bool F16, bool PH = false>
 __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
   // kSets groups of 8 pages per warp are loaded together (all page ids first, then all
   // summary pieces), so that each warp keeps kSets * 8 page summaries in flight.
@@ -244,7 +235,7 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
             const int phys = a.page_table[(size_t)tb * a.maxp + p];
             if (phys >= 0 && phys < a.n_phys)
               prefetch_l2(reinterpret_cast<const uint4*>(a.page_minmax) +
-                              ((size_t)phys * a.G + tg / a.kv_div) * kPieces,
+                              ((size_t)phys * a.G + (PH ? tg / a.kv_div : tg)) * kPieces,
                           kPieces * 16);
           }
         }
@@ -254,19 +245,34 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
   pdl_wait();
   pdl_trigger();
   const int r = bound_group(), b = blockIdx.z;  // selection row r reads KV head r / kv_div
-  const int g = r / a.kv_div;
+  const int g = PH ? r / a.kv_div : r;
   const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
   const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
   if (p0 >= npg) return;
-  const float* qb = a.qpn + ((size_t)b * a.Gs + r) * 2 * kD;
   float4 q0, q1;
-  if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
-    const float4* qv = reinterpret_cast<const float4*>(qb + (lane >> 4) * kD + 8 * (lane & 15));
-    q0 = qv[0];
-    q1 = qv[1];
-  } else {              // channels 4l..4l+3 of qneg and of qpos
-    q0 = reinterpret_cast<const float4*>(qb)[lane];
-    q1 = reinterpret_cast<const float4*>(qb + kD)[lane];
+  if constexpr (!PH) {
+    const float* qb = a.qpn + ((size_t)b * a.Gs + r) * 2 * kD;
+    if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
+      const float4* qv = reinterpret_cast<const float4*>(qb + (lane >> 4) * kD + 8 * (lane & 15));
+      q0 = qv[0];
+      q1 = qv[1];
+    } else {              // channels 4l..4l+3 of qneg and of qpos
+      q0 = reinterpret_cast<const float4*>(qb)[lane];
+      q1 = reinterpret_cast<const float4*>(qb + kD)[lane];
+    }
+  } else {  // one query head per row: fold its rotated query, qneg = min(q', 0), qpos = max
+    const float* qh = a.q_rot + ((size_t)b * a.Gs + r) * kD;
+    auto lo = [](float4 v) { return make_float4(fminf(v.x, 0.f), fminf(v.y, 0.f), fminf(v.z, 0.f), fminf(v.w, 0.f)); };
+    auto hi = [](float4 v) { return make_float4(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f), fmaxf(v.z, 0.f), fmaxf(v.w, 0.f)); };
+    if constexpr (F16) {
+      const float4* qv = reinterpret_cast<const float4*>(qh + 8 * (lane & 15));
+      q0 = lane < 16 ? lo(qv[0]) : hi(qv[0]);
+      q1 = lane < 16 ? lo(qv[1]) : hi(qv[1]);
+    } else {
+      const float4 v = reinterpret_cast<const float4*>(qh)[lane];
+      q0 = lo(v);
+      q1 = hi(v);
+    }
   }
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
   int my_phys = -1;  // lane i < kPagesPerWarp resolves page p0 + i
@@ -737,7 +743,8 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   constexpr int kBins = (kMaxGroup * 32 * CW + 2 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
-  const int b = row / a.Gs, g = (row % a.Gs) / a.kv_div;
+  const int b = row / a.Gs, r = row % a.Gs;
+  const int g = a.kv_div == 1 ? r : r / a.kv_div;  // no division on the grouped path
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.Gs;  // query heads of the row
   const int nbins = gs * 32 * CW + 2;
@@ -956,7 +963,8 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
   extern __shared__ uint32_t fsm[];
   const HammingArgs& h = a.h;
   const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
-  const int b = row / h.Gs, r = row % h.Gs, g = r / h.kv_div;
+  const int b = row / h.Gs, r = row % h.Gs;
+  const int g = h.kv_div == 1 ? r : r / h.kv_div;  // no division on the grouped path
   const int gs = h.Hq / h.Gs;  // query heads of the row
   if (threadIdx.x < gs * CW)  // visible after the selection's first barrier
     qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + r * gs) * CW + threadIdx.x];

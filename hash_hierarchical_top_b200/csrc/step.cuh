@@ -30,9 +30,8 @@ struct PrologueArgs {
   uint32_t* codes;
   float* q_rot;            // [B][Hq][d]
   uint32_t* q_code;        // [B][Hq][CW]
-  float* qpn;              // [B][G][2][d], or [B][Hq][2][d] per head
+  float* qpn;              // [B][G][2][d]
   int Hq, G, P, maxp, n_phys, summary_fp16;
-  int per_head;            // one folded query per query head instead of per KV group
 };
 
 
@@ -234,18 +233,9 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   }
   if (row_lead) {
     if (has_key) store_summary_row(a.page_minmax, a.summary_fp16, s.sbase, row, mn, mx);
-    if (!a.per_head) {
-      float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
-      o[row] = qneg;
-      o[kD + row] = qpos;
-    } else {  // each head's own folding of its rotated query
-#pragma unroll
-      for (int h = 0; h < GS; ++h) {
-        float* o = a.qpn + ((size_t)b * a.Hq + g * GS + h) * 2 * kD;
-        o[row] = fminf(y[1 + h], 0.f);
-        o[kD + row] = fmaxf(y[1 + h], 0.f);
-      }
-    }
+    float* o = a.qpn + ((size_t)b * a.G + g) * 2 * kD;
+    o[row] = qneg;
+    o[kD + row] = qpos;
   }
 }
 
