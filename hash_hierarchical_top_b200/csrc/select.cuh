@@ -727,7 +727,7 @@ __device__ __forceinline__ int hamming_delta(const QueryPlanes<NB, CW>& p, const
 struct HamShared {
   int scratch[66];
   int T, need_eq;
-  int tot[2];  // this CTA's (#below threshold, #equal) for the other ranks
+  int tot[2];  // lower-ranked CTAs' (#below threshold, #at threshold): this rank's output offsets
 };
 
 // Steps a3-a4 for one (sequence, group) row on the cluster's CTA `rank`, given the row's
@@ -758,7 +758,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   const int lo = min(C, rank * half), hi = min(C, lo + half);
   const int Cr = hi - lo;
   for (int i = tid; i < nbins; i += NT) hist[i] = 0;
-  if (tid == 0) { hs.T = -1; hs.need_eq = 0; }
+  if (tid == 0) { hs.T = -1; hs.need_eq = 0; hs.tot[0] = 0; hs.tot[1] = 0; }
   if (tid < 2 * CW) {
     const int kind = tid / CW, w = tid % CW;
     build_plane_word<NB>(qcs + w, CW, gs, kind, &planes[kind][w][0]);
@@ -810,33 +810,45 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   }
   cluster_sync_all();  // every rank's histogram is complete
   // Threshold bucket: smallest T with #(delta <= T) >= k_eff over the summed histograms.
-  // Thread t holds bins [kBins t, kBins (t + 1)) (fewer past nbins).
+  // Thread t holds bins [kBins t, kBins (t + 1)) (fewer past nbins). The same scan over the
+  // histograms of the lower-ranked CTAs gives this rank's output offsets: how many of their
+  // candidates lie below T (tot[0]) and at T (tot[1]).
   {
-    int hv[kBins], sum = 0;
+    int hv[kBins], lv[kBins], sum = 0, lsum = 0;
 #pragma unroll
     for (int q = 0; q < kBins; ++q) {
       const int i = kBins * tid + q;
       hv[q] = 0;
+      lv[q] = 0;
       if (i < nbins) {
 #pragma unroll
-        for (int r = 0; r < kHamRanks; ++r) hv[q] += cl.map_shared_rank(hist, r)[i];
+        for (int r = 0; r < kHamRanks; ++r) {
+          const int c = cl.map_shared_rank(hist, r)[i];
+          hv[q] += c;
+          if (r < rank) lv[q] += c;
+        }
       }
       sum += hv[q];
+      lsum += lv[q];
     }
-    int nvalid;
-    const int excl = block_excl_scan<false>(sum, hs.scratch, &nvalid);  // next use: after the barrier below
-    const int keff = min(a.top_k, nvalid);
-    if (keff > 0 && excl < keff && keff <= excl + sum) {
-      int run = excl;
+    cluster_arrive();  // no remote shared-memory access after this point
+    int2 nvalid;
+    const int2 excl = block_excl_scan2<false>(make_int2(sum, lsum), hs.scratch, &nvalid);
+    const int keff = min(a.top_k, nvalid.x);  // scratch's next use: after the barrier below
+    if (keff > 0 && excl.x < keff && keff <= excl.x + sum) {
+      int run = excl.x, lrun = excl.y;
       bool found = false;
 #pragma unroll
       for (int q = 0; q < kBins; ++q) {
         if (!found && keff <= run + hv[q]) {
           hs.T = kBins * tid + q;
           hs.need_eq = keff - run;
+          hs.tot[0] = lrun;   // lower ranks' candidates below T
+          hs.tot[1] = lv[q];  // and at T
           found = true;
         }
         run += hv[q];
+        lrun += lv[q];
       }
     }
     if (tid == 0) a.out_count[row] = keff;  // every rank writes the same value
@@ -844,7 +856,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
     for (int i = keff + rank * NT + tid; i < a.top_k; i += kHamRanks * NT)
       a.out_idx[(size_t)row * a.top_k + i] = -1;
   }
-  const int T = hs.T, need_eq = hs.need_eq;
+  const int T = hs.T, need_eq = hs.need_eq, lt_off = hs.tot[0], eq_off = hs.tot[1];
   // Ordered compaction of this rank's candidates: thread t owns [t*cpt, (t+1)*cpt), cpt a
   // multiple of 8, read as 16-byte groups of 8 distances.
   const int cpt = ((ceil_div(Cr, NT) + 7) / 8) * 8;
@@ -871,15 +883,6 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   }
   int2 tot;
   const int2 before = block_excl_scan2<false>(make_int2(lt, eq), hs.scratch, &tot);  // last use
-  if (tid == 0) { hs.tot[0] = tot.x; hs.tot[1] = tot.y; }
-  cluster_sync_all();  // every rank's totals are published
-  int lt_off = 0, eq_off = 0;
-  for (int r = 0; r < rank; ++r) {
-    const int* rt = cl.map_shared_rank(&hs.tot[0], r);
-    lt_off += rt[0];
-    eq_off += rt[1];
-  }
-  cluster_arrive();  // no remote shared-memory access after this point
   int32_t* out = a.out_idx + (size_t)row * a.top_k;
   {
     int e = eq_off + before.y;
