@@ -328,10 +328,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();  // every split's state is in its shared memory
-    if (cl.block_rank() == 0) {
-      const int ns = (int)cl.num_blocks();
+    {
+      // Rank r merges outputs [r n/ns, (r + 1) n/ns) of the group's n = gs * d (the same
+      // arithmetic per output as the combine kernel, split over the cluster's CTAs).
+      const int ns = (int)cl.num_blocks(), rk = (int)cl.block_rank();
+      const int per = (gs * kD + ns - 1) / ns;
+      const int lo = rk * per, hi = min(gs * kD, lo + per);
       float* res_local = reinterpret_cast<float*>(offs);
-      for (int i = tid; i < gs * kD; i += kAttnThreads) {
+      for (int i = lo + tid; i < hi; i += kAttnThreads) {
         const int h = i / kD, c = i % kD;
         float M = -INFINITY;
         for (int r = 0; r < ns; ++r)
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
         a.out[((size_t)b * a.Hq + g * gs + h) * kD + c] = (L > 0.f) ? O / L : 0.f;
       }
     }
-    cl.sync();  // keep every CTA's shared memory alive until rank 0 has read it
+    cl.sync();  // keep every CTA's shared memory alive until every rank has read it
   }
 }
 
