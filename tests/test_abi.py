@@ -120,6 +120,24 @@ def test_select_opts_validated(L):
     assert (o.sink_pages, o.local_pages) == (1, 2)
 
 
+def test_per_head_selection_sizes_and_validation(L):
+    """select_per_head: rows per sequence become the query heads (workspaces grow with them);
+    values other than 0/1, and the indexer mode, are rejected."""
+    d0, d1 = _d(), _d(select_per_head=1)
+    g = hhr.hhr_select_workspace_bytes(d0, hhr.HHR_MODE_HASH, 0, 16, 2048)
+    h = hhr.hhr_select_workspace_bytes(d1, hhr.HHR_MODE_HASH, 0, 16, 2048)
+    assert h > g > 0
+    # bounds [B][rows][max_pages], kept [B][rows][m_max]: 4x the rows at 32 heads / 8 groups
+    assert h - g >= (32 - 8) * (4096 + 256) * 4
+    assert hhr.hhr_attn_workspace_bytes(d1, 2048) > 0  # 4x the rows, fewer splits per row
+    assert hhr.hhr_decode_step_workspace_bytes(d1, 0, 16, 2048) > 0
+    assert hhr.sel_rows(d0) == 8 and hhr.sel_rows(d1) == 32
+    assert hhr.hhr_select_workspace_bytes(_d(select_per_head=2), hhr.HHR_MODE_HASH, 0, 16,
+                                          2048) == 0
+    di = _d(n_q_heads=64, n_kv_heads=1, page_size=128, max_pages_per_seq=1024, select_per_head=1)
+    assert hhr.hhr_select_workspace_bytes(di, hhr.HHR_MODE_INDEXER, 64, 0, 2048) == 0
+
+
 def test_select_validation_order(L):
     d = _d()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
