@@ -632,13 +632,14 @@ def run_oracle_timed(wl, inp, seconds=None, steps=None, warmup=0):
 
 def timing_events(n, stream):
     """n pairs of timing events, each recorded once so that the CUDA event exists
-    (torch creates it lazily) before its handle is given to the library's hook."""
+    (torch creates it lazily) before its handle is given to the library's hook. The stop
+    event is recorded first: a pair that no launch records again keeps a negative span."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n)]
     for a, b in evs:
-        a.record(stream)
         b.record(stream)
+        a.record(stream)
     stream.synchronize()
     return evs
 
@@ -851,10 +852,10 @@ def main():
         for name in names:
             a_, b_ = ev_k[name][r % L]
             kern[name].append(a_.elapsed_time(b_) * 1e3)
-    kern = {k: statistics.mean(v) for k, v in kern.items()}
     # Launches per step: every kernel of the breakdown that ran (an unlaunched kernel's
-    # events are the two pre-recorded ones, 0 us apart).
-    kernels_per_step = sum(1 for v in kern.values() if v > 0.5)
+    # events are the two pre-recorded ones, stop before start: a negative span).
+    kern = {k: statistics.mean(v) for k, v in kern.items() if min(v) > 0}
+    kernels_per_step = len(kern)
 
     # End to end through the public API with host buffers: every step copies its query and
     # newest K/V rows from pinned host memory and reads its output back to pinned host memory.
