@@ -604,16 +604,17 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
 // HHR page, Abstract (LHP: Hamming distance between binary codes ranks the keys of
 // the pages that survive pruning). Candidates are the valid keys of the kept pages, in
 // ascending token order.
-//   delta_t = sum over the group's heads of popcount(qcode_h ^ code_t)  (0..gs*128)
-// Selection of the k smallest (delta, t): a histogram of delta gives the threshold
-// bucket; an ordered compaction keeps every key below it and the first ones inside it
-// in token order. Output ascending; -1 past k_eff.
+//   delta_t = sum over the row's query heads of popcount(qcode_h ^ code_t)  (0..gs*32*CW)
+// Selection of the k smallest (delta, t): a histogram of the ranked distance (0 for a key of
+// a forced page, else 1 + delta) gives the threshold bucket; an ordered compaction keeps
+// every key below it and the first ones inside it in token order. Output ascending; -1 past
+// k_eff.
 //
 // Distance by bit planes: channel j of a candidate contributes z_j = #heads with query
 // bit 0 when the key bit is 1, else n_j = #heads with query bit 1. n and z are kept per
 // code word as NB bit planes (NB = bit width of gs), so one select per plane and word
-// gives the contributions' bits, and a carry-save step over the 4 words leaves 3
-// popcounts per plane: 3*NB popcounts per candidate instead of 4*gs.
+// gives the contributions' bits, and a carry-save step over each 4 words leaves 3
+// popcounts per plane: 3*NB popcounts per 4 words instead of 4*gs.
 constexpr int kHamRanks = 2;   // CTAs (a cluster) per (sequence, group)
 constexpr int kMaxCand = 131072;  // a flat top-k over 4096 pages of 32 keys
 constexpr int kMaxCodeWords = 8;  // 256-bit codes
@@ -927,7 +928,8 @@ inline size_t hamming_smem(int gs, int cw, int m_max, int P) {
 }
 
 // Top-m pages and the Hamming top-k fused in one cluster of kHamRanks CTAs per (sequence,
-// group): every rank selects the same kept pages (deterministic), resolving their physical
+// selection row: a KV group, or a query head): every rank selects the same kept pages
+// (deterministic), resolving their physical
 // pages during the compaction, so the kept list never leaves shared memory (rank 0 copies
 // it to `kept`/`kept_count` for inspection). Shared memory: [kept list: m_max words][their
 // physical pages: m_max words][union of: top-m keys (maxp words) | Hamming scratch].
