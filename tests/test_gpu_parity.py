@@ -198,6 +198,19 @@ def test_per_query_head_selection(heads):
     _check_all_groups(wl, inp_np, out)
 
 
+@pytest.mark.parametrize("case", [
+    dict(select_per_head=True, sink_pages=1, local_pages=2, code_bits=64),
+    dict(select_per_head=True, m_pages=4096, keep_div=0, code_bits=256),
+    dict(m_pages=4096, keep_div=0, sink_pages=2, local_pages=1, code_bits=256),
+], ids=["per_head+forced+64", "per_head+flat+256", "flat+forced+256"])
+def test_variant_combinations(case):
+    """Variants together: per-head rows with forced pages or a flat top-k, across code
+    lengths; every row against the oracle."""
+    wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(3000, 700), batch=2, top_k=300, **case)
+    inp, inp_np = _inputs(wl)
+    _check_all_groups(wl, inp_np, run_gpu(wl, inp, summary_fp16=1))
+
+
 def test_bulk_encoder_partial_start():
     """Tensor-core bulk append starting mid-page (merge with stored summaries)."""
     wl = S.scaled(S.WORKLOADS["llama8b_32k"], seq_lens=(20000, 13001), batch=2, top_k=500)
