@@ -61,8 +61,10 @@ inline int kv_div(const hhr_dims* d) { return sel_rows(d) / d->n_kv_heads; }
 inline int code_words(const hhr_dims* d) { return d->code_bits / 32; }
 inline int cw_index(int cw) { return cw == 2 ? 0 : cw == 4 ? 1 : 2; }
 
+// Group size, and selection rows per sequence (a grid dimension: at most 65535).
 int check_group(const hhr_dims* d) {
-  return (d->n_q_heads / d->n_kv_heads > kMaxGroup) ? HHR_ERR_UNSUPPORTED : HHR_OK;
+  if (d->n_q_heads / d->n_kv_heads > kMaxGroup) return HHR_ERR_UNSUPPORTED;
+  return sel_rows(d) > 65535 ? HHR_ERR_UNSUPPORTED : HHR_OK;
 }
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
@@ -145,6 +147,8 @@ int check_select_params(const hhr_dims* d, int mode, int m_pages, int keep_div, 
   if (mode == HHR_MODE_HASH) {
     if ((m_pages > 0) == (keep_div > 0)) return HHR_ERR_INVALID_ARG;
     if (check_group(d) != HHR_OK) return HHR_ERR_UNSUPPORTED;
+    // B x rows x ranks CTAs of the top-m + Hamming kernel form one grid dimension.
+    if ((long long)d->batch * sel_rows(d) * kHamRanks > 0x7fffffffLL) return HHR_ERR_UNSUPPORTED;
     if ((long long)kept_max(d, m_pages, keep_div) * d->page_size > kMaxCand)
       return HHR_ERR_UNSUPPORTED;
     if (topm_hamming_smem(d->n_q_heads / sel_rows(d), code_words(d),

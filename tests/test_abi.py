@@ -136,6 +136,12 @@ def test_per_head_selection_sizes_and_validation(L):
                                           2048) == 0
     di = _d(n_q_heads=64, n_kv_heads=1, page_size=128, max_pages_per_seq=1024, select_per_head=1)
     assert hhr.hhr_select_workspace_bytes(di, hhr.HHR_MODE_INDEXER, 64, 0, 2048) == 0
+    # Selection rows are a grid dimension: at most 65535 query heads with per-head rows.
+    big = _d(n_q_heads=8 * 10000, n_kv_heads=10000, select_per_head=1)
+    assert hhr.hhr_select_workspace_bytes(big, hhr.HHR_MODE_HASH, 0, 16, 2048) == 0
+    assert hhr.hhr_attn_workspace_bytes(big, 2048) == 0
+    ok = _d(n_q_heads=8 * 8000, n_kv_heads=8000, select_per_head=1)
+    assert hhr.hhr_attn_workspace_bytes(ok, 2048) > 0
 
 
 def test_select_validation_order(L):
