@@ -194,6 +194,15 @@ def check_codes_bruteforce(O, seed=4):
     for t in range(n):
         mism = sum(1 for h in range(gs) for j in range(bits) if qbits[h][j] != kbits[t][j])
         assert dist[t] == mism, t
+    # A square, non-symmetric projection (bits = d = 32): row j of W makes bit j.
+    d2 = 32
+    k2, _, pt2 = tiny_cache(rng, n, P, 1, d2)
+    R2 = orthogonal(rng, d2)
+    W2 = rng.standard_normal((d2, d2)).astype(np.float32)
+    enc2 = O.encode_group(k2, pt2, 0, n, P, R2, W2)
+    Kb2 = brute_logical(k2, pt2, 0, n, P)
+    for t in range(n):
+        assert words_to_bits(enc2["codes"][t], d2) == brute_code_bits(R2, W2, list(Kb2[t])), t
 
 
 def check_codes_identity_projection(O, seed=5):

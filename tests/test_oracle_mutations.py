@@ -111,6 +111,37 @@ def _per_head_uses_group(inp, *, P, m_pages, keep_div, top_k, scale=None, groups
     return {key: [r] * gs for key, r in res.items()}
 
 
+def _query_prep_unrotated_codes(R_g, W_g, Qg):
+    Qrot = _orig["rotate"](R_g, Qg)
+    proj = _orig["projections"](W_g, np.asarray(Qg, dtype=np.float64))  # hashes q, not q'
+    nrm = np.linalg.norm(Qg, axis=1, keepdims=True)
+    return Qrot, _orig["pack_sign_bits"](proj), np.abs(proj) < 1e-4 * nrm
+
+
+def _projections_transposed(W_g, Xrot):
+    # W applied transposed (possible only where W is square; elsewhere the shapes refuse).
+    W = np.asarray(W_g, dtype=np.float64)
+    return Xrot @ W if W.shape[0] == W.shape[1] else Xrot @ W.T
+
+
+def _logical_rows_ignore_table(cache_bits, page_table_row, g, n, P):
+    return _orig["logical_rows"](cache_bits, np.arange(len(page_table_row)), g, n, P)
+
+
+def _summaries_swapped(Krot, P):
+    kmin, kmax = _orig["page_summaries"](Krot, P)
+    return kmax, kmin
+
+
+def _indexer_pos_early(q, pos, K, mu, n, P, m_blocks, k):
+    return _orig["indexer_select_one"](q, max(pos - 1, 0), K, mu, n, P, m_blocks, k)
+
+
+def _bf16_wrong_shift(bits):
+    u32 = bits.astype(np.uint32) << np.uint32(15)
+    return u32.view(np.float32).astype(np.float64)
+
+
 MUTATIONS = {
     "rotate_transposed": ("rotate", _rotate_transposed),
     "bound_min_not_max": ("page_bounds", _bounds_min),
@@ -131,6 +162,12 @@ MUTATIONS = {
     "forced_budget_not_grown": ("top_m_forced", _forced_budget_fixed),
     "forced_keys_not_first": ("top_k_forced", _forced_keys_not_first),
     "per_head_uses_group": ("decode_step_hash", _per_head_uses_group),
+    "query_codes_unrotated": ("query_prep", _query_prep_unrotated_codes),
+    "projections_transposed": ("projections", _projections_transposed),
+    "page_table_ignored": ("logical_rows", _logical_rows_ignore_table),
+    "summaries_min_max_swapped": ("page_summaries", _summaries_swapped),
+    "indexer_causal_one_early": ("indexer_select_one", _indexer_pos_early),
+    "bf16_wrong_shift": ("bf16_to_f64", _bf16_wrong_shift),
 }
 
 
