@@ -89,12 +89,16 @@ def sign_codes(R_g, W_g, X):
     return pack_sign_bits(projections(W_g, rotate(R_g, X)))
 
 
-def fragile_bits(R_g, W_g, X, rel=1e-4):
+def fragile_mask(proj, X, rel=1e-4):
     """Bits whose projection is too close to zero to be fixed by the code tolerance:
-    |(W_g R_g x)_j| < rel * ||x||. Boolean [n][bits]."""
-    p = projections(W_g, rotate(R_g, X))
-    nrm = np.linalg.norm(X, axis=1, keepdims=True)
-    return np.abs(p) < rel * nrm
+    |proj_j| < rel * ||x|| for each row x of X. Boolean [n][bits]."""
+    nrm = np.linalg.norm(np.asarray(X, dtype=np.float64), axis=1, keepdims=True)
+    return np.abs(proj) < rel * nrm
+
+
+def fragile_bits(R_g, W_g, X, rel=1e-4):
+    """fragile_mask of the projections W_g R_g x of the rows of X."""
+    return fragile_mask(projections(W_g, rotate(R_g, X)), X, rel)
 
 
 def page_summaries(Krot, P):
@@ -132,17 +136,14 @@ def encode_group(k_bits, page_table_row, g, n, P, R_g, W_g):
     Krot = rotate(R_g, K)
     kmin, kmax = page_summaries(Krot, P)
     proj = projections(W_g, Krot)
-    nrm = np.linalg.norm(K, axis=1, keepdims=True)
-    return dict(kmin=kmin, kmax=kmax, codes=pack_sign_bits(proj),
-                fragile=np.abs(proj) < 1e-4 * nrm)
+    return dict(kmin=kmin, kmax=kmax, codes=pack_sign_bits(proj), fragile=fragile_mask(proj, K))
 
 
 def query_prep(R_g, W_g, Qg):
     """Step a1: rotated queries q'_h = R_g q_h and their codes, for the heads of one group."""
     Qrot = rotate(R_g, Qg)
     proj = projections(W_g, Qrot)
-    nrm = np.linalg.norm(Qg, axis=1, keepdims=True)
-    return Qrot, pack_sign_bits(proj), np.abs(proj) < 1e-4 * nrm
+    return Qrot, pack_sign_bits(proj), fragile_mask(proj, Qg)
 
 
 # --------------------------------------------------------------------------- step a2

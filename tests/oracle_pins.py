@@ -205,6 +205,46 @@ def check_codes_bruteforce(O, seed=4):
         assert words_to_bits(enc2["codes"][t], d2) == brute_code_bits(R2, W2, list(Kb2[t])), t
 
 
+def check_fragile_bits(O, seed=14):
+    """Fragile code bits (the only ones a GPU code may flip) are exactly those whose
+    projection lies within 1e-4 ||x|| of zero, by explicit sums; on Gaussian data they are
+    rare, and a bit placed on a zero projection is always fragile."""
+    rng = np.random.default_rng(seed)
+    d, bits, n = 16, 64, 40
+    R = orthogonal(rng, d)
+    W = rng.standard_normal((bits, d)).astype(np.float32)
+    X = bf(rand_bf16_bits(rng, (n, d)))
+    # Plant exact zeros: x orthogonal to the rotated row j of W (x = R^T v, v ⟂ W_j).
+    Wj = W[3].astype(np.float64)
+    v = rng.standard_normal(d)
+    v -= (v @ Wj) / (Wj @ Wj) * Wj
+    X[0] = R.astype(np.float64).T @ v
+    fr = O.fragile_bits(R, W, X)
+    for t in range(n):
+        xr = brute_rotate(R, list(X[t]))
+        nrm = math.sqrt(math.fsum(c * c for c in X[t]))
+        for j in range(bits):
+            p = math.fsum(float(W[j][i]) * xr[i] for i in range(d))
+            if abs(abs(p) - 1e-4 * nrm) > 1e-12 * nrm:  # away from the cut itself
+                assert bool(fr[t, j]) == (abs(p) < 1e-4 * nrm), (t, j)
+    assert fr[0, 3]
+    assert fr.mean() < 0.01
+    # The masks the encoder and the query preparation return are the same rule.
+    _, qmask = O.query_prep(R, W, X)[1:]
+    assert np.array_equal(qmask, fr)
+    P = 8
+    kc, _, pt = tiny_cache(rng, n, P, 1, d)
+    enc = O.encode_group(kc, pt, 0, n, P, R, W)
+    Kb = brute_logical(kc, pt, 0, n, P)
+    for t in range(n):
+        xr = brute_rotate(R, list(Kb[t]))
+        nrm = math.sqrt(math.fsum(c * c for c in Kb[t]))
+        for j in range(bits):
+            p = math.fsum(float(W[j][i]) * xr[i] for i in range(d))
+            if abs(abs(p) - 1e-4 * nrm) > 1e-12 * nrm:
+                assert bool(enc["fragile"][t, j]) == (abs(p) < 1e-4 * nrm), (t, j)
+
+
 def check_codes_identity_projection(O, seed=5):
     """W = I: the code is the sign pattern of the rotated key itself."""
     rng = np.random.default_rng(seed)
@@ -479,5 +519,5 @@ ALL_CHECKS = [
     check_codes_identity_projection, check_topk_bruteforce, check_kept_count,
     check_flat_hash_topk, check_dense_attention, check_single_key_attention,
     check_hand_example, check_hisa_block_size_one, check_hisa_all_blocks_and_causal,
-    check_forced_pages, check_per_head_selection,
+    check_forced_pages, check_per_head_selection, check_fragile_bits,
 ]

@@ -142,6 +142,14 @@ def _bf16_wrong_shift(bits):
     return u32.view(np.float32).astype(np.float64)
 
 
+def _fragile_everything(proj, X, rel=1e-4):
+    return np.ones(np.shape(proj), dtype=bool)
+
+
+def _fragile_wrong_scale(proj, X, rel=1e-4):
+    return _orig["fragile_mask"](proj, X, rel * 100)
+
+
 MUTATIONS = {
     "rotate_transposed": ("rotate", _rotate_transposed),
     "bound_min_not_max": ("page_bounds", _bounds_min),
@@ -168,6 +176,8 @@ MUTATIONS = {
     "summaries_min_max_swapped": ("page_summaries", _summaries_swapped),
     "indexer_causal_one_early": ("indexer_select_one", _indexer_pos_early),
     "bf16_wrong_shift": ("bf16_to_f64", _bf16_wrong_shift),
+    "fragile_everything": ("fragile_mask", _fragile_everything),
+    "fragile_wrong_scale": ("fragile_mask", _fragile_wrong_scale),
 }
 
 
