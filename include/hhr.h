@@ -169,6 +169,11 @@ size_t hhr_select_workspace_bytes(const hhr_dims* dims, int mode, int m_pages, i
  *       past k_eff are set to -1.
  *   Uses q, seq_len, page_table, R, W, page_minmax, codes; block_mean, k_cache and
  *   q_pos may be NULL.
+ *   With dims.select_per_head the rows are the query heads: "h in g" above becomes the
+ *   row's single head h, scoring KV group h / (Hq/G)'s summaries and codes.
+ *   When m_b covers every page (m_pages >= max_pages_per_seq, or keep_div == 1) no page
+ *   bound is needed (a flat hash top-k over every key): the bounds are then computed only
+ *   if trace->bounds asks for them.
  * HHR_MODE_INDEXER (HISA page, Abstract; n_kv_heads == 1, n_q_heads = T):
  *   a1' score_blk = q_i . block_mean_blk for blocks with blk*P <= q_pos[b][i];
  *       keep the m_b = min(m_pages, #eligible) best, ties to the lower block.
