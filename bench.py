@@ -96,6 +96,45 @@ def bound_kernel_bytes(wl, lens, sbytes=4):
     return tot
 
 
+def step_kernel_bytes(wl, lens, m_of, sbytes=4):
+    """Algorithmic bytes of each kernel of one fused step (the names of kernels_us):
+    encode = the prologue (R_g and W_g once per group, the new K/V rows and the queries read;
+    rotated queries and folded queries written); bound = bound_kernel_bytes; hamming = the
+    bounds, the kept pages' page-table entries and codes read, the selected ids and cache
+    rows written; attn = the selected rows' offsets, K and V read, the queries read and the
+    outputs written."""
+    G, Hq, d, P = wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.page_size
+    rows = Hq if wl.select_per_head else G
+    B = len(lens)
+    enc = G * (d * d + wl.code_bits * d) * 4 + B * G * 2 * d * 2 + B * Hq * d * (2 + 4) \
+        + B * G * 2 * d * 4
+    ham = attn = 0
+    for n in lens:
+        npg = -(-n // P)
+        m = m_of(npg)
+        cand = min(n, m * P)
+        k = min(wl.top_k, cand)
+        ham += rows * (npg * 4 + m * 4 + cand * (wl.code_bits // 8) + k * 8)
+        attn += rows * k * (4 + 2 * d * 2)
+    attn += B * Hq * d * (2 + 4)
+    return {"encode": enc, "bound": bound_kernel_bytes(wl, lens, sbytes), "hamming": ham,
+            "attn": attn}
+
+
+def kernel_table(kern_us, kbytes, peak_gbs):
+    """Per kernel: bracketed time, algorithmic bytes, GB/s and its fraction of 8 TB/s and of
+    the measured copy bandwidth (kernels without a byte figure get the time only)."""
+    out = {}
+    for name, us in kern_us.items():
+        row = {"us": us}
+        if name in kbytes and us > 0:
+            gbs = kbytes[name] / (us * 1e-6) / 1e9
+            row.update(algorithmic_bytes=kbytes[name], gbs=gbs, frac_of_8tbs=gbs / 8000.0,
+                       frac_of_measured=gbs / peak_gbs)
+        out[name] = row
+    return out
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -1047,6 +1086,7 @@ def main():
                          "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
                          "frac_of_measured": step_gbs / peak},
             "kernels_us": kern,
+            "kernels": kernel_table(kern, step_kernel_bytes(wl, lens, m_of, sbytes), peak),
             "prefill_encode": prefill,
             "other_workloads": other,
             "selection_quality": quality,

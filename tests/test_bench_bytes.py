@@ -52,3 +52,20 @@ def test_indexer_bytes():
     for name, T in (("hisa_128k_t1", 1), ("hisa_128k_t64", 64)):
         wl = S.WORKLOADS[name]
         assert bench.indexer_required_bytes(wl, [131072]) == 1024 * 512 + T * 64 * 128 * 256
+
+
+def test_step_kernel_bytes_and_table():
+    wl = S.WORKLOADS["llama8b_128k_b8"]
+    kb = bench.step_kernel_bytes(wl, [131072] * 8, KEEP_16, 2)
+    assert kb["bound"] == 135462912
+    # Attention: 8 x 8 groups x 2048 rows x (4-byte offset + 256 B K + 256 B V), plus 8 x 32
+    # queries read (bf16) and written (f32).
+    assert kb["attn"] == 8 * 8 * 2048 * 516 + 8 * 32 * 128 * 6
+    # Hamming: 4096 bounds + 256 page-table entries + 8192 codes of 16 B + 2048 x 8 B out.
+    assert kb["hamming"] == 8 * 8 * (4096 * 4 + 256 * 4 + 8192 * 16 + 2048 * 8)
+    assert kb["encode"] == 8 * (128 * 128 * 2) * 4 + 8 * 8 * 512 + 8 * 32 * 128 * 6 + 8 * 8 * 1024
+    t = bench.kernel_table({"bound": 25.0, "attn": 20.0, "combine": 2.0}, kb, 6548.0)
+    assert t["combine"] == {"us": 2.0}
+    assert abs(t["bound"]["gbs"] - 135462912 / 25e-6 / 1e9) < 1e-9
+    assert abs(t["bound"]["frac_of_measured"] - t["bound"]["gbs"] / 6548.0) < 1e-12
+    assert abs(t["attn"]["frac_of_8tbs"] - t["attn"]["gbs"] / 8000.0) < 1e-12
