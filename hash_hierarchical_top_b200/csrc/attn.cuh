@@ -10,14 +10,17 @@
 //      with 16-byte cp.async; consecutive threads copy consecutive pieces of a row,
 //      so the random row gather stays coalesced; two tiles are in flight while one
 //      is computed;
-//   2. logits: warp w takes 8 rows of the tile, lane l channels 4l..4l+3; the
-//      8 rows x 4 heads partial dot products are folded by one transposed warp
-//      reduction, so each lane ends up with one (row, head) logit;
+//   2. logits: warp w takes 8 rows of the tile; S = Q K^T on bf16 mma.sync
+//      (m16n8k16, the group's heads on M, the warp's 8 keys on N), so the
+//      accumulator fragment holds one (head, key pair) per lane;
 //   3. every warp keeps its own online softmax (running max, sum and output per
-//      head) over its rows; P.V runs with lanes over channels;
+//      head) over its rows; O^T += V^T P^T on mma.sync m16n8k8, the logit
+//      accumulator being directly the B operand (P split into bf16 hi + lo);
 //   4. the 8 warps are merged in shared memory; a split writes its partial (max,
-//      sum, output) per head, or the final output when the group is not split; a
-//      combine kernel merges the splits (standard split softmax rescaling).
+//      sum, output) per head, or the final output when the group is not split.
+//      The splits are merged either by a combine kernel, or (cluster variant) by
+//      the cluster's CTAs through distributed shared memory, each CTA merging its
+//      share of the group's outputs (standard split softmax rescaling).
 #pragma once
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
@@ -116,8 +119,9 @@ __device__ __forceinline__ int swz(int r, int chunk) { return r * kD + ((chunk ^
 // fragment of O^T = V^T P^T on mma.m16n8k8 (channels on M, heads on N). P is split into
 // bf16 hi + lo parts (two MMAs) so its rounding stays near 2^-16 relative.
 // kCluster: the splits of a group form one thread-block cluster; after each CTA has
-// merged its warps, the cluster's rank 0 merges the splits through distributed shared
-// memory and writes the output (no partials in global memory, no combine kernel).
+// merged its warps, every CTA merges its share of the group's outputs from all the
+// splits' states through distributed shared memory and writes them (no partials in
+// global memory, no combine kernel).
 template <bool kCluster>
 __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a) {
   extern __shared__ float4 at_smem[];
@@ -134,9 +138,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   const uint32_t gkv = (uint32_t)(a.kv_div == 1 ? g : g / a.kv_div);  // KV head of the row
   const int cnt = min(a.count[row], a.top_k);
   const int base = split * a.split_rows;
-  // A split past the selection does no work (in a cluster it still joins the merge).
+  // A split past the selection does no work (in a cluster it still joins the merge). An
+  // unsplit group with an empty selection writes its zero output here, since no merge follows.
   const int nrows = max(0, min(a.split_rows, cnt - base));
-  if (!kCluster && nrows == 0) return;
+  if (!kCluster && nrows == 0) {
+    if (a.n_splits == 1)
+      for (int i = tid; i < gs * kD; i += kAttnThreads)
+        a.out[((size_t)b * a.Hq + g * gs) * kD + i] = 0.f;
+    return;
+  }
   const int ntiles = (nrows + kTile - 1) / kTile;
   const int n = a.seq_len[b];
 

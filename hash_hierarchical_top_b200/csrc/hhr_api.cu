@@ -5,7 +5,6 @@
 #include <math.h>
 #include <stdio.h>
 
-#include <atomic>
 #include <initializer_list>
 
 #include "../../include/hhr.h"
@@ -474,22 +473,41 @@ size_t hhr_attn_workspace_bytes(const hhr_dims* d, int top_k) {
   return align256(rows * ns * gs * kD * 4) + align256(rows * ns * gs * 2 * 4);
 }
 
-int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cache,
+}  // extern "C"
+
+namespace {
+
+// Host-side validation of the attention arguments (everything but the workspace).
+int check_attn_args(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cache,
                     const uint16_t* v_cache, const int32_t* page_table, const int32_t* seq_len,
-                    const int32_t* idx, const int32_t* count, int top_k, float scale, float* out,
-                    void* workspace, size_t ws_bytes, void* stream) {
+                    const int32_t* idx, const int32_t* count, int top_k, float scale,
+                    const float* out) {
   int st = check_dims(d);
   if (st != HHR_OK) return st;
   if ((st = check_group(d)) != HHR_OK) return st;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || page_table == nullptr ||
-      seq_len == nullptr || idx == nullptr || count == nullptr || out == nullptr ||
-      workspace == nullptr)
+      seq_len == nullptr || idx == nullptr || count == nullptr || out == nullptr)
     return HHR_ERR_INVALID_ARG;
   if (top_k < 1 || !(scale == scale) || isinf(scale)) return HHR_ERR_INVALID_ARG;
   if (misaligned16({q, k_cache, v_cache, out})) return HHR_ERR_INVALID_ARG;
   // Cache rows are addressed with 32-bit row indices.
   if ((unsigned long long)d->n_phys_pages * d->n_kv_heads * d->page_size >= 0xffffffffull)
     return HHR_ERR_UNSUPPORTED;
+  return HHR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hhr_sparse_attn(const hhr_dims* d, const uint16_t* q, const uint16_t* k_cache,
+                    const uint16_t* v_cache, const int32_t* page_table, const int32_t* seq_len,
+                    const int32_t* idx, const int32_t* count, int top_k, float scale, float* out,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_attn_args(d, q, k_cache, v_cache, page_table, seq_len, idx, count, top_k,
+                           scale, out);
+  if (st != HHR_OK) return st;
+  if (workspace == nullptr) return HHR_ERR_INVALID_ARG;
   const size_t need = hhr_attn_workspace_bytes(d, top_k);
   if (ws_bytes < need) return HHR_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255) != 0) return HHR_ERR_INVALID_ARG;
@@ -698,15 +716,16 @@ int hhr_read_device_status(void* stream, int* bits) {
 // no workspace. Its scratch is the file-scope array below, which every GPU that
 // loads the library holds until the process exits. Host code cannot pass the
 // array's name to a kernel (in host code it names a host-side shadow, not device
-// memory), so the first call on each device looks up the array's device address
-// with cudaGetSymbolAddress while that device is current, and caches it.
+// memory), so every call looks up the array's device address with
+// cudaGetSymbolAddress in the current device's context: a host-side lookup once the
+// first call on that device has loaded the library's device code there, and right
+// after a device reset or in another context too, which a cached address would not be.
 }  // extern "C"
 
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
 
 }  // namespace
 
@@ -716,7 +735,8 @@ int hhr_sparse_attn_noalloc(const hhr_dims* d, const uint16_t* q, const uint16_t
                             const uint16_t* v_cache, const int32_t* page_table,
                             const int32_t* seq_len, const int32_t* idx, const int32_t* count,
                             int top_k, float scale, float* out, void* stream) {
-  // Size check first: the partials must fit in the fixed array.
+  // Size check first: the partials must fit in the fixed array. Then the other arguments,
+  // all before any CUDA call.
   const size_t need = hhr_attn_workspace_bytes(d, top_k);
   if (need == 0) {
     int st = check_dims(d);
@@ -725,21 +745,14 @@ int hhr_sparse_attn_noalloc(const hhr_dims* d, const uint16_t* q, const uint16_t
     return HHR_ERR_INVALID_ARG;
   }
   if (need > kNoAllocScratchBytes) return HHR_ERR_WORKSPACE;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    g_last_cuda = e;
+  const int st = check_attn_args(d, q, k_cache, v_cache, page_table, seq_len, idx, count, top_k,
+                                 scale, out);
+  if (st != HHR_OK) return st;
+  void* scratch = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+  if (e != cudaSuccess || scratch == nullptr) {
+    g_last_cuda = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
     return HHR_ERR_CUDA;
-  }
-  if (dev < 0 || dev >= kMaxDevices) return HHR_ERR_UNSUPPORTED;
-  void* scratch = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (scratch == nullptr) {
-    e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
-    if (e != cudaSuccess || scratch == nullptr) {
-      g_last_cuda = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
-      return HHR_ERR_CUDA;
-    }
-    g_noalloc_ptr[dev].store(scratch, std::memory_order_release);
   }
   // The partials are written by the chunk kernel before the merge kernel reads
   // them (same stream), so nothing in the array has to start at zero.

@@ -186,6 +186,26 @@ __device__ __forceinline__ float dot8_h(const uint4 h, const float4 q0, const fl
          q1.z * d.x + q1.w * d.y;
 }
 
+// f16 summaries saturate to -inf (min row) or +inf (max row) beyond the f16 range. A folded
+// query component that is exactly 0 (no head of the group on that side) then meets an
+// infinite summary and 0 * inf is NaN, while that channel's true contribution is 0 for every
+// key of the page. dot8_h is NaN exactly in that case (every other product is finite or
+// +inf: qneg <= 0 pairs with kmin, which only saturates to -inf, and qpos >= 0 with kmax,
+// which only saturates to +inf), and this slow path recomputes it with those terms at 0.
+__device__ __forceinline__ float dot8_h_zero_guarded(const uint4 h, const float4 q0,
+                                                  const float4 q1) {
+  const float q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 k = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    s += q[2 * i] == 0.f ? 0.f : q[2 * i] * k.x;
+    s += q[2 * i + 1] == 0.f ? 0.f : q[2 * i + 1] * k.y;
+  }
+  return s;
+}
+
 // 16-byte summary load; the variant is a build-time choice (streaming by default).
 #ifndef HHR_BOUND_LOAD
 #define HHR_BOUND_LOAD 0
@@ -305,7 +325,20 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
                q1.y * mx.y + q1.z * mx.z + q1.w * mx.w;
       }
     }
-    const float tot = warp_sum8_transposed(v, lane);
+    float tot = warp_sum8_transposed(v, lane);
+    if constexpr (F16) {
+      // Rare: a NaN total (a zero folded query component met a saturated summary). The
+      // page's pieces are loaded again and summed with those terms at 0.
+      unsigned nan_pages = __ballot_sync(kFull, lane < 8 && tot != tot);
+      while (nan_pages != 0u) {
+        const int l = __ffs(nan_pages) - 1;
+        nan_pages &= nan_pages - 1u;
+        const int phys = __shfl_sync(kFull, my_phys, st * 8 + l);
+        const uint4 piece = load_summary16(base4 + ((size_t)phys * a.G + g) * kPieces + lane);
+        const float s = warp_sum(dot8_h_zero_guarded(piece, q0, q1));
+        if (lane == l) tot = s;
+      }
+    }
     // Lane l (< 8) holds the bound of page p0 + st*8 + l; its page id is on lane st*8 + l.
     const int phys_l = __shfl_sync(kFull, my_phys, (st * 8 + lane) & 31);
     const int lp = p0 + st * 8 + lane;

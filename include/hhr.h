@@ -84,7 +84,9 @@ typedef struct {
   int n_phys_pages;       /* pages in the pool */
   int summary_fp16;       /* page_minmax element type: 0 = f32; 1 = f16 rounded outward
                              (min toward -inf, max toward +inf), so the page bound stays an
-                             upper bound; values beyond the f16 range saturate to -inf/+inf */
+                             upper bound; values beyond the f16 range saturate to -inf/+inf
+                             (a channel on which the group's folded query is exactly 0 then
+                             contributes 0 to the bound, as it does for every finite key) */
   int select_per_head;    /* hash mode: 0 = one selection per KV group (the default reading:
                              bounds and distances summed over the group's query heads);
                              1 = one per query head (a variant): head h scores the summaries
@@ -251,10 +253,12 @@ int hhr_decode_step(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_n
  *     library holds it until the process exits.
  *   - Limit: hhr_attn_workspace_bytes(dims, top_k) must be at most 8 MiB (8388608
  *     bytes), e.g. batch 8 x 8 KV heads x 4-head groups at top_k 2048 needs about
- *     2.1 MB; a larger problem returns HHR_ERR_WORKSPACE before any launch.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make that
- *     first call outside any stream capture.
+ *     2.1 MB; a larger problem returns HHR_ERR_WORKSPACE before any CUDA call.
+ *   - Every call looks up the array's device address in the current device's
+ *     context (cudaGetSymbolAddress), so the address stays right after a device
+ *     reset or in another context of the same device. The first call on a device
+ *     also loads the library's device code there (the set-up); make that first
+ *     call before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents.
  *     Nothing in it needs to start at zero (each partial is written before it is
  *     read, in stream order), but calls that can overlap on the GPU (different

@@ -219,3 +219,27 @@ def test_misaligned_pointers_rejected(L):
     step[7] = bad  # R
     assert L.hhr_decode_step(ctypes.byref(d), *step, 0, 16, 2048, None, ctypes.c_float(0.1),
                              p, p, p, p, 1 << 30, None) == hhr.HHR_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_sizes_beyond_the_array(L):
+    """hhr_sparse_attn_noalloc keeps its split-K partials in a fixed 8 MiB device array: a
+    problem whose partials need more is refused with HHR_ERR_WORKSPACE, and bad arguments
+    with HHR_ERR_INVALID_ARG, both before any CUDA call (null pointers here, so nothing
+    could ever be dereferenced)."""
+    batch = 32
+    while True:
+        d = hhr.make_dims(batch, 64, 8, 32, 4096, 4096 * 32)
+        if hhr.hhr_attn_workspace_bytes(d, 8192) > 8 * 1024 * 1024:
+            break
+        batch *= 2
+        assert batch <= 65535
+    nul = [None] * 7
+    st = L.hhr_sparse_attn_noalloc(ctypes.byref(d), *nul, 8192, ctypes.c_float(0.1), None, None)
+    assert st == hhr.HHR_ERR_WORKSPACE
+    small = _d(batch=2)
+    assert hhr.hhr_attn_workspace_bytes(small, 1024) <= 8 * 1024 * 1024
+    st = L.hhr_sparse_attn_noalloc(ctypes.byref(small), *nul, 1024, ctypes.c_float(0.1), None,
+                                   None)
+    assert st == hhr.HHR_ERR_INVALID_ARG
+    st = L.hhr_sparse_attn_noalloc(ctypes.byref(small), *nul, 0, ctypes.c_float(0.1), None, None)
+    assert st == hhr.HHR_ERR_INVALID_ARG

@@ -25,3 +25,4 @@ def test_reference_arm_json_line():
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["value"] == j["value"]
     assert j["config"]["workload"] == "llama8b_128k_b8"
+    assert j["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))

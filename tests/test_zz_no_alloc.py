@@ -5,12 +5,11 @@ with no device allocator of its own, code that runs while a memory pool is froze
 or a plugin whose host forbids cudaMalloc. For them the library keeps the
 attention's split-K scratch in a fixed 8 MiB device array. This test calls that
 entry point through the C ABI twice in a row and compares each result with the
-regular entry point (which takes a caller workspace), within the attention
-tolerance used by the parity tests. It lives in its own file, collected last, and
-passes both alone in a fresh process and after the other tests.
+regular entry point (which takes a caller workspace): both run the same kernels with
+the same split plan, so the outputs must be identical bit for bit. It lives in its own
+file, collected last, and passes both alone in a fresh process and after the other
+tests. (The size limit is checked on the host without a GPU, in test_abi.py.)
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -20,16 +19,6 @@ from hash_hierarchical_top_b200 import build, hhr
 from hash_hierarchical_top_b200.step import DecodeStep, LayerCache
 
 pytestmark = pytest.mark.gpu
-
-ATTN_TOL = 2e-3
-
-
-def _rel_err(a, b):
-    a = a.double()
-    b = b.double()
-    den = b.abs().amax(dim=-1).clamp_min(1e-30)
-    return float(((a - b).abs().amax(dim=-1) / den).max())
-
 
 def _selected(wl, layer):
     inp = S.make_inputs(wl, device="cuda", layer=layer)
@@ -60,23 +49,5 @@ def test_noalloc_matches_workspace_entry_point_twice():
         torch.cuda.synchronize()
         assert hhr.hhr_read_device_status() == (hhr.HHR_OK, 0)
         assert torch.isfinite(out).all(), f"call {call}: non-finite output"
-        err = _rel_err(out, ref)
-        assert err <= ATTN_TOL, f"call {call}: max relative error {err}"
-
-
-def test_noalloc_rejects_sizes_beyond_the_array():
-    build.build()
-    L = hhr.lib()
-    # Grow the batch (8 KV heads, 8-head groups, top_k 8192) until the split-K partials
-    # no longer fit in the 8 MiB array.
-    batch = 32
-    while True:
-        d = hhr.make_dims(batch, 64, 8, 32, 4096, 4096 * 32)
-        if hhr.hhr_attn_workspace_bytes(d, 8192) > 8 * 1024 * 1024:
-            break
-        batch *= 2
-        assert batch <= 65535
-    p = ctypes.c_void_p(256)  # never dereferenced: the size check comes first
-    st = L.hhr_sparse_attn_noalloc(ctypes.byref(d), p, p, p, p, p, p, p, 8192,
-                                   ctypes.c_float(0.1), p, None)
-    assert st == hhr.HHR_ERR_WORKSPACE
+        assert torch.equal(out.view(torch.int32), ref.view(torch.int32)), \
+            f"call {call}: output differs from hhr_sparse_attn"
