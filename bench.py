@@ -195,10 +195,10 @@ class Clocks:
                 "samples": len(mhz)}
 
 
-def traffic_from_profile(kernel_src_hash, fmt):
-    """(DRAM bytes, algorithmic bytes) of the profiled page-bound launch from the committed
-    ncu summary, or None if the kernel source changed since the counters were taken."""
-    p = os.path.join(ROOT, "profiles", f"page_bound_{fmt}_kernel_llama8b_128k_b8.txt")
+def traffic_from_profile(name, kernel_src_hash):
+    """(DRAM bytes, algorithmic bytes) of the profiled launch from the committed ncu summary
+    profiles/<name>, or None if the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     vals = {}
@@ -864,15 +864,16 @@ def main():
         raise RuntimeError(f"device status {bits}")
 
     # Each decode step is one CUDA graph replay (one launch from the host). NG graphs cycle
-    # over the L layer caches; graph j carries its own event pair around the page-bound
-    # kernel, so the last NG replays of the timed region give the kernel's duration.
+    # over the L layer caches; graph j carries its own event pair around the dominant kernel
+    # (the page bounds), so the last NG replays of the timed region give its duration.
+    rk = "bound"
     NG = L * max(1, 48 // L)
     ev_b = timing_events(NG, stream)
     graphs = []
     for j in range(NG):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            hhr.hhr_profile_next("bound", ev_b[j][0], ev_b[j][1])
+            hhr.hhr_profile_next(rk, ev_b[j][0], ev_b[j][1])
             run(j)
         graphs.append(gr)
     # The same steps without the event nodes (which sit between kernels and cut the
@@ -1082,12 +1083,14 @@ def main():
                    "peak_source": "measured bf16 dense (burst)" if mp else "fallback"}
 
     peak, peak_kind = measured_peaks()
-    bound_bytes = bound_kernel_bytes(wl, lens, sbytes)
+    kbytes = step_kernel_bytes(wl, lens, m_of, sbytes)
+    bound_bytes = kbytes[rk]
     bound_avg_ms = statistics.mean(bound_ms)
     achieved = bound_bytes / (bound_avg_ms / 1e3) / 1e9
     # DRAM bytes of the profiled launch, scaled to this launch's algorithmic bytes (the
-    # kernel's traffic grows in proportion to the pages it reads).
-    prof = traffic_from_profile(kernel_source_hash(), args.summary)
+    # kernel's traffic grows in proportion to the pages and rows it reads).
+    rk_name = f"page_bound_{args.summary}"
+    prof = traffic_from_profile(f"{rk_name}_kernel_{wl.name}.txt", kernel_source_hash())
     traffic = prof[0] * bound_bytes / prof[1] if prof is not None else None
     step_gbs = req / (ms_step / 1e3) / 1e9
 
@@ -1130,17 +1133,20 @@ def main():
                        "timing": f"CUDA-graph replay per step, CUDA events on the stream; the "
                                  f"last {nbr} of {K} replays carry event nodes around the page-bound "
                                  f"kernel (its duration for the roofline)"},
-            "roofline": {"bound": "hbm", "kernel": f"page_bound_{args.summary}_kernel",
+            "roofline": {"bound": "hbm", "kernel": f"{rk_name}_kernel",
+                         "scope": "the dominant kernel alone (its CUDA-event duration in "
+                                  "bracketed replays); the whole step's fraction is step_hbm",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
                          "traffic": traffic, "algorithmic_bytes": bound_bytes,
-                         "avg_launch_us": bound_avg_ms * 1e3},
+                         "avg_launch_us": bound_avg_ms * 1e3,
+                         "step_frac_of_measured": step_gbs / peak},
             "step_hbm": {"required_bytes": req, "summaries": summ_b, "codes": codes_b,
                          "kv_rows": kv_b, "achieved_gbs": step_gbs,
                          "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
                          "frac_of_measured": step_gbs / peak},
             "kernels_us": kern,
-            "kernels": kernel_table(kern, step_kernel_bytes(wl, lens, m_of, sbytes), peak),
+            "kernels": kernel_table(kern, kbytes, peak),
             "prefill_encode": prefill,
             "other_workloads": other,
             "selection_quality": quality,

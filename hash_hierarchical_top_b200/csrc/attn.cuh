@@ -122,31 +122,29 @@ __device__ __forceinline__ int swz(int r, int chunk) { return r * kD + ((chunk ^
 // merged its warps, every CTA merges its share of the group's outputs from all the
 // splits' states through distributed shared memory and writes them (no partials in
 // global memory, no combine kernel).
-template <bool kCluster>
-__global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a) {
-  extern __shared__ float4 at_smem[];
-  pdl_wait();
-  pdl_trigger();
-  uint16_t* stage_base = reinterpret_cast<uint16_t*>(at_smem);             // [kStages][2][kTile][d]
-  uint32_t* offs = reinterpret_cast<uint32_t*>(stage_base + (size_t)kStages * 2 * kTile * kD);
+// Barrier of the kAttnThreads threads that run one split: the whole CTA of the split kernel
+// (named barrier 0), or one half of a CTA of the fused step kernel (named barriers 1, 2).
+__device__ __forceinline__ void attn_sync(int bar_id) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(bar_id), "r"(kAttnThreads) : "memory");
+}
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;  // g: selection row
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// One split of one selection row, run by kAttnThreads threads (tid 0..255) behind barrier
+// bar_id: rows [base, base + nrows) of the row's selection are gathered and attended; the
+// split's softmax state is merged over its warps, and emit(h, c, M, L, O) is called once
+// for every (head h < gs, channel c) of the row, M the split's running max of head h (in
+// log2 units), L its sum of exponentials and O its output channel c before the division
+// by L. smem: the stage buffers followed by the row-offset table of split_rows entries.
+// Selection rows, counts and cache rows are read through L2 (they may have been written by
+// other CTAs of the same kernel).
+template <typename Emit>
+__device__ __forceinline__ void attn_split(const AttnArgs& a, int g, int b, int base, int nrows,
+                                           uint16_t* stage_base, int tid, int bar_id, Emit emit) {
+  uint32_t* offs = reinterpret_cast<uint32_t*>(stage_base + (size_t)kStages * 2 * kTile * kD);
+  const int lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;   // fragment coordinates
   const int gs = a.Hq / a.Gs;
   const int row = b * a.Gs + g;
   const uint32_t gkv = (uint32_t)(a.kv_div == 1 ? g : g / a.kv_div);  // KV head of the row
-  const int cnt = min(a.count[row], a.top_k);
-  const int base = split * a.split_rows;
-  // A split past the selection does no work (in a cluster it still joins the merge). An
-  // unsplit group with an empty selection writes its zero output here, since no merge follows.
-  const int nrows = max(0, min(a.split_rows, cnt - base));
-  if (!kCluster && nrows == 0) {
-    if (a.n_splits == 1)
-      for (int i = tid; i < gs * kD; i += kAttnThreads)
-        a.out[((size_t)b * a.Hq + g * gs) * kD + i] = 0.f;
-    return;
-  }
   const int ntiles = (nrows + kTile - 1) / kTile;
   const int n = a.seq_len[b];
 
@@ -154,9 +152,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
   for (int r = tid; r < ntiles * kTile; r += kAttnThreads) {
     uint32_t o = kNoRow;
     if (r < nrows && a.rows != nullptr) {
-      o = a.rows[(size_t)row * a.top_k + base + r];
+      o = __ldcg(a.rows + (size_t)row * a.top_k + base + r);
     } else if (r < nrows) {
-      const int t = a.idx[(size_t)row * a.top_k + base + r];
+      const int t = __ldcg(a.idx + (size_t)row * a.top_k + base + r);
       const int lp = t / a.P;
       if (t >= 0 && t < n && lp < a.maxp) {
         const int phys = a.page_table[(size_t)b * a.maxp + lp];
@@ -170,7 +168,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
     }
     offs[r] = o;
   }
-  __syncthreads();
+  attn_sync(bar_id);
 
   auto issue = [&](int t) {
     uint16_t* Ks = stage_base + (size_t)(t % kStages) * 2 * kTile * kD;
@@ -220,7 +218,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
 
   for (int t = 0; t < ntiles; ++t) {
     cp_async_wait<kStages - 2>();
-    __syncthreads();
+    attn_sync(bar_id);
     if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
     cp_async_commit();
     const uint32_t ks = smem0 + (uint32_t)((t % kStages) * 2 * kTile * kD) * 2;
@@ -275,7 +273,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
     }
   }
   cp_async_wait<0>();
-  __syncthreads();
+  attn_sync(bar_id);
 
   // Merge the 8 warps: o = sum_w 2^(m_w - M) o_w, l = sum_w 2^(m_w - M) l_w.
   float* mo = reinterpret_cast<float*>(stage_base);             // [warps][8 heads][d]
@@ -299,7 +297,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
       mml[(warp * kMaxGroup + gq) * 2 + 1] = l_run;
     }
   }
-  __syncthreads();
+  attn_sync(bar_id);
   for (int i = tid; i < gs * kD; i += kAttnThreads) {
     const int h = i / kD, c = i % kD;
     float M = -INFINITY;
@@ -315,6 +313,58 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
         O = fmaf(sc, mo[((size_t)w * kMaxGroup + h) * kD + c], O);
       }
     }
+    emit(h, c, M, L, O);
+  }
+}
+
+// Merge of the split partials of output (head hh, channel c) of selection row `row` over its
+// first ns splits: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s (0 for an empty set).
+// The same arithmetic, in the same order, wherever splits are merged.
+__device__ __forceinline__ float merge_splits(const float* part_o, const float* part_ml, int row,
+                                              int n_splits, int ns, int gs, int hh, int c) {
+  const float* ml = part_ml + ((size_t)row * n_splits * gs + hh) * 2;
+  const float* po = part_o + ((size_t)row * n_splits * gs + hh) * kD + c;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, __ldcg(ml + (size_t)s * gs * 2));
+  float L = 0.f, o = 0.f;
+  if (M > -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const float m = __ldcg(ml + (size_t)s * gs * 2);
+      const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      L = fmaf(w, __ldcg(ml + (size_t)s * gs * 2 + 1), L);
+      o = fmaf(w, __ldcg(po + (size_t)s * gs * kD), o);
+    }
+  }
+  return (L > 0.f) ? o / L : 0.f;
+}
+
+// kCluster: the splits of a group form one thread-block cluster; after each CTA has
+// merged its warps, every CTA merges its share of the group's outputs from all the
+// splits' states through distributed shared memory and writes them (no partials in
+// global memory, no combine kernel).
+template <bool kCluster>
+__global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a) {
+  extern __shared__ float4 at_smem[];
+  pdl_wait();
+  pdl_trigger();
+  uint16_t* stage_base = reinterpret_cast<uint16_t*>(at_smem);             // [kStages][2][kTile][d]
+  uint32_t* offs = reinterpret_cast<uint32_t*>(stage_base + (size_t)kStages * 2 * kTile * kD);
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;  // g: selection row
+  const int tid = threadIdx.x;
+  const int gs = a.Hq / a.Gs;
+  const int row = b * a.Gs + g;
+  const int cnt = min(__ldcg(a.count + row), a.top_k);
+  const int base = split * a.split_rows;
+  // A split past the selection does no work (in a cluster it still joins the merge). An
+  // unsplit group with an empty selection writes its zero output here, since no merge follows.
+  const int nrows = max(0, min(a.split_rows, cnt - base));
+  if (!kCluster && nrows == 0) {
+    if (a.n_splits == 1)
+      for (int i = tid; i < gs * kD; i += kAttnThreads)
+        a.out[((size_t)b * a.Hq + g * gs) * kD + i] = 0.f;
+    return;
+  }
+  attn_split(a, g, b, base, nrows, stage_base, tid, 0, [&](int h, int c, float M, float L, float O) {
     if constexpr (kCluster) {
       // This CTA's merged state, in the (now free) offset table: [gs][d] outputs, [gs][2].
       float* res = reinterpret_cast<float*>(offs);
@@ -333,14 +383,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) sparse_attn_kernel(AttnArgs a
         a.part_ml[p * 2 + 1] = L;
       }
     }
-  }
+  });
   if constexpr (kCluster) {
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();  // every split's state is in its shared memory
     {
       // Rank r merges outputs [r n/ns, (r + 1) n/ns) of the group's n = gs * d (the same
-      // arithmetic per output as the combine kernel, split over the cluster's CTAs).
+      // arithmetic per output as merge_splits, split over the cluster's CTAs).
       const int ns = (int)cl.num_blocks(), rk = (int)cl.block_rank();
       const int per = (gs * kD + ns - 1) / ns;
       const int lo = rk * per, hi = min(gs * kD, lo + per);
@@ -408,20 +458,8 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(CombineArgs a) {
   const int row = b * a.G + g;
   const int cnt = min(a.count[row], a.top_k);
   const int ns = min(a.n_splits, ceil_div(max(cnt, 0), a.split_rows));
-  const float* ml = a.part_ml + ((size_t)row * a.n_splits * gs + hh) * 2;
-  const float* po = a.part_o + ((size_t)row * a.n_splits * gs + hh) * kD + tid;
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, ml[(size_t)s * gs * 2]);
-  float L = 0.f, o = 0.f;
-  if (M > -INFINITY) {
-    for (int s = 0; s < ns; ++s) {
-      const float m = ml[(size_t)s * gs * 2];
-      const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      L = fmaf(w, ml[(size_t)s * gs * 2 + 1], L);
-      o = fmaf(w, po[(size_t)s * gs * kD], o);
-    }
-  }
-  a.out[((size_t)b * a.Hq + h) * kD + tid] = (L > 0.f) ? o / L : 0.f;
+  a.out[((size_t)b * a.Hq + h) * kD + tid] =
+      merge_splits(a.part_o, a.part_ml, row, a.n_splits, ns, gs, hh, tid);
 }
 
 }  // namespace hhr

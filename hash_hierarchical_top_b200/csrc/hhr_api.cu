@@ -25,6 +25,17 @@ constexpr int kMaxDevices = 64;
 constexpr int kTcMinBulk = 4096;  // appends at least this long use the tensor-core encoder
 constexpr int kTcSlots = 148;     // persistent encoder CTAs (one per SM of a B200)
 constexpr size_t kMaxKernelSmem = 200 * 1024;  // below the 227 KB opt-in of sm_100
+// Summaries of the first selection rows, about this many bytes, are prefetched into L2 by
+// the fused step's prologue for the page-bound kernel that follows it.
+#ifndef HHR_WARM_MB
+#define HHR_WARM_MB 44
+#endif
+constexpr size_t kWarmBytes = (size_t)HHR_WARM_MB << 20;
+// Page bounds: 1 = page_bound_stage_kernel (summaries staged page-major in shared memory by
+// bulk copies), 0 = page_bound_kernel (summaries loaded to registers).
+#ifndef HHR_BOUND_STAGE
+#define HHR_BOUND_STAGE 0
+#endif
 
 // Every device buffer is read with 16-byte vector loads somewhere on the path.
 bool misaligned16(std::initializer_list<const void*> ptrs) {
@@ -105,7 +116,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   return e;
 }
 
-bool g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
+bool g_smem_stage[2][kMaxDevices], g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
     g_smem_sel[kMaxDevices], g_smem_ham[3][2][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
     g_smem_attn_cl[kMaxDevices];
 
@@ -230,6 +241,35 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Launches the page bounds of every selection row (step a2), with programmatic stream
+// serialisation when `pdl`: page_bound_stage_kernel (summaries staged page-major in shared
+// memory by bulk copies; persistent, one CTA per SM), or page_bound_kernel (summaries loaded
+// to registers) where its shared-memory prefix does not fit or HHR_BOUND_STAGE is 0.
+cudaError_t launch_bounds_kernel(const hhr_dims* d, const BoundArgs& ba, bool pdl,
+                                 cudaStream_t s) {
+  const bool ph = kv_div(d) > 1, f16 = d->summary_fp16 != 0;
+  const int B = d->batch, Gs = sel_rows(d), maxp = d->max_pages_per_seq;
+  if (HHR_BOUND_STAGE && B <= kStageMaxBatch && stage_slots(d->n_kv_heads, f16) >= 2) {
+    void (*k)(BoundArgs, int) = f16 ? page_bound_stage_kernel<true> : page_bound_stage_kernel<false>;
+    const size_t smem = stage_smem(d->n_kv_heads, f16, B);
+    cudaError_t e = allow_smem(k, smem, g_smem_stage[f16 ? 1 : 0]);
+    if (e != cudaSuccess) return e;
+    const int S = stage_slots(d->n_kv_heads, f16);
+    const dim3 grid(sm_count());
+    if (pdl) return launch_pdl(k, grid, dim3(kStageThreads), smem, s, ba, S);
+    k<<<grid, kStageThreads, smem, s>>>(ba, S);
+    return cudaGetLastError();
+  }
+  const int ppc = bound_pages_per_cta(f16);
+  const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
+  void (*k)(BoundArgs) =
+      f16 ? (ph ? page_bound_kernel<true, true> : page_bound_kernel<true, false>)
+          : (ph ? page_bound_kernel<false, true> : page_bound_kernel<false, false>);
+  if (pdl) return launch_pdl(k, grid, dim3(kBoundWarps * 32), 0, s, ba);
+  k<<<grid, kBoundWarps * 32, 0, s>>>(ba);
+  return cudaGetLastError();
 }
 
 int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
@@ -384,19 +424,11 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
     const bool flat = m_max >= maxp;
     if (!flat || (trace != nullptr && trace->bounds != nullptr)) {
       const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                         d->n_phys_pages, 0, Gs, kv_div(d)};
-      const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
-      const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
+                         d->n_phys_pages, 0, Gs, kv_div(d), B};
       prof_begin(HHR_KERNEL_BOUND, s);
-      const dim3 blk(kBoundWarps * 32);
-      if (d->summary_fp16)
-        (kv_div(d) > 1 ? page_bound_kernel<true, true> : page_bound_kernel<true, false>)
-            <<<grid, blk, 0, s>>>(ba);
-      else
-        (kv_div(d) > 1 ? page_bound_kernel<false, true> : page_bound_kernel<false, false>)
-            <<<grid, blk, 0, s>>>(ba);
+      const cudaError_t e = launch_bounds_kernel(d, ba, false, s);
       prof_end(HHR_KERNEL_BOUND, s);
-      if ((st = launch_status()) != HHR_OK) return st;
+      if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
     }
     HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
                    Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, nullptr, sink, local,
@@ -593,6 +625,7 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
   float* part_ml = reinterpret_cast<float*>(aws + align256((size_t)B * Gs * ns * rh * kD * 4));
   uint32_t* row_buf = reinterpret_cast<uint32_t*>(aws + hhr_attn_workspace_bytes(d, top_k));
   const int cw = code_words(d);
+  const bool flat = m_max >= maxp;
   const size_t fsm = topm_hamming_smem(rh, cw, m_max, P, maxp);
   const int nt = topm_hamming_threads(cw, (long long)B * Gs * kHamRanks, sm_count());
   if (allow_smem(topm_hamming_for(rh, cw, nt), fsm,
@@ -604,29 +637,35 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     return HHR_ERR_CUDA;
   cudaError_t e;
 
-  // a0 + a1: append and encode the newest key rows, rotate and encode the queries.
+  // a0 + a1: append and encode the newest key rows, rotate and encode the queries. The staged
+  // bound kernel that follows starts each CTA at the beginning of its chunk range: the
+  // prologue prefetches those first units into L2 (about kWarmBytes in all; not when an event
+  // brackets the bound kernel, whose duration is then that of a cold L2).
+  int warm_units = 0, warm_ctas = 0;
+  const bool staged = HHR_BOUND_STAGE && B <= kStageMaxBatch &&
+                      stage_slots(G, d->summary_fp16 != 0) >= 2;
+  const int ub = stage_unit_bytes(G, d->summary_fp16 != 0);
+  if (!flat && staged && B <= 64 && g_prof[HHR_KERNEL_BOUND].start == nullptr) {
+    warm_ctas = sm_count();
+    warm_units = (int)min((size_t)kStageChunk * 64, kWarmBytes / ((size_t)warm_ctas * ub));
+  }
   prof_begin(HHR_KERNEL_ENCODE, s);
   step_prologue_for(gs, cw)<<<dim3(kPrologueRanks, G, B), kPrologueThreads, 0, s>>>(
       PrologueArgs{q, k_new, v_new, k_cache, v_cache, page_table, seq_len, R, W, page_minmax,
                    codes, q_rot, q_code, qpn, Hq, G, P, maxp, d->n_phys_pages,
-                   d->summary_fp16});
+                   d->summary_fp16, warm_units, warm_ctas, ub, kStageChunk});
   prof_end(HHR_KERNEL_ENCODE, s);
   if ((st = launch_status()) != HHR_OK) return st;
   // a2: page bounds (none when every page is kept: a flat hash top-k).
-  const bool flat = m_max >= maxp;
   if (!flat) {
-    // Launched behind the prologue: its first CTAs warm L2 while the prologue runs, unless
-    // an event is recorded between the two (profiling), which leaves no overlap to use.
+    // Launched behind the prologue. With f32 summaries (page_bound_kernel) its first CTAs
+    // warm L2 while the prologue runs, unless an event is recorded between the two
+    // (profiling), which leaves no overlap to use.
     const int early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
     const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                       d->n_phys_pages, early, Gs, kv_div(d)};
-    const int ppc = bound_pages_per_cta(d->summary_fp16 != 0);
-    const dim3 grid = bound_grid(Gs, (maxp + ppc - 1) / ppc, B);
+                       d->n_phys_pages, early, Gs, kv_div(d), B};
     prof_begin(HHR_KERNEL_BOUND, s);
-    void (*bk)(BoundArgs) =
-        d->summary_fp16 ? (kv_div(d) > 1 ? page_bound_kernel<true, true> : page_bound_kernel<true, false>)
-                        : (kv_div(d) > 1 ? page_bound_kernel<false, true> : page_bound_kernel<false, false>);
-    e = launch_pdl(bk, grid, dim3(kBoundWarps * 32), 0, s, ba);
+    e = launch_bounds_kernel(d, ba, true, s);
     prof_end(HHR_KERNEL_BOUND, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   }

@@ -96,10 +96,6 @@ inline size_t qprep_smem() { return 0; }
 // path, so this kernel is a pure streaming GEMV.
 // Tuned on B200 at 128K context, batch 8 (4096 pages x 8 groups x 8 sequences); the
 // macros below exist for such sweeps.
-// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
-}
 
 #ifndef HHR_BOUND_WARPS
 #define HHR_BOUND_WARPS 4
@@ -146,6 +142,7 @@ struct BoundArgs {
   int G, P, maxp, n_phys;
   int early;      // CTAs that warm L2 before the dependency wait (0: none)
   int Gs, kv_div; // selection rows per sequence (G, or Hq per head); row r uses KV head r / kv_div
+  int batch;      // B
 };
 
 // Sum over the warp of 8 per-lane partials (one per page): a butterfly over lane bits 4
@@ -226,61 +223,24 @@ __device__ __forceinline__ uint4 load_summary16(const uint4* p) {
 #endif
 }
 
-// PH: one query head per selection row (per-head selection), folded here from q_rot.
-template <bool F16, bool PH = false>
-__global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
-  // kSets groups of 8 pages per warp are loaded together (all page ids first, then all
-  // summary pieces), so that each warp keeps kSets * 8 page summaries in flight.
-  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
-  constexpr int kPagesPerWarp = 8 * kSets;
-  // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
-  constexpr int kPieces = F16 ? 32 : 64;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if constexpr (HHR_BOUND_LOOKAHEAD > 0) {
-    // Reads only inputs no earlier kernel of the step writes (page table, lengths); a
-    // prefetch of a summary that the previous kernel is updating is coherent in L2.
-    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-    const int total = gridDim.x * gridDim.y * gridDim.z;
-    if (lin < a.early && lane < kPagesPerWarp) {
-#pragma unroll
-      for (int j = 0; j < HHR_BOUND_LOOKAHEAD; ++j) {
-        const int t = lin + j * a.early;
-        if (t < total) {
-          const int tx = t % gridDim.x, ty = (t / gridDim.x) % gridDim.y;
-          const int tb = t / (gridDim.x * gridDim.y);
-          const int tg = bound_group_of(tx, ty);
-          const int p = bound_chunk_of(tx, ty) * kBoundWarps * kPagesPerWarp +
-                        warp * kPagesPerWarp + lane;
-          if (p < min(ceil_div(a.seq_len[tb], a.P), a.maxp)) {
-            const int phys = a.page_table[(size_t)tb * a.maxp + p];
-            if (phys >= 0 && phys < a.n_phys)
-              prefetch_l2(reinterpret_cast<const uint4*>(a.page_minmax) +
-                              ((size_t)phys * a.G + (PH ? tg / a.kv_div : tg)) * kPieces,
-                          kPieces * 16);
-          }
-        }
-      }
-    }
-  }
-  pdl_wait();
-  pdl_trigger();
-  const int r = bound_group(), b = blockIdx.z;  // selection row r reads KV head r / kv_div
-  const int g = PH ? r / a.kv_div : r;
-  const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
-  const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
-  if (p0 >= npg) return;
-  float4 q0, q1;
-  if constexpr (!PH) {
+// The folded query of selection row r of sequence b, as the lane's halves of the two bound
+// vectors (qneg paired with kmin, qpos with kmax): 8 channels of qneg (lanes 0-15) or qpos
+// (lanes 16-31) for f16 summaries, channels 4l..4l+3 of both for f32. per_head: the row is one
+// query head, folded here from its rotated query (qneg = min(q', 0), qpos = max(q', 0)).
+template <bool F16>
+__device__ __forceinline__ void bound_query(const BoundArgs& a, int b, int r, bool per_head,
+                                            int lane, float4& q0, float4& q1) {
+  if (!per_head) {
     const float* qb = a.qpn + ((size_t)b * a.Gs + r) * 2 * kD;
-    if constexpr (F16) {  // 8 channels of qneg (lanes 0-15) or qpos (lanes 16-31)
+    if constexpr (F16) {
       const float4* qv = reinterpret_cast<const float4*>(qb + (lane >> 4) * kD + 8 * (lane & 15));
       q0 = qv[0];
       q1 = qv[1];
-    } else {              // channels 4l..4l+3 of qneg and of qpos
+    } else {
       q0 = reinterpret_cast<const float4*>(qb)[lane];
       q1 = reinterpret_cast<const float4*>(qb + kD)[lane];
     }
-  } else {  // one query head per row: fold its rotated query, qneg = min(q', 0), qpos = max
+  } else {
     const float* qh = a.q_rot + ((size_t)b * a.Gs + r) * kD;
     auto lo = [](float4 v) { return make_float4(fminf(v.x, 0.f), fminf(v.y, 0.f), fminf(v.z, 0.f), fminf(v.w, 0.f)); };
     auto hi = [](float4 v) { return make_float4(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f), fmaxf(v.z, 0.f), fmaxf(v.w, 0.f)); };
@@ -294,6 +254,18 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
       q1 = hi(v);
     }
   }
+}
+
+// One warp's share of the page bounds of selection row r (KV head g) of sequence b: pages
+// [p0, p0 + kPagesPerWarp) (those below npg), written to a.bounds (-inf and a status bit for a
+// page id outside the pool). All page ids are loaded first, then all summary pieces, so that
+// the warp keeps kPagesPerWarp page summaries in flight.
+template <bool F16>
+__device__ __forceinline__ void bound_warp(const BoundArgs& a, int b, int r, int g, int p0,
+                                           int npg, int lane, float4 q0, float4 q1) {
+  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
+  constexpr int kPagesPerWarp = 8 * kSets;
+  constexpr int kPieces = F16 ? 32 : 64;
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
   int my_phys = -1;  // lane i < kPagesPerWarp resolves page p0 + i
   if (lane < kPagesPerWarp && p0 + lane < npg)
@@ -348,6 +320,261 @@ __global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs 
       out[lp] = ok ? tot : -INFINITY;
     }
   }
+}
+
+
+// Page bounds from summaries staged page-major in shared memory by bulk copies. A unit is
+// one physical page's summaries of every KV group, G x 2 x d values stored contiguously
+// (G x 512 B in f16, G x 1 KB in f32), so one 1-D bulk copy (cp.async.bulk, global -> this
+// CTA's shared memory, no multicast) moves it. A persistent CTA (one per SM) has one
+// producer warp and kStageConsumers consumer warps around a ring of unit slots: the producer
+// issues each unit's copy into the next free slot (its "empty" mbarrier) and the copy
+// completes on the slot's "full" mbarrier; consumer warp w folds units w, w + kStageConsumers,
+// ... of the CTA's stream into the bounds of every selection row of the unit's sequence (a
+// row reads its KV group's summary), with the arithmetic of bound_warp on the same 16-byte
+// pieces per lane, so the bounds are bit-identical; then it hands the slot back.
+// Work: chunks of kStageChunk consecutive pages of a sequence (every sequence's chunks below
+// its page count, sequences in order); CTA c takes a contiguous range of chunks.
+constexpr int kStageThreads = 512;
+constexpr int kStageConsumers = kStageThreads / 32 - 1;
+constexpr int kStageChunk = 16;
+constexpr int kStageMaxSlots = 256;
+constexpr int kStageMaxBatch = 4096;  // sequences whose chunk prefix fits in shared memory
+constexpr size_t kStageRingBytes = 192 * 1024;
+constexpr long long kStageWaitLimit = 1ll << 24;
+
+__host__ __device__ inline int stage_unit_bytes(int G, bool f16) { return G * 2 * kD * (f16 ? 2 : 4); }
+inline int stage_slots(int G, bool f16) {
+  const int n = (int)(kStageRingBytes / (size_t)stage_unit_bytes(G, f16));
+  return n < kStageMaxSlots ? n : kStageMaxSlots;
+}
+// Dynamic shared memory: the slots, their full and empty mbarriers, their page ids, and the
+// chunk prefix over the sequences.
+inline size_t stage_smem(int G, bool f16, int B) {
+  const int S = stage_slots(G, f16);
+  return (size_t)S * stage_unit_bytes(G, f16) + (size_t)S * 16 + (size_t)S * 4 +
+         (size_t)(2 * B + 1) * 4 + 16;
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(kStageThreads, 1) page_bound_stage_kernel(BoundArgs a, int S) {
+  extern __shared__ __align__(16) unsigned char st_smem[];
+  constexpr int Q = kStageChunk;
+  constexpr int kAhead = 4;  // producer batches whose page ids are loaded ahead
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int B = a.batch, G = a.G;
+  const int ub = stage_unit_bytes(G, F16);
+  unsigned char* slots = st_smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(st_smem + (size_t)S * ub);
+  uint64_t* empty = full + S;
+  int* slot_phys = reinterpret_cast<int*>(empty + S);
+  int* cpre = slot_phys + S;  // [B + 1] chunks of the sequences before b
+  int* npgs = cpre + B + 1;   // [B] pages of sequence b
+  for (int i = threadIdx.x; i < S; i += kStageThreads) {
+    mbar_init(smem_u32(full + i), 1);
+    mbar_init(smem_u32(empty + i), 1);
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  // Page counts and chunk prefix (the lengths are inputs: read before the dependency wait).
+  if (warp == 0) {
+    int run = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      const int np = b < B ? min(ceil_div(max(a.seq_len[b], 0), a.P), a.maxp) : 0;
+      const int nc = ceil_div(np, Q);
+      const int incl = warp_incl_scan(nc, lane);
+      if (b < B) {
+        cpre[b] = run + incl - nc;
+        npgs[b] = np;
+      }
+      run += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) cpre[B] = run;
+  }
+  __syncthreads();
+  const int C = cpre[B];
+  const int c0 = (int)((long long)blockIdx.x * C / gridDim.x);
+  const int c1 = (int)((long long)(blockIdx.x + 1) * C / gridDim.x);
+  const int n_units = (c1 - c0) * Q;
+  // Unit j of this CTA: sequence b and page p (a unit at p >= npgs[b] is past the end).
+  auto unit = [&](int j, int& b, int& p) {
+    const int id = c0 + j / Q;
+    int lo = 0, hi = B - 1;  // the last b with cpre[b] <= id
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cpre[mid] <= id) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    p = (id - cpre[b]) * Q + j % Q;
+  };
+  if (warp == 0) {
+    // Producer: lane l < PB takes units j0 + l of every batch; -1 marks a unit past its
+    // sequence's end, -2 a page id outside the pool (no copy for either). PB <= S keeps the
+    // lanes of one batch on distinct slots, so no lane waits for a slot that another lane of
+    // its batch must fill. Page ids are loaded kAhead batches ahead (the page table is an
+    // input: the first ones before the dependency wait).
+    const int PB = S < 32 ? S : 32;
+    auto page_id = [&](int j) {
+      int phys = -1;
+      if (lane < PB && j < n_units) {
+        int b, p;
+        unit(j, b, p);
+        if (p < npgs[b]) {
+          phys = a.page_table[(size_t)b * a.maxp + p];
+          if (phys < 0 || phys >= a.n_phys) phys = -2;
+        }
+      }
+      return phys;
+    };
+    int ahead[kAhead];
+#pragma unroll
+    for (int t = 0; t < kAhead; ++t) ahead[t] = page_id(t * PB + lane);
+    pdl_wait();
+    pdl_trigger();
+    for (int j0 = 0, t = 0; j0 < n_units; j0 += PB, ++t) {
+      const int phys = ahead[0];
+#pragma unroll
+      for (int u = 0; u + 1 < kAhead; ++u) ahead[u] = ahead[u + 1];
+      ahead[kAhead - 1] = page_id(j0 + kAhead * PB + lane);
+      const int j = j0 + lane;
+      if (lane < PB && j < n_units) {
+        const int slot = j % S;
+        if (!mbar_wait_bounded(smem_u32(empty + slot), ((j / S) & 1) ^ 1, kStageWaitLimit))
+          flag_status(kStatusWaitGaveUp);
+        slot_phys[slot] = phys;
+        mbar_arrive_expect_tx(smem_u32(full + slot), phys >= 0 ? (uint32_t)ub : 0u);
+        if (phys >= 0)
+          bulk_g2s(smem_u32(slots + (size_t)slot * ub),
+                   static_cast<const unsigned char*>(a.page_minmax) + (size_t)phys * ub,
+                   (uint32_t)ub, smem_u32(full + slot));
+      }
+    }
+    return;
+  }
+  pdl_wait();
+  pdl_trigger();
+  // Consumers. The folded queries of up to 8 rows of the current sequence stay in registers.
+  constexpr int kPiece = F16 ? 512 : 1024;  // bytes of one KV group's summary
+  const bool per_head = a.kv_div > 1;
+  const bool cache_q = a.Gs <= 8;
+  float4 qc0[8], qc1[8];
+  int qb = -1;
+  for (int j = warp - 1; j < n_units; j += kStageConsumers) {
+    const int slot = j % S;
+    int b, p;
+    unit(j, b, p);
+    if (cache_q && b != qb) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i < a.Gs) bound_query<F16>(a, b, i, per_head, lane, qc0[i], qc1[i]);
+      qb = b;
+    }
+    if (!mbar_wait_bounded(smem_u32(full + slot), (j / S) & 1, kStageWaitLimit) && lane == 0)
+      flag_status(kStatusWaitGaveUp);
+    const int phys = slot_phys[slot];
+    const unsigned char* u = slots + (size_t)slot * ub;
+    if (phys != -1) {
+      for (int r0 = 0; r0 < a.Gs; r0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = r0 + i;
+          v[i] = 0.f;
+          if (r < a.Gs && phys >= 0) {
+            float4 q0, q1;
+            if (cache_q) {
+              q0 = qc0[i];
+              q1 = qc1[i];
+            } else {
+              bound_query<F16>(a, b, r, per_head, lane, q0, q1);
+            }
+            const unsigned char* gp = u + (size_t)(a.kv_div == 1 ? r : r / a.kv_div) * kPiece;
+            if constexpr (F16) {
+              v[i] = dot8_h(*reinterpret_cast<const uint4*>(gp + lane * 16), q0, q1);
+            } else {
+              const float4 mn = *reinterpret_cast<const float4*>(gp + lane * 16);
+              const float4 mx = *reinterpret_cast<const float4*>(gp + 512 + lane * 16);
+              v[i] = q0.x * mn.x + q0.y * mn.y + q0.z * mn.z + q0.w * mn.w + q1.x * mx.x +
+                     q1.y * mx.y + q1.z * mx.z + q1.w * mx.w;
+            }
+          }
+        }
+        float tot = warp_sum8_transposed(v, lane);
+        if constexpr (F16) {
+          // Rare: a NaN total (a zero folded query component met a saturated summary): the
+          // row is summed again with those terms at 0.
+          unsigned nan_rows = __ballot_sync(kFull, lane < 8 && tot != tot);
+          while (nan_rows != 0u) {
+            const int l = __ffs(nan_rows) - 1;
+            nan_rows &= nan_rows - 1u;
+            const int r = r0 + l;
+            float4 q0, q1;
+            bound_query<F16>(a, b, r, per_head, lane, q0, q1);
+            const unsigned char* gp = u + (size_t)(a.kv_div == 1 ? r : r / a.kv_div) * kPiece;
+            const float sum = warp_sum(
+                dot8_h_zero_guarded(*reinterpret_cast<const uint4*>(gp + lane * 16), q0, q1));
+            if (lane == l) tot = sum;
+          }
+        }
+        const int r = r0 + lane;
+        if (lane < 8 && r < a.Gs) {
+          if (phys == -2 && r == 0) flag_status(kStatusBadPage);
+          a.bounds[((size_t)b * a.Gs + r) * a.maxp + p] = phys >= 0 ? tot : -INFINITY;
+        }
+      }
+    }
+    // The unit's shared-memory reads are complete (their values are folded): hand the slot
+    // back for its next bulk copy.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+  }
+}
+
+// PH: one query head per selection row (per-head selection), folded here from q_rot.
+template <bool F16, bool PH = false>
+__global__ void __launch_bounds__(kBoundWarps * 32) page_bound_kernel(BoundArgs a) {
+  // kSets groups of 8 pages per warp are loaded together (all page ids first, then all
+  // summary pieces), so that each warp keeps kSets * 8 page summaries in flight.
+  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
+  constexpr int kPagesPerWarp = 8 * kSets;
+  // A page's summary in units of 16-byte pieces: 64 (f32) or 32 (f16).
+  constexpr int kPieces = F16 ? 32 : 64;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if constexpr (HHR_BOUND_LOOKAHEAD > 0) {
+    // Reads only inputs no earlier kernel of the step writes (page table, lengths); a
+    // prefetch of a summary that the previous kernel is updating is coherent in L2.
+    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int total = gridDim.x * gridDim.y * gridDim.z;
+    if (lin < a.early && lane < kPagesPerWarp) {
+#pragma unroll
+      for (int j = 0; j < HHR_BOUND_LOOKAHEAD; ++j) {
+        const int t = lin + j * a.early;
+        if (t < total) {
+          const int tx = t % gridDim.x, ty = (t / gridDim.x) % gridDim.y;
+          const int tb = t / (gridDim.x * gridDim.y);
+          const int tg = bound_group_of(tx, ty);
+          const int p = bound_chunk_of(tx, ty) * kBoundWarps * kPagesPerWarp +
+                        warp * kPagesPerWarp + lane;
+          if (p < min(ceil_div(a.seq_len[tb], a.P), a.maxp)) {
+            const int phys = a.page_table[(size_t)tb * a.maxp + p];
+            if (phys >= 0 && phys < a.n_phys)
+              prefetch_l2(reinterpret_cast<const uint4*>(a.page_minmax) +
+                              ((size_t)phys * a.G + (PH ? tg / a.kv_div : tg)) * kPieces,
+                          kPieces * 16);
+          }
+        }
+      }
+    }
+  }
+  pdl_wait();
+  pdl_trigger();
+  const int r = bound_group(), b = blockIdx.z;  // selection row r reads KV head r / kv_div
+  const int npg = min(ceil_div(a.seq_len[b], a.P), a.maxp);
+  const int p0 = bound_chunk() * kBoundWarps * kPagesPerWarp + warp * kPagesPerWarp;
+  if (p0 >= npg) return;
+  float4 q0, q1;
+  bound_query<F16>(a, b, r, PH, lane, q0, q1);
+  bound_warp<F16>(a, b, r, PH ? r / a.kv_div : r, p0, npg, lane, q0, q1);
 }
 
 // Pages covered by one CTA of page_bound_kernel.
@@ -463,7 +690,7 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
 #pragma unroll
     for (int j = 0; j < kSelLoadUnroll; ++j) {
       const int i = base + j * NT + tid;
-      f[j] = i < n ? sc[i] : -INFINITY;
+      f[j] = i < n ? __ldcg(sc + i) : -INFINITY;  // may come from other CTAs of a kernel
     }
 #pragma unroll
     for (int j = 0; j < kSelLoadUnroll; ++j) {
@@ -766,13 +993,14 @@ struct HamShared {
 
 // Steps a3-a4 for one (sequence, group) row on the cluster's CTA `rank`, given the row's
 // kept logical pages klp[0..m) (ascending) and their physical pages kphys (-1 invalid),
-// in shared memory. CTA r scores candidates [r*half, (r+1)*half); the histograms and the
-// compaction offsets are combined through distributed shared memory.
+// in shared memory; n = the sequence's keys. CTA r scores candidates [r*half, (r+1)*half); the
+// histograms and the compaction offsets are combined through distributed shared memory.
 // hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
 template <int NB, int CW, int NT>
 __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
                                      const int32_t* kphys, int m, const uint32_t* qcs,
-                                     uint32_t (*planes)[CW][4], uint32_t* hsm, HamShared& hs) {
+                                     uint32_t (*planes)[CW][4], uint32_t* hsm, HamShared& hs,
+                                     int n) {
   // Ranked distance: 0 for a key of a forced page, else 1 + delta (bins 0 .. gs*32*CW + 1).
   constexpr int kBins = (kMaxGroup * 32 * CW + 2 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
@@ -785,7 +1013,6 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   m = min(m, a.m_max);
   int* hist = reinterpret_cast<int*>(hsm);                                // [nbins]
   uint16_t* dist = reinterpret_cast<uint16_t*>(hist + ((nbins + 31) & ~31));  // [half], 16B-aligned
-  const int n = a.seq_len[b];
   const int npg = min(ceil_div(max(n, 0), a.P), a.maxp);  // pages of the sequence
   const int C = min(m * a.P, kMaxCand);
   const int half = ((ceil_div(C, kHamRanks) + 7) / 8) * 8;
@@ -973,6 +1200,14 @@ struct TopmHammingArgs {
   int flat;             // every page is kept (flat hash top-k): no bounds, no top-m
 };
 
+// 1: the kept-page pass prefetches each kept page's codes into L2 for the Hamming stage.
+// Measured on B200 (128K context, batch 8, clock stamps per phase): the 256 bulk prefetches
+// per CTA slow the kept-page pass by 0.4 us and speed the Hamming stage by 0.26 us, so the
+// default is 0.
+#ifndef HHR_TOPM_CODE_PREFETCH
+#define HHR_TOPM_CODE_PREFETCH 0
+#endif
+
 // Per-warp ballots of the kept-page pass of topm_hamming_kernel: NT / 32 warps share the
 // 32768 pages a sequence may hold, in 32-page chunks.
 constexpr int kTopmPages = 32768;
@@ -986,31 +1221,41 @@ struct TopmShared {
   static_assert(kWarps <= 32, "the warp-prefix scan covers the warps with one warp");
 };
 
+// Static shared memory of one selection (top-m + Hamming top-k of one row).
+template <int NT>
+struct TopmSmem {
+  SelShared sh;
+  HamShared hs;
+  uint32_t qcs[kMaxGroup * kMaxCodeWords];   // the row's query codes
+  uint32_t planes[2][kMaxCodeWords][4];      // their bit planes
+  TopmShared<NT> ts;
+};
+
+// Top-m pages and the Hamming top-k of selection row `row`, on CTA `rank` of its cluster of
+// kHamRanks CTAs (NT threads each; call uniformly). fsm: topm_hamming_smem() bytes of dynamic
+// shared memory. Bounds are read through L2. The row's length and first page-table entries
+// (inputs that no earlier kernel writes) are loaded first; with dep_wait the programmatic
+// dependency wait comes after them, before anything an earlier kernel writes is read.
 template <int NB, int CW, int NT>
-__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_blocks<CW, NT>())
-    topm_hamming_kernel(TopmHammingArgs a) {
+__device__ __forceinline__ void topm_hamming_row(const TopmHammingArgs& a, int row, int rank,
+                                                 TopmSmem<NT>& S, uint32_t* fsm, bool dep_wait) {
   static_assert(NT == 512 || (NT == 1024 && CW <= 4), "512 threads, or 1024 up to 4 words");
   constexpr int kTopmWarps = NT / 32;
-  __shared__ SelShared sh;
-  __shared__ HamShared hs;
-  __shared__ uint32_t qcs[kMaxGroup * CW];     // the group's query codes
-  __shared__ uint32_t planes[2][CW][4];         // their bit planes
-  __shared__ TopmShared<NT> ts;
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ uint32_t fsm[];
+  SelShared& sh = S.sh;
+  HamShared& hs = S.hs;
+  uint32_t* qcs = S.qcs;
+  uint32_t(*planes)[CW][4] = reinterpret_cast<uint32_t(*)[CW][4]>(&S.planes[0][0][0]);
+  TopmShared<NT>& ts = S.ts;
   const HammingArgs& h = a.h;
-  const int row = blockIdx.x / kHamRanks, rank = blockIdx.x % kHamRanks;
   const int b = row / h.Gs, r = row % h.Gs;
   const int g = h.kv_div == 1 ? r : r / h.kv_div;  // no division on the grouped path
   const int gs = h.Hq / h.Gs;  // query heads of the row
-  if (threadIdx.x < gs * CW)  // visible after the selection's first barrier
-    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + r * gs) * CW + threadIdx.x];
   const int mw = (h.m_max + 3) & ~3;
   int32_t* kept_s = reinterpret_cast<int32_t*>(fsm);
   int32_t* kphys_s = kept_s + mw;
   uint32_t* work = fsm + 2 * mw;
-  const int n = min(ceil_div(max(h.seq_len[b], 0), h.P), h.maxp);
+  const int n_keys = h.seq_len[b];
+  const int n = min(ceil_div(max(n_keys, 0), h.P), h.maxp);
   // Kept pages: warp w owns pages [w R, (w + 1) R), R a multiple of 32, visited 32 at a time
   // (page w R + 32 j + lane), so that kept flags come from ballots and kept positions from
   // popcounts; every lane with a kept page then does its writes at once.
@@ -1023,6 +1268,9 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
   const uint32_t* code_g = h.codes + (size_t)g * h.P * CW;
   const size_t code_page = (size_t)h.G * h.P * CW;
   if (a.flat) {  // flat hash top-k: the kept list is every page of the sequence
+    if (dep_wait) pdl_wait();
+    if (threadIdx.x < gs * CW)  // visible after the barrier below
+      qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + r * gs) * CW + threadIdx.x];
     const int m = min(n, h.m_max);
     for (int p = threadIdx.x; p < m; p += NT) {
       int phys = ptab[p];
@@ -1036,7 +1284,8 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
     }
     if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
     __syncthreads();
-    hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
+    hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs,
+                                     n_keys);
     return;
   }
   int pt[kTopmPtPre];  // page-table entries of the first chunks, loaded with the bounds
@@ -1045,6 +1294,9 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
     const int p = wbase + 32 * j + lane;
     pt[j] = (j < J && p < n) ? ptab[p] : -1;
   }
+  if (dep_wait) pdl_wait();
+  if (threadIdx.x < gs * CW)  // visible after the selection's first barrier
+    qcs[threadIdx.x] = h.q_code[((size_t)b * h.Hq + r * gs) * CW + threadIdx.x];
   const SelCut cut = block_select_cut<NT>(a.bounds + (size_t)row * h.maxp, n, work, sh,
                                           true, a.m_pages, a.keep_div, 0, h.sink, h.local);
   int ng = 0, ne = 0;
@@ -1095,7 +1347,7 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
       if (phys < 0 || phys >= h.n_phys) {
         flag_status(kStatusBadPage);
         phys = -1;
-      } else {
+      } else if (HHR_TOPM_CODE_PREFETCH) {
         prefetch_l2(code_g + (size_t)phys * code_page, (unsigned)(h.P * CW * 4));
       }
       if (kpos < h.m_max) {
@@ -1108,7 +1360,17 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
   }
   if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
   __syncthreads();
-  hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs);
+  hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs,
+                                   n_keys);
+}
+
+template <int NB, int CW, int NT>
+__global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_blocks<CW, NT>())
+    topm_hamming_kernel(TopmHammingArgs a) {
+  __shared__ TopmSmem<NT> S;
+  pdl_trigger();
+  extern __shared__ uint32_t fsm[];
+  topm_hamming_row<NB, CW, NT>(a, blockIdx.x / kHamRanks, blockIdx.x % kHamRanks, S, fsm, true);
 }
 
 inline size_t topm_hamming_smem(int gs, int cw, int m_max, int P, int maxp) {

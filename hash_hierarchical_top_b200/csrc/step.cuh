@@ -32,6 +32,9 @@ struct PrologueArgs {
   uint32_t* q_code;        // [B][Hq][CW]
   float* qpn;              // [B][G][2][d]
   int Hq, G, P, maxp, n_phys, summary_fp16;
+  // L2 warm-up for page_bound_stage_kernel: the first warm_units units (pages, all groups'
+  // summaries, unit_bytes each) of each of its warm_ctas CTAs' chunk ranges; 0 = none.
+  int warm_units, warm_ctas, unit_bytes, chunk;
 };
 
 
@@ -134,6 +137,39 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
     if (w < CW) load_row16(a.W + (size_t)g * (32 * CW) * kD, w * 32 + lrow, wr[i]);
   }
   const int len = a.seq_len[b];
+  // L2 warm-up for the page-bound kernel that follows, while HBM is otherwise idle here:
+  // thread t of the grid takes unit t % warm_units of that kernel's CTA t / warm_units, whose
+  // range of chunks starts at chunk cta * C / warm_ctas (C chunks of `chunk` pages over the
+  // sequences in order, as that kernel cuts them). It reads only inputs (lengths, page table);
+  // a summary this kernel updates is prefetched coherently (L2 holds the update).
+  const int t_lin = ((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) *
+                        kPrologueThreads + tid;
+  const void* warm = nullptr;
+  if (a.warm_units > 0 && t_lin < a.warm_units * a.warm_ctas) {
+    const int B = gridDim.z;
+    auto chunks_of = [&](int bb) {
+      return ceil_div(min(ceil_div(max(a.seq_len[bb], 0), a.P), a.maxp), a.chunk);
+    };
+    int C = 0;
+    for (int bb = 0; bb < B; ++bb) C += chunks_of(bb);
+    const int cta = t_lin / a.warm_units, u = t_lin - cta * a.warm_units;
+    int id = (int)((long long)cta * C / a.warm_ctas) + u / a.chunk;
+    const int id_end = (int)((long long)(cta + 1) * C / a.warm_ctas);
+    if (id < id_end) {
+      int wb = 0;
+      for (; wb < B; ++wb) {
+        const int nc = chunks_of(wb);
+        if (id < nc) break;
+        id -= nc;
+      }
+      const int wp = id * a.chunk + u % a.chunk;
+      if (wb < B && wp < min(ceil_div(max(a.seq_len[wb], 0), a.P), a.maxp)) {
+        const int ph = a.page_table[(size_t)wb * a.maxp + wp];
+        if (ph >= 0 && ph < a.n_phys)
+          warm = static_cast<const char*>(a.page_minmax) + (size_t)ph * a.unit_bytes;
+      }
+    }
+  }
   // Threads [16v, 16v + 16) load vector v (k_new, then the queries) as 16-byte pieces of
   // 8 channels; threads [16 NV, 16 NV + 16) load v_new.
   const int pv = tid >> 4, c8 = (tid & 15) * 8;
@@ -163,6 +199,7 @@ __global__ void __cluster_dims__(kPrologueRanks, 1, 1) __launch_bounds__(kProlog
   float mn = INFINITY, mx = -INFINITY;
   if (has_key && s.slot > 0 && row_lead) load_summary_row(a.page_minmax, a.summary_fp16, s.sbase, row, mn, mx);
   __syncthreads();
+  if (warm != nullptr) prefetch_l2(warm, (unsigned)a.unit_bytes);
 
   // Rotation (steps a0 and a1) of every vector on this thread's row.
   float y[NV];
