@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "encode.cuh"
 #include "encode_tc.cuh"
+#include "indexer.cuh"
 #include "select.cuh"
 #include "step.cuh"
 
@@ -31,6 +32,11 @@ constexpr size_t kMaxKernelSmem = 200 * 1024;  // below the 227 KB opt-in of sm_
 #define HHR_WARM_MB 44
 #endif
 constexpr size_t kWarmBytes = (size_t)HHR_WARM_MB << 20;
+// Indexer mode runs as one cluster of kIxRanks CTAs per query (indexer_cluster_kernel) when
+// there are at most this many queries (B x T) and the sizes fit; else as four kernels.
+#ifndef HHR_IX_CLUSTER_MAX_QUERIES
+#define HHR_IX_CLUSTER_MAX_QUERIES 8
+#endif
 // Page bounds: 1 = page_bound_stage_kernel (summaries staged page-major in shared memory by
 // bulk copies), 0 = page_bound_kernel (summaries loaded to registers).
 #ifndef HHR_BOUND_STAGE
@@ -116,7 +122,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
   return e;
 }
 
-bool g_smem_stage[2][kMaxDevices], g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
+bool g_smem_ix[kMaxDevices], g_smem_stage[2][kMaxDevices], g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
     g_smem_sel[kMaxDevices], g_smem_ham[3][2][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
     g_smem_attn_cl[kMaxDevices];
 
@@ -270,6 +276,39 @@ cudaError_t launch_bounds_kernel(const hhr_dims* d, const BoundArgs& ba, bool pd
   if (pdl) return launch_pdl(k, grid, dim3(kBoundWarps * 32), 0, s, ba);
   k<<<grid, kBoundWarps * 32, 0, s>>>(ba);
   return cudaGetLastError();
+}
+
+// Whether a cluster of kIxRanks CTAs of indexer_cluster_kernel can be resident on this
+// device with `smem` bytes of dynamic shared memory (checked once per device; the kernel's
+// non-portable cluster size is enabled on the way). 0 unknown, 1 yes, -1 no.
+int g_ix_ok[kMaxDevices];
+bool indexer_cluster_ready(size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (allow_smem(indexer_cluster_kernel, smem, g_smem_ix) != cudaSuccess) return false;
+  if (g_ix_ok[dev] == 0) {
+    int ok = -1;
+    if (cudaFuncSetAttribute(indexer_cluster_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kIxRanks, 1);
+      cfg.blockDim = dim3(kIxThreads);
+      cfg.dynamicSmemBytes = ix_smem(kIxMaxBlocks, kIxMaxCand / 128, 128);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kIxRanks;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, indexer_cluster_kernel, &cfg) == cudaSuccess && n > 0)
+        ok = 1;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error
+    g_ix_ok[dev] = ok;
+  }
+  return g_ix_ok[dev] == 1;
 }
 
 int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
@@ -451,6 +490,38 @@ int hhr_select(const hhr_dims* d, int mode, const uint16_t* q, const int32_t* se
 
   // Indexer variant (HISA).
   const int T = Hq;
+  const size_t ixs = ix_smem(maxp, m_max, P);
+  if ((long long)B * T <= HHR_IX_CLUSTER_MAX_QUERIES && maxp <= kIxMaxBlocks &&
+      (long long)m_max * P <= kIxMaxCand && indexer_cluster_ready(ixs)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kIxRanks, B * T);
+    cfg.blockDim = dim3(kIxThreads);
+    cfg.dynamicSmemBytes = ixs;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kIxRanks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    prof_begin(HHR_KERNEL_BLOCK, s);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, indexer_cluster_kernel,
+        IxArgs{q, block_mean, k_cache, page_table, seq_len, q_pos, bounds, kept, kept_count,
+               reinterpret_cast<float*>(ws + L.tok), out_idx, out_count, T, P, maxp,
+               d->n_phys_pages, m_pages, m_max, top_k});
+    prof_end(HHR_KERNEL_BLOCK, s);
+    if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+    if (trace != nullptr) {
+      if ((st = copy_trace(trace->bounds, ws, L.bounds, (size_t)B * T * maxp * 4, s))) return st;
+      if ((st = copy_trace(trace->kept, ws, L.kept, (size_t)B * T * m_max * 4, s))) return st;
+      if ((st = copy_trace(trace->kept_count, ws, L.kept_count, (size_t)B * T * 4, s))) return st;
+    }
+    return HHR_OK;
+  }
   float* tok = reinterpret_cast<float*>(ws + L.tok);
   if (allow_smem(block_score_kernel, block_score_smem(), g_smem_blk) != cudaSuccess)
     return HHR_ERR_CUDA;

@@ -645,8 +645,15 @@ __device__ __forceinline__ void block_count_minmax(int cnt, uint32_t lo, uint32_
   if (kTailSync) __syncthreads();  // before sh is reused
 }
 
+// HC copies of each radix histogram: lane l adds into copy l % HC, so that lanes of one warp
+// whose keys share a digit contend less on one shared-memory address; the scan sums the
+// copies. Measured on B200: 4 copies take the standalone selection kernel of the 64-query
+// indexer chunk from 72.6 to 65.8 us; the 4096-bound top-m of the Hamming kernel is not faster
+// with them (2.32 -> 2.43 us of radix passes), so it keeps one.
+template <int HC = 1>
 struct SelShared {
-  int hist[2][256];  // double-buffered: a pass zeroes the next pass's histogram
+  static constexpr int kCopies = HC;
+  int hist[2][HC][256];  // double-buffered: a pass zeroes the next pass's histogram
   int scratch[66];
   uint32_t mm[96];
   int res[2][3];     // per pass (alternating): digit, rem, cnt
@@ -677,23 +684,24 @@ struct SelCut {
 // the scores in keys[0..n) (shared memory, 16-byte aligned). Forced entries i < sink and
 // i >= n - local take the largest key (above every finite score) and, when by_kept, k is at
 // least their number.
-template <int NT>
+// LU: score loads in flight per thread.
+template <int NT, int LU = kSelLoadUnroll, int HC = 1>
 __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint32_t* keys,
-                                                   SelShared& sh, bool by_kept, int m_pages,
+                                                   SelShared<HC>& sh, bool by_kept, int m_pages,
                                                    int keep_div, int top_k, int sink = 0,
                                                    int local = 0) {
   const int tid = threadIdx.x;
   int nfin = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int base = 0; base < n; base += kSelLoadUnroll * NT) {
-    float f[kSelLoadUnroll];
+  for (int base = 0; base < n; base += LU * NT) {
+    float f[LU];
 #pragma unroll
-    for (int j = 0; j < kSelLoadUnroll; ++j) {
+    for (int j = 0; j < LU; ++j) {
       const int i = base + j * NT + tid;
       f[j] = i < n ? __ldcg(sc + i) : -INFINITY;  // may come from other CTAs of a kernel
     }
 #pragma unroll
-    for (int j = 0; j < kSelLoadUnroll; ++j) {
+    for (int j = 0; j < LU; ++j) {
       const int i = base + j * NT + tid;
       const bool forced = i < n && (i < sink || i >= n - local);
       const bool live = forced || f[j] > -INFINITY;
@@ -730,20 +738,28 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
       // Two barriers per pass: the histogram and the pass result alternate between two
       // buffers, and a pass zeroes the other histogram while it fills its own.
       int cur = 0;
-      if (tid < 256) sh.hist[0][tid] = 0;
+      for (int i = tid; i < HC * 256; i += NT) (&sh.hist[0][0][0])[i] = 0;
       __syncthreads();
+      const int copy = (tid & 31) % HC;
       while (true) {
         for (int i = tid; i < n; i += NT) {
           const uint32_t kk = keys[i];
-          if (kk != 0u && (kk & mask) == prefix) atomicAdd(&sh.hist[cur][(kk >> shift) & 255], 1);
+          if (kk != 0u && (kk & mask) == prefix)
+            atomicAdd(&sh.hist[cur][copy][(kk >> shift) & 255], 1);
         }
-        if (tid < 256) sh.hist[cur ^ 1][tid] = 0;
+        for (int i = tid; i < HC * 256; i += NT) (&sh.hist[cur ^ 1][0][0])[i] = 0;
         __syncthreads();
         if (tid < 32) {
           // Lane l covers digits 255-8l .. 248-8l (descending).
           int cq[8], sum = 0;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { cq[q] = sh.hist[cur][255 - 8 * tid - q]; sum += cq[q]; }
+          for (int q = 0; q < 8; ++q) {
+            int c = 0;
+#pragma unroll
+            for (int cp = 0; cp < HC; ++cp) c += sh.hist[cur][cp][255 - 8 * tid - q];
+            cq[q] = c;
+            sum += c;
+          }
           const int incl = warp_incl_scan(sum, tid);
           const int excl = incl - sum;
           if (excl < rem && rem <= incl) {
@@ -786,14 +802,15 @@ __device__ __forceinline__ SelCut block_select_cut(const float* sc, int n, uint3
 // ties to the lower index, written in ascending index order to out[0..k) (global or shared
 // memory); see block_select_cut for k. unit > 0 maps index i to kept_units[i / unit] * unit
 // + i % unit. keys: shared scratch of n words (16-byte aligned). Returns k.
-template <int NT = kSelThreads>
+template <int NT = kSelThreads, int LU = kSelLoadUnroll, int HC = 1>
 __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint32_t* keys,
-                                                    SelShared& sh, bool by_kept, int m_pages,
-                                                    int keep_div, int top_k, int32_t* out,
-                                                    int out_stride, const int32_t* kept_units,
-                                                    int unit) {
+                                                    SelShared<HC>& sh, bool by_kept,
+                                                    int m_pages, int keep_div, int top_k,
+                                                    int32_t* out, int out_stride,
+                                                    const int32_t* kept_units, int unit) {
   const int tid = threadIdx.x;
-  const SelCut c = block_select_cut<NT>(sc, n, keys, sh, by_kept, m_pages, keep_div, top_k);
+  const SelCut c =
+      block_select_cut<NT, LU, HC>(sc, n, keys, sh, by_kept, m_pages, keep_div, top_k);
   // Compaction in index order over contiguous per-thread ranges. Before thread t's range
   // are gt_before keys above the cut and eq_before equal to it, of which the first
   // min(eq_before, rem) are taken.
@@ -838,7 +855,7 @@ __device__ __forceinline__ int block_select_largest(const float* sc, int n, uint
 __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ SelShared sh;
+  __shared__ SelShared<4> sh;
   extern __shared__ uint32_t keys[];  // [n], 16-byte aligned
   const int row = blockIdx.x, tid = threadIdx.x;
   const int b = row / a.rows_per_b;
@@ -851,7 +868,7 @@ __global__ void __launch_bounds__(kSelThreads) select_largest_kernel(SelectArgs 
     n = min(a.kept_count[row] * a.unit, a.stride);
   }
   int32_t* out = a.out + (size_t)row * a.out_stride;
-  const int k = block_select_largest(
+  const int k = block_select_largest<kSelThreads, kSelLoadUnroll, 4>(
       a.scores + (size_t)row * a.stride, n, keys, sh, a.mode == 0, a.m_pages, a.keep_div,
       a.top_k, out, a.out_stride,
       a.unit > 0 ? a.kept_units + (size_t)row * a.m_max : nullptr, a.unit);
@@ -1005,7 +1022,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   constexpr int kBins = (kMaxGroup * 32 * CW + 2 + NT - 1) / NT;  // threshold bins per thread
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
-  const int b = row / a.Gs, r = row % a.Gs;
+  const int r = row % a.Gs;
   const int g = a.kv_div == 1 ? r : r / a.kv_div;  // no division on the grouped path
   const int tid = threadIdx.x;
   const int gs = a.Hq / a.Gs;  // query heads of the row
@@ -1224,7 +1241,7 @@ struct TopmShared {
 // Static shared memory of one selection (top-m + Hamming top-k of one row).
 template <int NT>
 struct TopmSmem {
-  SelShared sh;
+  SelShared<1> sh;
   HamShared hs;
   uint32_t qcs[kMaxGroup * kMaxCodeWords];   // the row's query codes
   uint32_t planes[2][kMaxCodeWords][4];      // their bit planes
@@ -1241,7 +1258,7 @@ __device__ __forceinline__ void topm_hamming_row(const TopmHammingArgs& a, int r
                                                  TopmSmem<NT>& S, uint32_t* fsm, bool dep_wait) {
   static_assert(NT == 512 || (NT == 1024 && CW <= 4), "512 threads, or 1024 up to 4 words");
   constexpr int kTopmWarps = NT / 32;
-  SelShared& sh = S.sh;
+  SelShared<1>& sh = S.sh;
   HamShared& hs = S.hs;
   uint32_t* qcs = S.qcs;
   uint32_t(*planes)[CW][4] = reinterpret_cast<uint32_t(*)[CW][4]>(&S.planes[0][0][0]);

@@ -277,7 +277,8 @@ typedef enum {
   HHR_KERNEL_BOUND = 2,      /* hhr_select, hash mode, step a2 bounds */
   HHR_KERNEL_TOPM = 3,       /* hhr_select, indexer mode, top-m blocks */
   HHR_KERNEL_HAMMING = 4,    /* hhr_select, hash mode, top-m pages + steps a3-a4 (fused) */
-  HHR_KERNEL_BLOCK = 5,      /* hhr_select, indexer mode, block scores */
+  HHR_KERNEL_BLOCK = 5,      /* hhr_select, indexer mode, block scores (or the whole
+                                selection, when it runs as one cluster per query) */
   HHR_KERNEL_TOKEN = 6,      /* hhr_select, indexer mode, token scores */
   HHR_KERNEL_TOKEN_TOPK = 7, /* hhr_select, indexer mode, token top-k */
   HHR_KERNEL_ATTN = 8,       /* hhr_sparse_attn, split chunks */
