@@ -11,14 +11,23 @@
 // in fp32 in TMEM — enough for the 1e-4 ||k|| code tolerance, which plain bf16 or tf32
 // operands are not.
 //
-// One persistent CTA of 128 threads per (slot, KV group): it builds B_g once in shared
+// One persistent CTA of 512 threads per (slot, KV group): it builds B_g once in shared
 // memory (M = W_g R_g computed in fp32, then split), then loops over 128-key tiles of its
-// group (4 pages of 32 keys): cp.async gathers the tile's rows through the page table into
-// the 128-byte-swizzled K-major layout, one thread issues 8 k-steps x 3 splits of
-// tcgen05.mma (M=128, N=256, K=16) into a 256-column TMEM accumulator and commits to an
-// mbarrier, then warp w reads TMEM lanes 32w..32w+31 (= the keys of page w of the tile):
-// min/max of each rotated channel over the page by a transposed warp reduction, and the
-// 128 sign bits of each key packed per thread. All mbarrier waits are bounded.
+// group (4 pages of 32 keys) in a two-deep software pipeline. For tile k: the rows, already
+// in registers, are stored into the 128-byte-swizzled K-major A buffer; one thread issues 8
+// k-steps x 3 splits of tcgen05.mma (M=128, N=256, K=16) into one of two 256-column TMEM
+// accumulators and commits to that accumulator's mbarrier; while those MMAs run, the threads
+// load tile k+1's rows (through the page table) into registers and run the epilogue of tile
+// k-1 from the other accumulator: warp w reads TMEM lanes 32(w % 4)..32(w % 4)+31 (= the keys
+// of page w % 4 of the tile), columns of group c = w / 4: rotated channels 32c..32c+31, whose
+// min/max over the page a transposed warp reduction gives, and projections of code word c,
+// whose 32 sign bits each lane packs for its key. Then the CTA waits for tile k's MMAs (the A
+// buffer is free again). A shared-memory double buffer for A does not fit next to the 192 KB
+// of B; registers hold the next tile instead (4 x 16 B per thread).
+// Measured on B200 (prefill of 128K x 8 sequences x 8 groups): with 4 warps the epilogue was
+// instruction-bound (ncu: 6% of warp slots, tensor pipe 23.7% active) and the overlap alone
+// gained 3% (3.12 -> 3.04 ms); 16 warps: 1.89 ms, tensor pipe 40.5%; 32 warps (16 columns
+// each): 2.23 ms, tensor pipe 34%. All mbarrier waits are bounded.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -29,7 +38,7 @@ namespace hhr {
 
 constexpr int kTcTile = 128;               // keys per tile (MMA M)
 constexpr int kTcN = 256;                  // 128 rotated channels + 128 projections (MMA N)
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 512;             // 16 warps: 4 per TMEM lane quarter
 constexpr int kTcSplits = 3;
 constexpr int kTcPage = 32;                // page size served by this kernel
 constexpr uint32_t kTcBHalf = kTcN * 128;  // bytes of one 64-channel half of one split of B
@@ -37,7 +46,9 @@ constexpr uint32_t kTcBSplit = 2 * kTcBHalf;
 constexpr uint32_t kTcBBytes = kTcSplits * kTcBSplit;  // 192 KB
 constexpr uint32_t kTcAHalf = kTcTile * 128;
 constexpr uint32_t kTcABytes = 2 * kTcAHalf;           // 32 KB
-constexpr size_t kTcSmem = kTcBBytes + kTcABytes + 1024 /*alignment*/ + 64 /*barrier, tmem*/;
+constexpr size_t kTcSmem = kTcBBytes + kTcABytes + 1024 /*alignment*/ + 64 /*barriers, tmem*/;
+constexpr uint32_t kTcTmemCols = 2 * kTcN;             // two accumulators
+constexpr int kTcChunks = kTcTile * 16 / kTcThreads;   // 16-byte row chunks per thread
 constexpr int kStatusTimeout = 8;
 constexpr long long kTcWaitLimit = 1ll << 22;  // try_wait polls before giving up
 
@@ -144,7 +155,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
   uint8_t* gB = gbase;
   uint8_t* gA = gbase + kTcBBytes;
   uint32_t* taddr_p = reinterpret_cast<uint32_t*>(gbase + kTcBBytes + kTcABytes + 16);
-  const uint32_t bar = sA + kTcABytes;
+  const uint32_t bar0 = sA + kTcABytes;  // MMA completion of accumulator 0 (bar0 + 8: 1)
 
   // ---- B = [R_g ; W_g R_g] as three bf16 splits, in the swizzled K-major layout -------
   const float* Rg = a.R + (size_t)g * kD * kD;
@@ -160,15 +171,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
     *reinterpret_cast<__nv_bfloat16*>(gB + 2 * kTcBSplit + off) = __float2bfloat16_rn(lo);
   };
   for (int i = tid; i < kD * kD; i += kTcThreads) put_split(i >> 7, i & 127, Rg[i]);
-  // M = W_g R_g: warp w computes rows 32w..32w+31, 8 rows at a time, lane l columns 4l..4l+3.
-  for (int r0 = warp * 32; r0 < warp * 32 + 32; r0 += 8) {
-    float4 acc[8];
+  // M = W_g R_g: warp w computes rows kRowsW w .. kRowsW (w + 1) - 1, 8 rows at a time, lane l
+  // columns 4l..4l+3.
+  constexpr int kRowsW = kD / (kTcThreads / 32);
+  constexpr int kStepR = kRowsW < 8 ? kRowsW : 8;
+  static_assert(kRowsW % kStepR == 0, "whole steps of rows");
+  for (int r0 = warp * kRowsW; r0 < (warp + 1) * kRowsW; r0 += kStepR) {
+    float4 acc[kStepR];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < kStepR; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int l = 0; l < kD; ++l) {
       const float4 rv = __ldg(reinterpret_cast<const float4*>(Rg + (size_t)l * kD) + lane);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kStepR; ++j) {
         const float w = __ldg(Wg + (size_t)(r0 + j) * kD + l);
         acc[j].x = fmaf(w, rv.x, acc[j].x);
         acc[j].y = fmaf(w, rv.y, acc[j].y);
@@ -177,7 +192,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
       }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kStepR; ++j) {
       put_split(kD + r0 + j, 4 * lane + 0, acc[j].x);
       put_split(kD + r0 + j, 4 * lane + 1, acc[j].y);
       put_split(kD + r0 + j, 4 * lane + 2, acc[j].z);
@@ -187,11 +202,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
   // Tensor-core reads of shared memory go through the async proxy.
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 
-  if (tid == 0) mbar_init(bar, 1);
+  if (tid == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+  }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      (uint32_t)__cvta_generic_to_shared(taddr_p)),
-                 "r"((uint32_t)kTcN)
+                 "r"(kTcTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
@@ -201,72 +219,67 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   const uint32_t tmem = *taddr_p;
   const uint32_t idesc = tc_idesc();
-  uint32_t parity = 0;
+  uint32_t parity = 0u;  // bit i: the phase parity the next wait on accumulator i expects
   bool failed = false;
 
+  // This CTA's tiles: j = slot_cta, slot_cta + ctas_per_group, ... that hold appended keys.
   const int total_tiles = a.B * a.tiles_per_seq;
-  for (int j = slot_cta; j < total_tiles && !failed; j += a.ctas_per_group) {
+  auto tile_live = [&](int j) {
     const int b = j / a.tiles_per_seq, ti = j % a.tiles_per_seq;
     int nn = a.n_new[b];
     if (nn > a.max_new) nn = a.max_new;
     const int s0 = a.start[b];
-    if (nn <= 0 || s0 < 0) continue;
-    const int e0 = s0 + nn;
+    if (nn <= 0 || s0 < 0) return false;
     const int T0 = ti * kTcTile;
-    if (T0 >= e0 || T0 + kTcTile <= s0) continue;
-
-    // Gather the tile's rows (positions T0 .. T0+127): 16 chunks of 16 B per row.
-    for (int q = tid; q < kTcTile * 16; q += kTcThreads) {
+    return T0 < s0 + nn && T0 + kTcTile > s0;
+  };
+  auto next_tile = [&](int j) {
+    for (j += a.ctas_per_group; j < total_tiles; j += a.ctas_per_group)
+      if (tile_live(j)) return j;
+    return total_tiles;
+  };
+  // Rows of tile j into registers: thread tid takes chunks q = tid + i * kTcThreads (row q/16,
+  // 16-byte chunk q%16); rows outside the appended range (or of a bad page) are zero.
+  uint4 rows[kTcChunks];
+  auto load_rows = [&](int j) {
+    const int b = j / a.tiles_per_seq, T0 = (j % a.tiles_per_seq) * kTcTile;
+    int nn = a.n_new[b];
+    if (nn > a.max_new) nn = a.max_new;
+    const int s0 = a.start[b], e0 = s0 + nn;
+#pragma unroll
+    for (int i = 0; i < kTcChunks; ++i) {
+      const int q = tid + i * kTcThreads;
       const int r = q >> 4, ch = q & 15;
       const int t = T0 + r;
       const int lp = t / kTcPage;
       int phys = -1;
       if (t >= s0 && t < e0 && lp < a.maxp) {
         phys = a.page_table[(size_t)b * a.maxp + lp];
-        if (phys >= 0 && phys >= a.n_phys) phys = -1;
+        if (phys >= a.n_phys) phys = -1;
       }
-      const uint32_t off = sw128_offset(kTcAHalf, r, ch * 8);
-      if (phys >= 0) {
-        const uint16_t* src = a.k_cache + (((size_t)phys * a.G + g) * kTcPage + (t % kTcPage)) * kD +
-                              ch * 8;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sA + off), "l"(src));
-      } else {
-        *reinterpret_cast<uint4*>(gA + off) = make_uint4(0, 0, 0, 0);
-      }
+      rows[i] = make_uint4(0, 0, 0, 0);
+      if (phys >= 0)
+        rows[i] = __ldcs(reinterpret_cast<const uint4*>(
+            a.k_cache + (((size_t)phys * a.G + g) * kTcPage + (t % kTcPage)) * kD + ch * 8));
     }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-
-    if (tid == 0) {
-#pragma unroll 1
-      for (int s = 0; s < 8; ++s) {  // k-steps of 16 channels
-        const uint32_t koff = (uint32_t)(s & 3) * 32u;  // 16 channels = 32 B into the half
-        const uint64_t da = sw128_desc(sA + (uint32_t)(s >> 2) * kTcAHalf + koff);
+  };
+  auto store_rows = [&]() {
 #pragma unroll
-        for (int sp = 0; sp < kTcSplits; ++sp) {
-          const uint64_t db =
-              sw128_desc(sB + (uint32_t)sp * kTcBSplit + (uint32_t)(s >> 2) * kTcBHalf + koff);
-          tc_mma(tmem, da, db, idesc, (s > 0 || sp > 0) ? 1u : 0u);
-        }
-      }
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                       bar)
-                   : "memory");
+    for (int i = 0; i < kTcChunks; ++i) {
+      const int q = tid + i * kTcThreads;
+      *reinterpret_cast<uint4*>(gA + sw128_offset(kTcAHalf, q >> 4, (q & 15) * 8)) = rows[i];
     }
-    const bool ok = mbar_wait(bar, parity);
-    if (__syncthreads_or(!ok)) {  // one decision for the whole CTA
-      failed = true;
-      if (tid == 0) flag_status(kStatusTimeout);
-      break;
-    }
-    parity ^= 1u;
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-
-    // Epilogue: warp w holds the keys of page w of the tile (positions T0 + 32w + lane).
-    const int t = T0 + warp * 32 + lane;
+  };
+  // Epilogue of tile j from accumulator acc (its MMAs complete).
+  auto epilogue = [&](int j, int acc) {
+    const int b = j / a.tiles_per_seq, T0 = (j % a.tiles_per_seq) * kTcTile;
+    int nn = a.n_new[b];
+    if (nn > a.max_new) nn = a.max_new;
+    const int s0 = a.start[b], e0 = s0 + nn;
+    // Warp w holds the keys of page w % 4 of the tile (positions T0 + 32 (w % 4) + lane) and
+    // column group cb = w / 4 (rotated channels 32cb.., code word cb).
+    const int quarter = warp & 3, cb = warp >> 2;
+    const int t = T0 + quarter * 32 + lane;
     const int lp = t / kTcPage;
     const bool valid = t >= s0 && t < e0;
     int phys = -1;
@@ -275,13 +288,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
     const bool page_ok = __shfl_sync(kFull, phys, 0) >= 0;
     const int pstart = lp * kTcPage;
     const bool any_valid = __any_sync(kFull, valid);
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tmem + (uint32_t)(acc * kTcN) + ((uint32_t)(quarter * 32) << 16);
     // Rotated channels: per-page min/max (page-uniform phys: all lanes of the warp share lp).
     if (any_valid && page_ok) {
       const size_t sbase = ((size_t)phys * a.G + g) * 2 * kD;
       const bool merge = s0 > pstart;  // the page already held keys before this call
-#pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
+      {
         float v[32], w[32];
         tmem_ld32(trow + (uint32_t)(cb * 32), v);
 #pragma unroll
@@ -310,9 +322,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
           mm[kD + ch] = mx;
         }
       }
-      // Projections: 128 sign bits of this lane's key, 4 words.
-#pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
+      // Projections: code word cb of this lane's key (32 sign bits).
+      {
         float v[32];
         tmem_ld32(trow + (uint32_t)(kD + cb * 32), v);
         uint32_t word = 0;
@@ -324,16 +335,63 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(EncodeTcArgs a
     } else if (any_valid && lane == 0) {
       flag_status(kStatusBadPage);
     }
+  };
+
+  int cur = tile_live(slot_cta) ? slot_cta : next_tile(slot_cta);
+  int prev = -1, acc = 0;
+  if (cur < total_tiles) load_rows(cur);
+  while (cur < total_tiles) {
+    // The A buffer is free (the previous tile's MMAs completed): tile cur's rows go in.
+    store_rows();
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t bar = bar0 + 8u * (uint32_t)acc;
+    if (tid == 0) {
+      const uint32_t d = tmem + (uint32_t)(acc * kTcN);
+#pragma unroll 1
+      for (int s = 0; s < 8; ++s) {  // k-steps of 16 channels
+        const uint32_t koff = (uint32_t)(s & 3) * 32u;  // 16 channels = 32 B into the half
+        const uint64_t da = sw128_desc(sA + (uint32_t)(s >> 2) * kTcAHalf + koff);
+#pragma unroll
+        for (int sp = 0; sp < kTcSplits; ++sp) {
+          const uint64_t db =
+              sw128_desc(sB + (uint32_t)sp * kTcBSplit + (uint32_t)(s >> 2) * kTcBHalf + koff);
+          tc_mma(d, da, db, idesc, (s > 0 || sp > 0) ? 1u : 0u);
+        }
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                       bar)
+                   : "memory");
+    }
+    // While tile cur's MMAs run: the next tile's rows into registers, the previous tile's
+    // epilogue from the other accumulator.
+    const int nxt = next_tile(cur);
+    if (nxt < total_tiles) load_rows(nxt);
+    if (prev >= 0) epilogue(prev, acc ^ 1);
+    const bool ok = mbar_wait(bar, (parity >> acc) & 1u);
+    if (__syncthreads_or(!ok)) {  // one decision for the whole CTA
+      failed = true;
+      if (tid == 0) flag_status(kStatusTimeout);
+      break;
+    }
+    parity ^= 1u << acc;
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    prev = cur;
+    cur = nxt;
+    acc ^= 1;
   }
+  if (!failed && prev >= 0) epilogue(prev, acc ^ 1);
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
 
-  // On a time-out, give outstanding MMAs a bounded chance to finish before freeing TMEM.
-  if (failed) mbar_wait(bar, parity);
+  // On a time-out, give the outstanding MMAs a bounded chance to finish before freeing TMEM.
+  if (failed) mbar_wait(bar0 + 8u * (uint32_t)acc, (parity >> acc) & 1u);
   __syncthreads();
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
-                 "r"((uint32_t)kTcN)
+                 "r"(kTcTmemCols)
                  : "memory");
 }
 
