@@ -102,7 +102,7 @@ def step_kernel_bytes(wl, lens, m_of, sbytes=4):
     rotated queries and folded queries written); bound = bound_kernel_bytes; hamming = the
     bounds, the kept pages' page-table entries and codes read, the selected ids and cache
     rows written; attn = the selected rows' offsets, K and V read, the queries read and the
-    outputs written."""
+    outputs written; row = bound + hamming + attn (the small-batch kernel that does all three)."""
     G, Hq, d, P = wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.page_size
     rows = Hq if wl.select_per_head else G
     B = len(lens)
@@ -117,8 +117,9 @@ def step_kernel_bytes(wl, lens, m_of, sbytes=4):
         ham += rows * (npg * 4 + m * 4 + cand * (wl.code_bits // 8) + k * 8)
         attn += rows * k * (4 + 2 * d * 2)
     attn += B * Hq * d * (2 + 4)
-    return {"encode": enc, "bound": bound_kernel_bytes(wl, lens, sbytes), "hamming": ham,
-            "attn": attn}
+    bound = bound_kernel_bytes(wl, lens, sbytes)
+    return {"encode": enc, "bound": bound, "hamming": ham, "attn": attn,
+            "row": bound + ham + attn}
 
 
 def kernel_table(kern_us, kbytes, peak_gbs):
@@ -850,8 +851,12 @@ def main():
                   inp["R"], inp["W"], cache, start, one)
 
     fused = args.path == "fused" and not args.select_only
+    # Small batches: hhr_decode_step runs steps a2-a5 as one cluster per selection row.
+    row_path = fused and hhr.hhr_decode_step_kernels(d0, wl.m_pages, wl.keep_div, wl.top_k) == 2
     if args.select_only:
         names = ("encode", "qprep", "bound", "hamming")
+    elif row_path:
+        names = ("encode", "row")
     elif args.path == "fused":
         names = ("encode", "bound", "hamming", "attn", "combine")
     else:
@@ -865,8 +870,9 @@ def main():
 
     # Each decode step is one CUDA graph replay (one launch from the host). NG graphs cycle
     # over the L layer caches; graph j carries its own event pair around the dominant kernel
-    # (the page bounds), so the last NG replays of the timed region give its duration.
-    rk = "bound"
+    # (the page bounds, or the row clusters on the small-batch path), so the last NG replays
+    # of the timed region give its duration.
+    rk = "row" if row_path else "bound"
     NG = L * max(1, 48 // L)
     ev_b = timing_events(NG, stream)
     graphs = []
@@ -1095,7 +1101,7 @@ def main():
     achieved = bound_bytes / (bound_avg_ms / 1e3) / 1e9
     # DRAM bytes of the profiled launch, scaled to this launch's algorithmic bytes (the
     # kernel's traffic grows in proportion to the pages and rows it reads).
-    rk_name = f"page_bound_{args.summary}"
+    rk_name = "row_cluster" if row_path else f"page_bound_{args.summary}"
     prof = traffic_from_profile(f"{rk_name}_kernel_{wl.name}.txt", kernel_source_hash())
     traffic = prof[0] * bound_bytes / prof[1] if prof is not None else None
     step_gbs = req / (ms_step / 1e3) / 1e9
@@ -1137,8 +1143,9 @@ def main():
                        "api": "hhr_decode_step" if args.path == "fused" else
                               "hhr_encode_keys + hhr_select + hhr_sparse_attn",
                        "timing": f"CUDA-graph replay per step, CUDA events on the stream; the "
-                                 f"last {nbr} of {K} replays carry event nodes around the page-bound "
-                                 f"kernel (its duration for the roofline)"},
+                                 f"last {nbr} of {K} replays carry event nodes around the "
+                                 f"{'row-cluster' if row_path else 'page-bound'} kernel (its "
+                                 f"duration for the roofline)"},
             "roofline": {"bound": "hbm", "kernel": f"{rk_name}_kernel",
                          "scope": "the dominant kernel alone (its CUDA-event duration in "
                                   "bracketed replays); the whole step's fraction is step_hbm",

@@ -34,7 +34,10 @@ constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kTile = 64;                        // selected rows per pipeline stage
 constexpr int kStages = 3;
 constexpr int kMaxSplitRows = 2048;              // rows of one split (offsets in smem)
-constexpr int kTargetCtas = 2 * 148;             // two resident CTAs on each of 148 SMs
+#ifndef HHR_ATTN_TARGET_CTAS
+#define HHR_ATTN_TARGET_CTAS (2 * 148)             // two resident CTAs on each of 148 SMs
+#endif
+constexpr int kTargetCtas = HHR_ATTN_TARGET_CTAS;
 constexpr uint32_t kNoRow = 0xffffffffu;          // offset table: row to skip
 
 struct AttnArgs {

@@ -13,6 +13,7 @@
 #include "encode.cuh"
 #include "encode_tc.cuh"
 #include "indexer.cuh"
+#include "row_cluster.cuh"
 #include "select.cuh"
 #include "step.cuh"
 
@@ -39,6 +40,21 @@ constexpr size_t kWarmBytes = (size_t)HHR_WARM_MB << 20;
 #endif
 // Page bounds: 1 = page_bound_stage_kernel (summaries staged page-major in shared memory by
 // bulk copies), 0 = page_bound_kernel (summaries loaded to registers).
+// 1: hhr_decode_step runs steps a2-a5 of small batches (at most one wave of row clusters)
+// in row_cluster_kernel; 0: always the chain of separate kernels.
+#ifndef HHR_ROW_CLUSTER
+#define HHR_ROW_CLUSTER 1
+#endif
+// Largest batch x selection rows x pages per sequence for the row-cluster path. Its bounds
+// run on the rows' clusters only (64 SMs for 8 rows of 8 CTAs), at about the per-SM rate of
+// the page-bound kernel, so past a few MB of summaries the separate page-bound kernel on every
+// SM wins. Measured on B200 (one sequence of 8 KV groups, f16 summaries, L2-cold): 32K context
+// (8 x 1024 pages) 34.7 us per step against 36.5 us for the kernel chain; 128K (8 x 4096
+// pages) 39.1 against 35.2 us.
+#ifndef HHR_ROW_MAX_PAGES
+#define HHR_ROW_MAX_PAGES 16384
+#endif
+
 #ifndef HHR_BOUND_STAGE
 #define HHR_BOUND_STAGE 0
 #endif
@@ -124,7 +140,7 @@ cudaError_t allow_smem(K kernel, size_t bytes, bool* done_per_dev) {
 
 bool g_smem_ix[kMaxDevices], g_smem_stage[2][kMaxDevices], g_smem_tc[kMaxDevices], g_smem_encode[3][kMaxDevices], g_smem_qprep[3][kMaxDevices],
     g_smem_sel[kMaxDevices], g_smem_ham[3][2][4][kMaxDevices], g_smem_blk[kMaxDevices], g_smem_attn[kMaxDevices],
-    g_smem_attn_cl[kMaxDevices];
+    g_smem_attn_cl[kMaxDevices], g_smem_row[kRowVariants][kMaxDevices];
 
 struct SelectLayout {
   size_t qpn, q_rot, q_code, bounds, kept, kept_count, tok, total;
@@ -309,6 +325,69 @@ bool indexer_cluster_ready(size_t smem) {
     g_ix_ok[dev] = ok;
   }
   return g_ix_ok[dev] == 1;
+}
+
+// How many clusters of row_cluster_kernel instantiation `index` (`ranks` CTAs of
+// kRowThreads threads) can be resident at once on this device: checked once per device and
+// instantiation (a non-portable cluster size is enabled on the way); 0 when it cannot run
+// or `smem` bytes of dynamic shared memory do not fit.
+int g_row_cap[kMaxDevices][kRowVariants];
+int row_cluster_capacity(RowClusterFn fn, int index, int ranks, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (allow_smem(fn, smem, g_smem_row[index]) != cudaSuccess) return 0;
+  int& cap = g_row_cap[dev][index];
+  if (cap == 0) {
+    int n = -1;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(ranks);
+      cfg.blockDim = dim3(kRowThreads);
+      cfg.dynamicSmemBytes = attn_smem();
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = ranks;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) n = -1;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error
+    cap = n;
+  }
+  return cap > 0 ? cap : 0;
+}
+
+// hhr_decode_step's steps a2-a5 as row_cluster_kernel: used when the codes are 128-bit, the
+// batch's rows hold at most HHR_ROW_MAX_PAGES pages in all, the row's attention splits fit
+// the cluster and every selection row's cluster is resident at once: clusters of 16 CTAs
+// where they all fit, else of 8.
+struct RowPlan {
+  bool use;
+  int ranks;
+  RowClusterFn fn;
+  size_t smem;
+  AttnPlan attn;
+};
+RowPlan row_plan(const hhr_dims* d, int m_max, int top_k) {
+  RowPlan p{};
+  if (!HHR_ROW_CLUSTER || code_words(d) != 4) return p;
+  const int Gs = sel_rows(d), rh = d->n_q_heads / Gs;
+  const bool f16 = d->summary_fp16 != 0;
+  const long long rows = (long long)d->batch * Gs;
+  if (rows * d->max_pages_per_seq > HHR_ROW_MAX_PAGES) return p;
+  for (int ranks : {16, 8}) {
+    p.ranks = ranks;
+    p.attn = attn_plan(d->batch, Gs, top_k, ranks);
+    p.fn = row_cluster_for(rh, f16, ranks);
+    p.smem = row_cluster_smem(rh, 4, m_max, d->page_size, d->max_pages_per_seq, ranks);
+    p.use = p.attn.n_splits <= ranks &&
+            rows <= row_cluster_capacity(p.fn, row_cluster_index(rh, f16, ranks), ranks, p.smem);
+    if (p.use) break;
+  }
+  return p;
 }
 
 int copy_trace(void* dst, const char* ws, size_t off, size_t bytes, cudaStream_t s) {
@@ -727,24 +806,62 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
                    d->summary_fp16, warm_units, warm_ctas, ub, kStageChunk});
   prof_end(HHR_KERNEL_ENCODE, s);
   if ((st = launch_status()) != HHR_OK) return st;
+  const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
+                     d->n_phys_pages, 0, Gs, kv_div(d), B};
+  HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
+                 Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, row_buf, sink, local,
+                 Gs, kv_div(d)};
+  ha.pf_k = k_cache;
+  ha.pf_v = v_cache;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  // a2-a5 of small batches: one cluster per selection row.
+  {
+    const RowPlan rp = row_plan(d, m_max, top_k);
+    if (rp.use) {
+      ha.pf_split = rp.attn.split_rows;
+      const AttnArgs aa{q, k_cache, v_cache, page_table, seq_len, out_idx, out_count, nullptr,
+                        nullptr, out, scale_log2, Hq, G, P, maxp, d->n_phys_pages, top_k,
+                        rp.attn.n_splits, rp.attn.split_rows, row_buf, Gs, kv_div(d)};
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(rp.ranks * B * Gs);
+      cfg.blockDim = dim3(kRowThreads);
+      cfg.dynamicSmemBytes = rp.smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = rp.ranks;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      prof_begin(HHR_KERNEL_ROW, s);
+      e = cudaLaunchKernelEx(&cfg, rp.fn,
+                             RowClusterArgs{ba, TopmHammingArgs{ha, bounds, m_pages, keep_div,
+                                                                flat ? 1 : 0},
+                                            aa, kv_div(d) > 1 ? 1 : 0});
+      prof_end(HHR_KERNEL_ROW, s);
+      if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
+      return HHR_OK;
+    }
+  }
   // a2: page bounds (none when every page is kept: a flat hash top-k).
   if (!flat) {
     // Launched behind the prologue. With f32 summaries (page_bound_kernel) its first CTAs
     // warm L2 while the prologue runs, unless an event is recorded between the two
     // (profiling), which leaves no overlap to use.
-    const int early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
-    const BoundArgs ba{qpn, q_rot, page_minmax, page_table, seq_len, bounds, G, P, maxp,
-                       d->n_phys_pages, early, Gs, kv_div(d), B};
+    BoundArgs bw = ba;
+    bw.early = g_prof[HHR_KERNEL_BOUND].start != nullptr ? 0 : 3 * sm_count();
     prof_begin(HHR_KERNEL_BOUND, s);
-    e = launch_bounds_kernel(d, ba, true, s);
+    e = launch_bounds_kernel(d, bw, true, s);
     prof_end(HHR_KERNEL_BOUND, s);
     if (e != cudaSuccess) { g_last_cuda = e; return HHR_ERR_CUDA; }
   }
   // a2 top-m + a3 + a4: kept pages, Hamming distances, deterministic top-k.
   {
-    HammingArgs ha{q_code, codes, page_table, seq_len, kept, kept_count, out_idx, out_count,
-                   Hq, G, P, maxp, d->n_phys_pages, m_max, top_k, row_buf, sink, local,
-                   Gs, kv_div(d)};
+    const AttnPlan cp = attn_plan(B, Gs, top_k, kMaxClusterSplits);
+    ha.pf_split = cp.n_splits <= kMaxClusterSplits ? cp.split_rows : plan.split_rows;
     prof_begin(HHR_KERNEL_HAMMING, s);
     e = launch_pdl(topm_hamming_for(rh, cw, nt), dim3(B * Gs * kHamRanks), dim3(nt), fsm, s,
                    TopmHammingArgs{ha, bounds, m_pages, keep_div, flat ? 1 : 0});
@@ -797,6 +914,18 @@ int hhr_decode_step(const hhr_dims* d, const uint16_t* q, const uint16_t* k_new,
     }
   }
   return HHR_OK;
+}
+
+int hhr_decode_step_kernels(const hhr_dims* d, int m_pages, int keep_div, int top_k) {
+  const int st = check_select_params(d, HHR_MODE_HASH, m_pages, keep_div, top_k);
+  if (st != HHR_OK) return st;
+  const int m_max = kept_max(d, m_pages, keep_div);
+  if (row_plan(d, m_max, top_k).use) return 2;
+  const bool flat = m_max >= d->max_pages_per_seq;
+  const int ns = attn_plan(d->batch, sel_rows(d), top_k).n_splits;
+  const bool cluster = attn_plan(d->batch, sel_rows(d), top_k, kMaxClusterSplits).n_splits <=
+                       kMaxClusterSplits;
+  return 2 + (flat ? 0 : 1) + (cluster || ns == 1 ? 1 : 2);
 }
 
 int hhr_read_device_status(void* stream, int* bits) {

@@ -259,11 +259,13 @@ __device__ __forceinline__ void bound_query(const BoundArgs& a, int b, int r, bo
 // One warp's share of the page bounds of selection row r (KV head g) of sequence b: pages
 // [p0, p0 + kPagesPerWarp) (those below npg), written to a.bounds (-inf and a status bit for a
 // page id outside the pool). All page ids are loaded first, then all summary pieces, so that
-// the warp keeps kPagesPerWarp page summaries in flight.
-template <bool F16>
+// the warp keeps kPagesPerWarp = 8 * kSets page summaries in flight (SETS: kSets, or 0 for
+// the page-bound kernel's setting).
+template <bool F16, int SETS = 0>
 __device__ __forceinline__ void bound_warp(const BoundArgs& a, int b, int r, int g, int p0,
                                            int npg, int lane, float4 q0, float4 q1) {
-  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
+  constexpr int kSets = SETS > 0 ? SETS : F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
+  static_assert(8 * kSets <= 32, "one page id per lane");
   constexpr int kPagesPerWarp = 8 * kSets;
   constexpr int kPieces = F16 ? 32 : 64;
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);
@@ -923,7 +925,17 @@ struct HammingArgs {
                              // sequence uses the KV head r / kv_div and query heads
                              // [r Hq/Gs, (r + 1) Hq/Gs); bounds, kept lists and outputs are
                              // indexed by (sequence, row)
+  // With out_rows: the K/V rows of output positions p with p % pf_split < HHR_ATTN_PREFETCH_ROWS
+  // (the first tiles of each attention split) are prefetched into L2 (pf_split 0: none).
+  const uint16_t* pf_k = nullptr;
+  const uint16_t* pf_v = nullptr;
+  int pf_split = 0;
 };
+
+// Selected K/V rows prefetched into L2 per attention split by the compaction (0: none).
+#ifndef HHR_ATTN_PREFETCH_ROWS
+#define HHR_ATTN_PREFETCH_ROWS 0
+#endif
 
 inline int hamming_planes(int gs) { return 32 - __builtin_clz((unsigned)gs); }
 
@@ -1008,12 +1020,14 @@ struct HamShared {
   int tot[2];  // lower-ranked CTAs' (#below threshold, #at threshold): this rank's output offsets
 };
 
-// Steps a3-a4 for one (sequence, group) row on the cluster's CTA `rank`, given the row's
-// kept logical pages klp[0..m) (ascending) and their physical pages kphys (-1 invalid),
+// Steps a3-a4 for one (sequence, group) row on the cluster's CTA `rank` (of RANKS), given the
+// row's kept logical pages klp[0..m) (ascending) and their physical pages kphys (-1 invalid),
 // in shared memory; n = the sequence's keys. CTA r scores candidates [r*half, (r+1)*half); the
 // histograms and the compaction offsets are combined through distributed shared memory.
-// hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads.
-template <int NB, int CW, int NT>
+// hsm: hamming_smem() bytes of shared memory. Call uniformly by all threads. Ends with the
+// cluster's shared memory released (a cluster barrier that does not order the compaction's
+// global writes: a caller that reads them in other CTAs synchronises the cluster again).
+template <int NB, int CW, int NT, int RANKS = kHamRanks>
 __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int row, int rank, const int32_t* klp,
                                      const int32_t* kphys, int m, const uint32_t* qcs,
                                      uint32_t (*planes)[CW][4], uint32_t* hsm, HamShared& hs,
@@ -1032,7 +1046,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   uint16_t* dist = reinterpret_cast<uint16_t*>(hist + ((nbins + 31) & ~31));  // [half], 16B-aligned
   const int npg = min(ceil_div(max(n, 0), a.P), a.maxp);  // pages of the sequence
   const int C = min(m * a.P, kMaxCand);
-  const int half = ((ceil_div(C, kHamRanks) + 7) / 8) * 8;
+  const int half = ((ceil_div(C, RANKS) + 7) / 8) * 8;
   const int lo = min(C, rank * half), hi = min(C, lo + half);
   const int Cr = hi - lo;
   for (int i = tid; i < nbins; i += NT) hist[i] = 0;
@@ -1100,7 +1114,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
       lv[q] = 0;
       if (i < nbins) {
 #pragma unroll
-        for (int r = 0; r < kHamRanks; ++r) {
+        for (int r = 0; r < RANKS; ++r) {
           const int c = cl.map_shared_rank(hist, r)[i];
           hv[q] += c;
           if (r < rank) lv[q] += c;
@@ -1131,7 +1145,7 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
     }
     if (tid == 0) a.out_count[row] = keff;  // every rank writes the same value
     __syncthreads();
-    for (int i = keff + rank * NT + tid; i < a.top_k; i += kHamRanks * NT)
+    for (int i = keff + rank * NT + tid; i < a.top_k; i += RANKS * NT)
       a.out_idx[(size_t)row * a.top_k + i] = -1;
   }
   const int T = hs.T, need_eq = hs.need_eq, lt_off = hs.tot[0], eq_off = hs.tot[1];
@@ -1184,9 +1198,16 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
           const int pi = (a.P == 1) ? i : (int)__umulhi((uint32_t)i, magic);
           const int slot = i - pi * a.P;
           out[pos] = klp[pi] * a.P + slot;
-          if (a.out_rows != nullptr)
-            a.out_rows[(size_t)row * a.top_k + pos] =
+          if (a.out_rows != nullptr) {
+            const uint32_t crow =
                 ((uint32_t)kphys[pi] * (uint32_t)a.G + (uint32_t)g) * (uint32_t)a.P + (uint32_t)slot;
+            a.out_rows[(size_t)row * a.top_k + pos] = crow;
+            if (HHR_ATTN_PREFETCH_ROWS > 0 && a.pf_split > 0 &&
+                pos % a.pf_split < HHR_ATTN_PREFETCH_ROWS && kphys[pi] >= 0) {
+              prefetch_l2(a.pf_k + (size_t)crow * kD, kD * 2);
+              prefetch_l2(a.pf_v + (size_t)crow * kD, kD * 2);
+            }
+          }
           ++pos;
         }
       }
@@ -1195,12 +1216,12 @@ __device__ __forceinline__ void hamming_topk_cluster(const HammingArgs& a, int r
   cluster_wait();  // keep this CTA's shared memory alive until every rank has read it
 }
 
-inline size_t hamming_smem(int gs, int cw, int m_max, int P) {
+inline size_t hamming_smem(int gs, int cw, int m_max, int P, int ranks = kHamRanks) {
   const int nbins = gs * 32 * cw + 2;
   const size_t ints = (size_t)((nbins + 31) & ~31);
   // This rank's distances, padded so the 16-byte group reads of the last thread stay inside.
   const size_t c = (size_t)m_max * P < (size_t)kMaxCand ? (size_t)m_max * P : (size_t)kMaxCand;
-  const size_t half = ((c + kHamRanks - 1) / kHamRanks + 7) & ~(size_t)7;
+  const size_t half = ((c + ranks - 1) / ranks + 7) & ~(size_t)7;
   return ints * 4 + (half + 8) * 2 + 16;
 }
 
@@ -1249,11 +1270,11 @@ struct TopmSmem {
 };
 
 // Top-m pages and the Hamming top-k of selection row `row`, on CTA `rank` of its cluster of
-// kHamRanks CTAs (NT threads each; call uniformly). fsm: topm_hamming_smem() bytes of dynamic
+// RANKS CTAs (NT threads each; call uniformly). fsm: topm_hamming_smem() bytes of dynamic
 // shared memory. Bounds are read through L2. The row's length and first page-table entries
 // (inputs that no earlier kernel writes) are loaded first; with dep_wait the programmatic
 // dependency wait comes after them, before anything an earlier kernel writes is read.
-template <int NB, int CW, int NT>
+template <int NB, int CW, int NT, int RANKS = kHamRanks>
 __device__ __forceinline__ void topm_hamming_row(const TopmHammingArgs& a, int row, int rank,
                                                  TopmSmem<NT>& S, uint32_t* fsm, bool dep_wait) {
   static_assert(NT == 512 || (NT == 1024 && CW <= 4), "512 threads, or 1024 up to 4 words");
@@ -1301,8 +1322,8 @@ __device__ __forceinline__ void topm_hamming_row(const TopmHammingArgs& a, int r
     }
     if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
     __syncthreads();
-    hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs,
-                                     n_keys);
+    hamming_topk_cluster<NB, CW, NT, RANKS>(h, row, rank, kept_s, kphys_s, m, qcs, planes,
+                                            work, hs, n_keys);
     return;
   }
   int pt[kTopmPtPre];  // page-table entries of the first chunks, loaded with the bounds
@@ -1377,8 +1398,8 @@ __device__ __forceinline__ void topm_hamming_row(const TopmHammingArgs& a, int r
   }
   if (rank == 0 && threadIdx.x == 0) const_cast<int32_t*>(h.kept_count)[row] = m;
   __syncthreads();
-  hamming_topk_cluster<NB, CW, NT>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work, hs,
-                                   n_keys);
+  hamming_topk_cluster<NB, CW, NT, RANKS>(h, row, rank, kept_s, kphys_s, m, qcs, planes, work,
+                                          hs, n_keys);
 }
 
 template <int NB, int CW, int NT>
@@ -1390,9 +1411,10 @@ __global__ void __cluster_dims__(kHamRanks, 1, 1) __launch_bounds__(NT, ham_min_
   topm_hamming_row<NB, CW, NT>(a, blockIdx.x / kHamRanks, blockIdx.x % kHamRanks, S, fsm, true);
 }
 
-inline size_t topm_hamming_smem(int gs, int cw, int m_max, int P, int maxp) {
+inline size_t topm_hamming_smem(int gs, int cw, int m_max, int P, int maxp,
+                                int ranks = kHamRanks) {
   const size_t sel = (size_t)maxp * 4;
-  const size_t ham = hamming_smem(gs, cw, m_max, P);
+  const size_t ham = hamming_smem(gs, cw, m_max, P, ranks);
   return (size_t)((m_max + 3) & ~3) * 8 + (sel > ham ? sel : ham);
 }
 

@@ -29,11 +29,11 @@ EXPORTED = [
     "hhr_encode_keys", "hhr_kept_max", "hhr_select_workspace_bytes", "hhr_select",
     "hhr_attn_workspace_bytes", "hhr_sparse_attn", "hhr_read_device_status",
     "hhr_status_string", "hhr_profile_next", "hhr_last_cuda_error", "hhr_sparse_attn_noalloc",
-    "hhr_decode_step_workspace_bytes", "hhr_decode_step",
+    "hhr_decode_step_workspace_bytes", "hhr_decode_step", "hhr_decode_step_kernels",
 ]
 
 KERNELS = ["encode", "qprep", "bound", "topm", "hamming", "block", "token", "token_topk", "attn",
-           "combine"]
+           "combine", "row"]
 KERNEL_ID = {name: i for i, name in enumerate(KERNELS)}
 
 
@@ -105,6 +105,8 @@ def lib():
         L.hhr_decode_step.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
                                       i32, po, ctypes.c_float, vp, vp, vp, vp, sz, vp]
         L.hhr_decode_step.restype = i32
+        L.hhr_decode_step_kernels.argtypes = [pd, i32, i32, i32]
+        L.hhr_decode_step_kernels.restype = i32
         L.hhr_sparse_attn_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp, i32,
                                               ctypes.c_float, vp, vp]
         L.hhr_sparse_attn_noalloc.restype = i32
@@ -237,6 +239,15 @@ def hhr_profile_next(kernel, start_event, stop_event):
     k = KERNEL_ID[kernel] if isinstance(kernel, str) else int(kernel)
     ev = lambda e: ctypes.c_void_p(e.cuda_event) if e is not None else None
     _check("hhr_profile_next", lib().hhr_profile_next(k, ev(start_event), ev(stop_event)))
+
+
+def hhr_decode_step_kernels(d, m_pages, keep_div, top_k) -> int:
+    """Kernels one hhr_decode_step call launches (2 on the small-batch row-cluster path)."""
+    n = int(lib().hhr_decode_step_kernels(ctypes.byref(d), int(m_pages), int(keep_div),
+                                          int(top_k)))
+    if n < 0:
+        raise HHRError("hhr_decode_step_kernels", n)
+    return n
 
 
 def hhr_sparse_attn_noalloc(d, q, k_cache, v_cache, page_table, seq_len, idx, count, top_k,

@@ -221,12 +221,25 @@ size_t hhr_decode_step_workspace_bytes(const hhr_dims* dims, int m_pages, int ke
                                        int top_k);
 
 /* One whole HHR decode step (steps a0-a5) in one call, for a decode loop that appends one
- * key/value row per sequence and then attends: equal, bit for bit, to
+ * key/value row per sequence and then attends: the same codes, summaries, selections and
+ * counts, bit for bit, as
  *   hhr_encode_keys(start = seq_len - 1, n_new = 1) + hhr_select(HHR_MODE_HASH) +
  *   hhr_sparse_attn,
  * but with the append encoder and the query preparation fused into one kernel (one read
- * of R and W), top-m fused with the Hamming top-k, and the kernels chained with
- * programmatic dependent launch.
+ * of R and W) and the kernels chained with programmatic dependent launch. Steps a2-a5 run
+ * in one of two ways:
+ *   - small batches (128-bit codes, every selection row's cluster resident at once, at most
+ *     16384 pages over all rows: e.g. one sequence of 8 KV groups up to 64K keys): one
+ *     kernel, a cluster of 16 CTAs (where all rows' clusters fit) or 8 CTAs per selection row
+ *     doing its bounds, top-m, Hamming top-k and attention (at most 16 or 8 attention splits
+ *     per row, merged in the cluster);
+ *   - otherwise: the page bounds, top-m fused with the Hamming top-k, and the attention, its
+ *     splits merged inside a cluster of at most 8 CTAs (or by a combine kernel).
+ * The attention output is identical bit for bit to hhr_sparse_attn's wherever the latter's
+ * split plan has no more splits than the fused path's cluster (16 or 8 CTAs; every size of
+ * the tests); otherwise the fused call merges fewer, larger splits and its outputs can differ in
+ * the last bits (both within the attention tolerance). hhr_decode_step_kernels tells how
+ * many kernels a call launches.
  *   seq_len : lengths after the append; the newest row of sequence b is position
  *             seq_len[b] - 1 (its page must be mapped in page_table).
  *   k_new, v_new : bf16 [B][G][d] newest rows, written into k_cache/v_cache at that
@@ -240,6 +253,12 @@ int hhr_decode_step(const hhr_dims* dims, const uint16_t* q, const uint16_t* k_n
                     int keep_div, int top_k, const hhr_select_opts* opts, float scale,
                     int32_t* out_idx, int32_t* out_count, float* out, void* workspace,
                     size_t ws_bytes, void* stream);
+
+/* Number of kernels one hhr_decode_step call with these dims and budgets launches on the
+ * current device: 2 when steps a2-a5 run as one cluster per selection row (small batches),
+ * else 3 to 5 (the bound kernel is skipped when every page is kept, the combine kernel runs
+ * when a row's attention splits exceed one cluster). Negative status on invalid input. */
+int hhr_decode_step_kernels(const hhr_dims* dims, int m_pages, int keep_div, int top_k);
 
 /* hhr_sparse_attn without a workspace argument, for callers that cannot allocate
  * device memory themselves: runtimes without a device allocator, code running
@@ -283,7 +302,9 @@ typedef enum {
   HHR_KERNEL_TOKEN_TOPK = 7, /* hhr_select, indexer mode, token top-k */
   HHR_KERNEL_ATTN = 8,       /* hhr_sparse_attn, split chunks */
   HHR_KERNEL_COMBINE = 9,    /* hhr_sparse_attn, merge of the chunks */
-  HHR_KERNEL_COUNT = 10
+  HHR_KERNEL_ROW = 10,       /* hhr_decode_step, small batches: bounds, top-m, Hamming top-k
+                                and attention of each selection row in one cluster */
+  HHR_KERNEL_COUNT = 11
 } hhr_kernel;
 
 /* Measurement hook (no counterpart on the pages): the next launch of `kernel` by

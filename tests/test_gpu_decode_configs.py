@@ -1,7 +1,8 @@
 """hhr_decode_step, the call the benchmark times, against the fp64 oracle on the full-size
 configurations: Llama-3.1-8B shapes at 128K context and batch 8 (4096 pages of 32 keys per
-sequence, keep 1/16, top-2048, 128-bit codes, f16 summaries), and the ragged batch of 32
-sequences of 8K..128K keys in a permuted page pool (top-1024).
+sequence, keep 1/16, top-2048, 128-bit codes, f16 summaries), the same at batch 1 and at 32K
+context (keep 1/8, top-3276; on the small-batch path, one cluster per selection row),
+and the ragged batch of 32 sequences of 8K..128K keys in a permuted page pool (top-1024).
 
 The cache is built as a serving loop holds it at a decode step: positions [0, n - 1) of every
 sequence are prefilled with the bulk (tensor-core) encoder, and the newest key/value rows are
@@ -23,7 +24,7 @@ from parity_helpers import check_hash_group, dims_of
 pytestmark = pytest.mark.gpu
 
 
-def _decode_step_outputs(wl):
+def _decode_step_outputs(wl, expect_kernels=None):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
     d = dims_of(wl, inp, 1)
@@ -36,6 +37,8 @@ def _decode_step_outputs(wl):
     # The newest rows are not in the cache yet: only the decode step can put them there.
     inp["k_cache"][phys, :, t % P] = 0
     inp["v_cache"][phys, :, t % P] = 0
+    if expect_kernels is not None:
+        assert hhr.hhr_decode_step_kernels(d, wl.m_pages, wl.keep_div, wl.top_k) == expect_kernels
     cache = LayerCache(d, "cuda")
     step = DecodeStep(d, hhr.HHR_MODE_HASH, wl.m_pages, wl.keep_div, wl.top_k, "cuda")
     z = torch.zeros(B, dtype=torch.int32, device="cuda")
@@ -97,4 +100,29 @@ def test_decode_step_ragged_batch32():
     for j, b in enumerate(picks):
         for g in (j % 8, (j + 5) % 8):
             check_hash_group(wl, inp_np, g_out, b, g, rep)
+    print(rep)
+
+
+def test_decode_step_llama8b_128k_batch1():
+    """One sequence at 128K (32768 pages over its 8 KV groups: the kernel chain, not the
+    row-cluster path). Every group."""
+    wl = S.WORKLOADS["llama8b_128k_b1"]
+    inp, g_out = _decode_step_outputs(wl, expect_kernels=4)
+    assert np.all(g_out["count"] == wl.top_k)
+    inp_np = S.to_numpy_inputs(inp)
+    rep = {}
+    for g in range(8):
+        check_hash_group(wl, inp_np, g_out, 0, g, rep)
+    print(rep)
+
+
+def test_decode_step_llama8b_32k():
+    """32K context, keep 1/8 (128 of 1024 pages), top-3276 over the 4096 kept keys; small-batch
+    path. Groups 0, 3 and 7."""
+    wl = S.WORKLOADS["llama8b_32k"]
+    inp, g_out = _decode_step_outputs(wl, expect_kernels=2)
+    inp_np = S.to_numpy_inputs(inp)
+    rep = {}
+    for g in (0, 3, 7):
+        check_hash_group(wl, inp_np, g_out, 0, g, rep)
     print(rep)

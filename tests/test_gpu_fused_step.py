@@ -80,10 +80,36 @@ def test_fused_step_per_head(heads):
     _fused_vs_separate(wl, 1, True)
 
 
-def _fused_vs_separate(wl, f16, with_new_rows):
+@pytest.mark.parametrize("case", ["groups", "f32", "forced", "per_head", "flat", "gs2",
+                                  "short_seq"])
+def test_fused_step_row_cluster(case):
+    """Small batches run steps a2-a5 as one cluster of 16 or 8 CTAs per selection row (2
+    kernels per call). With at most 8 attention splits per row in both plans (top-k <= 512),
+    the fused call equals the separate calls bit for bit."""
+    kw = dict(batch=1, ragged=(12000, 20000), top_k=512)
+    f16 = 1
+    if case == "f32":
+        f16 = 0
+    elif case == "forced":
+        kw.update(sink_pages=1, local_pages=2)
+    elif case == "per_head":
+        kw.update(n_q_heads=8, n_kv_heads=1, select_per_head=True)
+    elif case == "flat":
+        kw.update(m_pages=4096, keep_div=0, ragged=(5000, 9000), top_k=512)
+    elif case == "gs2":
+        kw.update(batch=2, n_q_heads=8, n_kv_heads=4, top_k=448)
+    elif case == "short_seq":
+        kw.update(batch=4, n_q_heads=4, n_kv_heads=2, ragged=(33, 3000), top_k=300)
+    wl = S.scaled(S.WORKLOADS["ragged_b32"], **kw)
+    _fused_vs_separate(wl, f16, True, expect_kernels=2)
+
+
+def _fused_vs_separate(wl, f16, with_new_rows, expect_kernels=None):
     build.build()
     inp = S.make_inputs(wl, device="cuda")
     d = dims_of(wl, inp, f16)
+    if expect_kernels is not None:
+        assert hhr.hhr_decode_step_kernels(d, wl.m_pages, wl.keep_div, wl.top_k) == expect_kernels
     lens = inp["seq_len"]
     G, P = wl.n_kv_heads, wl.page_size
     # The newest row of each sequence: remember it, and (for the k_new path) wipe it from
