@@ -314,11 +314,12 @@ def popcount32(x):
     return ((x * 0x01010101) & 0xFFFFFFFF) >> 24
 
 
-def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=None):
+def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=None, hot=None):
     """Encode layer inputs `inp` with rotation R (and projection W, default inp["W"], of
     wl.code_bits rows), select wl.top_k keys with the given page budget and score the
     selection against the exact group logits' top-k_true (default wl.top_k; see
-    selection_quality)."""
+    selection_quality). hot: {sequence: [planted hot pages of each KV group]}, for the share
+    of them the page stage keeps."""
     import statistics
     import torch
     from hash_hierarchical_top_b200 import hhr
@@ -343,7 +344,7 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
     st.select(inp["q"], inp["seq_len"], inp["page_table"], cache, R=R, W=W,
               trace=hhr.make_trace(q_code=qcode, kept=kept, kept_count=kcnt))
     torch.cuda.synchronize()
-    rec, mass, page_rec, ham_rec, rho = [], [], [], [], []
+    rec, mass, page_rec, ham_rec, rho, hot_kept = [], [], [], [], [], []
     scale = 1.0 / math.sqrt(wl.head_dim)
     gen = torch.Generator(device=dev).manual_seed(0)
     for b in range(B):
@@ -376,6 +377,9 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
             page_rec.append(float(in_kept.float().mean().item()))
             if bool(in_kept.any()):
                 ham_rec.append(recall_at_k(sel, true[in_kept]))
+            if hot is not None:
+                hp = torch.tensor(hot[b][g], device=dev, dtype=torch.long)
+                hot_kept.append(float(torch.isin(hp, kp).float().mean().item()))
             if full:
                 codes = cache.codes[pages, g].reshape(npg * P, CW)[:n]
                 qc = qcode[b, g * gs:(g + 1) * gs]                        # [gs][CW]
@@ -388,6 +392,8 @@ def hhr_quality(wl, inp, dev, R, m_pages, keep_div, full=True, W=None, k_true=No
            "hamming_recall_within_kept_pages": statistics.mean(ham_rec) if ham_rec else None,
            "k": wl.top_k, "k_true": k_true or wl.top_k, "kept_pages": st.m_max,
            "rows": B * rows}
+    if hot_kept:
+        res["hot_pages_kept"] = statistics.mean(hot_kept)
     if full:
         res["spearman_minus_hamming_vs_logit"] = statistics.mean(rho)
         res["random_selection_mass"] = wl.top_k / float(inp["seq_len"].float().mean())
@@ -448,8 +454,24 @@ def selection_quality(dev):
                                               full=False),
         f"flat_all_{npg}_pages": hhr_quality(wl, inp, dev, inp["R"], npg, 0, full=False)}
     del inp
+    # Planted page locality: the keys each query attends to cluster in a few pages (8 runs of 8
+    # hot pages per KV group, 2048 hot keys); the same stages and budgets as above.
+    wl = S.WORKLOADS["llama8b_128k_planted"]
+    inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
+    hot = {b: S.hot_pages(wl, b, int(inp["seq_len"][b]), 0) for b in range(wl.batch)}
+    every = S.scaled(wl, top_k=256 * wl.page_size)
+    out["hhr_planted_llama8b_128k_b2"] = {
+        "gkr_keep_1/16": hhr_quality(wl, inp, dev, inp["R"], 0, 16, hot=hot),
+        "quest_R_identity_keep_1/16": hhr_quality(wl, inp, dev, eye, 0, 16, full=False, hot=hot),
+        "gkr_keep_1/32": hhr_quality(wl, inp, dev, inp["R"], 0, 32, full=False, hot=hot),
+        "flat_all_4096_pages": hhr_quality(wl, inp, dev, inp["R"], 4096, 0, full=False),
+        "gkr_only_keep_1/16_attend_kept_pages": hhr_quality(
+            every, inp, dev, inp["R"], 0, 16, full=False, k_true=wl.top_k, hot=hot),
+        "planted": f"{wl.hot_runs} runs of {wl.hot_run_pages} hot pages per KV group, keys "
+                   f"shifted by {wl.hot_scale} sqrt(d) along the group's mean query direction"}
+    del inp
     # HISA: hierarchical selection against the flat indexer's causal top-k over all keys.
-    for name in ("hisa_128k_t1", "hisa_128k_t64"):
+    for name in ("hisa_128k_t1", "hisa_128k_t64", "hisa_128k_t1_planted"):
         wl = S.WORKLOADS[name]
         inp = S.make_inputs(wl, device=dev, layer=0, with_values=False)
         d = hhr.make_dims(wl.batch, wl.n_queries, 1, wl.page_size, inp["max_pages"], inp["n_phys"])

@@ -10,7 +10,7 @@
 // drain times on top. Here the rows' clusters cover the GPU and each step runs across the
 // cluster:
 //   1. rank r computes the bounds of its slice of the row's pages (bound_warp, one warp per
-//      8 * kRowBoundSets pages at a time) and writes them;
+//      16 pages at a time) and writes them;
 //   2. after a cluster barrier every rank selects the same top-m pages from all the bounds
 //      (read back through L2) and scores its 1/RANKS share of the kept pages' keys; the
 //      distance histograms are summed and the top-k compacted in token order across the
@@ -32,11 +32,6 @@
 namespace hhr {
 
 constexpr int kRowThreads = 512;   // 16 warps: bound warps, then the selection, then attention
-// Page summaries in flight per bound warp: 8 * kRowBoundSets pages.
-#ifndef HHR_ROW_BOUND_SETS
-#define HHR_ROW_BOUND_SETS 2
-#endif
-constexpr int kRowBoundSets = HHR_ROW_BOUND_SETS;
 constexpr int kRowWarps = kRowThreads / 32;
 static_assert(kRowThreads >= kAttnThreads, "one attention split per CTA");
 
@@ -71,7 +66,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(RowClusterA
 
   // 1. Bounds of this rank's pages: slices of whole 16-page warp units.
   if (!a.sel.flat) {
-    constexpr int kWarpPages = 8 * kRowBoundSets;
+    constexpr int kWarpPages = 8 * (F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32);
     const int npg = min(ceil_div(ba.seq_len[b], ba.P), ba.maxp);
     const int per = ceil_div(ceil_div(npg, RANKS), kWarpPages) * kWarpPages;
     const int lo = rank * per, hi = min(npg, lo + per);
@@ -79,8 +74,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(RowClusterA
       float4 q0, q1;
       bound_query<F16>(ba, b, r, a.per_head != 0, lane, q0, q1);
       for (int p0 = lo + warp * kWarpPages; p0 < hi; p0 += kRowWarps * kWarpPages)
-        bound_warp<F16, kRowBoundSets>(ba, b, r, a.per_head ? r / ba.kv_div : r, p0, hi, lane,
-                                       q0, q1);
+        bound_warp<F16>(ba, b, r, a.per_head ? r / ba.kv_div : r, p0, hi, lane, q0, q1);
     }
     cluster_sync_all();  // every rank's bounds are written (visible cluster-wide)
   }

@@ -259,13 +259,11 @@ __device__ __forceinline__ void bound_query(const BoundArgs& a, int b, int r, bo
 // One warp's share of the page bounds of selection row r (KV head g) of sequence b: pages
 // [p0, p0 + kPagesPerWarp) (those below npg), written to a.bounds (-inf and a status bit for a
 // page id outside the pool). All page ids are loaded first, then all summary pieces, so that
-// the warp keeps kPagesPerWarp = 8 * kSets page summaries in flight (SETS: kSets, or 0 for
-// the page-bound kernel's setting).
-template <bool F16, int SETS = 0>
+// the warp keeps kPagesPerWarp page summaries in flight.
+template <bool F16>
 __device__ __forceinline__ void bound_warp(const BoundArgs& a, int b, int r, int g, int p0,
                                            int npg, int lane, float4 q0, float4 q1) {
-  constexpr int kSets = SETS > 0 ? SETS : F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
-  static_assert(8 * kSets <= 32, "one page id per lane");
+  constexpr int kSets = F16 ? HHR_BOUND_SETS_F16 : HHR_BOUND_SETS_F32;
   constexpr int kPagesPerWarp = 8 * kSets;
   constexpr int kPieces = F16 ? 32 : 64;
   const uint4* base4 = reinterpret_cast<const uint4*>(a.page_minmax);

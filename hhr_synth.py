@@ -62,6 +62,13 @@ class Workload:
     sink_pages: int = 0              # selection variant: forced first pages of a sequence
     local_pages: int = 0             # selection variant: forced last pages of a sequence
     select_per_head: bool = False    # selection variant: one selection per query head
+    # Planted page locality (quality workloads only): per sequence and KV group, hot_runs runs
+    # of hot_run_pages consecutive logical pages whose keys are shifted by
+    # hot_scale * sqrt(head_dim) along the group's mean query direction, so that the keys a
+    # query attends to cluster in a few pages, as relevant context does in real attention.
+    hot_runs: int = 0
+    hot_run_pages: int = 0
+    hot_scale: float = 0.0
 
     @property
     def group_size(self):
@@ -125,6 +132,16 @@ for _bits in (64, 256):
     _n = f"llama8b_128k_b8_codes{_bits}"
     WORKLOADS[_n] = dataclasses.replace(WORKLOADS["llama8b_128k_b8"], name=_n, code_bits=_bits)
 
+# Quality workloads with planted page locality (selection_quality only): the 128K decode at
+# batch 2 with 8 runs of 8 hot pages per KV group (2048 hot keys, as many as the top-k), and
+# the HISA single query with 4 runs of 4 hot 128-key blocks (2048 hot keys).
+WORKLOADS["llama8b_128k_planted"] = dataclasses.replace(
+    WORKLOADS["llama8b_128k_b8"], name="llama8b_128k_planted", cfg_id=6, batch=2,
+    seq_lens=(131072,) * 2, hot_runs=8, hot_run_pages=8, hot_scale=2.5)
+WORKLOADS["hisa_128k_t1_planted"] = dataclasses.replace(
+    WORKLOADS["hisa_128k_t1"], name="hisa_128k_t1_planted", cfg_id=7, n_needles=0,
+    hot_runs=4, hot_run_pages=4, hot_scale=0.5)
+
 
 def scaled(wl: Workload, **changes) -> Workload:
     """A copy of ``wl`` with some fields replaced (e.g. shorter contexts for parity tests)."""
@@ -132,7 +149,7 @@ def scaled(wl: Workload, **changes) -> Workload:
 
 
 # Seed streams: key = 1000*cfg_id + j, j as below, plus the sequence index and layer.
-J_KEYS, J_VALUES, J_QUERIES, J_R, J_W, J_OUTLIER, J_DRIFT, J_LAYOUT, J_NEEDLE = range(9)
+J_KEYS, J_VALUES, J_QUERIES, J_R, J_W, J_OUTLIER, J_DRIFT, J_LAYOUT, J_NEEDLE, J_HOT = range(10)
 
 
 def _gen(device, wl, j, *extra):
@@ -218,6 +235,8 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0, with_values: bool = 
             u = q[b].float().mean(0)
             u = u / u.norm()
             k[:, pos, :] = (wl.needle_scale * math.sqrt(d) * u)[None, None, :]
+        if wl.hot_runs > 0:
+            k = k + _hot_shift(wl, q[b], b, n, layer, device)
         _scatter(k_cache, page_table[b].to(device), k.to(torch.bfloat16), P)
         del k
         if with_values:
@@ -248,6 +267,37 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0, with_values: bool = 
                           dtype=torch.int32)
         out["q_pos"] = qp.to(device)
     return out
+
+
+def hot_pages(wl: Workload, b: int, n: int, layer: int = 0) -> list:
+    """The planted hot logical pages of sequence b (n keys), per KV group: hot_runs runs of
+    hot_run_pages consecutive pages, at distinct run-aligned starts drawn from the sequence's
+    hot stream."""
+    npg = -(-n // wl.page_size)
+    slots = max(npg // wl.hot_run_pages, 1)
+    gh = _gen("cpu", wl, J_HOT, b, layer)
+    out = []
+    for _ in range(wl.n_kv_heads):
+        starts = torch.randperm(slots, generator=gh)[: wl.hot_runs] * wl.hot_run_pages
+        pages = sorted(int(s0) + i for s0 in starts for i in range(wl.hot_run_pages)
+                       if int(s0) + i < npg)
+        out.append(pages)
+    return out
+
+
+def _hot_shift(wl: Workload, qb: torch.Tensor, b: int, n: int, layer: int, device):
+    """Key shift [G][n][d] of the planted hot pages of sequence b: hot_scale * sqrt(d) times
+    the unit mean query direction of each KV group (its query heads, or the chunk queries of
+    the one indexer head)."""
+    G, d, P = wl.n_kv_heads, wl.head_dim, wl.page_size
+    per = qb.shape[0] // G
+    shift = torch.zeros(G, n, d, device=device)
+    for g, pages in enumerate(hot_pages(wl, b, n, layer)):
+        u = qb[g * per:(g + 1) * per].float().mean(0)
+        u = u / u.norm()
+        for p in pages:
+            shift[g, p * P: min((p + 1) * P, n)] = wl.hot_scale * math.sqrt(d) * u
+    return shift
 
 
 def lhp_projection(wl: Workload, layer: int = 0) -> torch.Tensor:
