@@ -243,3 +243,16 @@ def test_noalloc_rejects_sizes_beyond_the_array(L):
     assert st == hhr.HHR_ERR_INVALID_ARG
     st = L.hhr_sparse_attn_noalloc(ctypes.byref(small), *nul, 0, ctypes.c_float(0.1), None, None)
     assert st == hhr.HHR_ERR_INVALID_ARG
+
+
+def test_decode_step_kernel_count_on_the_host(L):
+    """hhr_decode_step_kernels validates like the decode step and, with no GPU to host the
+    small-batch clusters, counts the kernel chain: prologue, bounds (none when every page is
+    kept), top-m + Hamming, attention."""
+    d = hhr.make_dims(8, 32, 8, 32, 4096, 8 * 4096, summary_fp16=1)
+    assert hhr.hhr_decode_step_kernels(d, 0, 16, 2048) == 4
+    assert hhr.hhr_decode_step_kernels(d, 4096, 0, 2048) == 3  # flat: no bound kernel
+    with pytest.raises(hhr.HHRError):
+        hhr.hhr_decode_step_kernels(d, 0, 0, 2048)  # neither m_pages nor keep_div
+    with pytest.raises(hhr.HHRError):
+        hhr.hhr_decode_step_kernels(d, 0, 16, 0)
