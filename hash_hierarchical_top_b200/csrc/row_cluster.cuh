@@ -7,8 +7,9 @@
 // hash codes rank the keys of the pages that survive, and attention runs over the selected
 // keys. With few rows (a batch of one or two sequences) each of the separate kernels runs on a
 // few SMs as a latency chain, and the chain of four launches costs their start-up and
-// drain times on top. Here the rows' clusters cover the GPU and each step runs across the
-// cluster:
+// drain times on top. Here each row's steps run across its cluster, with no kernel boundary
+// (the bounds then use only the clusters' SMs, so the host takes this path only for a few MB
+// of summaries):
 //   1. rank r computes the bounds of its slice of the row's pages (bound_warp, one warp per
 //      16 pages at a time) and writes them;
 //   2. after a cluster barrier every rank selects the same top-m pages from all the bounds
