@@ -84,6 +84,12 @@ def required_bytes(wl, lens, m_of, sbytes=4):
     return summ, codes, kv
 
 
+def dense_kv_bytes(wl, lens):
+    """K and V bytes one dense (full-context) decode step reads: every key and value row of
+    every KV group, for comparison with the step's required bytes."""
+    return sum(lens) * wl.n_kv_heads * wl.head_dim * 2 * 2
+
+
 def bound_kernel_bytes(wl, lens, sbytes=4):
     """Algorithmic bytes of one page-bound launch: per (page, group) the summary read
     (2 x 128 x sbytes) and the 4-byte bound write; per page its 4-byte page-table entry;
@@ -1179,7 +1185,9 @@ def main():
             "step_hbm": {"required_bytes": req, "summaries": summ_b, "codes": codes_b,
                          "kv_rows": kv_b, "achieved_gbs": step_gbs,
                          "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
-                         "frac_of_measured": step_gbs / peak},
+                         "frac_of_measured": step_gbs / peak,
+                         "dense_kv_bytes": dense_kv_bytes(wl, lens),
+                         "dense_over_required": dense_kv_bytes(wl, lens) / req},
             "kernels_us": kern,
             "kernels": kernel_table(kern, kbytes, peak),
             "prefill_encode": prefill,

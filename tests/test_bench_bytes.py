@@ -69,3 +69,13 @@ def test_step_kernel_bytes_and_table():
     assert abs(t["bound"]["gbs"] - 135462912 / 25e-6 / 1e9) < 1e-9
     assert abs(t["bound"]["frac_of_measured"] - t["bound"]["gbs"] / 6548.0) < 1e-12
     assert abs(t["attn"]["frac_of_8tbs"] - t["attn"]["gbs"] / 8000.0) < 1e-12
+
+
+def test_dense_kv_bytes():
+    """A dense step at 128K reads every K and V row of the 8 KV groups: 537 MB per sequence,
+    20.5x the hierarchical step's required bytes with f16 summaries."""
+    wl = S.WORKLOADS["llama8b_128k_b8"]
+    dense = bench.dense_kv_bytes(wl, [131072] * 8)
+    assert dense == 8 * 131072 * 8 * 128 * 2 * 2
+    req = sum(bench.required_bytes(wl, [131072] * 8, KEEP_16, 2))
+    assert abs(dense / req - 20.48) < 0.01
