@@ -239,7 +239,9 @@ size_t hhr_decode_step_workspace_bytes(const hhr_dims* dims, int m_pages, int ke
  * split plan has no more splits than the fused path's cluster (16 or 8 CTAs; every size of
  * the tests); otherwise the fused call merges fewer, larger splits and its outputs can differ in
  * the last bits (both within the attention tolerance). hhr_decode_step_kernels tells how
- * many kernels a call launches.
+ * many kernels a call launches. The first call on a device sets kernel attributes and queries
+ * how many row clusters fit the device (host-side, once per device): make it before capturing
+ * the call into a CUDA graph.
  *   seq_len : lengths after the append; the newest row of sequence b is position
  *             seq_len[b] - 1 (its page must be mapped in page_table).
  *   k_new, v_new : bf16 [B][G][d] newest rows, written into k_cache/v_cache at that
