@@ -510,6 +510,54 @@ def selection_quality(dev):
 
 # ----------------------------------------------------------------------------- other workloads
 
+def measure_dense_attention(layers, wl, dev, stream, steps=200):
+    """Dense decode attention over the whole cache with the library's own attention kernel
+    (every key of every sequence selected: top_k = the context), graph-timed over the same
+    layer caches as the step: the full attention the hierarchical step replaces."""
+    import torch
+    from hash_hierarchical_top_b200 import hhr
+    B, G, Hq, d0 = wl.batch, wl.n_kv_heads, wl.n_q_heads, layers[0][1]
+    L = len(layers)
+    lens = layers[0][0]["seq_len"]
+    n = int(lens.max())
+    idx = torch.arange(n, dtype=torch.int32, device=dev).expand(B, G, n).contiguous()
+    count = lens.to(torch.int32).view(B, 1).expand(B, G).contiguous()
+    ws = torch.empty(hhr.hhr_attn_workspace_bytes(d0, n), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, Hq, wl.head_dim, device=dev)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+
+    def run(l):
+        inp, d = layers[l % L][0], layers[l % L][1]
+        hhr.hhr_sparse_attn(d, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
+                            inp["seq_len"], idx, count, n, scale, out, ws)
+
+    for l in range(L):
+        run(l)
+    torch.cuda.synchronize()
+    st_, bits = hhr.hhr_read_device_status()
+    if st_ != hhr.HHR_OK or not bool(torch.isfinite(out).all()):
+        raise RuntimeError(f"dense attention: device status {bits}")
+    graphs = []
+    for l in range(L):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            run(l)
+        graphs.append(gr)
+    for i in range(2 * L):
+        graphs[i % L].replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        graphs[i % L].replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    kv = dense_kv_bytes(wl, [int(x) for x in lens.tolist()])
+    del graphs
+    return {"api": "hhr_sparse_attn with every key selected (top_k = context)",
+            "us_per_step": ms * 1e3, "kv_bytes": kv, "achieved_gbs": kv / (ms / 1e3) / 1e9}
+
+
 SECONDARY = ("llama8b_128k_b1", "ragged_b32", "llama8b_32k", "tiny_1h_4k", "hisa_128k_t1",
              "hisa_128k_t64", "llama8b_128k_b8_codes64", "llama8b_128k_b8_codes256",
              "llama8b_128k_b8_flat", "llama8b_128k_b8_sink1_local2", "llama8b_128k_b8_per_head")
@@ -1140,6 +1188,14 @@ def main():
     if (rank == 0 and world == 1 and not args.no_secondary and fused and args.batch == 0
             and args.workload == "llama8b_128k_b8"):
         other = {w: measure_secondary(w, dev, l2, f16, 2000, stream, 24 << 30) for w in SECONDARY}
+    dense = None
+    if (rank == 0 and world == 1 and not args.no_secondary and fused and args.batch == 0
+            and args.workload == "llama8b_128k_b8"):
+        try:
+            dense = measure_dense_attention(layers, wl, dev, stream)
+            dense["hhr_step_speedup"] = dense["us_per_step"] / (ms_step * 1e3)
+        except Exception as exc:  # context only: never fail the run over it
+            dense = {"error": f"{type(exc).__name__}: {exc}"}
     quality = None
     if (rank == 0 and world == 1 and not args.no_quality and fused and args.batch == 0
             and args.workload == "llama8b_128k_b8"):
@@ -1192,6 +1248,7 @@ def main():
             "kernels": kernel_table(kern, kbytes, peak),
             "prefill_encode": prefill,
             "other_workloads": other,
+            "dense_attention": dense,
             "selection_quality": quality,
             "cpu_baseline": cpu,
             "e2e": e2e,
